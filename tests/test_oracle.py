@@ -1,0 +1,310 @@
+"""Pins for the fp64 oracle (CPU only).
+
+Each test checks the oracle against something other than itself: a second
+formulation written differently (explicit transition matrices, the chunked
+WY/UT form), or a closed form that the gated delta rule, the conv, the gates or
+the norm fix exactly.  A dropped term, a wrong sign, index or tap order, or a
+transposed operand in the C oracle fails at least one of them.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from hybrid_linear_attention_mixer_b200 import inputs
+
+ACTS = "qkvabz"
+
+
+def _run(shape, w, acts, conv_state, rec_state, cu, **kw):
+    return oracle.forward(shape, w, *[acts[n] for n in ACTS], conv_state, rec_state, cu, **kw)
+
+
+def _random_case(rng, Hk=1, G=2, d=4, T=7, n_seqs=2, K=4, state_std=0.3):
+    Hv = Hk * G
+    shape = oracle.Shape(Hk, Hv, d, d, K)
+    C = shape.channels
+    lens = rng.integers(1, T + 1, n_seqs)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    Tt = int(cu[-1])
+    w = {"conv_w": rng.normal(0, 0.7, (C, K)), "A_log": rng.uniform(-1, 1, Hv),
+         "dt_bias": rng.normal(0, 0.3, Hv), "norm_w": rng.normal(1, 0.2, d)}
+    acts = {"q": rng.normal(size=(Tt, Hk * d)), "k": rng.normal(size=(Tt, Hk * d)),
+            "v": rng.normal(size=(Tt, Hv * d)), "z": rng.normal(size=(Tt, Hv * d)),
+            "a": rng.normal(size=(Tt, Hv)), "b": rng.normal(size=(Tt, Hv))}
+    cs = rng.normal(size=(n_seqs, C, K - 1))
+    rs = rng.normal(0, state_std, (n_seqs, Hv, d, d))
+    return shape, w, acts, cs, rs, cu
+
+
+@pytest.mark.parametrize("seed", [0, 1, 2])
+def test_brute_force_explicit_matrices(seed):
+    """C oracle (rank-1 update) == numpy with explicit alpha (I - beta k k^T) products."""
+    rng = np.random.default_rng(seed)
+    shape, w, acts, cs, rs, cu = _random_case(rng, Hk=2, G=2, d=4, T=8, n_seqs=3)
+    r = _run(shape, w, acts, cs, rs, cu, want_o_pre=True)
+    bf = oracle.brute_force(shape, w, *[acts[n] for n in ACTS], cs, rs, cu)
+    np.testing.assert_allclose(r["o_pre"], bf["o_pre"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r["out"], bf["out"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(r["rec_state"], bf["rec_state"], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("chunk", [1, 3, 16, 64])
+def test_chunked_equals_sequential(chunk):
+    """The chunked WY/UT algebra the GPU kernel uses reaches the sequential result."""
+    rng = np.random.default_rng(10 + chunk)
+    shape, w, acts, cs, rs, cu = _random_case(rng, Hk=2, G=3, d=8, T=150, n_seqs=3)
+    r = _run(shape, w, acts, cs, rs, cu, want_o_pre=True)
+    ch = oracle.chunked(shape, w, *[acts[n] for n in ACTS], cs, rs, cu, chunk=chunk)
+    assert np.abs(ch["o_pre"] - r["o_pre"]).max() <= 1e-10
+    assert np.abs(ch["rec_state"] - r["rec_state"]).max() <= 1e-10
+
+
+def test_chunked_tiny_workload_chunk16():
+    """The tiny workload (T=64, chunk 16): chunked form == sequential oracle."""
+    c = inputs.make_case("tiny")
+    shape = oracle.Shape(c.n_k_heads, c.n_v_heads, c.d_k, c.d_v)
+    r = _run(shape, c.weights, c.acts, c.conv_state, c.rec_state, c.cu_seqlens)
+    ch = oracle.chunked(shape, c.weights, *[c.acts[n] for n in ACTS], c.conv_state,
+                        c.rec_state, c.cu_seqlens, chunk=c.chunk)
+    assert np.abs(ch["out"] - r["out"]).max() <= 1e-10
+    assert np.abs(ch["rec_state"] - r["rec_state"]).max() <= 1e-10
+
+
+def _identity_conv(shape, scale=1.0):
+    w = np.zeros((shape.channels, shape.conv_kernel))
+    w[:, -1] = scale          # only the current token's tap
+    return w
+
+
+def _silu(x):
+    return x / (1.0 + math.exp(-x))
+
+
+def test_exact_overwrite():
+    """alpha = beta = 1 and a unit key: S' k = v after the write, whatever S was."""
+    rng = np.random.default_rng(3)
+    d = 8
+    shape = oracle.Shape(1, 1, d, d, l2_eps=0.0)
+    w = {"conv_w": rng.normal(0, 0.7, (shape.channels, 4)), "A_log": np.array([-1000.0]),
+         "dt_bias": np.zeros(1), "norm_w": np.ones(d)}
+    T = 5
+    acts = {"q": rng.normal(size=(T, d)), "k": rng.normal(size=(T, d)), "v": rng.normal(size=(T, d)),
+            "z": rng.normal(size=(T, d)), "a": rng.normal(size=(T, 1)), "b": np.full((T, 1), 60.0)}
+    cs = rng.normal(size=(1, shape.channels, 3))
+    rs = rng.normal(size=(1, 1, d, d))
+    cu = np.array([0, T], np.int32)
+    r = _run(shape, w, acts, cs, rs, cu)
+    _, kh, vh, la, beta = oracle.features(shape, w, acts["q"], acts["k"], acts["v"], acts["a"],
+                                          acts["b"], cs, cu)
+    assert np.all(la == 0.0) and np.all(beta == 1.0)
+    S = r["rec_state"][0, 0]
+    np.testing.assert_allclose(S @ kh[-1, 0], vh[-1, 0], rtol=0, atol=1e-13)
+
+
+def test_pure_decay_and_gate_closed_form():
+    """beta = 0: S_T = prod(alpha) S_0, o_t = gamma_t S_0 q_t / sqrt(d).
+
+    A_log = ln 2 and a + dt_bias = 0 give alpha = exp(-2 ln 2) = 1/4 exactly
+    (softplus(0) = ln 2), so S_T = 4^-T S_0."""
+    rng = np.random.default_rng(4)
+    d, T = 4, 6
+    shape = oracle.Shape(1, 1, d, d, l2_eps=0.0)
+    w = {"conv_w": rng.normal(0, 0.7, (shape.channels, 4)), "A_log": np.array([math.log(2.0)]),
+         "dt_bias": np.array([1.0]), "norm_w": np.ones(d)}
+    acts = {"q": rng.normal(size=(T, d)), "k": rng.normal(size=(T, d)), "v": rng.normal(size=(T, d)),
+            "z": rng.normal(size=(T, d)), "a": np.full((T, 1), -1.0), "b": np.full((T, 1), -800.0)}
+    cs = rng.normal(size=(1, shape.channels, 3))
+    S0 = rng.normal(size=(1, 1, d, d))
+    cu = np.array([0, T], np.int32)
+    r = _run(shape, w, acts, cs, S0, cu, want_o_pre=True)
+    np.testing.assert_allclose(r["rec_state"][0, 0], S0[0, 0] * 0.25 ** T, rtol=1e-14, atol=0)
+    qh, *_ = oracle.features(shape, w, acts["q"], acts["k"], acts["v"], acts["a"], acts["b"], cs, cu)
+    for t in range(T):
+        expect = 0.25 ** (t + 1) * S0[0, 0] @ qh[t, 0] / math.sqrt(d)
+        np.testing.assert_allclose(r["o_pre"][t, 0], expect, rtol=1e-13, atol=1e-300)
+
+
+def test_alpha_one_beta_zero_keeps_state():
+    rng = np.random.default_rng(5)
+    shape, w, acts, cs, rs, cu = _random_case(rng, Hk=1, G=3, d=4, T=9, n_seqs=2)
+    w["A_log"][:] = -1000.0
+    acts["b"][:] = -800.0
+    r = _run(shape, w, acts, cs, rs, cu)
+    np.testing.assert_array_equal(r["rec_state"], rs)
+
+
+def _recall_setup(d=4, Hk=2, G=2, shift=1):
+    """Orthonormal keys: conv passes only the current token, raw k of key head j at
+    token t is 5 on channel (t + j*shift) % d and 0 elsewhere, so k^ is that basis
+    vector exactly (SiLU(0) = 0).  q = k.  alpha = beta = 1."""
+    Hv = Hk * G
+    shape = oracle.Shape(Hk, Hv, d, d, l2_eps=0.0, norm_eps=0.0)
+    T = d
+    k = np.zeros((T, Hk * d))
+    for t in range(T):
+        for j in range(Hk):
+            k[t, j * d + (t + j * shift) % d] = 5.0
+    rng = np.random.default_rng(6)
+    v = rng.normal(size=(T, Hv * d))
+    w = {"conv_w": _identity_conv(shape), "A_log": np.full(Hv, -1000.0), "dt_bias": np.zeros(Hv),
+         "norm_w": np.ones(d)}
+    acts = {"q": k.copy(), "k": k, "v": v, "z": rng.normal(size=(T, Hv * d)),
+            "a": np.zeros((T, Hv)), "b": np.full((T, Hv), 60.0)}
+    cs = np.zeros((1, shape.channels, 3))
+    rs = np.zeros((1, Hv, d, d))
+    return shape, w, acts, cs, rs, np.array([0, T], np.int32)
+
+
+def test_orthonormal_recall_and_head_map():
+    """Writing d orthonormal keys once recalls every value exactly; value head h
+    reads key head h // (H_v / H_k)."""
+    d, Hk, G = 4, 2, 2
+    shape, w, acts, cs, rs, cu = _recall_setup(d, Hk, G)
+    r = _run(shape, w, acts, cs, rs, cu, want_o_pre=True)
+    silu_v = np.vectorize(_silu)(acts["v"]).reshape(d, Hk * G, d)
+    for h in range(Hk * G):
+        j = h // G
+        S = r["rec_state"][0, h]
+        for t in range(d):
+            e = np.zeros(d)
+            e[(t + j) % d] = 1.0
+            np.testing.assert_allclose(S @ e, silu_v[t, h], rtol=0, atol=1e-14)
+            # q = k: o_t = S_t e_t / sqrt(d) = v_t / sqrt(d)
+            np.testing.assert_allclose(r["o_pre"][t, h], silu_v[t, h] / math.sqrt(d),
+                                       rtol=0, atol=1e-14)
+
+
+def test_conv_tap_order_impulse():
+    """An impulse on token 0 of a v channel comes out of the conv as the taps in
+    reverse order: y_t = SiLU(w[c, K-1-t]).  Read back exactly through recall."""
+    d, Hk, G = 4, 1, 1
+    shape, w, acts, cs, rs, cu = _recall_setup(d, Hk, G)
+    taps = np.array([0.3, -0.7, 1.1, 0.9])
+    c = 2 * d + 1                       # v channel 1 of value head 0
+    w["conv_w"][c] = taps
+    acts["v"][:] = 0.0
+    acts["v"][0, 1] = 1.0
+    r = _run(shape, w, acts, cs, rs, cu)
+    S = r["rec_state"][0, 0]
+    for t in range(d):
+        e = np.zeros(d)
+        e[t] = 1.0
+        assert abs((S @ e)[1] - _silu(taps[3 - t])) < 1e-15
+
+
+def test_conv_state_carry_and_short_sequences():
+    """conv_state after a call holds the last K-1 raw inputs (oldest first), and
+    continues the old state for sequences shorter than K-1."""
+    rng = np.random.default_rng(7)
+    shape, w, acts, cs, rs, cu = _random_case(rng, Hk=1, G=2, d=4, T=6, n_seqs=3)
+    cu = np.array([0, 1, 3, 8], np.int32)
+    for n in ACTS:
+        acts[n] = rng.normal(size=(8, acts[n].shape[1]))
+    r = _run(shape, w, acts, cs, rs, cu)
+    x = np.concatenate([acts["q"], acts["k"], acts["v"]], axis=1)
+    hist = [np.concatenate([cs[s].T, x[cu[s]:cu[s + 1]]], axis=0)[-3:].T for s in range(3)]
+    np.testing.assert_array_equal(r["conv_state"], np.stack(hist))
+
+
+def test_constant_output_rmsnorm_closed_form():
+    """beta = 0 and S_0 with identical rows make o = c * 1; the gated norm then gives
+    sign(c) * w * SiLU(z) exactly when norm_eps = 0."""
+    rng = np.random.default_rng(8)
+    d, T = 8, 4
+    shape = oracle.Shape(1, 1, d, d, norm_eps=0.0)
+    w = {"conv_w": rng.normal(0, 0.7, (shape.channels, 4)), "A_log": np.array([0.0]),
+         "dt_bias": np.array([0.0]), "norm_w": rng.normal(1, 0.3, d)}
+    acts = {"q": rng.normal(size=(T, d)), "k": rng.normal(size=(T, d)), "v": rng.normal(size=(T, d)),
+            "z": rng.normal(size=(T, d)), "a": rng.normal(size=(T, 1)), "b": np.full((T, 1), -800.0)}
+    row = rng.normal(size=d)
+    S0 = np.tile(row, (d, 1))[None, None]
+    cs = rng.normal(size=(1, shape.channels, 3))
+    cu = np.array([0, T], np.int32)
+    r = _run(shape, w, acts, cs, S0, cu, want_o_pre=True)
+    for t in range(T):
+        o = r["o_pre"][t, 0]
+        assert np.ptp(o) <= 1e-15 * np.abs(o).max()
+        expect = np.sign(o[0]) * w["norm_w"] * np.vectorize(_silu)(acts["z"][t])
+        np.testing.assert_allclose(r["out"][t, 0], expect, rtol=1e-13, atol=0)
+
+
+def test_l2_norm_unit_and_features_closed_forms():
+    rng = np.random.default_rng(9)
+    shape, w, acts, cs, rs, cu = _random_case(rng, Hk=2, G=2, d=8, T=10, n_seqs=2)
+    shape.l2_eps = 0.0
+    qh, kh, vh, la, beta = oracle.features(shape, w, acts["q"], acts["k"], acts["v"], acts["a"],
+                                           acts["b"], cs, cu)
+    np.testing.assert_allclose(np.linalg.norm(qh, axis=-1), 1.0, rtol=0, atol=1e-14)
+    np.testing.assert_allclose(np.linalg.norm(kh, axis=-1), 1.0, rtol=0, atol=1e-14)
+    # gates: a + dt_bias = 0 -> softplus = ln 2; b = 0 -> beta = 1/2
+    a0 = -np.broadcast_to(w["dt_bias"], acts["a"].shape)
+    _, _, _, la0, b0 = oracle.features(shape, w, acts["q"], acts["k"], acts["v"], a0,
+                                       np.zeros_like(acts["b"]), cs, cu)
+    np.testing.assert_allclose(la0, -np.exp(w["A_log"])[None, :] * math.log(2.0) * np.ones_like(la0),
+                               rtol=1e-15)
+    np.testing.assert_array_equal(b0, 0.5)
+
+
+def test_split_prefill_and_decode_equal_one_prefill():
+    """prefill(T1) then prefill(T2), or prefill then one-token decode steps, equal
+    prefill(T1 + T2): both states carry everything the layer needs."""
+    rng = np.random.default_rng(11)
+    shape, w, acts, cs, rs, cu = _random_case(rng, Hk=2, G=3, d=8, T=12, n_seqs=1)
+    T = int(cu[-1])
+    full = _run(shape, w, acts, cs, rs, np.array([0, T], np.int32))
+    T1 = T // 2
+    first = _run(shape, w, {n: a[:T1] for n, a in acts.items()}, cs, rs, np.array([0, T1], np.int32))
+    second = _run(shape, w, {n: a[T1:] for n, a in acts.items()}, first["conv_state"],
+                  first["rec_state"], np.array([0, T - T1], np.int32))
+    np.testing.assert_allclose(np.concatenate([first["out"], second["out"]]), full["out"],
+                               rtol=0, atol=1e-12)
+    np.testing.assert_allclose(second["rec_state"], full["rec_state"], rtol=0, atol=1e-12)
+    np.testing.assert_array_equal(second["conv_state"], full["conv_state"])
+    # token-by-token decode after the first half
+    st = first
+    outs = [first["out"]]
+    for t in range(T1, T):
+        st = _run(shape, w, {n: a[t:t + 1] for n, a in acts.items()}, st["conv_state"],
+                  st["rec_state"], np.array([0, 1], np.int32))
+        outs.append(st["out"])
+    np.testing.assert_allclose(np.concatenate(outs), full["out"], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(st["rec_state"], full["rec_state"], rtol=0, atol=1e-12)
+
+
+def test_packed_varlen_equals_separate_calls():
+    rng = np.random.default_rng(12)
+    shape, w, acts, cs, rs, cu = _random_case(rng, Hk=1, G=2, d=4, T=9, n_seqs=4)
+    packed = _run(shape, w, acts, cs, rs, cu)
+    for s in range(4):
+        t0, t1 = int(cu[s]), int(cu[s + 1])
+        one = _run(shape, w, {n: a[t0:t1] for n, a in acts.items()}, cs[s:s + 1], rs[s:s + 1],
+                   np.array([0, t1 - t0], np.int32))
+        np.testing.assert_array_equal(one["out"], packed["out"][t0:t1])
+        np.testing.assert_array_equal(one["rec_state"][0], packed["rec_state"][s])
+        np.testing.assert_array_equal(one["conv_state"][0], packed["conv_state"][s])
+
+
+def test_head_subset_matches_all_heads():
+    rng = np.random.default_rng(13)
+    shape, w, acts, cs, rs, cu = _random_case(rng, Hk=2, G=3, d=4, T=6, n_seqs=2)
+    full = _run(shape, w, acts, cs, rs, cu)
+    heads = np.array([5, 1, 3], np.int32)
+    sub = _run(shape, w, acts, cs, rs[:, heads], cu, heads=heads)
+    np.testing.assert_array_equal(sub["out"], full["out"][:, heads])
+    np.testing.assert_array_equal(sub["rec_state"], full["rec_state"][:, heads])
+
+
+def test_bf16_inputs_are_read_exactly():
+    """bf16 bit patterns reach the oracle as the exact values they encode."""
+    rng = np.random.default_rng(14)
+    shape, w, acts, cs, rs, cu = _random_case(rng, Hk=1, G=2, d=4, T=5, n_seqs=1)
+    bits = {n: inputs.f32_to_bf16_bits(a.astype(np.float32)) for n, a in acts.items()}
+    vals = {n: inputs.bf16_bits_to_f32(b).astype(np.float64) for n, b in bits.items()}
+    r1 = _run(shape, w, bits, cs, rs, cu)
+    r2 = _run(shape, w, vals, cs, rs, cu)
+    np.testing.assert_array_equal(r1["out"], r2["out"])
+    np.testing.assert_array_equal(r1["rec_state"], r2["rec_state"])
+    assert inputs.bf16_bits_to_f32(inputs.f32_to_bf16_bits(np.array([1.0, -2.5, 1 + 2 ** -9],
+                                                                     np.float32))).tolist() == [1.0, -2.5, 1.0]
