@@ -1,0 +1,173 @@
+// Fused one-token decode step of the Gated DeltaNet mixer.
+//
+// One CTA per (sequence, key head): it rolls the conv state of the key head's
+// q/k channels and of its G value heads' v channels, runs conv + SiLU, the L2
+// norm of q and k, the gates, and then streams the G value-head states
+// (G x d_v rows of d_k fp32, one contiguous block) through registers once.
+// Row r of S gives row r of S' and o_r with no other row involved:
+//     u_r   = S_r . k,   p_r = S_r . q
+//     d_r   = beta (v_r - alpha u_r)
+//     S'_r  = alpha S_r + d_r k^T
+//     o_r   = (alpha p_r + d_r (k . q)) / sqrt(d_k)         (= S'_r . q / sqrt(d_k))
+// which is S' = alpha S (I - beta k k^T) + beta v k^T applied row by row.  The
+// gated RMSNorm over the d_v entries of o follows.  HBM-bound: 2 x 64 KiB of
+// state per value head per step against ~1 KiB of everything else.
+#pragma once
+#include "device.cuh"
+
+namespace gdn {
+namespace dec {
+
+constexpr int NT = 256;
+constexpr int NW = NT / 32;
+
+struct Args {
+    const void *q, *k, *v, *a, *b, *z;   // act dtype; q,k [N][Hk*dk], v,z [N][Hv*dv], a,b [N][Hv]
+    const float* conv_w;                 // [Ctot][4]
+    const float* A_log;
+    const float* dt_bias;
+    const float* norm_w;
+    void* conv_state;                    // [N][Ctot][3] act dtype, in/out
+    float* rec_state;                    // [N][Hv][dv][dk], in/out
+    void* out;                           // [N][Hv][dv] out dtype
+    int Hk, Hv, dk, dv;
+    float l2_eps, norm_eps;
+};
+
+__host__ __device__ constexpr size_t smem_floats(int dk, int G, int dv) {
+    return (size_t)2 * dk + (size_t)2 * G * dv + 2 * G;
+}
+
+template <typename TA, typename TO, int DK>
+__global__ void __launch_bounds__(NT) gdn_decode_kernel(Args p) {
+    constexpr int LPR = DK / 4;        // lanes per state row (4 fp32 each)
+    constexpr int RPP = 32 / LPR;      // rows per warp pass
+    constexpr int U = DK == 128 ? 8 : 4;   // passes in flight per warp
+    extern __shared__ float sm[];
+    const int Hk = p.Hk, Hv = p.Hv, dv = p.dv, G = Hv / Hk;
+    const int Cq = Hk * DK, Cv = Hv * dv, Ctot = 2 * Cq + Cv;
+    const int seq = blockIdx.x / Hk, j = blockIdx.x % Hk;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    float* sq = sm;                 // [DK]
+    float* sk = sq + DK;            // [DK]
+    float* sv = sk + DK;            // [G*dv]
+    float* so = sv + G * dv;        // [G*dv]
+    float* s_al = so + G * dv;      // [G]
+    float* s_be = s_al + G;         // [G]
+
+    // ---- conv + SiLU with the conv-state roll (channels of this key-head group) ----
+    const TA* pq = static_cast<const TA*>(p.q);
+    const TA* pk = static_cast<const TA*>(p.k);
+    const TA* pv = static_cast<const TA*>(p.v);
+    TA* cst = static_cast<TA*>(p.conv_state);
+    const int nch = 2 * DK + G * dv;
+    for (int i = tid; i < nch; i += NT) {
+        int ch;
+        const TA* src;
+        if (i < DK) {
+            ch = j * DK + i;
+            src = pq + (int64_t)seq * Cq + ch;
+        } else if (i < 2 * DK) {
+            ch = Cq + j * DK + (i - DK);
+            src = pk + (int64_t)seq * Cq + (ch - Cq);
+        } else {
+            const int vi = j * G * dv + (i - 2 * DK);
+            ch = 2 * Cq + vi;
+            src = pv + (int64_t)seq * Cv + vi;
+        }
+        TA* st = cst + ((int64_t)seq * Ctot + ch) * 3;
+        const TA xr = *src, h0 = st[0], h1 = st[1], h2 = st[2];
+        const float4 w = reinterpret_cast<const float4*>(p.conv_w)[ch];
+        float acc = w.x * to_f32(h0);
+        acc = fmaf(w.y, to_f32(h1), acc);
+        acc = fmaf(w.z, to_f32(h2), acc);
+        acc = fmaf(w.w, to_f32(xr), acc);
+        sm[i] = silu_f(acc);
+        st[0] = h1;
+        st[1] = h2;
+        st[2] = xr;
+    }
+    if (tid < G) {
+        const int h = j * G + tid;
+        const float av = to_f32(static_cast<const TA*>(p.a)[(int64_t)seq * Hv + h]);
+        const float bv = to_f32(static_cast<const TA*>(p.b)[(int64_t)seq * Hv + h]);
+        s_al[tid] = __expf(-__expf(p.A_log[h]) * softplus_f(av + p.dt_bias[h]));
+        s_be[tid] = sigmoid_f(bv);
+    }
+    __syncthreads();
+    if (warp < 2) {   // L2 norm: warp 0 -> q, warp 1 -> k
+        float* x = warp == 0 ? sq : sk;
+        float ss = 0.f;
+        for (int i = lane; i < DK; i += 32) ss = fmaf(x[i], x[i], ss);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float r = rsqrtf(ss + p.l2_eps);
+        for (int i = lane; i < DK; i += 32) x[i] *= r;
+    }
+    __syncthreads();
+
+    // ---- stream the state rows ----
+    const int col = 4 * (lane % LPR);
+    const int sub = lane / LPR;
+    const float4 k4 = *reinterpret_cast<const float4*>(sk + col);
+    const float4 q4 = *reinterpret_cast<const float4*>(sq + col);
+    float kq = k4.x * q4.x + k4.y * q4.y + k4.z * q4.z + k4.w * q4.w;
+#pragma unroll
+    for (int off = LPR / 2; off >= 1; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
+    const float inv_sqrt_dk = rsqrtf((float)DK);
+    float* Sb = p.rec_state + ((int64_t)seq * Hv + (int64_t)j * G) * dv * DK;
+    const int rows = G * dv;
+    for (int R0 = warp * RPP * U; R0 < rows; R0 += NW * RPP * U) {
+        float4 s[U];
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const int R = R0 + u * RPP + sub;
+            s[u] = R < rows ? __ldcs(reinterpret_cast<const float4*>(Sb + (int64_t)R * DK + col))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const int R = R0 + u * RPP + sub;
+            const int g = min(R, rows - 1) / dv;
+            float uk = s[u].x * k4.x + s[u].y * k4.y + s[u].z * k4.z + s[u].w * k4.w;
+            float up = s[u].x * q4.x + s[u].y * q4.y + s[u].z * q4.z + s[u].w * q4.w;
+#pragma unroll
+            for (int off = LPR / 2; off >= 1; off >>= 1) {
+                uk += __shfl_xor_sync(0xffffffffu, uk, off);
+                up += __shfl_xor_sync(0xffffffffu, up, off);
+            }
+            if (R < rows) {
+                const float al = s_al[g], be = s_be[g];
+                const float d = be * (sv[R] - al * uk);
+                float4 o4;
+                o4.x = fmaf(al, s[u].x, d * k4.x);
+                o4.y = fmaf(al, s[u].y, d * k4.y);
+                o4.z = fmaf(al, s[u].z, d * k4.z);
+                o4.w = fmaf(al, s[u].w, d * k4.w);
+                __stcs(reinterpret_cast<float4*>(Sb + (int64_t)R * DK + col), o4);
+                if (lane % LPR == 0) so[R] = (al * up + d * kq) * inv_sqrt_dk;
+            }
+        }
+    }
+    __syncthreads();
+
+    // ---- gated RMSNorm per value head ----
+    const TA* pz = static_cast<const TA*>(p.z);
+    TO* po = static_cast<TO*>(p.out);
+    for (int g = warp; g < G; g += NW) {
+        float ss = 0.f;
+        for (int r = lane; r < dv; r += 32) ss = fmaf(so[g * dv + r], so[g * dv + r], ss);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float rs = rsqrtf(ss / (float)dv + p.norm_eps);
+        const int h = j * G + g;
+        for (int r = lane; r < dv; r += 32) {
+            const int64_t off = ((int64_t)seq * Hv + h) * dv + r;
+            const float zz = to_f32(pz[off]);
+            from_f32(so[g * dv + r] * rs * p.norm_w[r] * silu_f(zz), po + off);
+        }
+    }
+}
+
+}  // namespace dec
+}  // namespace gdn

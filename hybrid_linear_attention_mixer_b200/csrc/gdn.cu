@@ -1,0 +1,247 @@
+// C ABI of the Gated DeltaNet mixer (include/gdn.h): argument checks and
+// kernel launches.  One translation unit holds every kernel.
+#include "gdn.h"
+
+#include <cmath>
+#include <cstring>
+
+#include "chunk.cuh"
+#include "conv.cuh"
+#include "decode.cuh"
+#include "device.cuh"
+
+namespace {
+
+using gdn::ConvArgs;
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+gdn_status check_config(const gdn_config* c) {
+    if (!c) return GDN_ERR_INVALID_ARG;
+    if (c->n_k_heads <= 0 || c->n_v_heads <= 0 || c->d_k <= 0 || c->d_v <= 0) return GDN_ERR_INVALID_ARG;
+    if (!(c->l2_eps >= 0.f) || !(c->norm_eps >= 0.f) || !std::isfinite(c->l2_eps) ||
+        !std::isfinite(c->norm_eps))
+        return GDN_ERR_INVALID_ARG;
+    if (c->act_dtype != GDN_BF16 && c->act_dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (c->out_dtype != GDN_BF16 && c->out_dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (c->n_v_heads % c->n_k_heads != 0) return GDN_ERR_UNSUPPORTED;
+    if (!dim_ok(c->d_k) || !dim_ok(c->d_v)) return GDN_ERR_UNSUPPORTED;
+    if (c->conv_kernel != 4 || c->chunk != gdn::chunk::C) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+gdn_status check_weights(const gdn_weights* w) {
+    if (!w || !w->conv_weight || !w->A_log || !w->dt_bias || !w->norm_weight) return GDN_ERR_INVALID_ARG;
+    if (!aligned(w->conv_weight, 16)) return GDN_ERR_INVALID_ARG;
+    return GDN_OK;
+}
+
+struct Layout {
+    size_t q_off, k_off, v_off, total;
+};
+
+Layout workspace_layout(const gdn_config* c, int64_t T) {
+    Layout L;
+    const size_t qb = align_up((size_t)T * c->n_k_heads * c->d_k * sizeof(__half), 256);
+    const size_t vb = align_up((size_t)T * c->n_v_heads * c->d_v * sizeof(__half), 256);
+    L.q_off = 0;
+    L.k_off = qb;
+    L.v_off = 2 * qb;
+    L.total = 2 * qb + vb;
+    return L;
+}
+
+// Opt in to > 48 KiB of dynamic shared memory, once per device and kernel.
+template <typename K>
+cudaError_t ensure_smem(K kernel, int variant, size_t bytes) {
+    static bool done[64][8];
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 64 && done[dev][variant]) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess && dev < 64) done[dev][variant] = true;
+    return e;
+}
+
+template <typename TA, typename TO>
+cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void* q, const void* k,
+                           const void* v, const void* a, const void* b, const void* z, void* conv_state,
+                           float* rec_state, const int32_t* cu, int n_seqs, int64_t T, void* out,
+                           void* ws, int variant, cudaStream_t st) {
+    const Layout L = workspace_layout(c, T);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    ConvArgs ca;
+    ca.q = q; ca.k = k; ca.v = v;
+    ca.conv_w = w->conv_weight;
+    ca.conv_state = conv_state;
+    ca.cu = cu;
+    ca.n_seqs = n_seqs;
+    ca.T = T;
+    ca.Hk = c->n_k_heads; ca.Hv = c->n_v_heads; ca.dk = c->d_k; ca.dv = c->d_v;
+    ca.l2_eps = c->l2_eps;
+    ca.qh = reinterpret_cast<__half*>(wsb + L.q_off);
+    ca.kh = reinterpret_cast<__half*>(wsb + L.k_off);
+    ca.vh = reinterpret_cast<__half*>(wsb + L.v_off);
+    const int Ctot = 2 * c->n_k_heads * c->d_k + c->n_v_heads * c->d_v;
+    const int cblocks = (Ctot / 8 + gdn::kConvThreads - 1) / gdn::kConvThreads;
+    const int64_t tblocks = (T + gdn::kConvTokens - 1) / gdn::kConvTokens;
+    if (tblocks > 0x7fffffff) return cudaErrorInvalidValue;
+    gdn::conv_silu_norm_kernel<TA><<<dim3((unsigned)tblocks, cblocks), gdn::kConvThreads, 0, st>>>(ca);
+    gdn::conv_state_update_kernel<TA><<<dim3(n_seqs, (Ctot + 255) / 256), 256, 0, st>>>(ca, conv_state);
+
+    gdn::chunk::Args pa;
+    pa.qh = ca.qh; pa.kh = ca.kh; pa.vh = ca.vh;
+    pa.a = a; pa.b = b; pa.z = z;
+    pa.A_log = w->A_log; pa.dt_bias = w->dt_bias; pa.norm_w = w->norm_weight;
+    pa.rec_state = rec_state;
+    pa.cu = cu;
+    pa.out = out;
+    pa.Hk = c->n_k_heads; pa.Hv = c->n_v_heads; pa.dk = c->d_k; pa.dv = c->d_v;
+    pa.norm_eps = c->norm_eps;
+    auto kern = gdn::chunk::gdn_chunk_kernel<TA, TO>;
+    cudaError_t e = ensure_smem(kern, variant, gdn::chunk::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    kern<<<(unsigned)n_seqs * c->n_v_heads, gdn::chunk::NT, gdn::chunk::SMEM_BYTES, st>>>(pa);
+    return cudaGetLastError();
+}
+
+template <typename TA, typename TO, int DK>
+cudaError_t launch_decode_dk(const gdn::dec::Args& a, int n_seqs, cudaStream_t st) {
+    const int G = a.Hv / a.Hk;
+    const size_t smem = gdn::dec::smem_floats(DK, G, a.dv) * sizeof(float);
+    auto kern = gdn::dec::gdn_decode_kernel<TA, TO, DK>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<(unsigned)n_seqs * a.Hk, gdn::dec::NT, smem, st>>>(a);
+    return cudaGetLastError();
+}
+
+template <typename TA, typename TO>
+cudaError_t launch_decode(const gdn::dec::Args& a, int n_seqs, cudaStream_t st) {
+    switch (a.dk) {
+        case 32: return launch_decode_dk<TA, TO, 32>(a, n_seqs, st);
+        case 64: return launch_decode_dk<TA, TO, 64>(a, n_seqs, st);
+        default: return launch_decode_dk<TA, TO, 128>(a, n_seqs, st);
+    }
+}
+
+}  // namespace
+
+extern "C" {
+
+void gdn_config_default(gdn_config* cfg) {
+    if (!cfg) return;
+    cfg->n_k_heads = 16;
+    cfg->n_v_heads = 48;
+    cfg->d_k = 128;
+    cfg->d_v = 128;
+    cfg->conv_kernel = 4;
+    cfg->chunk = 64;
+    cfg->l2_eps = 1e-6f;
+    cfg->norm_eps = 1e-6f;
+    cfg->act_dtype = GDN_BF16;
+    cfg->out_dtype = GDN_BF16;
+}
+
+size_t gdn_prefill_workspace_size(const gdn_config* cfg, int64_t T_total, int32_t n_seqs) {
+    if (check_config(cfg) != GDN_OK || T_total < 0 || n_seqs < 0) return 0;
+    return workspace_layout(cfg, T_total).total;
+}
+
+gdn_status gdn_prefill(const gdn_config* cfg, const gdn_weights* w, const void* q, const void* k,
+                       const void* v, const void* a, const void* b, const void* z, void* conv_state,
+                       float* rec_state, const int32_t* cu_seqlens, int32_t n_seqs, int64_t T_total,
+                       void* out, void* workspace, size_t workspace_bytes, void* stream) {
+    gdn_status s = check_config(cfg);
+    if (s != GDN_OK) return s;
+    if ((s = check_weights(w)) != GDN_OK) return s;
+    if (n_seqs < 0 || T_total < 0) return GDN_ERR_INVALID_ARG;
+    if (T_total == 0 || n_seqs == 0) return GDN_OK;
+    if (!q || !k || !v || !a || !b || !z || !conv_state || !rec_state || !cu_seqlens || !out || !workspace)
+        return GDN_ERR_INVALID_ARG;
+    const void* a16[] = {q, k, v, z, out, rec_state};
+    for (const void* p : a16)
+        if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)n_seqs * cfg->n_v_heads > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (workspace_bytes < workspace_layout(cfg, T_total).total) return GDN_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    const bool abf = cfg->act_dtype == GDN_BF16, obf = cfg->out_dtype == GDN_BF16;
+    if (abf && obf)
+        e = launch_prefill<__nv_bfloat16, __nv_bfloat16>(cfg, w, q, k, v, a, b, z, conv_state, rec_state,
+                                                          cu_seqlens, n_seqs, T_total, out, workspace, 0, st);
+    else if (abf)
+        e = launch_prefill<__nv_bfloat16, float>(cfg, w, q, k, v, a, b, z, conv_state, rec_state, cu_seqlens,
+                                                 n_seqs, T_total, out, workspace, 1, st);
+    else if (obf)
+        e = launch_prefill<float, __nv_bfloat16>(cfg, w, q, k, v, a, b, z, conv_state, rec_state, cu_seqlens,
+                                                 n_seqs, T_total, out, workspace, 2, st);
+    else
+        e = launch_prefill<float, float>(cfg, w, q, k, v, a, b, z, conv_state, rec_state, cu_seqlens, n_seqs,
+                                         T_total, out, workspace, 3, st);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w, const void* q, const void* k,
+                      const void* v, const void* a, const void* b, const void* z, void* conv_state,
+                      float* rec_state, int32_t n_seqs, void* out, void* stream) {
+    gdn_status s = check_config(cfg);
+    if (s != GDN_OK) return s;
+    if ((s = check_weights(w)) != GDN_OK) return s;
+    if (n_seqs < 0) return GDN_ERR_INVALID_ARG;
+    if (n_seqs == 0) return GDN_OK;
+    if (!q || !k || !v || !a || !b || !z || !conv_state || !rec_state || !out) return GDN_ERR_INVALID_ARG;
+    const void* a16[] = {q, k, v, z, out, rec_state};
+    for (const void* p : a16)
+        if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+    if ((int64_t)n_seqs * cfg->n_k_heads > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    gdn::dec::Args da;
+    da.q = q; da.k = k; da.v = v; da.a = a; da.b = b; da.z = z;
+    da.conv_w = w->conv_weight; da.A_log = w->A_log; da.dt_bias = w->dt_bias; da.norm_w = w->norm_weight;
+    da.conv_state = conv_state;
+    da.rec_state = rec_state;
+    da.out = out;
+    da.Hk = cfg->n_k_heads; da.Hv = cfg->n_v_heads; da.dk = cfg->d_k; da.dv = cfg->d_v;
+    da.l2_eps = cfg->l2_eps; da.norm_eps = cfg->norm_eps;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    const bool abf = cfg->act_dtype == GDN_BF16, obf = cfg->out_dtype == GDN_BF16;
+    if (abf && obf) e = launch_decode<__nv_bfloat16, __nv_bfloat16>(da, n_seqs, st);
+    else if (abf) e = launch_decode<__nv_bfloat16, float>(da, n_seqs, st);
+    else if (obf) e = launch_decode<float, __nv_bfloat16>(da, n_seqs, st);
+    else e = launch_decode<float, float>(da, n_seqs, st);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_check_device_error(void* stream) {
+    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDN_ERR_CUDA;
+    unsigned int v = 0;
+    if (cudaMemcpyFromSymbol(&v, gdn::g_device_error, sizeof v) != cudaSuccess) return GDN_ERR_CUDA;
+    if (v) {
+        const unsigned int zero = 0;
+        if (cudaMemcpyToSymbol(gdn::g_device_error, &zero, sizeof zero) != cudaSuccess) return GDN_ERR_CUDA;
+        return GDN_ERR_DEVICE_TIMEOUT;
+    }
+    return GDN_OK;
+}
+
+const char* gdn_status_string(gdn_status s) {
+    switch (s) {
+        case GDN_OK: return "ok";
+        case GDN_ERR_INVALID_ARG: return "invalid argument";
+        case GDN_ERR_UNSUPPORTED: return "unsupported shape or dtype";
+        case GDN_ERR_CUDA: return "CUDA error";
+        case GDN_ERR_DEVICE_TIMEOUT: return "device wait timed out";
+        case GDN_ERR_WORKSPACE: return "workspace too small";
+    }
+    return "unknown status";
+}
+
+}  // extern "C"

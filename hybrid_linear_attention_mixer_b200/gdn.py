@@ -1,0 +1,200 @@
+"""Python binding of the C-ABI library ``libgdn_b200.so`` (include/gdn.h).
+
+Argument marshalling only: every step of the layer runs in the library's CUDA
+kernels.  PyTorch supplies device memory and the stream.  If the library is
+missing this module raises; there is no other implementation to fall back to.
+
+Tensors (all contiguous, on one CUDA device):
+  q, k        [T, H_k*d_k]  (or [T, H_k, d_k])   activation dtype
+  v, z        [T, H_v*d_v]                       activation dtype
+  a, b        [T, H_v]                           activation dtype
+  conv_state  [N, 2*H_k*d_k + H_v*d_v, 3]        activation dtype, updated in place
+  rec_state   [N, H_v, d_v, d_k] float32         updated in place
+  cu_seqlens  [N + 1] int32                      (prefill only)
+  weights     dict: conv_w [C, 4], A_log [H_v], dt_bias [H_v], norm_w [d_v], float32
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libgdn_b200.so")
+
+_DT = {torch.bfloat16: 0, torch.float32: 1}
+
+
+class GdnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        super().__init__("%s: %s (status %d)" % (what, status_string(status), status))
+        self.status = status
+
+
+class _CConfig(ctypes.Structure):
+    _fields_ = [("n_k_heads", ctypes.c_int32), ("n_v_heads", ctypes.c_int32),
+                ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32),
+                ("conv_kernel", ctypes.c_int32), ("chunk", ctypes.c_int32),
+                ("l2_eps", ctypes.c_float), ("norm_eps", ctypes.c_float),
+                ("act_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
+
+
+class _CWeights(ctypes.Structure):
+    _fields_ = [("conv_weight", ctypes.c_void_p), ("A_log", ctypes.c_void_p),
+                ("dt_bias", ctypes.c_void_p), ("norm_weight", ctypes.c_void_p)]
+
+
+_lib = None
+EXPORTS = ("gdn_config_default", "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode",
+           "gdn_check_device_error", "gdn_status_string")
+
+
+def lib() -> ctypes.CDLL:
+    """Load libgdn_b200.so (built in place by ``build.py``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libgdn_b200.so is not built; run `python -m "
+                               "hybrid_linear_attention_mixer_b200.build` (needs nvcc)")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+        L.gdn_config_default.argtypes = [vp]
+        L.gdn_config_default.restype = None
+        L.gdn_prefill_workspace_size.argtypes = [vp, i64, i32]
+        L.gdn_prefill_workspace_size.restype = sz
+        L.gdn_prefill.argtypes = [vp, vp] + [vp] * 8 + [vp, i32, i64, vp, vp, sz, vp]
+        L.gdn_prefill.restype = ctypes.c_int
+        L.gdn_decode.argtypes = [vp, vp] + [vp] * 8 + [i32, vp, vp]
+        L.gdn_decode.restype = ctypes.c_int
+        L.gdn_check_device_error.argtypes = [vp]
+        L.gdn_check_device_error.restype = ctypes.c_int
+        L.gdn_status_string.argtypes = [ctypes.c_int]
+        L.gdn_status_string.restype = ctypes.c_char_p
+        _lib = L
+    return _lib
+
+
+def status_string(s: int) -> str:
+    return lib().gdn_status_string(int(s)).decode()
+
+
+@dataclass
+class Config:
+    """Layer shape; the defaults are the published layer (16 / 48 heads of 128, K = 4)."""
+    n_k_heads: int = 16
+    n_v_heads: int = 48
+    d_k: int = 128
+    d_v: int = 128
+    conv_kernel: int = 4
+    chunk: int = 64
+    l2_eps: float = 1e-6
+    norm_eps: float = 1e-6
+    act_dtype: torch.dtype = torch.bfloat16
+    out_dtype: torch.dtype = torch.bfloat16
+
+    @property
+    def channels(self) -> int:
+        return 2 * self.n_k_heads * self.d_k + self.n_v_heads * self.d_v
+
+    def c(self) -> _CConfig:
+        return _CConfig(self.n_k_heads, self.n_v_heads, self.d_k, self.d_v, self.conv_kernel,
+                        self.chunk, self.l2_eps, self.norm_eps, _DT[self.act_dtype],
+                        _DT[self.out_dtype])
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(t, name, dtype, device):
+    if t.dtype != dtype:
+        raise TypeError("%s: dtype %s, expected %s" % (name, t.dtype, dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+
+
+def _weights(w: dict, device) -> _CWeights:
+    for n in ("conv_w", "A_log", "dt_bias", "norm_w"):
+        _check(w[n], n, torch.float32, device)
+    return _CWeights(w["conv_w"].data_ptr(), w["A_log"].data_ptr(), w["dt_bias"].data_ptr(),
+                     w["norm_w"].data_ptr())
+
+
+def workspace_size(cfg: Config, T_total: int, n_seqs: int) -> int:
+    c = cfg.c()
+    return int(lib().gdn_prefill_workspace_size(ctypes.byref(c), int(T_total), int(n_seqs)))
+
+
+def prefill(cfg: Config, w: dict, q, k, v, a, b, z, conv_state, rec_state, cu_seqlens,
+            out=None, workspace=None, stream=None):
+    """Packed variable-length prefill; returns out [T, H_v*d_v] (out_dtype)."""
+    dev = q.device
+    T = q.shape[0]
+    for n, t in (("q", q), ("k", k), ("v", v), ("a", a), ("b", b), ("z", z),
+                 ("conv_state", conv_state)):
+        _check(t, n, cfg.act_dtype, dev)
+    _check(rec_state, "rec_state", torch.float32, dev)
+    _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
+    n_seqs = cu_seqlens.shape[0] - 1
+    if out is None:
+        out = torch.empty((T, cfg.n_v_heads * cfg.d_v), dtype=cfg.out_dtype, device=dev)
+    _check(out, "out", cfg.out_dtype, dev)
+    need = workspace_size(cfg, T, n_seqs)
+    if workspace is None:
+        workspace = torch.empty(max(need, 1), dtype=torch.uint8, device=dev)
+    c, cw = cfg.c(), _weights(w, dev)
+    s = lib().gdn_prefill(ctypes.byref(c), ctypes.byref(cw), _ptr(q), _ptr(k), _ptr(v), _ptr(a),
+                          _ptr(b), _ptr(z), _ptr(conv_state), _ptr(rec_state), _ptr(cu_seqlens),
+                          n_seqs, T, _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_prefill")
+    return out
+
+
+def decode(cfg: Config, w: dict, q, k, v, a, b, z, conv_state, rec_state, out=None, stream=None):
+    """One token per sequence; returns out [N, H_v*d_v] (out_dtype)."""
+    dev = q.device
+    N = q.shape[0]
+    for n, t in (("q", q), ("k", k), ("v", v), ("a", a), ("b", b), ("z", z),
+                 ("conv_state", conv_state)):
+        _check(t, n, cfg.act_dtype, dev)
+    _check(rec_state, "rec_state", torch.float32, dev)
+    if out is None:
+        out = torch.empty((N, cfg.n_v_heads * cfg.d_v), dtype=cfg.out_dtype, device=dev)
+    _check(out, "out", cfg.out_dtype, dev)
+    c, cw = cfg.c(), _weights(w, dev)
+    s = lib().gdn_decode(ctypes.byref(c), ctypes.byref(cw), _ptr(q), _ptr(k), _ptr(v), _ptr(a),
+                         _ptr(b), _ptr(z), _ptr(conv_state), _ptr(rec_state), N, _ptr(out),
+                         _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_decode")
+    return out
+
+
+def check_device_error(stream=None) -> None:
+    """Synchronise the stream and raise if a kernel's bounded wait ran out."""
+    s = lib().gdn_check_device_error(_stream(stream))
+    if s != 0:
+        raise GdnError(s, "device")
+
+
+def prefill_host(cfg: Config, w: dict, host: dict, conv_state, rec_state, stream=None):
+    """End-to-end prefill from host buffers: copies the step's inputs (pinned host
+    tensors q, k, v, a, b, z, cu_seqlens) to the device, runs the layer, and copies
+    ``out`` back into host['out'] (pinned).  States stay resident on the device."""
+    dev = rec_state.device
+    d = {n: host[n].to(dev, non_blocking=True) for n in ("q", "k", "v", "a", "b", "z", "cu_seqlens")}
+    out = prefill(cfg, w, d["q"], d["k"], d["v"], d["a"], d["b"], d["z"], conv_state, rec_state,
+                  d["cu_seqlens"], stream=stream)
+    host["out"].copy_(out, non_blocking=True)
+    return host["out"]

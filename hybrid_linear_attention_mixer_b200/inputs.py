@@ -25,12 +25,14 @@ Workloads (head shape of the layer: 16 key heads, 48 value heads, d_k = d_v =
 """
 from __future__ import annotations
 
+import os
 import zlib
+from concurrent.futures import ThreadPoolExecutor
 from dataclasses import dataclass, field
 
 import numpy as np
 
-ROW_BLOCK = 2048
+ROW_BLOCK = 1024
 
 
 def f32_to_bf16_bits(x: np.ndarray) -> np.ndarray:
@@ -49,15 +51,29 @@ def _rng(seed: int, name: str, block: int = 0) -> np.random.Generator:
     return np.random.Generator(np.random.PCG64([seed, key, block]))
 
 
+def _workers() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
 def _normal_rows(seed, name, rows, cols, std=1.0, mean=0.0, bf16=True):
-    """[rows, cols] N(mean, std^2), drawn in independent row blocks."""
+    """[rows, cols] N(mean, std^2), drawn in independent row blocks (threaded)."""
     out = np.empty((rows, cols), dtype=np.uint16 if bf16 else np.float32)
-    for blk, r0 in enumerate(range(0, rows, ROW_BLOCK)):
+
+    def fill(blk):
+        r0 = blk * ROW_BLOCK
         r1 = min(rows, r0 + ROW_BLOCK)
         x = _rng(seed, name, blk).standard_normal((r1 - r0, cols), dtype=np.float32)
         if std != 1.0 or mean != 0.0:
             x = x * np.float32(std) + np.float32(mean)
         out[r0:r1] = f32_to_bf16_bits(x) if bf16 else x
+
+    nblk = (rows + ROW_BLOCK - 1) // ROW_BLOCK
+    if nblk <= 1:
+        for blk in range(nblk):
+            fill(blk)
+    else:
+        with ThreadPoolExecutor(min(_workers(), nblk)) as ex:
+            list(ex.map(fill, range(nblk)))
     return out
 
 

@@ -1,0 +1,143 @@
+/*
+ * gdn.h -- C ABI of the B200 (sm_100a) Gated DeltaNet token mixer.
+ *
+ * The layer (one of the 36 linear-attention layers of the hybrid decoder
+ * described in "Qwen3.8-Flash-Next" (llm-architectures-explained), "Every
+ * architecture field": mixers.linear.type deltanet, 16 key heads, 48 value
+ * heads, key/value head dim 128, conv kernel 4; "Qwen3.8-Flash-Next anatomy"
+ * (frontier-model-atlas), "Decoder microscope"):
+ *
+ *   x_t   = [q_t | k_t | v_t]                      (2*H_k*d_k + H_v*d_v channels)
+ *   y_t   = SiLU(sum_i w[c,i] x_{t-K+1+i}[c])      depthwise causal conv, no bias;
+ *                                                  the K-1 inputs before a sequence
+ *                                                  start come from conv_state
+ *   q^,k^ = y_q / sqrt(|y_q|^2 + l2_eps), same for k, per key head
+ *   alpha = exp(-exp(A_log[h]) * softplus(a_t + dt_bias[h])),  beta = sigmoid(b_t)
+ *   S_t   = alpha S_{t-1} (I - beta k^ k^T) + beta v^ k^T    (S: d_v x d_k, fp32)
+ *   o_t   = S_t q^ / sqrt(d_k)
+ *   out_t = o_t * rsqrt(mean(o_t^2) + norm_eps) * norm_weight * SiLU(z_t)
+ *
+ * Value head h reads key head h / (H_v / H_k).  The recurrent state is kept in
+ * float32 (mamba_ssm_dtype float32, "Qwen3.8-Flash-Next" (llm-atlas-9r2),
+ * "Raw config fields"); norm_eps defaults to rms_norm_eps = 1e-6 from the same
+ * table.  The pages name the gated delta rule without printing it; the
+ * recurrence above is its standard statement.
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers, contiguous, row-major, owned by
+ *     the caller.  The library allocates no memory and never synchronises the
+ *     stream (gdn_check_device_error excepted).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t passed as void*; NULL
+ *     is the legacy default stream).  conv_state and rec_state are read and
+ *     updated in place.
+ *   - Activation tensors q, k, v, a, b, z and conv_state are all of
+ *     config->act_dtype; out is of config->out_dtype.  Parameters are float32.
+ *   - Pointers q, k, v, z, out, rec_state, conv_state and workspace must be
+ *     16-byte aligned.
+ *   - Argument errors are returned synchronously and launch nothing.  Launch
+ *     failures return GDN_ERR_CUDA.  Kernels never trap: a bounded wait that
+ *     runs out records a device error word and the kernel returns;
+ *     gdn_check_device_error reports it as GDN_ERR_DEVICE_TIMEOUT.
+ *   - No C++ exception crosses this interface.
+ *
+ * Supported shapes: d_k, d_v in {32, 64, 128}; n_v_heads a multiple of
+ * n_k_heads; conv_kernel == 4; chunk == 64 (the chunk length never changes the
+ * result, only how prefill is computed).  Anything else: GDN_ERR_UNSUPPORTED.
+ */
+#ifndef GDN_B200_H
+#define GDN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    GDN_OK = 0,
+    GDN_ERR_INVALID_ARG = 1,     /* null pointer, bad size, misaligned pointer   */
+    GDN_ERR_UNSUPPORTED = 2,     /* shape or dtype outside the supported set     */
+    GDN_ERR_CUDA = 3,            /* a CUDA launch or runtime call failed          */
+    GDN_ERR_DEVICE_TIMEOUT = 4,  /* a kernel's bounded wait ran out               */
+    GDN_ERR_WORKSPACE = 5        /* workspace smaller than gdn_prefill_workspace_size */
+} gdn_status;
+
+typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
+
+typedef struct {
+    int32_t n_k_heads;    /* H_k, default 16  */
+    int32_t n_v_heads;    /* H_v, default 48  */
+    int32_t d_k;          /* default 128      */
+    int32_t d_v;          /* default 128      */
+    int32_t conv_kernel;  /* K, default 4     */
+    int32_t chunk;        /* prefill chunk, default 64 */
+    float l2_eps;         /* default 1e-6     */
+    float norm_eps;       /* default 1e-6     */
+    int32_t act_dtype;    /* gdn_dtype of q, k, v, a, b, z, conv_state; default GDN_BF16 */
+    int32_t out_dtype;    /* gdn_dtype of out; default GDN_BF16 */
+} gdn_config;
+
+typedef struct {
+    const float* conv_weight;  /* [2*H_k*d_k + H_v*d_v][K], channel order q | k | v;
+                                  tap K-1 multiplies the current token            */
+    const float* A_log;        /* [H_v]                                           */
+    const float* dt_bias;      /* [H_v]                                           */
+    const float* norm_weight;  /* [d_v], shared by all value heads               */
+} gdn_weights;
+
+/* Fills *cfg with the layer's published shape (16/48 heads of 128, K = 4,
+ * chunk 64, eps 1e-6, bf16 activations and output). */
+void gdn_config_default(gdn_config* cfg);
+
+/* Bytes of device workspace gdn_prefill needs for T_total packed tokens.
+ * Returns 0 for an invalid or unsupported config. */
+size_t gdn_prefill_workspace_size(const gdn_config* cfg, int64_t T_total, int32_t n_seqs);
+
+/*
+ * Packed variable-length prefill.
+ *   q, k        [T_total][H_k][d_k]    act_dtype
+ *   v, z        [T_total][H_v][d_v]    act_dtype
+ *   a, b        [T_total][H_v]         act_dtype
+ *   conv_state  [n_seqs][2*H_k*d_k + H_v*d_v][K-1]  act_dtype, in/out, oldest first
+ *   rec_state   [n_seqs][H_v][d_v][d_k] float32, in/out
+ *   cu_seqlens  [n_seqs + 1] int32 device, cu_seqlens[0] = 0, non-decreasing,
+ *               cu_seqlens[n_seqs] = T_total (not checked on the host: it is
+ *               device memory and reading it would synchronise)
+ *   out         [T_total][H_v][d_v]    out_dtype
+ *   workspace   >= gdn_prefill_workspace_size(cfg, T_total, n_seqs) bytes,
+ *               256-byte aligned; contents need not be initialised
+ * Sequences of length 0 leave their states unchanged.  T_total == 0 is a no-op.
+ */
+gdn_status gdn_prefill(const gdn_config* cfg, const gdn_weights* w,
+                       const void* q, const void* k, const void* v,
+                       const void* a, const void* b, const void* z,
+                       void* conv_state, float* rec_state,
+                       const int32_t* cu_seqlens, int32_t n_seqs, int64_t T_total,
+                       void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * One decode step: one new token for each of n_seqs sequences.
+ *   q, k [n_seqs][H_k][d_k]; v, z [n_seqs][H_v][d_v]; a, b [n_seqs][H_v]  act_dtype
+ *   conv_state [n_seqs][C][K-1] act_dtype in/out; rec_state [n_seqs][H_v][d_v][d_k]
+ *   float32 in/out; out [n_seqs][H_v][d_v] out_dtype.  No workspace.
+ * Equal to gdn_prefill with every sequence of length 1.
+ */
+gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w,
+                      const void* q, const void* k, const void* v,
+                      const void* a, const void* b, const void* z,
+                      void* conv_state, float* rec_state, int32_t n_seqs,
+                      void* out, void* stream);
+
+/* Synchronises `stream`, then reads and clears the device error word that
+ * bounded waits write.  GDN_OK, GDN_ERR_DEVICE_TIMEOUT or GDN_ERR_CUDA. */
+gdn_status gdn_check_device_error(void* stream);
+
+/* Static string for a status code. */
+const char* gdn_status_string(gdn_status s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GDN_B200_H */

@@ -1,0 +1,95 @@
+"""The C-ABI library loads and exports every symbol include/gdn.h declares, and its
+host-side argument checks answer without touching a GPU (CPU only)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from hybrid_linear_attention_mixer_b200 import build, gdn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+OK, INVALID, UNSUPPORTED, CUDA, TIMEOUT, WORKSPACE = range(6)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return gdn.lib()
+
+
+def declared_functions():
+    names = []
+    for h in os.listdir(os.path.join(ROOT, "include")):
+        if h.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", h)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"\b(gdn_\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"gdn_prefill", "gdn_decode", "gdn_prefill_workspace_size"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(gdn.EXPORTS) <= set(names)
+
+
+def test_default_config_is_the_published_shape(lib):
+    c = gdn._CConfig()
+    lib.gdn_config_default(ctypes.byref(c))
+    assert (c.n_k_heads, c.n_v_heads, c.d_k, c.d_v, c.conv_kernel, c.chunk) == (16, 48, 128, 128, 4, 64)
+    assert abs(c.norm_eps - 1e-6) < 1e-12 and abs(c.l2_eps - 1e-6) < 1e-12
+    assert c.act_dtype == 0 and c.out_dtype == 0
+
+
+def test_workspace_size(lib):
+    cfg = gdn.Config()
+    T = 4096
+    # fp16 q^, k^ [T, 16*128] and v^ [T, 48*128], each rounded up to 256 bytes
+    assert gdn.workspace_size(cfg, T, 1) == 2 * T * 2048 * 2 + T * 6144 * 2
+    assert gdn.workspace_size(cfg, 0, 0) == 0
+    assert gdn.workspace_size(gdn.Config(d_k=48), T, 1) == 0
+
+
+def _call_prefill(lib, cfg, w=True, ptr=0x1000, T=16, n=1, ws_bytes=1 << 30, ws=0x100000):
+    c = cfg.c()
+    cw = gdn._CWeights(0x2000, 0x3000, 0x4000, 0x5000) if w else None
+    P = ctypes.c_void_p
+    ptrs = [P(ptr)] * 8
+    return lib.gdn_prefill(ctypes.byref(c), ctypes.byref(cw) if cw else None, *ptrs, P(0x6000), n, T,
+                           P(0x7000), P(ws), ws_bytes, None)
+
+
+def test_argument_errors_are_synchronous_and_launch_nothing(lib):
+    cfg = gdn.Config()
+    assert _call_prefill(lib, cfg, w=False) == INVALID
+    assert _call_prefill(lib, gdn.Config(d_k=48)) == UNSUPPORTED
+    assert _call_prefill(lib, gdn.Config(n_k_heads=5)) == UNSUPPORTED
+    assert _call_prefill(lib, gdn.Config(conv_kernel=3)) == UNSUPPORTED
+    assert _call_prefill(lib, gdn.Config(chunk=32)) == UNSUPPORTED
+    assert _call_prefill(lib, cfg, ptr=0x1001) == INVALID          # misaligned activation
+    assert _call_prefill(lib, cfg, ws=0x100010) == INVALID         # workspace not 256-aligned
+    assert _call_prefill(lib, cfg, ws_bytes=1000) == WORKSPACE
+    assert _call_prefill(lib, cfg, T=0) == OK                      # nothing to do
+    assert _call_prefill(lib, cfg, n=-1) == INVALID
+    c = cfg.c()
+    cw = gdn._CWeights(0x2000, 0x3000, 0x4000, 0x5000)
+    P = ctypes.c_void_p
+    assert lib.gdn_decode(ctypes.byref(c), ctypes.byref(cw), *[P(0)] * 8, 4, P(0x7000), None) == INVALID
+    assert lib.gdn_decode(ctypes.byref(c), ctypes.byref(cw), *[P(0x1000)] * 8, 0, P(0x7000), None) == OK
+    assert lib.gdn_decode(None, ctypes.byref(cw), *[P(0x1000)] * 8, 4, P(0x7000), None) == INVALID
+
+
+def test_status_strings(lib):
+    for s in range(6):
+        assert gdn.status_string(s)
+    assert gdn.status_string(99) == "unknown status"
+
+
+def test_binding_fails_loudly_without_library(monkeypatch):
+    monkeypatch.setattr(gdn, "_lib", None)
+    monkeypatch.setattr(gdn, "LIB_PATH", "/nonexistent/libgdn_b200.so")
+    with pytest.raises(RuntimeError):
+        gdn.lib()
