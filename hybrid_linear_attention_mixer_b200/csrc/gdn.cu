@@ -245,3 +245,43 @@ const char* gdn_status_string(gdn_status s) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// gdn_prefill_noalloc: gdn_prefill with its workspace in a fixed device array,
+// for callers that cannot allocate device memory (see gdn.h).
+// ---------------------------------------------------------------------------
+#include <mutex>
+
+static __device__ __align__(256) uint8_t g_noalloc_scratch[GDN_NOALLOC_SCRATCH_BYTES];
+
+namespace {
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[64];   // device address of g_noalloc_scratch, per device
+}  // namespace
+
+extern "C" gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const gdn_weights* w, const void* q,
+                                          const void* k, const void* v, const void* a, const void* b,
+                                          const void* z, void* conv_state, float* rec_state,
+                                          const int32_t* cu_seqlens, int32_t n_seqs, int64_t T_total,
+                                          void* out, void* stream) {
+    gdn_status s = check_config(cfg);
+    if (s != GDN_OK) return s;
+    if (n_seqs < 0 || T_total < 0) return GDN_ERR_INVALID_ARG;
+    if (workspace_layout(cfg, T_total).total > GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;
+    void* scratch = nullptr;
+    if (T_total > 0 && n_seqs > 0) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+        if (dev < 0 || dev >= 64) return GDN_ERR_UNSUPPORTED;
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_addr[dev]) {
+            // The array's name is a host-side stand-in; the kernels need its device address.
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GDN_ERR_CUDA;
+            g_noalloc_addr[dev] = p;
+        }
+        scratch = g_noalloc_addr[dev];
+    }
+    return gdn_prefill(cfg, w, q, k, v, a, b, z, conv_state, rec_state, cu_seqlens, n_seqs, T_total, out,
+                       scratch, GDN_NOALLOC_SCRATCH_BYTES, stream);
+}

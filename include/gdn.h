@@ -129,6 +129,48 @@ gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w,
                       void* conv_state, float* rec_state, int32_t n_seqs,
                       void* out, void* stream);
 
+/* Capacity, in bytes, of the fixed scratch array used by gdn_prefill_noalloc. */
+#define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * gdn_prefill_noalloc -- gdn_prefill for callers that cannot allocate device
+ * memory.  The pages have no counterpart of this call; it exists only for such
+ * callers.  Examples: a server whose device memory is all carved into its own
+ * pool at start-up, or a latency-critical caller that cannot afford the
+ * implicit device synchronisation of cudaMalloc/cudaFree.  Either way the caller
+ * cannot provide a gdn_prefill workspace.
+ *
+ * Arguments and results are those of gdn_prefill without `workspace` /
+ * `workspace_bytes`.  The caller still provides every input and output buffer.
+ * The scratch is one file-scope device array of GDN_NOALLOC_SCRATCH_BYTES
+ * (64 MiB).  It is allocated when the library's module is loaded on a GPU, and
+ * every GPU that loads the library keeps it until the process exits.  This call
+ * allocates nothing itself: no cudaMalloc, no cudaFree, no allocating library
+ * routine.
+ *
+ *   - Size limit: a request needing more than GDN_NOALLOC_SCRATCH_BYTES of
+ *     workspace is rejected with GDN_ERR_WORKSPACE, before any launch.  The
+ *     needed size is gdn_prefill_workspace_size(cfg, T_total, n_seqs); at the
+ *     published shape that is 20,480 bytes per token, so up to 3,276 tokens.
+ *     Longer prompts can be split into consecutive calls, since the states
+ *     carry from one call to the next.
+ *   - First call on a device: it looks up the array's device address with
+ *     cudaGetSymbolAddress (with that device current), then reuses it.  Make
+ *     this first call before any stream capture.
+ *   - Shared contents: all calls on a device share the one array, which keeps
+ *     the last call's contents.  Nothing in it needs to start at zero: each
+ *     call writes every scratch element it reads.
+ *   - Races: calls whose work overlaps on the GPU (different streams, no
+ *     ordering between them) race on the array.  Order them on one stream, or
+ *     with events.
+ */
+gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const gdn_weights* w,
+                               const void* q, const void* k, const void* v,
+                               const void* a, const void* b, const void* z,
+                               void* conv_state, float* rec_state,
+                               const int32_t* cu_seqlens, int32_t n_seqs, int64_t T_total,
+                               void* out, void* stream);
+
 /* Synchronises `stream`, then reads and clears the device error word that
  * bounded waits write.  GDN_OK, GDN_ERR_DEVICE_TIMEOUT or GDN_ERR_CUDA. */
 gdn_status gdn_check_device_error(void* stream);
