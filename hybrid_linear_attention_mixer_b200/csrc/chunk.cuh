@@ -50,17 +50,23 @@ constexpr uint32_t OFF_W = 81920;       // -W^T: 128 d_k rows x 64 chunk columns
 constexpr uint32_t OFF_S16 = 98304;     // S (fp16 copy): 128 d_v rows x d_k, halves of 16384
 constexpr uint32_t OFF_UT = 131072;     // U^T: 128 d_v rows x 64 chunk columns
 constexpr uint32_t OFF_P = 147456;      // P: 64 x 64 (row r, col j)
+constexpr uint32_t OFF_ZT = 155648;    // z (bf16): 64 token rows x d_v, halves of 8192; the
+                                        // gated output is staged in place before its store
 constexpr int LDA = 65;                 // fp32 64 x 64 work matrices, padded rows
-constexpr uint32_t OFF_A = 155648;
+constexpr uint32_t OFF_A = 172032;
 constexpr uint32_t OFF_X = OFF_A + 64 * LDA * 4;
 constexpr uint32_t OFF_Z = OFF_X + 64 * LDA * 4;
 constexpr uint32_t OFF_G = OFF_Z + 64 * LDA * 4;   // g[64]
 constexpr uint32_t OFF_B = OFF_G + 256;            // beta[64]
 constexpr uint32_t OFF_RED = OFF_B + 256;          // [4][64] partial sums of o^2
 constexpr uint32_t OFF_RS = OFF_RED + 1024;        // rsqrt(mean o^2 + eps) [64]
-constexpr uint32_t OFF_BAR = OFF_RS + 256;         // mbarrier, TMEM address, abort flag
+constexpr uint32_t OFF_BAR = OFF_RS + 256;         // mbarriers, TMEM address, abort flag
 constexpr uint32_t SMEM_USED = OFF_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;  // slack for the 1024-byte alignment
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+// Bytes one chunk's TMA loads deliver: q, k, v halves (6 boxes) and z halves (2 boxes)
+constexpr uint32_t QKV_BYTES = 6 * 8192, Z_BYTES = 2 * 8192;
 
 // Tensor-memory columns (fp32 accumulators, 128 lanes each)
 constexpr uint32_t ACC_QK = 0, ACC_W = 64, ACC_U = 128, ACC_O1 = 192, ACC_O2 = 256, ACC_SI = 320;
@@ -71,10 +77,10 @@ constexpr uint32_t ID_MK_64 = idesc_f16(128, 64, 1, 0);
 constexpr uint32_t ID_KM_64 = idesc_f16(128, 64, 0, 1);
 constexpr uint32_t ID_KM_128 = idesc_f16(128, 128, 0, 1);
 
+// The q^, k^ (unit norm, fp16), v^ (fp16) and z (bf16) tiles arrive through 3-D
+// TMA tensor maps over [T][H][d] with boxes of 64 (d) x 1 (head) x 64 (tokens)
+// and the 128-byte swizzle; columns past d and rows past T read as zero.
 struct Args {
-    const __half* qh;        // [T][Hk][dk] unit-norm q
-    const __half* kh;        // [T][Hk][dk] unit-norm k
-    const __half* vh;        // [T][Hv][dv]
     const void* a;           // [T][Hv] act dtype
     const void* b;           // [T][Hv]
     const void* z;           // [T][Hv][dv]
@@ -109,7 +115,11 @@ __device__ __forceinline__ uint4 scale8(uint4 v, float s) {
 }
 
 template <typename TA, typename TO>
-__global__ void __launch_bounds__(NT, 1) gdn_chunk_kernel(Args p) {
+__global__ void __launch_bounds__(NT, 1)
+gdn_chunk_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                 const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_z, Args p) {
+    constexpr bool kZTile = sizeof(TA) == 2;                  // z through TMA (bf16 activations)
+    constexpr bool kOutStage = kZTile && sizeof(TO) == 2;     // out staged in the z tile
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sb = (raw + 1023u) & ~1023u;
@@ -121,7 +131,9 @@ __global__ void __launch_bounds__(NT, 1) gdn_chunk_kernel(Args p) {
     float* Am = reinterpret_cast<float*>(smem + OFF_A);
     float* Xm = reinterpret_cast<float*>(smem + OFF_X);
     float* Zm = reinterpret_cast<float*>(smem + OFF_Z);
-    const uint32_t bar = sb + OFF_BAR;
+    const uint32_t bar = sb + OFF_BAR;          // tensor-core commits
+    const uint32_t bar_ld = sb + OFF_BAR + 24;  // q, k, v tiles of a chunk
+    const uint32_t bar_z = sb + OFF_BAR + 32;   // z tile of a chunk
     volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 8);
     volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 16);
 
@@ -132,13 +144,23 @@ __global__ void __launch_bounds__(NT, 1) gdn_chunk_kernel(Args p) {
     const int seq = blockIdx.x / Hv, h = blockIdx.x % Hv;
     const int j = h / (Hv / Hk);
     const int64_t s0 = p.cu[seq], s1 = p.cu[seq + 1];
+    const TA* __restrict__ pa = static_cast<const TA*>(p.a);
+    const TA* __restrict__ pb = static_cast<const TA*>(p.b);
+    const TA* __restrict__ pz = static_cast<const TA*>(p.z);
+    TO* __restrict__ pout = static_cast<TO*>(p.out);
     const int nchunks = (int)((s1 - s0 + C - 1) / C);
     if (nchunks <= 0) return;
 
     if (tid == 0) {
         mbar_init(bar, 1);
+        mbar_init(bar_ld, 1);
+        mbar_init(bar_z, 1);
         fence_mbar_init();
         *s_abort = 0;
+        prefetch_tmap(&tm_q);
+        prefetch_tmap(&tm_k);
+        prefetch_tmap(&tm_v);
+        if (kZTile) prefetch_tmap(&tm_z);
     }
     if (warp == 0) {
         tmem_alloc(sb + OFF_BAR + 8, TMEM_COLS);
@@ -150,6 +172,35 @@ __global__ void __launch_bounds__(NT, 1) gdn_chunk_kernel(Args p) {
     const uint32_t tmem = *s_tmem;
     const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);   // this warp's lane quadrant
     uint32_t phase = 0;
+
+    int ld_issued = 0, z_issued = 0;   // TMA loads issued (thread 0) ...
+    int ld_ok = 0, z_ok = 0;           // ... and completed waits on them
+    auto issue_qkv = [&](int64_t t) {   // one thread: the q, k, v tiles of the chunk at token t
+        ld_issued++;
+        mbar_arrive_expect_tx(bar_ld, QKV_BYTES);
+#pragma unroll
+        for (int hf = 0; hf < 2; hf++) {
+            tma_load_3d(sb + OFF_QK + hf * 16384, &tm_q, 64 * hf, j, (int)t, bar_ld);
+            tma_load_3d(sb + OFF_QK + hf * 16384 + C * 128, &tm_k, 64 * hf, j, (int)t, bar_ld);
+            tma_load_3d(sb + OFF_V + hf * 8192, &tm_v, 64 * hf, h, (int)t, bar_ld);
+        }
+    };
+    auto issue_z = [&](int64_t t) {
+        z_issued++;
+        mbar_arrive_expect_tx(bar_z, Z_BYTES);
+#pragma unroll
+        for (int hf = 0; hf < 2; hf++) tma_load_3d(sb + OFF_ZT + hf * 8192, &tm_z, 64 * hf, h, (int)t, bar_z);
+    };
+    if (tid == 0) {
+        issue_qkv(s0);
+        if (kZTile) issue_z(s0);
+    }
+    // gate inputs of the next chunk, loaded one chunk ahead (threads 0..63)
+    float a_nx = 0.f, b_nx = 0.f;
+    if (tid < C && s0 + tid < s1) {
+        a_nx = to_f32(pa[(s0 + tid) * Hv + h]);
+        b_nx = to_f32(pb[(s0 + tid) * Hv + h]);
+    }
 
     // fp32 state: this thread owns row dv_r, columns [64*half, 64*half + 64)
     const int dv_r = 32 * qd + lane;
@@ -165,15 +216,11 @@ __global__ void __launch_bounds__(NT, 1) gdn_chunk_kernel(Args p) {
     const float dtb = p.dt_bias[h];
     const float inv_sqrt_dk = rsqrtf((float)dk);
     const float wn = dv_r < dv ? p.norm_w[dv_r] : 0.f;
-    const int64_t ldq = (int64_t)Hk * dk, ldv = (int64_t)Hv * dv;
-    const TA* pa = static_cast<const TA*>(p.a);
-    const TA* pb = static_cast<const TA*>(p.b);
-    const TA* pz = static_cast<const TA*>(p.z);
-    TO* pout = static_cast<TO*>(p.out);
+    const int64_t ldv = (int64_t)Hv * dv;
 
 #define GDN_MMA_WAIT()                                        \
     do {                                                      \
-        if (!mbar_wait_bounded(bar, phase)) *s_abort = 1;     \
+        if (!mbar_wait_bounded(bar, phase)) atomicOr((unsigned*)s_abort, 1u); \
         phase ^= 1;                                           \
         __syncthreads();                                      \
         if (*s_abort) goto abort_;                            \
@@ -195,10 +242,14 @@ __global__ void __launch_bounds__(NT, 1) gdn_chunk_kernel(Args p) {
         if (tid < C) {
             float la = 0.f, bt = 0.f;
             if (tid < n) {
-                const float av = to_f32(pa[(t0 + tid) * Hv + h]);
-                const float bv = to_f32(pb[(t0 + tid) * Hv + h]);
-                la = -expA * softplus_f(av + dtb);
-                bt = sigmoid_f(bv);
+                la = -expA * softplus_f(a_nx + dtb);
+                bt = sigmoid_f(b_nx);
+            }
+            const int64_t tn = t0 + C + tid;   // prefetch the next chunk's a, b
+            a_nx = b_nx = 0.f;
+            if (tn < s1) {
+                a_nx = to_f32(pa[tn * Hv + h]);
+                b_nx = to_f32(pb[tn * Hv + h]);
             }
             float g = la;
 #pragma unroll
@@ -214,29 +265,19 @@ __global__ void __launch_bounds__(NT, 1) gdn_chunk_kernel(Args p) {
         __syncthreads();
         const float g_last = s_g[C - 1];
 
-        // ---- operand tiles: [Q;K], K~ (scaled keys), V ----
+        // ---- wait for this chunk's q, k, v tiles; K~ = diag(e^{g_C - g}) K from the k rows ----
+        if (mbar_wait_bounded(bar_ld, ci & 1)) ld_ok++; else atomicOr((unsigned*)s_abort, 2u);
         for (int idx = tid; idx < C * 16; idx += NT) {
             const int r = idx >> 4, c16 = idx & 15;
             const int hf = c16 >> 3, cc = c16 & 7;
-            uint4 qv = make_uint4(0, 0, 0, 0), kv = qv, vv = qv;
-            if (r < n) {
-                if (c16 * 8 < dk) {
-                    qv = *reinterpret_cast<const uint4*>(p.qh + (t0 + r) * ldq + j * dk + c16 * 8);
-                    kv = *reinterpret_cast<const uint4*>(p.kh + (t0 + r) * ldq + j * dk + c16 * 8);
-                }
-                if (c16 * 8 < dv)
-                    vv = *reinterpret_cast<const uint4*>(p.vh + (t0 + r) * ldv + (int64_t)h * dv + c16 * 8);
-            }
-            const float sc = r < n ? __expf(g_last - s_g[r]) : 0.f;
-            const uint4 kt = scale8(kv, sc);
-            sts128(sb + OFF_QK + hf * 16384 + swz128(r, cc), qv.x, qv.y, qv.z, qv.w);
-            sts128(sb + OFF_QK + hf * 16384 + swz128(C + r, cc), kv.x, kv.y, kv.z, kv.w);
+            const uint4 kv = lds128(sb + OFF_QK + hf * 16384 + swz128(C + r, cc));
+            const uint4 kt = scale8(kv, r < n ? __expf(g_last - s_g[r]) : 0.f);
             sts128(sb + OFF_KT + hf * 8192 + swz128(r, cc), kt.x, kt.y, kt.z, kt.w);
-            sts128(sb + OFF_V + hf * 8192 + swz128(r, cc), vv.x, vv.y, vv.z, vv.w);
         }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
+        if (*s_abort) goto abort_;
 
         // ---- (a) [Q;K] K^T and (e) S Q^T ----
         if (tid == 0) {
@@ -372,6 +413,11 @@ __global__ void __launch_bounds__(NT, 1) gdn_chunk_kernel(Args p) {
             mma_commit(bar);
         }
         GDN_MMA_WAIT();
+        // (a), (b), (c), (e) are done with the q, k, v tiles: fetch the next chunk's
+        if (tid == 0 && ci + 1 < nchunks) {
+            fence_async_smem();
+            issue_qkv(t0 + C);
+        }
 
         // ---- -W^T -> fp16 tile (row d_k, chunk columns) ----
         {
@@ -476,15 +522,49 @@ __global__ void __launch_bounds__(NT, 1) gdn_chunk_kernel(Args p) {
                 s_rs[tid] = rsqrtf(ss / (float)dv + p.norm_eps);
             }
             __syncthreads();
-            if (dv_r < dv) {
-#pragma unroll 4
+            if constexpr (kZTile) {
+                if (mbar_wait_bounded(bar_z, ci & 1)) z_ok++; else atomicOr((unsigned*)s_abort, 2u);
+                // z[r][dv_r] from the swizzled tile; the result overwrites it in place
+                const uint32_t zcol = (uint32_t)(dv_r >> 6) * 8192 + (uint32_t)(dv_r & 7) * 2;
+#pragma unroll
                 for (int i = 0; i < 32; i++) {
                     const int r = 32 * half + i;
-                    if (r < n) {
-                        const int64_t off = (t0 + r) * ldv + (int64_t)h * dv + dv_r;
-                        const float zz = to_f32(pz[off]);
-                        from_f32(o[i] * s_rs[r] * wn * silu_f(zz), pout + off);
+                    __nv_bfloat16* zp = reinterpret_cast<__nv_bfloat16*>(smem + OFF_ZT + zcol +
+                                                                         swz128(r, (dv_r & 63) >> 3));
+                    const float y = o[i] * s_rs[r] * wn * silu_f(__bfloat162float(*zp));
+                    if constexpr (kOutStage) {
+                        *zp = __float2bfloat16_rn(y);
+                    } else {
+                        if (r < n && dv_r < dv) from_f32(y, pout + (t0 + r) * ldv + (int64_t)h * dv + dv_r);
                     }
+                }
+                if constexpr (kOutStage) {
+                    __syncthreads();
+                    for (int idx = tid; idx < C * 16; idx += NT) {   // 16-byte row pieces
+                        const int r = idx >> 4, c16 = idx & 15;
+                        if (r < n && c16 * 8 < dv) {
+                            const uint4 v4 = lds128(sb + OFF_ZT + (c16 >> 3) * 8192 + swz128(r, c16 & 7));
+                            __stcs(reinterpret_cast<uint4*>(pout + (t0 + r) * ldv + (int64_t)h * dv + c16 * 8), v4);
+                        }
+                    }
+                }
+                __syncthreads();
+                if (*s_abort) goto abort_;
+                if (tid == 0 && ci + 1 < nchunks) {   // the z tile is free: fetch the next chunk's
+                    fence_async_smem();
+                    issue_z(t0 + C);
+                }
+            } else if (dv_r < dv) {
+                float zz[32];
+#pragma unroll
+                for (int i = 0; i < 32; i++) {
+                    const int r = 32 * half + i;
+                    zz[i] = r < n ? to_f32(pz[(t0 + r) * ldv + (int64_t)h * dv + dv_r]) : 0.f;
+                }
+#pragma unroll
+                for (int i = 0; i < 32; i++) {
+                    const int r = 32 * half + i;
+                    if (r < n) from_f32(o[i] * s_rs[r] * wn * silu_f(zz[i]), pout + (t0 + r) * ldv + (int64_t)h * dv + dv_r);
                 }
             }
         }
@@ -505,11 +585,17 @@ __global__ void __launch_bounds__(NT, 1) gdn_chunk_kernel(Args p) {
     return;
 
 abort_:
-    // A tensor-core commit never arrived: report it, give in-flight MMAs one more
-    // bounded wait, release tensor memory and return.  The state is left as it was.
-    if (tid == 0) record_error(kErrMmaTimeout);
+    // A tensor-core commit or a TMA load never arrived: report it, give whatever
+    // is still in flight one more bounded wait, release tensor memory and return.
+    // The recurrent state is left as it was.
+    if (tid == 0) {
+        record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));
+        for (int k = ld_ok; k < ld_issued; k++) mbar_wait_bounded(bar_ld, k & 1);
+        for (int k = z_ok; k < z_issued; k++) mbar_wait_bounded(bar_z, k & 1);
+    }
     if (warp == 0) {
-        mbar_wait_bounded(bar, phase ^ 1u);   // the phase that did not complete
+        mbar_wait_bounded(bar, phase ^ 1u);   // the tensor-core phase that did not complete, if any
+        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }

@@ -30,24 +30,55 @@ struct ConvArgs {
     __half* vh;              // [T][Cv]
 };
 
-constexpr int kConvTokens = 16;
 constexpr int kConvThreads = 128;   // 8 channels per thread
+// tokens per CTA: every thread keeps TT + 3 rows of 8 inputs in registers
+template <typename TA> __host__ __device__ constexpr int conv_tokens() { return sizeof(TA) == 2 ? 16 : 8; }
 
 template <typename TA>
-__device__ __forceinline__ const TA* conv_channel_ptr(const ConvArgs& p, int64_t t, int c, int Cq, int Cv) {
+__device__ __forceinline__ const TA* __restrict__ conv_channel_ptr(const ConvArgs& p, int64_t t, int c, int Cq, int Cv) {
     if (c < Cq) return static_cast<const TA*>(p.q) + t * Cq + c;
     if (c < 2 * Cq) return static_cast<const TA*>(p.k) + t * Cq + (c - Cq);
     return static_cast<const TA*>(p.v) + t * Cv + (c - 2 * Cq);
 }
 
+// 8 consecutive activations of one token, kept packed until used.
+template <typename TA> struct Raw8;
+template <> struct Raw8<__nv_bfloat16> {
+    uint4 u;
+    __device__ __forceinline__ void load(const __nv_bfloat16* __restrict__ p) { u = __ldg(reinterpret_cast<const uint4*>(p)); }
+    __device__ __forceinline__ void zero() { u = make_uint4(0, 0, 0, 0); }
+    __device__ __forceinline__ void get(float (&f)[8]) const {
+        const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const float2 t = __bfloat1622float2(h[i]);
+            f[2 * i] = t.x;
+            f[2 * i + 1] = t.y;
+        }
+    }
+};
+template <> struct Raw8<float> {
+    float4 a, b;
+    __device__ __forceinline__ void load(const float* __restrict__ p) {
+        a = __ldg(reinterpret_cast<const float4*>(p));
+        b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+    }
+    __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+    __device__ __forceinline__ void get(float (&f)[8]) const {
+        f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+        f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+    }
+};
+
 template <typename TA>
 __global__ void __launch_bounds__(kConvThreads) conv_silu_norm_kernel(ConvArgs p) {
+    constexpr int TT = conv_tokens<TA>();
     const int Cq = p.Hk * p.dk, Cv = p.Hv * p.dv, Ctot = 2 * Cq + Cv;
     const int c = (blockIdx.y * kConvThreads + threadIdx.x) * 8;   // first of 8 channels
-    const int64_t t_begin = (int64_t)blockIdx.x * kConvTokens;
-    __shared__ int s_seq[kConvTokens];
-    __shared__ long long s_start[kConvTokens];
-    if (threadIdx.x < kConvTokens) {
+    const int64_t t_begin = (int64_t)blockIdx.x * TT;
+    __shared__ int s_seq[TT];
+    __shared__ long long s_start[TT];
+    if (threadIdx.x < TT) {
         const int64_t t = t_begin + threadIdx.x;
         int lo = 0, hi = p.n_seqs - 1;              // last s with cu[s] <= t
         while (lo < hi) {
@@ -57,48 +88,44 @@ __global__ void __launch_bounds__(kConvThreads) conv_silu_norm_kernel(ConvArgs p
         s_seq[threadIdx.x] = lo;
         s_start[threadIdx.x] = p.cu[lo];
     }
-    __syncthreads();
-
     const bool active = c < Ctot;
     const bool is_qk = c < 2 * Cq;
-    const int group = p.dk >> 3;                    // threads per key head (4, 8 or 16)
+    // All TT + 3 input rows of this thread's 8 channels are requested before any
+    // is used, so their latencies overlap.
+    Raw8<TA> raw[TT + 3];
+#pragma unroll
+    for (int s = 0; s < TT + 3; s++) {
+        const int64_t t = t_begin - 3 + s;
+        raw[s].zero();
+        if (active && t >= 0 && t < p.T) raw[s].load(conv_channel_ptr<TA>(p, t, c, Cq, Cv));
+    }
     float w[8][4];
-    float win[3][8];                                // x_{t-3}, x_{t-2}, x_{t-1}
 #pragma unroll
     for (int i = 0; i < 8; i++) {
         float4 t4 = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (active) t4 = reinterpret_cast<const float4*>(p.conv_w)[c + i];
+        if (active) t4 = __ldg(reinterpret_cast<const float4*>(p.conv_w) + c + i);
         w[i][0] = t4.x; w[i][1] = t4.y; w[i][2] = t4.z; w[i][3] = t4.w;
     }
-#pragma unroll
-    for (int s = 0; s < 3; s++) {
-        const int64_t t = t_begin - 3 + s;
-#pragma unroll
-        for (int i = 0; i < 8; i++) win[s][i] = 0.f;
-        if (active && t >= 0 && t < p.T) load8(conv_channel_ptr<TA>(p, t, c, Cq, Cv), win[s]);
-    }
+    __syncthreads();
 
-    for (int it = 0; it < kConvTokens; it++) {
+    const int group = p.dk >> 3;                    // threads per key head (4, 8 or 16)
+#pragma unroll
+    for (int it = 0; it < TT; it++) {
         const int64_t t = t_begin + it;
         const bool valid = active && t < p.T;
-        float x[8];
-#pragma unroll
-        for (int i = 0; i < 8; i++) x[i] = 0.f;
-        if (valid) load8(conv_channel_ptr<TA>(p, t, c, Cq, Cv), x);
-        // taps before the sequence start come from its conv_state
-        float tap[3][8];
+        float x[8], tap[3][8];
+        raw[it + 3].get(x);
         const int64_t s0 = s_start[it];
 #pragma unroll
         for (int s = 0; s < 3; s++) {
             const int64_t u = t - 3 + s;
-            if (valid && u < s0) {
+            if (valid && u < s0) {     // taps before the sequence start come from its conv_state
                 const int slot = 3 - (int)(s0 - u);
                 const TA* st = static_cast<const TA*>(p.conv_state) + ((int64_t)s_seq[it] * Ctot + c) * 3 + slot;
 #pragma unroll
                 for (int i = 0; i < 8; i++) tap[s][i] = to_f32(st[i * 3]);
             } else {
-#pragma unroll
-                for (int i = 0; i < 8; i++) tap[s][i] = win[s][i];
+                raw[it + s].get(tap[s]);
             }
         }
         float y[8];
@@ -128,13 +155,7 @@ __global__ void __launch_bounds__(kConvThreads) conv_silu_norm_kernel(ConvArgs p
             __half* dst = c < Cq ? p.qh + t * Cq + c
                         : c < 2 * Cq ? p.kh + t * Cq + (c - Cq)
                                      : p.vh + t * Cv + (c - 2 * Cq);
-            *reinterpret_cast<uint4*>(dst) = o;
-        }
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-            win[0][i] = win[1][i];
-            win[1][i] = win[2][i];
-            win[2][i] = x[i];
+            __stcs(reinterpret_cast<uint4*>(dst), o);
         }
     }
 }

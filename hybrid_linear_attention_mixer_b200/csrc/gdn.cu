@@ -2,8 +2,11 @@
 // kernel launches.  One translation unit holds every kernel.
 #include "gdn.h"
 
+#include <cudaTypedefs.h>
+
 #include <cmath>
 #include <cstring>
+#include <mutex>
 
 #include "chunk.cuh"
 #include "conv.cuh"
@@ -67,6 +70,35 @@ cudaError_t ensure_smem(K kernel, int variant, size_t bytes) {
     return e;
 }
 
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime.
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+    });
+    return fn;
+}
+
+// 3-D map over a row-major [T][H][d] tensor: boxes of 64 (d) x 1 (head) x 64
+// (tokens), 128-byte swizzle; elements past d or T read as zero.
+bool head_tile_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem_bytes, int d, int H,
+                   int64_t T) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T};
+    cuuint64_t strides[2] = {(cuuint64_t)d * elem_bytes, (cuuint64_t)H * d * elem_bytes};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)gdn::chunk::C};
+    cuuint32_t estr[3] = {1, 1, 1};
+    return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <typename TA, typename TO>
 cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void* q, const void* k,
                            const void* v, const void* a, const void* b, const void* z, void* conv_state,
@@ -86,15 +118,28 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     ca.qh = reinterpret_cast<__half*>(wsb + L.q_off);
     ca.kh = reinterpret_cast<__half*>(wsb + L.k_off);
     ca.vh = reinterpret_cast<__half*>(wsb + L.v_off);
+    // Set-up first: nothing is launched unless the tensor maps encode and the
+    // chunk kernel's shared-memory opt-in succeeds.
+    auto kern = gdn::chunk::gdn_chunk_kernel<TA, TO>;
+    cudaError_t e = ensure_smem(kern, variant, gdn::chunk::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    CUtensorMap tm_q, tm_k, tm_v, tm_z;
+    std::memset(&tm_z, 0, sizeof tm_z);
+    const int Hk = c->n_k_heads, Hv = c->n_v_heads;
+    if (!head_tile_map(&tm_q, ca.qh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, Hk, T) ||
+        !head_tile_map(&tm_k, ca.kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, Hk, T) ||
+        !head_tile_map(&tm_v, ca.vh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_v, Hv, T))
+        return cudaErrorInvalidValue;
+    if (sizeof(TA) == 2 && !head_tile_map(&tm_z, z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c->d_v, Hv, T))
+        return cudaErrorInvalidValue;
     const int Ctot = 2 * c->n_k_heads * c->d_k + c->n_v_heads * c->d_v;
     const int cblocks = (Ctot / 8 + gdn::kConvThreads - 1) / gdn::kConvThreads;
-    const int64_t tblocks = (T + gdn::kConvTokens - 1) / gdn::kConvTokens;
+    const int64_t tblocks = (T + gdn::conv_tokens<TA>() - 1) / gdn::conv_tokens<TA>();
     if (tblocks > 0x7fffffff) return cudaErrorInvalidValue;
     gdn::conv_silu_norm_kernel<TA><<<dim3((unsigned)tblocks, cblocks), gdn::kConvThreads, 0, st>>>(ca);
     gdn::conv_state_update_kernel<TA><<<dim3(n_seqs, (Ctot + 255) / 256), 256, 0, st>>>(ca, conv_state);
 
     gdn::chunk::Args pa;
-    pa.qh = ca.qh; pa.kh = ca.kh; pa.vh = ca.vh;
     pa.a = a; pa.b = b; pa.z = z;
     pa.A_log = w->A_log; pa.dt_bias = w->dt_bias; pa.norm_w = w->norm_weight;
     pa.rec_state = rec_state;
@@ -102,10 +147,7 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     pa.out = out;
     pa.Hk = c->n_k_heads; pa.Hv = c->n_v_heads; pa.dk = c->d_k; pa.dv = c->d_v;
     pa.norm_eps = c->norm_eps;
-    auto kern = gdn::chunk::gdn_chunk_kernel<TA, TO>;
-    cudaError_t e = ensure_smem(kern, variant, gdn::chunk::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    kern<<<(unsigned)n_seqs * c->n_v_heads, gdn::chunk::NT, gdn::chunk::SMEM_BYTES, st>>>(pa);
+    kern<<<(unsigned)n_seqs * c->n_v_heads, gdn::chunk::NT, gdn::chunk::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v, tm_z, pa);
     return cudaGetLastError();
 }
 
@@ -170,6 +212,7 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_weights* w, const void* 
         if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;
     if (!aligned(workspace, 256)) return GDN_ERR_INVALID_ARG;
     if ((int64_t)n_seqs * cfg->n_v_heads > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    if (T_total > 0x7fffffffLL - 64) return GDN_ERR_UNSUPPORTED;   // token coordinates are int32
     if (workspace_bytes < workspace_layout(cfg, T_total).total) return GDN_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;

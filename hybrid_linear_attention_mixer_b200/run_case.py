@@ -1,0 +1,59 @@
+"""Run one synthetic workload through the public API (no timing, no oracle).
+
+    python -m hybrid_linear_attention_mixer_b200.run_case --case prefill_4k --iters 2
+    python -m hybrid_linear_attention_mixer_b200.run_case --case decode_256 --batch 64 --iters 3
+
+A small, fixed-size target for profilers such as ncu: it builds the seeded
+inputs of the named workload, runs the layer `iters` times on cuda:0 and checks
+the device error word.
+"""
+from __future__ import annotations
+
+import argparse
+
+import numpy as np
+import torch
+
+from hybrid_linear_attention_mixer_b200 import gdn, inputs
+
+
+def _act(x, dev):
+    x = np.ascontiguousarray(x)
+    if x.dtype == np.uint16:
+        return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+    return torch.from_numpy(x).to(dev)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--case", default="prefill_4k", choices=inputs.CASES)
+    ap.add_argument("--iters", type=int, default=2)
+    ap.add_argument("--tokens", type=int, default=None, help="shrink a prefill workload to T tokens")
+    ap.add_argument("--batch", type=int, default=None, help="decode batch (sequences)")
+    args = ap.parse_args()
+    dev = torch.device("cuda:0")
+    if args.case == "decode_256":
+        c = inputs.make_case(args.case, n_seqs=args.batch, T=1)
+    else:
+        c = inputs.make_case(args.case, T=args.tokens)
+    act = torch.bfloat16 if c.bf16 else torch.float32
+    cfg = gdn.Config(c.n_k_heads, c.n_v_heads, c.d_k, c.d_v, c.conv_kernel, 64, c.l2_eps, c.norm_eps,
+                     act, act)
+    w = {n: torch.from_numpy(np.ascontiguousarray(c.weights[n])).to(dev)
+         for n in ("conv_w", "A_log", "dt_bias", "norm_w")}
+    d = {n: _act(c.acts[n], dev) for n in "qkvabz"}
+    cs = _act(c.conv_state, dev)
+    rs = torch.from_numpy(c.rec_state).to(dev)
+    for _ in range(args.iters):
+        if args.case == "decode_256":
+            gdn.decode(cfg, w, d["q"], d["k"], d["v"], d["a"], d["b"], d["z"], cs, rs)
+        else:
+            cu = torch.from_numpy(c.cu_seqlens).to(dev)
+            gdn.prefill(cfg, w, d["q"], d["k"], d["v"], d["a"], d["b"], d["z"], cs, rs, cu)
+    gdn.check_device_error()
+    torch.cuda.synchronize()
+    print("ok", args.case, "T=%d" % c.T, "seqs=%d" % c.n_seqs)
+
+
+if __name__ == "__main__":
+    main()
