@@ -32,7 +32,7 @@ struct ConvArgs {
 
 constexpr int kConvThreads = 128;   // 8 channels per thread
 // tokens per CTA: every thread keeps TT + 3 rows of 8 inputs in registers
-template <typename TA> __host__ __device__ constexpr int conv_tokens() { return sizeof(TA) == 2 ? 16 : 8; }
+template <typename TA> __host__ __device__ constexpr int conv_tokens() { return sizeof(TA) == 2 ? 8 : 4; }
 
 template <typename TA>
 __device__ __forceinline__ const TA* __restrict__ conv_channel_ptr(const ConvArgs& p, int64_t t, int c, int Cq, int Cv) {

@@ -8,10 +8,11 @@
 #include <cstring>
 #include <mutex>
 
-#include "chunk.cuh"
 #include "conv.cuh"
 #include "decode.cuh"
 #include "device.cuh"
+#include "intra.cuh"
+#include "scan.cuh"
 
 namespace {
 
@@ -32,7 +33,7 @@ gdn_status check_config(const gdn_config* c) {
     if (c->out_dtype != GDN_BF16 && c->out_dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
     if (c->n_v_heads % c->n_k_heads != 0) return GDN_ERR_UNSUPPORTED;
     if (!dim_ok(c->d_k) || !dim_ok(c->d_v)) return GDN_ERR_UNSUPPORTED;
-    if (c->conv_kernel != 4 || c->chunk != gdn::chunk::C) return GDN_ERR_UNSUPPORTED;
+    if (c->conv_kernel != 4 || c->chunk != gdn::intra::C) return GDN_ERR_UNSUPPORTED;
     return GDN_OK;
 }
 
@@ -42,18 +43,24 @@ gdn_status check_weights(const gdn_weights* w) {
     return GDN_OK;
 }
 
+// Prefill workspace: fp16 q^, k^, v^ (conv output), the first chunk of each
+// sequence, and one intra-chunk record per (chunk, value head).
 struct Layout {
-    size_t q_off, k_off, v_off, total;
+    size_t q_off, k_off, v_off, coff_off, rec_off, total;
 };
 
-Layout workspace_layout(const gdn_config* c, int64_t T) {
+Layout workspace_layout(const gdn_config* c, int64_t T, int64_t n_seqs) {
     Layout L;
     const size_t qb = align_up((size_t)T * c->n_k_heads * c->d_k * sizeof(__half), 256);
     const size_t vb = align_up((size_t)T * c->n_v_heads * c->d_v * sizeof(__half), 256);
+    const size_t cb = align_up((size_t)(n_seqs + 1) * sizeof(int32_t), 256);
+    const size_t max_chunks = (size_t)((T + gdn::intra::C - 1) / gdn::intra::C) + (size_t)n_seqs;
     L.q_off = 0;
     L.k_off = qb;
     L.v_off = 2 * qb;
-    L.total = 2 * qb + vb;
+    L.coff_off = 2 * qb + vb;
+    L.rec_off = L.coff_off + cb;
+    L.total = L.rec_off + max_chunks * c->n_v_heads * gdn::intra::REC_BYTES;
     return L;
 }
 
@@ -92,7 +99,7 @@ bool head_tile_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)T};
     cuuint64_t strides[2] = {(cuuint64_t)d * elem_bytes, (cuuint64_t)H * d * elem_bytes};
-    cuuint32_t box[3] = {64, 1, (cuuint32_t)gdn::chunk::C};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)gdn::intra::C};
     cuuint32_t estr[3] = {1, 1, 1};
     return enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -104,7 +111,7 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
                            const void* v, const void* a, const void* b, const void* z, void* conv_state,
                            float* rec_state, const int32_t* cu, int n_seqs, int64_t T, void* out,
                            void* ws, int variant, cudaStream_t st) {
-    const Layout L = workspace_layout(c, T);
+    const Layout L = workspace_layout(c, T, n_seqs);
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     ConvArgs ca;
     ca.q = q; ca.k = k; ca.v = v;
@@ -119,9 +126,12 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     ca.kh = reinterpret_cast<__half*>(wsb + L.k_off);
     ca.vh = reinterpret_cast<__half*>(wsb + L.v_off);
     // Set-up first: nothing is launched unless the tensor maps encode and the
-    // chunk kernel's shared-memory opt-in succeeds.
-    auto kern = gdn::chunk::gdn_chunk_kernel<TA, TO>;
-    cudaError_t e = ensure_smem(kern, variant, gdn::chunk::SMEM_BYTES);
+    // kernels' shared-memory opt-ins succeed.
+    auto k_intra = gdn::intra::gdn_intra_kernel<TA>;
+    auto k_scan = gdn::scan::gdn_scan_kernel<TA, TO>;
+    cudaError_t e = ensure_smem(k_intra, 4 + (sizeof(TA) == 2 ? 0 : 1), gdn::intra::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    e = ensure_smem(k_scan, variant, gdn::scan::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     CUtensorMap tm_q, tm_k, tm_v, tm_z;
     std::memset(&tm_z, 0, sizeof tm_z);
@@ -135,19 +145,31 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     const int Ctot = 2 * c->n_k_heads * c->d_k + c->n_v_heads * c->d_v;
     const int cblocks = (Ctot / 8 + gdn::kConvThreads - 1) / gdn::kConvThreads;
     const int64_t tblocks = (T + gdn::conv_tokens<TA>() - 1) / gdn::conv_tokens<TA>();
-    if (tblocks > 0x7fffffff) return cudaErrorInvalidValue;
+    const int64_t max_chunks = (T + gdn::intra::C - 1) / gdn::intra::C + n_seqs;
+    if (tblocks > 0x7fffffff || max_chunks * Hv > 0x7fffffff) return cudaErrorInvalidValue;
+    int32_t* chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off);
+    uint8_t* recs = wsb + L.rec_off;
+
     gdn::conv_silu_norm_kernel<TA><<<dim3((unsigned)tblocks, cblocks), gdn::kConvThreads, 0, st>>>(ca);
     gdn::conv_state_update_kernel<TA><<<dim3(n_seqs, (Ctot + 255) / 256), 256, 0, st>>>(ca, conv_state);
+    gdn::intra::chunk_offsets_kernel<<<1, 1024, 0, st>>>(cu, n_seqs, chunk_off);
 
-    gdn::chunk::Args pa;
-    pa.a = a; pa.b = b; pa.z = z;
-    pa.A_log = w->A_log; pa.dt_bias = w->dt_bias; pa.norm_w = w->norm_weight;
-    pa.rec_state = rec_state;
-    pa.cu = cu;
-    pa.out = out;
-    pa.Hk = c->n_k_heads; pa.Hv = c->n_v_heads; pa.dk = c->d_k; pa.dv = c->d_v;
-    pa.norm_eps = c->norm_eps;
-    kern<<<(unsigned)n_seqs * c->n_v_heads, gdn::chunk::NT, gdn::chunk::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v, tm_z, pa);
+    gdn::intra::Args ia;
+    ia.a = a; ia.b = b;
+    ia.A_log = w->A_log; ia.dt_bias = w->dt_bias;
+    ia.cu = cu; ia.chunk_off = chunk_off; ia.n_seqs = n_seqs;
+    ia.Hk = Hk; ia.Hv = Hv;
+    ia.rec = recs;
+    k_intra<<<(unsigned)(max_chunks * Hv), gdn::intra::NT, gdn::intra::SMEM_BYTES, st>>>(tm_q, tm_k, ia);
+
+    gdn::scan::Args sa;
+    sa.z = z; sa.norm_w = w->norm_weight;
+    sa.rec_state = rec_state;
+    sa.cu = cu; sa.chunk_off = chunk_off; sa.rec = recs;
+    sa.out = out;
+    sa.Hk = Hk; sa.Hv = Hv; sa.dk = c->d_k; sa.dv = c->d_v;
+    sa.norm_eps = c->norm_eps;
+    k_scan<<<(unsigned)n_seqs * Hv, gdn::scan::NT, gdn::scan::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v, tm_z, sa);
     return cudaGetLastError();
 }
 
@@ -193,7 +215,7 @@ void gdn_config_default(gdn_config* cfg) {
 
 size_t gdn_prefill_workspace_size(const gdn_config* cfg, int64_t T_total, int32_t n_seqs) {
     if (check_config(cfg) != GDN_OK || T_total < 0 || n_seqs < 0) return 0;
-    return workspace_layout(cfg, T_total).total;
+    return workspace_layout(cfg, T_total, n_seqs).total;
 }
 
 gdn_status gdn_prefill(const gdn_config* cfg, const gdn_weights* w, const void* q, const void* k,
@@ -213,7 +235,7 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_weights* w, const void* 
     if (!aligned(workspace, 256)) return GDN_ERR_INVALID_ARG;
     if ((int64_t)n_seqs * cfg->n_v_heads > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
     if (T_total > 0x7fffffffLL - 64) return GDN_ERR_UNSUPPORTED;   // token coordinates are int32
-    if (workspace_bytes < workspace_layout(cfg, T_total).total) return GDN_ERR_WORKSPACE;
+    if (workspace_bytes < workspace_layout(cfg, T_total, n_seqs).total) return GDN_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     const bool abf = cfg->act_dtype == GDN_BF16, obf = cfg->out_dtype == GDN_BF16;
@@ -310,7 +332,7 @@ extern "C" gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const gdn_weigh
     gdn_status s = check_config(cfg);
     if (s != GDN_OK) return s;
     if (n_seqs < 0 || T_total < 0) return GDN_ERR_INVALID_ARG;
-    if (workspace_layout(cfg, T_total).total > GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;
+    if (workspace_layout(cfg, T_total, n_seqs).total > GDN_NOALLOC_SCRATCH_BYTES) return GDN_ERR_WORKSPACE;
     void* scratch = nullptr;
     if (T_total > 0 && n_seqs > 0) {
         int dev = 0;

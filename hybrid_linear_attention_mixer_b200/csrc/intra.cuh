@@ -1,0 +1,339 @@
+// Intra-chunk part of the chunked gated delta rule: everything inside a chunk
+// that does not depend on the recurrent state, for every (chunk, value head)
+// pair in parallel.
+//
+// For a chunk of C = 64 tokens of one sequence and one value head h (key head
+// j = h / G), with g_r = sum_{i<=r} log alpha_i (the in-chunk gate prefix sum):
+//     A_rj = beta_r e^{g_r - g_j} k_r.k_j   (j < r),   T = (I + A)^-1 diag(beta)
+//     P_rj = q_r.k_j e^{g_r - g_j}          (j <= r)
+//     W    = T diag(e^g) K
+// These are the state-independent factors of the chunk's update (see scan.cuh
+// for the state chain that consumes them).  [Q;K] K^T and K^T (T diag(e^g))^T
+// run as tcgen05 MMAs (fp16 operands, fp32 accumulators in TMEM); the
+// triangular solve runs in fp32 on the CUDA cores.
+//
+// Each (chunk, value head) record written to the workspace holds the operand
+// tiles exactly as the scan kernel's tensor cores read them (128-byte swizzled
+// shared-memory images), so the scan brings a whole record in with one bulk copy:
+//     +0      -W   MN-major [d_k rows][64 chunk columns] fp16   16384 B
+//     +16384  T    K-major  [64 rows c][64 columns j]    fp16    8192 B
+//     +24576  P    K-major  [64 rows r][64 columns j]    fp16    8192 B
+//     +32768  g    [64] fp32 (rows past the sequence end repeat the last g)
+#pragma once
+#include "device.cuh"
+
+namespace gdn {
+namespace intra {
+
+constexpr int C = 64;
+constexpr int NT = 256;
+constexpr uint32_t REC_W = 0, REC_T = 16384, REC_P = 24576, REC_G = 32768;
+constexpr uint32_t REC_BYTES = 33792;   // 33 x 1024: keeps every tile of a record 1024-aligned
+
+constexpr uint32_t OFF_QK = 0;          // [Q;K]: 128 token rows x d_k, halves of 16384
+constexpr uint32_t OFF_TP = 32768;      // T' = T diag(e^g)
+constexpr int LDA = 65;
+constexpr uint32_t OFF_A = 40960;
+constexpr uint32_t OFF_X = OFF_A + 64 * LDA * 4;
+constexpr uint32_t OFF_Z = OFF_X + 64 * LDA * 4;
+constexpr uint32_t OFF_G = OFF_Z + 64 * LDA * 4;   // g[64]
+constexpr uint32_t OFF_B = OFF_G + 256;            // beta[64]
+constexpr uint32_t OFF_BAR = OFF_B + 256;          // mbarriers, TMEM address, abort flag
+constexpr uint32_t SMEM_USED = OFF_BAR + 64;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
+static_assert(2 * SMEM_BYTES <= 232448, "two CTAs per SM");
+constexpr uint32_t ACC_QK = 0, ACC_W = 64, TMEM_COLS = 128;
+
+struct Args {
+    const void* a;            // [T][Hv] act dtype
+    const void* b;            // [T][Hv]
+    const float* A_log;       // [Hv]
+    const float* dt_bias;     // [Hv]
+    const int32_t* cu;        // [N+1]
+    const int32_t* chunk_off; // [N+1] first chunk of each sequence; chunk_off[N] = total
+    int n_seqs;
+    int Hk, Hv;
+    uint8_t* rec;             // [total chunks][Hv][REC_BYTES]
+};
+
+__device__ __forceinline__ void stg128(void* p, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    *reinterpret_cast<uint4*>(p) = make_uint4(x, y, z, w);
+}
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w)
+                 : "memory");
+}
+
+// chunk_off[s] = sum_{i<s} ceil(len_i / C) (one CTA, any number of sequences)
+__global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int32_t* cu, int n_seqs, int32_t* chunk_off) {
+    __shared__ int32_t s_sum[32];
+    __shared__ int32_t s_carry;
+    if (threadIdx.x == 0) s_carry = 0;
+    __syncthreads();
+    for (int base = 0; base < n_seqs; base += 1024) {
+        const int s = base + threadIdx.x;
+        int32_t v = 0;
+        if (s < n_seqs) v = (cu[s + 1] - cu[s] + C - 1) / C;
+        int32_t x = v;   // inclusive scan within the warp
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int32_t y = __shfl_up_sync(0xffffffffu, x, off);
+            if ((threadIdx.x & 31) >= off) x += y;
+        }
+        if ((threadIdx.x & 31) == 31) s_sum[threadIdx.x >> 5] = x;
+        __syncthreads();
+        if (threadIdx.x < 32) {
+            int32_t w = s_sum[threadIdx.x];
+#pragma unroll
+            for (int off = 1; off < 32; off <<= 1) {
+                const int32_t y = __shfl_up_sync(0xffffffffu, w, off);
+                if (threadIdx.x >= off) w += y;
+            }
+            s_sum[threadIdx.x] = w;   // inclusive warp totals
+        }
+        __syncthreads();
+        const int32_t warp_base = (threadIdx.x >> 5) ? s_sum[(threadIdx.x >> 5) - 1] : 0;
+        if (s < n_seqs) chunk_off[s] = s_carry + warp_base + x - v;
+        __syncthreads();
+        if (threadIdx.x == 1023) s_carry += warp_base + x;
+        __syncthreads();
+    }
+    if (threadIdx.x == 0) chunk_off[n_seqs] = s_carry;
+}
+
+template <typename TA>
+__global__ void __launch_bounds__(NT, 2)
+gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, Args p) {
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sb = (raw + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (sb - raw);
+    float* s_g = reinterpret_cast<float*>(smem + OFF_G);
+    float* s_b = reinterpret_cast<float*>(smem + OFF_B);
+    float* Am = reinterpret_cast<float*>(smem + OFF_A);
+    float* Xm = reinterpret_cast<float*>(smem + OFF_X);
+    float* Zm = reinterpret_cast<float*>(smem + OFF_Z);
+    const uint32_t bar = sb + OFF_BAR, bar_ld = sb + OFF_BAR + 8;
+    volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 16);
+    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 20);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int qd = warp & 3, half = warp >> 2;
+    const int Hv = p.Hv;
+    const int h = blockIdx.x % Hv;
+    const int gc = blockIdx.x / Hv;
+    if (gc >= p.chunk_off[p.n_seqs]) return;
+    int lo = 0, hi = p.n_seqs - 1;   // sequence of this chunk: last s with chunk_off[s] <= gc
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.chunk_off[mid] <= gc) lo = mid; else hi = mid - 1;
+    }
+    const int seq = lo;
+    const int64_t t0 = (int64_t)p.cu[seq] + (int64_t)(gc - p.chunk_off[seq]) * C;
+    const int64_t rem = (int64_t)p.cu[seq + 1] - t0;
+    const int n = (int)(rem < C ? rem : C);
+    const int j = h / (Hv / p.Hk);
+    uint8_t* rec = p.rec + ((int64_t)gc * Hv + h) * REC_BYTES;
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init(bar_ld, 1);
+        fence_mbar_init();
+        *s_abort = 0;
+        mbar_arrive_expect_tx(bar_ld, 4 * 8192);
+#pragma unroll
+        for (int hf = 0; hf < 2; hf++) {
+            tma_load_3d(sb + OFF_QK + hf * 16384, &tm_q, 64 * hf, j, (int)t0, bar_ld);
+            tma_load_3d(sb + OFF_QK + hf * 16384 + C * 128, &tm_k, 64 * hf, j, (int)t0, bar_ld);
+        }
+    }
+    if (warp == 0) {
+        tmem_alloc(sb + OFF_BAR + 16, TMEM_COLS);
+        tmem_relinquish();
+    }
+    // gates: log alpha, beta and the in-chunk prefix sum g
+    if (tid < C) {
+        float la = 0.f, bt = 0.f;
+        if (tid < n) {
+            const float av = to_f32(static_cast<const TA*>(p.a)[(t0 + tid) * Hv + h]);
+            const float bv = to_f32(static_cast<const TA*>(p.b)[(t0 + tid) * Hv + h]);
+            la = -__expf(p.A_log[h]) * softplus_f(av + p.dt_bias[h]);
+            bt = sigmoid_f(bv);
+        }
+        float g = la;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const float o = __shfl_up_sync(0xffffffffu, g, off);
+            if (lane >= off) g += o;
+        }
+        s_g[tid] = g;
+        s_b[tid] = bt;
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid >= 32 && tid < C) s_g[tid] += s_g[31];
+    const uint32_t tmem = *s_tmem;
+    const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
+    if (!mbar_wait_bounded(bar_ld, 0)) atomicOr((unsigned*)s_abort, 2u);
+    __syncthreads();
+    if (tid < C) reinterpret_cast<float*>(rec + REC_G)[tid] = s_g[tid];
+    bool ok = *s_abort == 0;
+
+    // ---- [Q;K] K^T ----
+    if (ok && tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 8; ks++) {
+            const uint32_t o = (ks >> 2) * 16384 + (ks & 3) * 32;
+            mma_f16(tmem + ACC_QK, sdesc(sb + OFF_QK + o, 16, 1024), sdesc(sb + OFF_QK + o + C * 128, 16, 1024),
+                    idesc_f16(128, 64, 0, 0), ks > 0);
+        }
+        mma_commit(bar);
+    }
+    if (ok && !mbar_wait_bounded(bar, 0)) atomicOr((unsigned*)s_abort, 1u);
+    __syncthreads();
+    ok = *s_abort == 0;
+    if (ok) {
+        tc_fence_after();
+        uint32_t r32[32];
+        tmem_ld32(tl + ACC_QK + 32 * half, r32);
+        const int j0 = 32 * half;
+        if (qd < 2) {   // P rows -> the record
+            const int r = 32 * qd + lane;
+            const float gr = s_g[r];
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const int jj = j0 + 2 * i;
+                const float e0 = __expf(fminf(gr - s_g[jj], 0.f));
+                const float e1 = __expf(fminf(gr - s_g[jj + 1], 0.f));
+                pk[i] = pack_half2(jj <= r ? __uint_as_float(r32[2 * i]) * e0 : 0.f,
+                                   jj + 1 <= r ? __uint_as_float(r32[2 * i + 1]) * e1 : 0.f);
+            }
+#pragma unroll
+            for (int c4 = 0; c4 < 4; c4++)
+                stg128(rec + REC_P + swz128(r, j0 / 8 + c4), pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
+        } else {        // A rows -> shared memory
+            const int r = 32 * (qd - 2) + lane;
+            const float gr = s_g[r], br = s_b[r];
+#pragma unroll
+            for (int i = 0; i < 32; i++) {
+                const int jj = j0 + i;
+                const float e = __expf(fminf(gr - s_g[jj], 0.f));
+                Am[r * LDA + jj] = jj < r ? br * __uint_as_float(r32[i]) * e : 0.f;
+            }
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- X = (I + A)^-1, unit lower triangular, fp32 ----
+    if (ok && tid < 64) {   // diagonal 16 x 16 blocks: one column per thread
+        const int base = 16 * (tid >> 4), c = tid & 15;
+        float x[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            float acc = (i == c) ? 1.f : 0.f;
+#pragma unroll
+            for (int m = 0; m < i; m++) acc = fmaf(-Am[(base + i) * LDA + base + m], x[m], acc);
+            x[i] = acc;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; i++) Xm[(base + i) * LDA + base + c] = x[i];
+    }
+    __syncthreads();
+    if (ok) {   // Z_{bi,m} = X_{bi,bi} A_{bi,m} for the six blocks below the diagonal
+        const int i = tid >> 4, jj = tid & 15;
+#pragma unroll
+        for (int blk = 0; blk < 6; blk++) {
+            const int bi = blk < 1 ? 1 : blk < 3 ? 2 : 3;
+            const int m = blk < 1 ? 0 : blk < 3 ? blk - 1 : blk - 3;
+            float acc = 0.f;
+#pragma unroll
+            for (int l = 0; l < 16; l++)
+                acc = fmaf(Xm[(16 * bi + i) * LDA + 16 * bi + l], Am[(16 * bi + l) * LDA + 16 * m + jj], acc);
+            Zm[(16 * bi + i) * LDA + 16 * m + jj] = acc;
+        }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int dd = 1; dd < 4; dd++) {   // X_{bi,bj} = -sum_{m=bj}^{bi-1} Z_{bi,m} X_{m,bj}
+        if (ok) {
+            const int i = tid >> 4, jj = tid & 15;
+            for (int bj = 0; bj + dd < 4; bj++) {
+                const int bi = bj + dd;
+                float acc = 0.f;
+                for (int m = bj; m < bi; m++) {
+#pragma unroll
+                    for (int l = 0; l < 16; l++)
+                        acc = fmaf(Zm[(16 * bi + i) * LDA + 16 * m + l], Xm[(16 * m + l) * LDA + 16 * bj + jj], acc);
+                }
+                Xm[(16 * bi + i) * LDA + 16 * bj + jj] = -acc;
+            }
+        }
+        __syncthreads();
+    }
+    if (ok) {   // T = X diag(beta) -> the record; T' = T diag(e^g) -> shared memory
+        const int c = tid >> 2, jq = (tid & 3) * 16;
+        uint32_t tp[8], tq[8];
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            const int jj = jq + 2 * i;
+            const float x0 = jj <= c ? Xm[c * LDA + jj] * s_b[jj] : 0.f;
+            const float x1 = jj + 1 <= c ? Xm[c * LDA + jj + 1] * s_b[jj + 1] : 0.f;
+            tp[i] = pack_half2(x0, x1);
+            tq[i] = pack_half2(x0 * __expf(s_g[jj]), x1 * __expf(s_g[jj + 1]));
+        }
+#pragma unroll
+        for (int c2 = 0; c2 < 2; c2++) {
+            stg128(rec + REC_T + swz128(c, jq / 8 + c2), tp[4 * c2], tp[4 * c2 + 1], tp[4 * c2 + 2], tp[4 * c2 + 3]);
+            sts128(sb + OFF_TP + swz128(c, jq / 8 + c2), tq[4 * c2], tq[4 * c2 + 1], tq[4 * c2 + 2], tq[4 * c2 + 3]);
+        }
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+
+    // ---- W^T = K^T T'^T (M = d_k, N = 64 chunk columns, K = 64 tokens) ----
+    if (ok && tid == 0) {
+        tc_fence_after();
+#pragma unroll
+        for (int ks = 0; ks < 4; ks++)
+            mma_f16(tmem + ACC_W, sdesc(sb + OFF_QK + C * 128 + ks * 2048, 16384, 1024),
+                    sdesc(sb + OFF_TP + ks * 32, 16, 1024), idesc_f16(128, 64, 1, 0), ks > 0);
+        mma_commit(bar);
+    }
+    if (ok && !mbar_wait_bounded(bar, 1)) atomicOr((unsigned*)s_abort, 1u);
+    __syncthreads();
+    ok = *s_abort == 0;
+    if (ok) {   // -W^T -> the record (row d_k, chunk columns)
+        tc_fence_after();
+        uint32_t r32[32];
+        tmem_ld32(tl + ACC_W + 32 * half, r32);
+        const int row = 32 * qd + lane;
+#pragma unroll
+        for (int c4 = 0; c4 < 4; c4++) {
+            uint32_t w4[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++)
+                w4[i] = pack_half2(-__uint_as_float(r32[8 * c4 + 2 * i]), -__uint_as_float(r32[8 * c4 + 2 * i + 1]));
+            stg128(rec + REC_W + swz128(row, 4 * half + c4), w4[0], w4[1], w4[2], w4[3]);
+        }
+    } else if (tid == 0) {
+        record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));
+        // one more bounded wait for whatever may still be in flight
+        mbar_wait_bounded(bar_ld, 0);
+        mbar_wait_bounded(bar, 0);
+        mbar_wait_bounded(bar, 1);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+}
+
+}  // namespace intra
+}  // namespace gdn

@@ -1,0 +1,421 @@
+// State chain of the chunked gated delta rule on the sm_100a tensor cores.
+//
+// One CTA (512 threads) walks one (sequence, value head) chain chunk by chunk
+// (C = 64 tokens) and carries the d_v x d_k fp32 state in registers (row = TMEM
+// lane, a quarter of d_k per warp).  The state-independent factors of every
+// chunk come from the intra-chunk kernel's records (intra.cuh: -W, T, P, g).
+// With S0 the state at the chunk start:
+//     U   = T V - W S0^T                                    (exact per-token updates)
+//     O   = (diag(e^g) Q S0^T + P U) / sqrt(d_k)
+//     S_C = e^{g_C} S0 + U^T diag(e^{g_C - g}) K
+// followed by the layer's gated RMSNorm o * rsqrt(mean(o^2) + eps) * w * SiLU(z).
+//
+// Products (tcgen05.mma kind::f16, fp16 operands, fp32 accumulators in TMEM,
+// M = 128 = d_v always, the chunk is the N side):
+//   (c) V^T T^T           -> U^T accumulator            [A: V, MN-major]
+//   (d) S (-W)^T          accumulated into (c)           [B: -W, MN-major]
+//   (e) S Q^T             -> O1^T                        [double-buffered]
+//   (f) U^T P^T           -> O2^T                        [double-buffered]
+//   (g) U^T K~            -> state increment, K~ = diag(e^{g_C - g}) K [B: MN-major]
+// The chain per chunk is (c,d,e) -> U^T to fp16 -> (f,g) -> state update -> S to
+// fp16.  The gated-RMSNorm epilogue of chunk c-1 runs while (c,d,e) of chunk c
+// are on the tensor cores.  q^, k^, v^ and z tiles arrive by TMA and a chunk's
+// record by one bulk copy, all issued a chunk or more ahead.
+#pragma once
+#include "device.cuh"
+#include "intra.cuh"
+
+namespace gdn {
+namespace scan {
+
+constexpr int C = 64;
+constexpr int NT = 512;   // 16 warps: 4 per TMEM lane quadrant
+constexpr uint32_t REC_COPY = intra::REC_G + 256;   // bytes of a record brought in
+
+constexpr uint32_t OFF_REC = 0;               // two record buffers of REC_BYTES
+constexpr uint32_t OFF_QK = 2 * intra::REC_BYTES;   // [Q;K] 128 rows x d_k, halves of 16384
+constexpr uint32_t OFF_V = OFF_QK + 32768;    // V: 64 rows x d_v, halves of 8192
+constexpr uint32_t OFF_ZT = OFF_V + 16384;    // z (bf16), gated output staged in place
+constexpr uint32_t OFF_S16 = OFF_ZT + 16384;  // S (fp16): 128 d_v rows x d_k, halves of 16384
+constexpr uint32_t OFF_UT = OFF_S16 + 32768;  // U^T: 128 d_v rows x 64 chunk columns
+constexpr uint32_t OFF_KT = OFF_UT + 16384;   // K~: 64 rows x d_k, halves of 8192
+constexpr uint32_t OFF_G = OFF_KT + 16384;    // g [2][64]
+constexpr uint32_t OFF_EG = OFF_G + 512;      // e^g [2][64]
+constexpr uint32_t OFF_KS = OFF_EG + 512;     // e^{g_C - g} [64]
+constexpr uint32_t OFF_RED = OFF_KS + 256;    // [4][64] partial sums of o^2
+constexpr uint32_t OFF_RS = OFF_RED + 1024;   // rsqrt(mean o^2 + eps) [64]
+constexpr uint32_t OFF_BAR = OFF_RS + 256;    // mbarriers, TMEM address, abort flag
+constexpr uint32_t SMEM_USED = OFF_BAR + 64;
+constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
+static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+
+constexpr uint32_t ACC_U = 0, ACC_O1 = 64, ACC_O2 = 192, ACC_SI = 320, TMEM_COLS = 512;
+constexpr uint32_t QKV_BYTES = 6 * 8192, Z_BYTES = 2 * 8192;
+
+struct Args {
+    const void* z;              // [T][Hv][dv] act dtype
+    const float* norm_w;        // [dv]
+    float* rec_state;           // [N][Hv][dv][dk] in/out
+    const int32_t* cu;          // [N+1]
+    const int32_t* chunk_off;   // [N+1]
+    const uint8_t* rec;         // intra-chunk records
+    void* out;                  // [T][Hv][dv] out dtype
+    int Hk, Hv, dk, dv;
+    float norm_eps;
+};
+
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w)
+                 : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+__device__ __forceinline__ uint4 scale8(uint4 v, float s) {
+    const float2 a = unpack_half2(v.x), b = unpack_half2(v.y), c = unpack_half2(v.z), d = unpack_half2(v.w);
+    return make_uint4(pack_half2(a.x * s, a.y * s), pack_half2(b.x * s, b.y * s),
+                      pack_half2(c.x * s, c.y * s), pack_half2(d.x * s, d.y * s));
+}
+
+template <typename TA, typename TO>
+__global__ void __launch_bounds__(NT, 1)
+gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_z, Args p) {
+    constexpr bool kZTile = sizeof(TA) == 2;                  // z through TMA (bf16 activations)
+    constexpr bool kOutStage = kZTile && sizeof(TO) == 2;     // out staged in the z tile
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    const uint32_t sb = (raw + 1023u) & ~1023u;
+    uint8_t* smem = smem_raw + (sb - raw);
+    float* s_g = reinterpret_cast<float*>(smem + OFF_G);
+    float* s_eg = reinterpret_cast<float*>(smem + OFF_EG);
+    float* s_ks = reinterpret_cast<float*>(smem + OFF_KS);
+    float* s_red = reinterpret_cast<float*>(smem + OFF_RED);
+    float* s_rs = reinterpret_cast<float*>(smem + OFF_RS);
+    const uint32_t bar = sb + OFF_BAR, bar_qkv = sb + OFF_BAR + 8, bar_z = sb + OFF_BAR + 16;
+    const uint32_t bar_rec0 = sb + OFF_BAR + 24;   // + 8 * buffer
+    volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 40);
+    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 44);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int qd = warp & 3;      // TMEM lane quadrant
+    const int cs = warp >> 2;     // column slice 0..3
+    const int Hv = p.Hv, dk = p.dk, dv = p.dv;
+    const int seq = blockIdx.x / Hv, h = blockIdx.x % Hv;
+    const int j = h / (Hv / p.Hk);
+    const int64_t s0 = p.cu[seq], s1 = p.cu[seq + 1];
+    const int nchunks = (int)((s1 - s0 + C - 1) / C);
+    if (nchunks <= 0) return;
+    const uint8_t* rec0 = p.rec + ((int64_t)p.chunk_off[seq] * Hv + h) * intra::REC_BYTES;
+    const int64_t rec_stride = (int64_t)Hv * intra::REC_BYTES;
+    const TA* __restrict__ pz = static_cast<const TA*>(p.z);
+    TO* __restrict__ pout = static_cast<TO*>(p.out);
+    const int64_t ldv = (int64_t)Hv * dv;
+
+    int qkv_issued = 0, qkv_ok = 0, z_issued = 0, z_ok = 0;
+    int rec_issued[2] = {0, 0}, rec_ok[2] = {0, 0};
+    auto issue_qkv = [&](int ci) {
+        const int t = (int)(s0 + (int64_t)ci * C);
+        qkv_issued++;
+        mbar_arrive_expect_tx(bar_qkv, QKV_BYTES);
+#pragma unroll
+        for (int hf = 0; hf < 2; hf++) {
+            tma_load_3d(sb + OFF_QK + hf * 16384, &tm_q, 64 * hf, j, t, bar_qkv);
+            tma_load_3d(sb + OFF_QK + hf * 16384 + C * 128, &tm_k, 64 * hf, j, t, bar_qkv);
+            tma_load_3d(sb + OFF_V + hf * 8192, &tm_v, 64 * hf, h, t, bar_qkv);
+        }
+    };
+    auto issue_rec = [&](int ci) {
+        const int b = ci & 1;
+        rec_issued[b]++;
+        mbar_arrive_expect_tx(bar_rec0 + 8 * b, REC_COPY);
+        bulk_g2s(sb + OFF_REC + b * intra::REC_BYTES, rec0 + ci * rec_stride, REC_COPY, bar_rec0 + 8 * b);
+    };
+    auto issue_z = [&](int ci) {
+        z_issued++;
+        mbar_arrive_expect_tx(bar_z, Z_BYTES);
+#pragma unroll
+        for (int hf = 0; hf < 2; hf++)
+            tma_load_3d(sb + OFF_ZT + hf * 8192, &tm_z, 64 * hf, h, (int)(s0 + (int64_t)ci * C), bar_z);
+    };
+
+    if (tid == 0) {
+        mbar_init(bar, 1);
+        mbar_init(bar_qkv, 1);
+        mbar_init(bar_z, 1);
+        mbar_init(bar_rec0, 1);
+        mbar_init(bar_rec0 + 8, 1);
+        fence_mbar_init();
+        *s_abort = 0;
+        issue_qkv(0);
+        issue_rec(0);
+        if (nchunks > 1) issue_rec(1);
+        if (kZTile) issue_z(0);
+    }
+    if (warp == 0) {
+        tmem_alloc(sb + OFF_BAR + 40, TMEM_COLS);
+        tmem_relinquish();
+    }
+
+    // fp32 state: row dv_r, columns [32 cs, 32 cs + 32)
+    const int dv_r = 32 * qd + lane;
+    float S[32];
+    float* gstate = p.rec_state + ((int64_t)seq * Hv + h) * dv * dk;
+#pragma unroll
+    for (int i = 0; i < 32; i++) {
+        const int col = 32 * cs + i;
+        S[i] = (dv_r < dv && col < dk) ? gstate[(int64_t)dv_r * dk + col] : 0.f;
+    }
+    auto write_s16 = [&]() {
+#pragma unroll
+        for (int c4 = 0; c4 < 4; c4++)
+            sts128(sb + OFF_S16 + (cs >> 1) * 16384 + swz128(dv_r, (cs & 1) * 4 + c4),
+                   pack_half2(S[8 * c4 + 0], S[8 * c4 + 1]), pack_half2(S[8 * c4 + 2], S[8 * c4 + 3]),
+                   pack_half2(S[8 * c4 + 4], S[8 * c4 + 5]), pack_half2(S[8 * c4 + 6], S[8 * c4 + 7]));
+    };
+    write_s16();
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *s_tmem;
+    const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
+    const float inv_sqrt_dk = rsqrtf((float)dk);
+    const float wn = dv_r < dv ? p.norm_w[dv_r] : 0.f;
+    uint32_t mphase = 0;
+
+    // Gated RMSNorm epilogue of chunk ce (O accumulators of buffer ce & 1).
+    auto epilogue = [&](int ce) -> bool {
+        const int be = ce & 1;
+        const int64_t te = s0 + (int64_t)ce * C;
+        const int ne = (int)((s1 - te) < (int64_t)C ? (s1 - te) : (int64_t)C);
+        float o[16], v[16];
+        {
+            uint32_t o1[16], o2[16];
+            tmem_ld16(tl + ACC_O1 + 64 * be + 16 * cs, o1);
+            tmem_ld16(tl + ACC_O2 + 64 * be + 16 * cs, o2);
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const int r = 16 * cs + i;
+                o[i] = (s_eg[64 * be + r] * __uint_as_float(o1[i]) + __uint_as_float(o2[i])) * inv_sqrt_dk;
+                v[i] = o[i] * o[i];
+            }
+        }
+        // transpose-reduce: lanes L and L^16 end with the warp's sum for column 16 cs + (L & 15)
+#pragma unroll
+        for (int off = 8; off >= 1; off >>= 1) {
+            const bool upper = (lane & off) != 0;
+#pragma unroll
+            for (int i = 0; i < off; i++) {
+                const float send = upper ? v[i] : v[i + off];
+                const float keep = upper ? v[i + off] : v[i];
+                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
+            }
+        }
+        v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
+        if (lane < 16) s_red[qd * 64 + 16 * cs + lane] = v[0];
+        tc_fence_before();
+        __syncthreads();
+        if (tid < C) s_rs[tid] = rsqrtf((s_red[tid] + s_red[64 + tid] + s_red[128 + tid] + s_red[192 + tid]) /
+                                        (float)dv + p.norm_eps);
+        __syncthreads();
+        if constexpr (kZTile) {
+            if (mbar_wait_bounded(bar_z, ce & 1)) z_ok++; else atomicOr((unsigned*)s_abort, 2u);
+            const uint32_t zcol = (uint32_t)(dv_r >> 6) * 8192 + (uint32_t)(dv_r & 7) * 2;
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const int r = 16 * cs + i;
+                __nv_bfloat16* zp =
+                    reinterpret_cast<__nv_bfloat16*>(smem + OFF_ZT + zcol + swz128(r, (dv_r & 63) >> 3));
+                const float y = o[i] * s_rs[r] * wn * silu_f(__bfloat162float(*zp));
+                if constexpr (kOutStage) {
+                    *zp = __float2bfloat16_rn(y);
+                } else {
+                    if (r < ne && dv_r < dv) from_f32(y, pout + (te + r) * ldv + (int64_t)h * dv + dv_r);
+                }
+            }
+            if constexpr (kOutStage) {
+                __syncthreads();
+                for (int idx = tid; idx < C * 16; idx += NT) {   // 16-byte row pieces
+                    const int r = idx >> 4, c16 = idx & 15;
+                    if (r < ne && c16 * 8 < dv) {
+                        const uint4 v4 = lds128(sb + OFF_ZT + (c16 >> 3) * 8192 + swz128(r, c16 & 7));
+                        __stcs(reinterpret_cast<uint4*>(pout + (te + r) * ldv + (int64_t)h * dv + c16 * 8), v4);
+                    }
+                }
+            }
+            __syncthreads();
+            if (*s_abort) return false;
+            if (tid == 0 && ce + 1 < nchunks) {   // the z tile is free: fetch the next chunk's
+                fence_async_smem();
+                issue_z(ce + 1);
+            }
+        } else if (dv_r < dv) {
+            float zz[16];
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const int r = 16 * cs + i;
+                zz[i] = r < ne ? to_f32(pz[(te + r) * ldv + (int64_t)h * dv + dv_r]) : 0.f;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; i++) {
+                const int r = 16 * cs + i;
+                if (r < ne) from_f32(o[i] * s_rs[r] * wn * silu_f(zz[i]), pout + (te + r) * ldv + (int64_t)h * dv + dv_r);
+            }
+        }
+        return true;
+    };
+
+#define GDN_MMA_WAIT()                                                         \
+    do {                                                                       \
+        if (!mbar_wait_bounded(bar, mphase)) atomicOr((unsigned*)s_abort, 1u); \
+        mphase ^= 1u;                                                          \
+        __syncthreads();                                                       \
+        if (*s_abort) goto abort_;                                             \
+        tc_fence_after();                                                      \
+    } while (0)
+
+    for (int ci = 0; ci < nchunks; ci++) {
+        const int b = ci & 1;
+        const uint32_t rb = sb + OFF_REC + b * intra::REC_BYTES;
+        const int64_t t0 = s0 + (int64_t)ci * C;
+        const int n = (int)((s1 - t0) < (int64_t)C ? (s1 - t0) : (int64_t)C);
+
+        // ---- this chunk's tiles and record ----
+        if (mbar_wait_bounded(bar_qkv, ci & 1)) qkv_ok++; else atomicOr((unsigned*)s_abort, 2u);
+        if (mbar_wait_bounded(bar_rec0 + 8 * b, (ci >> 1) & 1)) rec_ok[b]++; else atomicOr((unsigned*)s_abort, 2u);
+        if (tid < C) {
+            const float* rg = reinterpret_cast<const float*>(smem + OFF_REC + b * intra::REC_BYTES + intra::REC_G);
+            const float g = rg[tid], gl = rg[C - 1];
+            s_g[64 * b + tid] = g;
+            s_eg[64 * b + tid] = __expf(g);
+            s_ks[tid] = tid < n ? __expf(gl - g) : 0.f;
+        }
+        __syncthreads();
+        if (*s_abort) goto abort_;
+
+        // ---- (c) U^T = V^T T^T, (d) U^T += S (-W)^T, (e) O1^T = S Q^T ----
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ks++)
+                mma_f16(tmem + ACC_U, sdesc(sb + OFF_V + ks * 2048, 8192, 1024),
+                        sdesc(rb + intra::REC_T + ks * 32, 16, 1024), idesc_f16(128, 64, 1, 0), ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ks++)
+                mma_f16(tmem + ACC_U, sdesc(sb + OFF_S16 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
+                        sdesc(rb + intra::REC_W + ks * 2048, 8192, 1024), idesc_f16(128, 64, 0, 1), 1);
+#pragma unroll
+            for (int ks = 0; ks < 8; ks++) {
+                const uint32_t o = (ks >> 2) * 16384 + (ks & 3) * 32;
+                mma_f16(tmem + ACC_O1 + 64 * b, sdesc(sb + OFF_S16 + o, 16, 1024), sdesc(sb + OFF_QK + o, 16, 1024),
+                        idesc_f16(128, 64, 0, 0), ks > 0);
+            }
+            mma_commit(bar);
+        }
+        // ---- K~ = diag(e^{g_C - g}) K (rows past the chunk's end are zero) ----
+        for (int idx = tid; idx < C * 16; idx += NT) {
+            const int r = idx >> 4, c16 = idx & 15;
+            const int hf = c16 >> 3, cc = c16 & 7;
+            const uint4 kt = scale8(lds128(sb + OFF_QK + hf * 16384 + swz128(C + r, cc)), s_ks[r]);
+            sts128(sb + OFF_KT + hf * 8192 + swz128(r, cc), kt.x, kt.y, kt.z, kt.w);
+        }
+        fence_async_smem();
+        // ---- the previous chunk's output, while (c, d, e) run ----
+        if (ci > 0 && !epilogue(ci - 1)) goto abort_;
+        GDN_MMA_WAIT();
+        if (tid == 0 && ci + 1 < nchunks) {   // q, k, v tiles consumed: fetch the next chunk's
+            fence_async_smem();
+            issue_qkv(ci + 1);
+        }
+
+        // ---- U^T -> fp16 ----
+        {
+            uint32_t r16[16];
+            tmem_ld16(tl + ACC_U + 16 * cs, r16);
+            uint32_t u[8];
+#pragma unroll
+            for (int i = 0; i < 8; i++) u[i] = pack_half2(__uint_as_float(r16[2 * i]), __uint_as_float(r16[2 * i + 1]));
+            sts128(sb + OFF_UT + swz128(dv_r, 2 * cs), u[0], u[1], u[2], u[3]);
+            sts128(sb + OFF_UT + swz128(dv_r, 2 * cs + 1), u[4], u[5], u[6], u[7]);
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- (f) O2^T = U^T P^T, (g) increment = U^T K~ ----
+        if (tid == 0) {
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ks++)
+                mma_f16(tmem + ACC_O2 + 64 * b, sdesc(sb + OFF_UT + ks * 32, 16, 1024),
+                        sdesc(rb + intra::REC_P + ks * 32, 16, 1024), idesc_f16(128, 64, 0, 0), ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ks++)
+                mma_f16(tmem + ACC_SI, sdesc(sb + OFF_UT + ks * 32, 16, 1024),
+                        sdesc(sb + OFF_KT + ks * 2048, 8192, 1024), idesc_f16(128, 128, 0, 1), ks > 0);
+            mma_commit(bar);
+        }
+        GDN_MMA_WAIT();
+        if (tid == 0 && ci + 2 < nchunks) {   // record buffer b consumed: fetch chunk ci + 2's
+            fence_async_smem();
+            issue_rec(ci + 2);
+        }
+
+        // ---- S <- e^{g_C} S + U^T K~, and its fp16 copy for the next chunk ----
+        {
+            const float eg = s_eg[64 * b + C - 1];
+            uint32_t r32[32];
+            tmem_ld32(tl + ACC_SI + 32 * cs, r32);
+#pragma unroll
+            for (int i = 0; i < 32; i++) S[i] = fmaf(eg, S[i], __uint_as_float(r32[i]));
+            write_s16();
+        }
+        fence_async_smem();
+        tc_fence_before();
+        __syncthreads();
+        (void)n;
+    }
+    if (!epilogue(nchunks - 1)) goto abort_;
+
+    // ---- final state ----
+#pragma unroll
+    for (int i = 0; i < 32; i++) {
+        const int col = 32 * cs + i;
+        if (dv_r < dv && col < dk) gstate[(int64_t)dv_r * dk + col] = S[i];
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+    return;
+
+abort_:
+    // A tensor-core commit or a copy never arrived: report it, give whatever is
+    // still in flight one more bounded wait, free tensor memory and return.  The
+    // recurrent state is left as it was.
+    if (tid == 0) {
+        record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));
+        for (int k = qkv_ok; k < qkv_issued; k++) mbar_wait_bounded(bar_qkv, k & 1);
+        for (int k = z_ok; k < z_issued; k++) mbar_wait_bounded(bar_z, k & 1);
+        for (int bb = 0; bb < 2; bb++)
+            for (int k = rec_ok[bb]; k < rec_issued[bb]; k++) mbar_wait_bounded(bar_rec0 + 8 * bb, k & 1);
+    }
+    if (warp == 0) {
+        mbar_wait_bounded(bar, mphase ^ 1u);
+        __syncwarp();
+        tc_fence_after();
+        tmem_dealloc(tmem, TMEM_COLS);
+    }
+#undef GDN_MMA_WAIT
+}
+
+}  // namespace scan
+}  // namespace gdn

@@ -150,10 +150,11 @@ gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w,
  *
  *   - Size limit: a request needing more than GDN_NOALLOC_SCRATCH_BYTES of
  *     workspace is rejected with GDN_ERR_WORKSPACE, before any launch.  The
- *     needed size is gdn_prefill_workspace_size(cfg, T_total, n_seqs); at the
- *     published shape that is 20,480 bytes per token, so up to 3,276 tokens.
- *     Longer prompts can be split into consecutive calls, since the states
- *     carry from one call to the next.
+ *     needed size is gdn_prefill_workspace_size(cfg, T_total, n_seqs).  At the
+ *     published shape that is 45,824 bytes per token plus about 1.6 MB per
+ *     sequence, so up to 1,408 tokens in one sequence.  Longer prompts can be
+ *     split into consecutive calls, since the states carry from one call to
+ *     the next.
  *   - First call on a device: it looks up the array's device address with
  *     cudaGetSymbolAddress (with that device current), then reuses it.  Make
  *     this first call before any stream capture.

@@ -47,9 +47,13 @@ def test_default_config_is_the_published_shape(lib):
 def test_workspace_size(lib):
     cfg = gdn.Config()
     T = 4096
-    # fp16 q^, k^ [T, 16*128] and v^ [T, 48*128], each rounded up to 256 bytes
-    assert gdn.workspace_size(cfg, T, 1) == 2 * T * 2048 * 2 + T * 6144 * 2
-    assert gdn.workspace_size(cfg, 0, 0) == 0
+    # fp16 q^, k^ [T, 16*128] and v^ [T, 48*128]; chunk offsets [N+1] int32 (256-byte
+    # rounded); one 33 KiB intra-chunk record per (chunk, value head), with at most
+    # ceil(T / 64) + N chunks
+    conv = 2 * T * 2048 * 2 + T * 6144 * 2
+    assert gdn.workspace_size(cfg, T, 1) == conv + 256 + (T // 64 + 1) * 48 * 33792
+    assert gdn.workspace_size(cfg, T, 3) == conv + 256 + (T // 64 + 3) * 48 * 33792
+    assert gdn.workspace_size(cfg, 0, 0) == 256
     assert gdn.workspace_size(gdn.Config(d_k=48), T, 1) == 0
 
 
