@@ -12,6 +12,7 @@
 #include "decode.cuh"
 #include "device.cuh"
 #include "intra.cuh"
+#include "norm.cuh"
 #include "scan.cuh"
 
 namespace {
@@ -44,9 +45,10 @@ gdn_status check_weights(const gdn_weights* w) {
 }
 
 // Prefill workspace: fp16 q^, k^, v^ (conv output), the first chunk of each
-// sequence, and one intra-chunk record per (chunk, value head).
+// sequence, one intra-chunk record per (chunk, value head), and the o tile
+// ([64][128], out dtype) of each (chunk, value head) before the gated norm.
 struct Layout {
-    size_t q_off, k_off, v_off, coff_off, rec_off, total;
+    size_t q_off, k_off, v_off, coff_off, rec_off, o_off, total;
 };
 
 Layout workspace_layout(const gdn_config* c, int64_t T, int64_t n_seqs) {
@@ -55,12 +57,14 @@ Layout workspace_layout(const gdn_config* c, int64_t T, int64_t n_seqs) {
     const size_t vb = align_up((size_t)T * c->n_v_heads * c->d_v * sizeof(__half), 256);
     const size_t cb = align_up((size_t)(n_seqs + 1) * sizeof(int32_t), 256);
     const size_t max_chunks = (size_t)((T + gdn::intra::C - 1) / gdn::intra::C) + (size_t)n_seqs;
+    const size_t o_tile = (size_t)gdn::intra::C * 128 * (c->out_dtype == GDN_F32 ? 4 : 2);
     L.q_off = 0;
     L.k_off = qb;
     L.v_off = 2 * qb;
     L.coff_off = 2 * qb + vb;
     L.rec_off = L.coff_off + cb;
-    L.total = L.rec_off + max_chunks * c->n_v_heads * gdn::intra::REC_BYTES;
+    L.o_off = L.rec_off + max_chunks * c->n_v_heads * gdn::intra::REC_BYTES;
+    L.total = L.o_off + max_chunks * c->n_v_heads * o_tile;
     return L;
 }
 
@@ -128,19 +132,16 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     // Set-up first: nothing is launched unless the tensor maps encode and the
     // kernels' shared-memory opt-ins succeed.
     auto k_intra = gdn::intra::gdn_intra_kernel<TA>;
-    auto k_scan = gdn::scan::gdn_scan_kernel<TA, TO>;
+    auto k_scan = gdn::scan::gdn_scan_kernel<TO>;
     cudaError_t e = ensure_smem(k_intra, 4 + (sizeof(TA) == 2 ? 0 : 1), gdn::intra::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = ensure_smem(k_scan, variant, gdn::scan::SMEM_BYTES);
+    e = ensure_smem(k_scan, 6 + (sizeof(TO) == 2 ? 0 : 1), gdn::scan::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    CUtensorMap tm_q, tm_k, tm_v, tm_z;
-    std::memset(&tm_z, 0, sizeof tm_z);
+    CUtensorMap tm_q, tm_k, tm_v;
     const int Hk = c->n_k_heads, Hv = c->n_v_heads;
     if (!head_tile_map(&tm_q, ca.qh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, Hk, T) ||
         !head_tile_map(&tm_k, ca.kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, Hk, T) ||
         !head_tile_map(&tm_v, ca.vh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_v, Hv, T))
-        return cudaErrorInvalidValue;
-    if (sizeof(TA) == 2 && !head_tile_map(&tm_z, z, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, c->d_v, Hv, T))
         return cudaErrorInvalidValue;
     const int Ctot = 2 * c->n_k_heads * c->d_k + c->n_v_heads * c->d_v;
     const int cblocks = (Ctot / 8 + gdn::kConvThreads - 1) / gdn::kConvThreads;
@@ -149,6 +150,7 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     if (tblocks > 0x7fffffff || max_chunks * Hv > 0x7fffffff) return cudaErrorInvalidValue;
     int32_t* chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off);
     uint8_t* recs = wsb + L.rec_off;
+    void* otiles = wsb + L.o_off;
 
     gdn::conv_silu_norm_kernel<TA><<<dim3((unsigned)tblocks, cblocks), gdn::kConvThreads, 0, st>>>(ca);
     gdn::conv_state_update_kernel<TA><<<dim3(n_seqs, (Ctot + 255) / 256), 256, 0, st>>>(ca, conv_state);
@@ -163,13 +165,17 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     k_intra<<<(unsigned)(max_chunks * Hv), gdn::intra::NT, gdn::intra::SMEM_BYTES, st>>>(tm_q, tm_k, ia);
 
     gdn::scan::Args sa;
-    sa.z = z; sa.norm_w = w->norm_weight;
     sa.rec_state = rec_state;
     sa.cu = cu; sa.chunk_off = chunk_off; sa.rec = recs;
-    sa.out = out;
+    sa.o = otiles;
     sa.Hk = Hk; sa.Hv = Hv; sa.dk = c->d_k; sa.dv = c->d_v;
-    sa.norm_eps = c->norm_eps;
-    k_scan<<<(unsigned)n_seqs * Hv, gdn::scan::NT, gdn::scan::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v, tm_z, sa);
+    k_scan<<<(unsigned)n_seqs * Hv, gdn::scan::NT, gdn::scan::SMEM_BYTES, st>>>(tm_q, tm_k, tm_v, sa);
+
+    gdn::norm::Args na;
+    na.o = otiles; na.z = z; na.norm_w = w->norm_weight;
+    na.cu = cu; na.chunk_off = chunk_off; na.out = out;
+    na.n_seqs = n_seqs; na.Hv = Hv; na.dv = c->d_v; na.eps = c->norm_eps;
+    gdn::norm::gdn_gated_norm_kernel<TA, TO><<<(unsigned)(max_chunks * Hv), gdn::norm::NT, 0, st>>>(na);
     return cudaGetLastError();
 }
 

@@ -8,7 +8,8 @@
 //     U   = T V - W S0^T                                    (exact per-token updates)
 //     O   = (diag(e^g) Q S0^T + P U) / sqrt(d_k)
 //     S_C = e^{g_C} S0 + U^T diag(e^{g_C - g}) K
-// followed by the layer's gated RMSNorm o * rsqrt(mean(o^2) + eps) * w * SiLU(z).
+// o goes out as [chunk][head][64][128] tiles; the gated RMSNorm that follows
+// runs in norm.cuh, in parallel over all tiles.
 //
 // Products (tcgen05.mma kind::f16, fp16 operands, fp32 accumulators in TMEM,
 // M = 128 = d_v always, the chunk is the N side):
@@ -18,9 +19,10 @@
 //   (f) U^T P^T           -> O2^T                        [double-buffered]
 //   (g) U^T K~            -> state increment, K~ = diag(e^{g_C - g}) K [B: MN-major]
 // The chain per chunk is (c,d,e) -> U^T to fp16 -> (f,g) -> state update -> S to
-// fp16.  The gated-RMSNorm epilogue of chunk c-1 runs while (c,d,e) of chunk c
-// are on the tensor cores.  q^, k^, v^ and z tiles arrive by TMA and a chunk's
-// record by one bulk copy, all issued a chunk or more ahead.
+// fp16.  The output tile of chunk c-1 is formed and stored (one bulk copy)
+// while (c,d,e) of chunk c are on the tensor cores.  q^, k^, v^ tiles arrive by
+// TMA and a chunk's record by one bulk copy, issued a chunk or more ahead.  One
+// thread waits on each mbarrier; the others meet it at the CTA barrier.
 #pragma once
 #include "device.cuh"
 #include "intra.cuh"
@@ -35,33 +37,27 @@ constexpr uint32_t REC_COPY = intra::REC_G + 256;   // bytes of a record brought
 constexpr uint32_t OFF_REC = 0;               // two record buffers of REC_BYTES
 constexpr uint32_t OFF_QK = 2 * intra::REC_BYTES;   // [Q;K] 128 rows x d_k, halves of 16384
 constexpr uint32_t OFF_V = OFF_QK + 32768;    // V: 64 rows x d_v, halves of 8192
-constexpr uint32_t OFF_ZT = OFF_V + 16384;    // z (bf16), gated output staged in place
-constexpr uint32_t OFF_S16 = OFF_ZT + 16384;  // S (fp16): 128 d_v rows x d_k, halves of 16384
+constexpr uint32_t OFF_OST = OFF_V + 16384;   // o tile staging: [64][128] out dtype (<= 32 KiB)
+constexpr uint32_t OFF_S16 = OFF_OST + 32768; // S (fp16): 128 d_v rows x d_k, halves of 16384
 constexpr uint32_t OFF_UT = OFF_S16 + 32768;  // U^T: 128 d_v rows x 64 chunk columns
 constexpr uint32_t OFF_KT = OFF_UT + 16384;   // K~: 64 rows x d_k, halves of 8192
-constexpr uint32_t OFF_G = OFF_KT + 16384;    // g [2][64]
-constexpr uint32_t OFF_EG = OFF_G + 512;      // e^g [2][64]
+constexpr uint32_t OFF_EG = OFF_KT + 16384;   // e^g [2][64]
 constexpr uint32_t OFF_KS = OFF_EG + 512;     // e^{g_C - g} [64]
-constexpr uint32_t OFF_RED = OFF_KS + 256;    // [4][64] partial sums of o^2
-constexpr uint32_t OFF_RS = OFF_RED + 1024;   // rsqrt(mean o^2 + eps) [64]
-constexpr uint32_t OFF_BAR = OFF_RS + 256;    // mbarriers, TMEM address, abort flag
+constexpr uint32_t OFF_BAR = OFF_KS + 256;    // mbarriers, TMEM address, abort flag
 constexpr uint32_t SMEM_USED = OFF_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
 constexpr uint32_t ACC_U = 0, ACC_O1 = 64, ACC_O2 = 192, ACC_SI = 320, TMEM_COLS = 512;
-constexpr uint32_t QKV_BYTES = 6 * 8192, Z_BYTES = 2 * 8192;
+constexpr uint32_t QKV_BYTES = 6 * 8192;
 
 struct Args {
-    const void* z;              // [T][Hv][dv] act dtype
-    const float* norm_w;        // [dv]
     float* rec_state;           // [N][Hv][dv][dk] in/out
     const int32_t* cu;          // [N+1]
     const int32_t* chunk_off;   // [N+1]
     const uint8_t* rec;         // intra-chunk records
-    void* out;                  // [T][Hv][dv] out dtype
+    void* o;                    // [chunks][Hv][64][128] out dtype: o before the gated norm
     int Hk, Hv, dk, dv;
-    float norm_eps;
 };
 
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
@@ -82,23 +78,19 @@ __device__ __forceinline__ uint4 scale8(uint4 v, float s) {
                       pack_half2(c.x * s, c.y * s), pack_half2(d.x * s, d.y * s));
 }
 
-template <typename TA, typename TO>
+template <typename TO>
 __global__ void __launch_bounds__(NT, 1)
 gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_z, Args p) {
-    constexpr bool kZTile = sizeof(TA) == 2;                  // z through TMA (bf16 activations)
-    constexpr bool kOutStage = kZTile && sizeof(TO) == 2;     // out staged in the z tile
+                const __grid_constant__ CUtensorMap tm_v, Args p) {
+    constexpr uint32_t O_BYTES = C * 128 * sizeof(TO);
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sb = (raw + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (sb - raw);
-    float* s_g = reinterpret_cast<float*>(smem + OFF_G);
     float* s_eg = reinterpret_cast<float*>(smem + OFF_EG);
     float* s_ks = reinterpret_cast<float*>(smem + OFF_KS);
-    float* s_red = reinterpret_cast<float*>(smem + OFF_RED);
-    float* s_rs = reinterpret_cast<float*>(smem + OFF_RS);
-    const uint32_t bar = sb + OFF_BAR, bar_qkv = sb + OFF_BAR + 8, bar_z = sb + OFF_BAR + 16;
-    const uint32_t bar_rec0 = sb + OFF_BAR + 24;   // + 8 * buffer
+    const uint32_t bar = sb + OFF_BAR, bar_qkv = sb + OFF_BAR + 8;
+    const uint32_t bar_rec0 = sb + OFF_BAR + 16, bar_rec1 = sb + OFF_BAR + 24;
     volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 40);
     volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 44);
 
@@ -111,14 +103,14 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const int64_t s0 = p.cu[seq], s1 = p.cu[seq + 1];
     const int nchunks = (int)((s1 - s0 + C - 1) / C);
     if (nchunks <= 0) return;
-    const uint8_t* rec0 = p.rec + ((int64_t)p.chunk_off[seq] * Hv + h) * intra::REC_BYTES;
+    const int64_t first = (int64_t)p.chunk_off[seq] * Hv + h;   // (chunk, head) index of chunk 0
+    const uint8_t* rec0 = p.rec + first * intra::REC_BYTES;
     const int64_t rec_stride = (int64_t)Hv * intra::REC_BYTES;
-    const TA* __restrict__ pz = static_cast<const TA*>(p.z);
-    TO* __restrict__ pout = static_cast<TO*>(p.out);
-    const int64_t ldv = (int64_t)Hv * dv;
+    uint8_t* otile0 = static_cast<uint8_t*>(p.o) + first * O_BYTES;
+    const int64_t o_stride = (int64_t)Hv * O_BYTES;
 
-    int qkv_issued = 0, qkv_ok = 0, z_issued = 0, z_ok = 0;
-    int rec_issued[2] = {0, 0}, rec_ok[2] = {0, 0};
+    // TMA / bulk loads issued (by thread 0) and waited for, for the abort path
+    int qkv_issued = 0, qkv_ok = 0, rec0_issued = 0, rec0_ok = 0, rec1_issued = 0, rec1_ok = 0;
     auto issue_qkv = [&](int ci) {
         const int t = (int)(s0 + (int64_t)ci * C);
         qkv_issued++;
@@ -131,31 +123,22 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
     };
     auto issue_rec = [&](int ci) {
-        const int b = ci & 1;
-        rec_issued[b]++;
-        mbar_arrive_expect_tx(bar_rec0 + 8 * b, REC_COPY);
-        bulk_g2s(sb + OFF_REC + b * intra::REC_BYTES, rec0 + ci * rec_stride, REC_COPY, bar_rec0 + 8 * b);
-    };
-    auto issue_z = [&](int ci) {
-        z_issued++;
-        mbar_arrive_expect_tx(bar_z, Z_BYTES);
-#pragma unroll
-        for (int hf = 0; hf < 2; hf++)
-            tma_load_3d(sb + OFF_ZT + hf * 8192, &tm_z, 64 * hf, h, (int)(s0 + (int64_t)ci * C), bar_z);
+        const uint32_t bb = (ci & 1) ? bar_rec1 : bar_rec0;
+        if (ci & 1) rec1_issued++; else rec0_issued++;
+        mbar_arrive_expect_tx(bb, REC_COPY);
+        bulk_g2s(sb + OFF_REC + (ci & 1) * intra::REC_BYTES, rec0 + ci * rec_stride, REC_COPY, bb);
     };
 
     if (tid == 0) {
         mbar_init(bar, 1);
         mbar_init(bar_qkv, 1);
-        mbar_init(bar_z, 1);
         mbar_init(bar_rec0, 1);
-        mbar_init(bar_rec0 + 8, 1);
+        mbar_init(bar_rec1, 1);
         fence_mbar_init();
         *s_abort = 0;
         issue_qkv(0);
         issue_rec(0);
         if (nchunks > 1) issue_rec(1);
-        if (kZTile) issue_z(0);
     }
     if (warp == 0) {
         tmem_alloc(sb + OFF_BAR + 40, TMEM_COLS);
@@ -186,98 +169,38 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t tmem = *s_tmem;
     const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
     const float inv_sqrt_dk = rsqrtf((float)dk);
-    const float wn = dv_r < dv ? p.norm_w[dv_r] : 0.f;
     uint32_t mphase = 0;
 
-    // Gated RMSNorm epilogue of chunk ce (O accumulators of buffer ce & 1).
-    auto epilogue = [&](int ce) -> bool {
+    // o = (e^{g_r} O1 + O2) / sqrt(d_k) of chunk ce -> [64][128] tile -> one bulk store
+    auto store_o = [&](int ce) {
         const int be = ce & 1;
-        const int64_t te = s0 + (int64_t)ce * C;
-        const int ne = (int)((s1 - te) < (int64_t)C ? (s1 - te) : (int64_t)C);
-        float o[16], v[16];
-        {
-            uint32_t o1[16], o2[16];
-            tmem_ld16(tl + ACC_O1 + 64 * be + 16 * cs, o1);
-            tmem_ld16(tl + ACC_O2 + 64 * be + 16 * cs, o2);
+        if (tid == 0) bulk_wait_read<0>();   // the previous tile's store has read the staging buffer
+        __syncthreads();
+        uint32_t o1[16], o2[16];
+        tmem_ld16(tl + ACC_O1 + 64 * be + 16 * cs, o1);
+        tmem_ld16(tl + ACC_O2 + 64 * be + 16 * cs, o2);
 #pragma unroll
-            for (int i = 0; i < 16; i++) {
-                const int r = 16 * cs + i;
-                o[i] = (s_eg[64 * be + r] * __uint_as_float(o1[i]) + __uint_as_float(o2[i])) * inv_sqrt_dk;
-                v[i] = o[i] * o[i];
-            }
+        for (int i = 0; i < 16; i++) {
+            const int r = 16 * cs + i;
+            const float o = (s_eg[64 * be + r] * __uint_as_float(o1[i]) + __uint_as_float(o2[i])) * inv_sqrt_dk;
+            from_f32(o, reinterpret_cast<TO*>(smem + OFF_OST) + r * 128 + dv_r);
         }
-        // transpose-reduce: lanes L and L^16 end with the warp's sum for column 16 cs + (L & 15)
-#pragma unroll
-        for (int off = 8; off >= 1; off >>= 1) {
-            const bool upper = (lane & off) != 0;
-#pragma unroll
-            for (int i = 0; i < off; i++) {
-                const float send = upper ? v[i] : v[i + off];
-                const float keep = upper ? v[i + off] : v[i];
-                v[i] = keep + __shfl_xor_sync(0xffffffffu, send, off);
-            }
-        }
-        v[0] += __shfl_xor_sync(0xffffffffu, v[0], 16);
-        if (lane < 16) s_red[qd * 64 + 16 * cs + lane] = v[0];
+        fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        if (tid < C) s_rs[tid] = rsqrtf((s_red[tid] + s_red[64 + tid] + s_red[128 + tid] + s_red[192 + tid]) /
-                                        (float)dv + p.norm_eps);
-        __syncthreads();
-        if constexpr (kZTile) {
-            if (mbar_wait_bounded(bar_z, ce & 1)) z_ok++; else atomicOr((unsigned*)s_abort, 2u);
-            const uint32_t zcol = (uint32_t)(dv_r >> 6) * 8192 + (uint32_t)(dv_r & 7) * 2;
-#pragma unroll
-            for (int i = 0; i < 16; i++) {
-                const int r = 16 * cs + i;
-                __nv_bfloat16* zp =
-                    reinterpret_cast<__nv_bfloat16*>(smem + OFF_ZT + zcol + swz128(r, (dv_r & 63) >> 3));
-                const float y = o[i] * s_rs[r] * wn * silu_f(__bfloat162float(*zp));
-                if constexpr (kOutStage) {
-                    *zp = __float2bfloat16_rn(y);
-                } else {
-                    if (r < ne && dv_r < dv) from_f32(y, pout + (te + r) * ldv + (int64_t)h * dv + dv_r);
-                }
-            }
-            if constexpr (kOutStage) {
-                __syncthreads();
-                for (int idx = tid; idx < C * 16; idx += NT) {   // 16-byte row pieces
-                    const int r = idx >> 4, c16 = idx & 15;
-                    if (r < ne && c16 * 8 < dv) {
-                        const uint4 v4 = lds128(sb + OFF_ZT + (c16 >> 3) * 8192 + swz128(r, c16 & 7));
-                        __stcs(reinterpret_cast<uint4*>(pout + (te + r) * ldv + (int64_t)h * dv + c16 * 8), v4);
-                    }
-                }
-            }
-            __syncthreads();
-            if (*s_abort) return false;
-            if (tid == 0 && ce + 1 < nchunks) {   // the z tile is free: fetch the next chunk's
-                fence_async_smem();
-                issue_z(ce + 1);
-            }
-        } else if (dv_r < dv) {
-            float zz[16];
-#pragma unroll
-            for (int i = 0; i < 16; i++) {
-                const int r = 16 * cs + i;
-                zz[i] = r < ne ? to_f32(pz[(te + r) * ldv + (int64_t)h * dv + dv_r]) : 0.f;
-            }
-#pragma unroll
-            for (int i = 0; i < 16; i++) {
-                const int r = 16 * cs + i;
-                if (r < ne) from_f32(o[i] * s_rs[r] * wn * silu_f(zz[i]), pout + (te + r) * ldv + (int64_t)h * dv + dv_r);
-            }
+        if (tid == 0) {
+            bulk_s2g(otile0 + ce * o_stride, sb + OFF_OST, O_BYTES);
+            bulk_commit();
         }
-        return true;
     };
 
-#define GDN_MMA_WAIT()                                                         \
-    do {                                                                       \
-        if (!mbar_wait_bounded(bar, mphase)) atomicOr((unsigned*)s_abort, 1u); \
-        mphase ^= 1u;                                                          \
-        __syncthreads();                                                       \
-        if (*s_abort) goto abort_;                                             \
-        tc_fence_after();                                                      \
+#define GDN_MMA_WAIT()                                                                        \
+    do {                                                                                      \
+        if (tid == 0 && !mbar_wait_bounded(bar, mphase)) atomicOr((unsigned*)s_abort, 1u);  \
+        mphase ^= 1u;                                                                         \
+        __syncthreads();                                                                      \
+        if (*s_abort) goto abort_;                                                            \
+        tc_fence_after();                                                                     \
     } while (0)
 
     for (int ci = 0; ci < nchunks; ci++) {
@@ -286,13 +209,16 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int64_t t0 = s0 + (int64_t)ci * C;
         const int n = (int)((s1 - t0) < (int64_t)C ? (s1 - t0) : (int64_t)C);
 
-        // ---- this chunk's tiles and record ----
-        if (mbar_wait_bounded(bar_qkv, ci & 1)) qkv_ok++; else atomicOr((unsigned*)s_abort, 2u);
-        if (mbar_wait_bounded(bar_rec0 + 8 * b, (ci >> 1) & 1)) rec_ok[b]++; else atomicOr((unsigned*)s_abort, 2u);
+        // ---- this chunk's tiles and record (the 64 threads that read the record wait) ----
         if (tid < C) {
+            if (mbar_wait_bounded(bar_qkv, ci & 1)) qkv_ok++; else atomicOr((unsigned*)s_abort, 2u);
+            if (mbar_wait_bounded(b ? bar_rec1 : bar_rec0, (ci >> 1) & 1)) {
+                if (b) rec1_ok++; else rec0_ok++;
+            } else {
+                atomicOr((unsigned*)s_abort, 2u);
+            }
             const float* rg = reinterpret_cast<const float*>(smem + OFF_REC + b * intra::REC_BYTES + intra::REC_G);
             const float g = rg[tid], gl = rg[C - 1];
-            s_g[64 * b + tid] = g;
             s_eg[64 * b + tid] = __expf(g);
             s_ks[tid] = tid < n ? __expf(gl - g) : 0.f;
         }
@@ -326,8 +252,8 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             sts128(sb + OFF_KT + hf * 8192 + swz128(r, cc), kt.x, kt.y, kt.z, kt.w);
         }
         fence_async_smem();
-        // ---- the previous chunk's output, while (c, d, e) run ----
-        if (ci > 0 && !epilogue(ci - 1)) goto abort_;
+        // ---- the previous chunk's o tile, while (c, d, e) run ----
+        if (ci > 0) store_o(ci - 1);
         GDN_MMA_WAIT();
         if (tid == 0 && ci + 1 < nchunks) {   // q, k, v tiles consumed: fetch the next chunk's
             fence_async_smem();
@@ -381,7 +307,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         __syncthreads();
         (void)n;
     }
-    if (!epilogue(nchunks - 1)) goto abort_;
+    store_o(nchunks - 1);
 
     // ---- final state ----
 #pragma unroll
@@ -389,6 +315,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int col = 32 * cs + i;
         if (dv_r < dv && col < dk) gstate[(int64_t)dv_r * dk + col] = S[i];
     }
+    if (tid == 0) bulk_wait<0>();   // every o tile has reached global memory
     tc_fence_before();
     __syncthreads();
     if (warp == 0) {
@@ -404,9 +331,9 @@ abort_:
     if (tid == 0) {
         record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));
         for (int k = qkv_ok; k < qkv_issued; k++) mbar_wait_bounded(bar_qkv, k & 1);
-        for (int k = z_ok; k < z_issued; k++) mbar_wait_bounded(bar_z, k & 1);
-        for (int bb = 0; bb < 2; bb++)
-            for (int k = rec_ok[bb]; k < rec_issued[bb]; k++) mbar_wait_bounded(bar_rec0 + 8 * bb, k & 1);
+        for (int k = rec0_ok; k < rec0_issued; k++) mbar_wait_bounded(bar_rec0, k & 1);
+        for (int k = rec1_ok; k < rec1_issued; k++) mbar_wait_bounded(bar_rec1, k & 1);
+        bulk_wait<0>();
     }
     if (warp == 0) {
         mbar_wait_bounded(bar, mphase ^ 1u);
