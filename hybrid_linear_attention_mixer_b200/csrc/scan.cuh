@@ -171,28 +171,61 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const float inv_sqrt_dk = rsqrtf((float)dk);
     uint32_t mphase = 0;
 
-    // o = (e^{g_r} O1 + O2) / sqrt(d_k) of chunk ce -> [64][128] tile -> one bulk store
-    auto store_o = [&](int ce) {
+    // Staging for the o tiles: two buffers when a tile is 16 KiB (bf16), one when 32 KiB.
+    constexpr int kOBufs = O_BYTES <= 16384 ? 2 : 1;
+    // o = (e^{g_r} O1 + O2) / sqrt(d_k) of chunk ce -> staging buffer; tid 0 stores it
+    // with one bulk copy after the next CTA barrier (issue_o).
+    auto stage_o = [&](int ce) {
         const int be = ce & 1;
-        if (tid == 0) bulk_wait_read<0>();   // the previous tile's store has read the staging buffer
-        __syncthreads();
         uint32_t o1[16], o2[16];
         tmem_ld16(tl + ACC_O1 + 64 * be + 16 * cs, o1);
         tmem_ld16(tl + ACC_O2 + 64 * be + 16 * cs, o2);
+        TO* st = reinterpret_cast<TO*>(smem + OFF_OST + (ce % kOBufs) * 16384);
 #pragma unroll
         for (int i = 0; i < 16; i++) {
             const int r = 16 * cs + i;
             const float o = (s_eg[64 * be + r] * __uint_as_float(o1[i]) + __uint_as_float(o2[i])) * inv_sqrt_dk;
-            from_f32(o, reinterpret_cast<TO*>(smem + OFF_OST) + r * 128 + dv_r);
+            from_f32(o, st + r * 128 + dv_r);
         }
         fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
-            bulk_s2g(otile0 + ce * o_stride, sb + OFF_OST, O_BYTES);
-            bulk_commit();
-        }
     };
+    auto issue_o = [&](int ce) {   // tid 0, after a CTA barrier that follows stage_o(ce)
+        bulk_s2g(otile0 + ce * o_stride, sb + OFF_OST + (ce % kOBufs) * 16384, O_BYTES);
+        bulk_commit();
+    };
+    // Record-derived per-chunk vectors of chunk ce: e^g and e^{g_C - g} (zero past the end).
+    // Threads 0..63 only; they first wait for the record.
+    auto chunk_vectors = [&](int ce) {
+        const int be = ce & 1;
+        if (mbar_wait_bounded(be ? bar_rec1 : bar_rec0, (ce >> 1) & 1)) {
+            if (be) rec1_ok++; else rec0_ok++;
+        } else {
+            atomicOr((unsigned*)s_abort, 2u);
+        }
+        const float* rg = reinterpret_cast<const float*>(smem + OFF_REC + be * intra::REC_BYTES + intra::REC_G);
+        const float g = rg[tid], gl = rg[C - 1];
+        const int64_t te = s0 + (int64_t)ce * C;
+        s_eg[64 * be + tid] = __expf(g);
+        s_ks[tid] = te + tid < s1 ? __expf(gl - g) : 0.f;
+    };
+
+    // Shared-memory descriptors (thread 0 issues every MMA); per-step offsets are
+    // added to the start-address field (addresses stay below 256 KiB).
+    const uint64_t dV = sdesc(sb + OFF_V, 8192, 1024);
+    const uint64_t dS = sdesc(sb + OFF_S16, 16, 1024);
+    const uint64_t dQ = sdesc(sb + OFF_QK, 16, 1024);
+    const uint64_t dUT = sdesc(sb + OFF_UT, 16, 1024);
+    const uint64_t dKT = sdesc(sb + OFF_KT, 8192, 1024);
+    const uint64_t dT0 = sdesc(sb + OFF_REC + intra::REC_T, 16, 1024);
+    const uint64_t dW0 = sdesc(sb + OFF_REC + intra::REC_W, 8192, 1024);
+    const uint64_t dP0 = sdesc(sb + OFF_REC + intra::REC_P, 16, 1024);
+    constexpr uint64_t kRecStep = intra::REC_BYTES >> 4;
+    constexpr uint32_t ID_MK = idesc_f16(128, 64, 1, 0), ID_KM = idesc_f16(128, 64, 0, 1);
+    constexpr uint32_t ID_KK = idesc_f16(128, 64, 0, 0), ID_KM128 = idesc_f16(128, 128, 0, 1);
+
+    if (tid < C) chunk_vectors(0);
+    __syncthreads();
+    if (*s_abort) goto abort_;
 
 #define GDN_MMA_WAIT()                                                                        \
     do {                                                                                      \
@@ -205,62 +238,36 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     for (int ci = 0; ci < nchunks; ci++) {
         const int b = ci & 1;
-        const uint32_t rb = sb + OFF_REC + b * intra::REC_BYTES;
-        const int64_t t0 = s0 + (int64_t)ci * C;
-        const int n = (int)((s1 - t0) < (int64_t)C ? (s1 - t0) : (int64_t)C);
-
-        // ---- this chunk's tiles and record (the 64 threads that read the record wait) ----
-        if (tid < C) {
-            if (mbar_wait_bounded(bar_qkv, ci & 1)) qkv_ok++; else atomicOr((unsigned*)s_abort, 2u);
-            if (mbar_wait_bounded(b ? bar_rec1 : bar_rec0, (ci >> 1) & 1)) {
-                if (b) rec1_ok++; else rec0_ok++;
-            } else {
-                atomicOr((unsigned*)s_abort, 2u);
-            }
-            const float* rg = reinterpret_cast<const float*>(smem + OFF_REC + b * intra::REC_BYTES + intra::REC_G);
-            const float g = rg[tid], gl = rg[C - 1];
-            s_eg[64 * b + tid] = __expf(g);
-            s_ks[tid] = tid < n ? __expf(gl - g) : 0.f;
-        }
-        __syncthreads();
-        if (*s_abort) goto abort_;
+        const uint64_t rs = b ? kRecStep : 0;
 
         // ---- (c) U^T = V^T T^T, (d) U^T += S (-W)^T, (e) O1^T = S Q^T ----
         if (tid == 0) {
+            if (mbar_wait_bounded(bar_qkv, ci & 1)) qkv_ok++; else atomicOr((unsigned*)s_abort, 2u);
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 4; ks++)
-                mma_f16(tmem + ACC_U, sdesc(sb + OFF_V + ks * 2048, 8192, 1024),
-                        sdesc(rb + intra::REC_T + ks * 32, 16, 1024), idesc_f16(128, 64, 1, 0), ks > 0);
+                mma_f16(tmem + ACC_U, dV + ks * 128, dT0 + rs + ks * 2, ID_MK, ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 8; ks++)
-                mma_f16(tmem + ACC_U, sdesc(sb + OFF_S16 + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-                        sdesc(rb + intra::REC_W + ks * 2048, 8192, 1024), idesc_f16(128, 64, 0, 1), 1);
+                mma_f16(tmem + ACC_U, dS + (ks >> 2) * 1024 + (ks & 3) * 2, dW0 + rs + ks * 128, ID_KM, 1);
 #pragma unroll
-            for (int ks = 0; ks < 8; ks++) {
-                const uint32_t o = (ks >> 2) * 16384 + (ks & 3) * 32;
-                mma_f16(tmem + ACC_O1 + 64 * b, sdesc(sb + OFF_S16 + o, 16, 1024), sdesc(sb + OFF_QK + o, 16, 1024),
-                        idesc_f16(128, 64, 0, 0), ks > 0);
-            }
+            for (int ks = 0; ks < 8; ks++)
+                mma_f16(tmem + ACC_O1 + 64 * b, dS + (ks >> 2) * 1024 + (ks & 3) * 2,
+                        dQ + (ks >> 2) * 1024 + (ks & 3) * 2, ID_KK, ks > 0);
             mma_commit(bar);
         }
-        // ---- K~ = diag(e^{g_C - g}) K (rows past the chunk's end are zero) ----
+        // ---- the previous chunk's o tile, while (c, d, e) run ----
+        if (ci > 0) stage_o(ci - 1);
+        GDN_MMA_WAIT();
+        if (tid == 0 && ci > 0) issue_o(ci - 1);
+
+        // ---- K~ = diag(e^{g_C - g}) K, and U^T -> fp16 ----
         for (int idx = tid; idx < C * 16; idx += NT) {
             const int r = idx >> 4, c16 = idx & 15;
             const int hf = c16 >> 3, cc = c16 & 7;
             const uint4 kt = scale8(lds128(sb + OFF_QK + hf * 16384 + swz128(C + r, cc)), s_ks[r]);
             sts128(sb + OFF_KT + hf * 8192 + swz128(r, cc), kt.x, kt.y, kt.z, kt.w);
         }
-        fence_async_smem();
-        // ---- the previous chunk's o tile, while (c, d, e) run ----
-        if (ci > 0) store_o(ci - 1);
-        GDN_MMA_WAIT();
-        if (tid == 0 && ci + 1 < nchunks) {   // q, k, v tiles consumed: fetch the next chunk's
-            fence_async_smem();
-            issue_qkv(ci + 1);
-        }
-
-        // ---- U^T -> fp16 ----
         {
             uint32_t r16[16];
             tmem_ld16(tl + ACC_U + 16 * cs, r16);
@@ -279,21 +286,17 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 4; ks++)
-                mma_f16(tmem + ACC_O2 + 64 * b, sdesc(sb + OFF_UT + ks * 32, 16, 1024),
-                        sdesc(rb + intra::REC_P + ks * 32, 16, 1024), idesc_f16(128, 64, 0, 0), ks > 0);
+                mma_f16(tmem + ACC_O2 + 64 * b, dUT + ks * 2, dP0 + rs + ks * 2, ID_KK, ks > 0);
 #pragma unroll
             for (int ks = 0; ks < 4; ks++)
-                mma_f16(tmem + ACC_SI, sdesc(sb + OFF_UT + ks * 32, 16, 1024),
-                        sdesc(sb + OFF_KT + ks * 2048, 8192, 1024), idesc_f16(128, 128, 0, 1), ks > 0);
+                mma_f16(tmem + ACC_SI, dUT + ks * 2, dKT + ks * 128, ID_KM128, ks > 0);
             mma_commit(bar);
+            if (ci + 1 < nchunks) issue_qkv(ci + 1);   // q, k, v tiles consumed: fetch the next chunk's
         }
         GDN_MMA_WAIT();
-        if (tid == 0 && ci + 2 < nchunks) {   // record buffer b consumed: fetch chunk ci + 2's
-            fence_async_smem();
-            issue_rec(ci + 2);
-        }
+        if (tid == 0 && ci + 2 < nchunks) issue_rec(ci + 2);   // record buffer b consumed
 
-        // ---- S <- e^{g_C} S + U^T K~, and its fp16 copy for the next chunk ----
+        // ---- S <- e^{g_C} S + U^T K~ and its fp16 copy; next chunk's vectors ----
         {
             const float eg = s_eg[64 * b + C - 1];
             uint32_t r32[32];
@@ -302,12 +305,20 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int i = 0; i < 32; i++) S[i] = fmaf(eg, S[i], __uint_as_float(r32[i]));
             write_s16();
         }
+        if (tid < C && ci + 1 < nchunks) chunk_vectors(ci + 1);
+        // the staging buffer the next chunk writes has been read by its last bulk store
+        if (tid == 0) {
+            if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();
+        }
         fence_async_smem();
         tc_fence_before();
         __syncthreads();
-        (void)n;
+        if (*s_abort) goto abort_;
     }
-    store_o(nchunks - 1);
+    stage_o(nchunks - 1);
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0) issue_o(nchunks - 1);
 
     // ---- final state ----
 #pragma unroll
