@@ -31,17 +31,20 @@ constexpr uint32_t REC_W = 0, REC_T = 16384, REC_P = 24576, REC_G = 32768;
 constexpr uint32_t REC_BYTES = 33792;   // 33 x 1024: keeps every tile of a record 1024-aligned
 
 constexpr uint32_t OFF_QK = 0;          // [Q;K]: 128 token rows x d_k, halves of 16384
-constexpr uint32_t OFF_TP = 32768;      // T' = T diag(e^g)
-constexpr int LDA = 65;
-constexpr uint32_t OFF_A = 40960;
-constexpr uint32_t OFF_X = OFF_A + 64 * LDA * 4;
-constexpr uint32_t OFF_Z = OFF_X + 64 * LDA * 4;
-constexpr uint32_t OFF_G = OFF_Z + 64 * LDA * 4;   // g[64]
+constexpr int LDA = 68;                 // fp32 64 x 64 work matrices: 16-byte aligned rows
+constexpr int LDY = 36;
+constexpr uint32_t OFF_A = 32768;       // A; after the solve, T' = T diag(e^g) (fp16 tile)
+constexpr uint32_t OFF_TP = OFF_A;
+constexpr uint32_t OFF_X = OFF_A + 64 * LDA * 4;   // X = (I + A)^-1
+constexpr uint32_t OFF_Y = OFF_X + 64 * LDA * 4;   // products of the doubling steps [32][LDY]
+constexpr uint32_t OFF_G = OFF_Y + 32 * LDY * 4;   // g[64]
 constexpr uint32_t OFF_B = OFF_G + 256;            // beta[64]
-constexpr uint32_t OFF_BAR = OFF_B + 256;          // mbarriers, TMEM address, abort flag
+constexpr uint32_t OFF_EG = OFF_B + 256;           // e^g [64]
+constexpr uint32_t OFF_BAR = OFF_EG + 256;         // mbarriers, TMEM address, abort flag
 constexpr uint32_t SMEM_USED = OFF_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
-static_assert(2 * SMEM_BYTES <= 232448, "two CTAs per SM");
+static_assert(3 * SMEM_BYTES <= 232448, "three CTAs per SM");
+static_assert(OFF_A % 1024 == 0, "T' tile alignment");
 constexpr uint32_t ACC_QK = 0, ACC_W = 64, TMEM_COLS = 128;
 
 struct Args {
@@ -101,8 +104,32 @@ __global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int32_t* cu, 
     if (threadIdx.x == 0) chunk_off[n_seqs] = s_carry;
 }
 
+// C = sgn * L R for n x n blocks (n = 16 or 32; rows 16-byte aligned), 1 x 4
+// register tiles: thread t of nt takes tiles t, t + nt, ...
+__device__ __forceinline__ void block_mm(const float* L, int ldl, const float* R, int ldr, float* Cm, int ldc,
+                                         int n, float sgn, int t, int nt) {
+    const int tpr = n >> 2;
+    for (int tile = t; tile < n * tpr; tile += nt) {
+        const int i = tile / tpr, j0 = (tile % tpr) * 4;
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int l0 = 0; l0 < n; l0 += 4) {
+            const float4 a = *reinterpret_cast<const float4*>(L + i * ldl + l0);
+            const float av[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+            for (int u = 0; u < 4; u++) {
+                const float4 r = *reinterpret_cast<const float4*>(R + (l0 + u) * ldr + j0);
+                acc.x = fmaf(av[u], r.x, acc.x);
+                acc.y = fmaf(av[u], r.y, acc.y);
+                acc.z = fmaf(av[u], r.z, acc.z);
+                acc.w = fmaf(av[u], r.w, acc.w);
+            }
+        }
+        *reinterpret_cast<float4*>(Cm + i * ldc + j0) = make_float4(sgn * acc.x, sgn * acc.y, sgn * acc.z, sgn * acc.w);
+    }
+}
+
 template <typename TA>
-__global__ void __launch_bounds__(NT, 2)
+__global__ void __launch_bounds__(NT, 3)
 gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k, Args p) {
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -112,7 +139,8 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     float* s_b = reinterpret_cast<float*>(smem + OFF_B);
     float* Am = reinterpret_cast<float*>(smem + OFF_A);
     float* Xm = reinterpret_cast<float*>(smem + OFF_X);
-    float* Zm = reinterpret_cast<float*>(smem + OFF_Z);
+    float* Ym = reinterpret_cast<float*>(smem + OFF_Y);
+    float* s_eg = reinterpret_cast<float*>(smem + OFF_EG);
     const uint32_t bar = sb + OFF_BAR, bar_ld = sb + OFF_BAR + 8;
     volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 16);
     volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 20);
@@ -173,11 +201,16 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc_fence_after();
     if (tid >= 32 && tid < C) s_g[tid] += s_g[31];
+    for (int i = tid; i < 64 * LDA / 4; i += NT)   // X starts as zero above its diagonal blocks
+        reinterpret_cast<float4*>(Xm)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     const uint32_t tmem = *s_tmem;
     const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
     if (!mbar_wait_bounded(bar_ld, 0)) atomicOr((unsigned*)s_abort, 2u);
     __syncthreads();
-    if (tid < C) reinterpret_cast<float*>(rec + REC_G)[tid] = s_g[tid];
+    if (tid < C) {
+        reinterpret_cast<float*>(rec + REC_G)[tid] = s_g[tid];
+        s_eg[tid] = __expf(s_g[tid]);
+    }
     bool ok = *s_abort == 0;
 
     // ---- [Q;K] K^T ----
@@ -218,10 +251,15 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const int r = 32 * (qd - 2) + lane;
             const float gr = s_g[r], br = s_b[r];
 #pragma unroll
-            for (int i = 0; i < 32; i++) {
-                const int jj = j0 + i;
-                const float e = __expf(fminf(gr - s_g[jj], 0.f));
-                Am[r * LDA + jj] = jj < r ? br * __uint_as_float(r32[i]) * e : 0.f;
+            for (int i4 = 0; i4 < 8; i4++) {
+                float a4[4];
+#pragma unroll
+                for (int u = 0; u < 4; u++) {
+                    const int jj = j0 + 4 * i4 + u;
+                    const float e = __expf(fminf(gr - s_g[jj], 0.f));
+                    a4[u] = jj < r ? br * __uint_as_float(r32[4 * i4 + u]) * e : 0.f;
+                }
+                *reinterpret_cast<float4*>(Am + r * LDA + j0 + 4 * i4) = make_float4(a4[0], a4[1], a4[2], a4[3]);
             }
         }
     }
@@ -229,51 +267,45 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
 
     // ---- X = (I + A)^-1, unit lower triangular, fp32 ----
-    if (ok && tid < 64) {   // diagonal 16 x 16 blocks: one column per thread
+    // 16 x 16 diagonal blocks by substitution, then two doubling steps: for
+    // diagonal blocks [[L1, 0], [A21, L2]] the inverse is [[X1, 0], [-X2 A21 X1, X2]].
+    if (ok && tid < 64) {   // one column of one diagonal block per thread
         const int base = 16 * (tid >> 4), c = tid & 15;
         float x[16];
 #pragma unroll
         for (int i = 0; i < 16; i++) {
             float acc = (i == c) ? 1.f : 0.f;
+            const float* arow = Am + (base + i) * LDA + base;
 #pragma unroll
-            for (int m = 0; m < i; m++) acc = fmaf(-Am[(base + i) * LDA + base + m], x[m], acc);
+            for (int m4 = 0; m4 < 16; m4 += 4) {
+                if (m4 < i) {
+                    const float4 a = *reinterpret_cast<const float4*>(arow + m4);
+                    if (m4 + 0 < i) acc = fmaf(-a.x, x[m4 + 0], acc);
+                    if (m4 + 1 < i) acc = fmaf(-a.y, x[m4 + 1], acc);
+                    if (m4 + 2 < i) acc = fmaf(-a.z, x[m4 + 2], acc);
+                    if (m4 + 3 < i) acc = fmaf(-a.w, x[m4 + 3], acc);
+                }
+            }
             x[i] = acc;
         }
 #pragma unroll
         for (int i = 0; i < 16; i++) Xm[(base + i) * LDA + base + c] = x[i];
     }
     __syncthreads();
-    if (ok) {   // Z_{bi,m} = X_{bi,bi} A_{bi,m} for the six blocks below the diagonal
-        const int i = tid >> 4, jj = tid & 15;
-#pragma unroll
-        for (int blk = 0; blk < 6; blk++) {
-            const int bi = blk < 1 ? 1 : blk < 3 ? 2 : 3;
-            const int m = blk < 1 ? 0 : blk < 3 ? blk - 1 : blk - 3;
-            float acc = 0.f;
-#pragma unroll
-            for (int l = 0; l < 16; l++)
-                acc = fmaf(Xm[(16 * bi + i) * LDA + 16 * bi + l], Am[(16 * bi + l) * LDA + 16 * m + jj], acc);
-            Zm[(16 * bi + i) * LDA + 16 * m + jj] = acc;
-        }
+    if (ok && tid < 128) {   // size 16 -> 32: Y = A21 X1 for the block pairs (0,1) and (2,3)
+        const int o1 = tid < 64 ? 0 : 32, o2 = o1 + 16;
+        block_mm(Am + o2 * LDA + o1, LDA, Xm + o1 * LDA + o1, LDA, Ym + (o1 >> 1), LDY, 16, 1.f, tid & 63, 64);
     }
     __syncthreads();
-#pragma unroll
-    for (int dd = 1; dd < 4; dd++) {   // X_{bi,bj} = -sum_{m=bj}^{bi-1} Z_{bi,m} X_{m,bj}
-        if (ok) {
-            const int i = tid >> 4, jj = tid & 15;
-            for (int bj = 0; bj + dd < 4; bj++) {
-                const int bi = bj + dd;
-                float acc = 0.f;
-                for (int m = bj; m < bi; m++) {
-#pragma unroll
-                    for (int l = 0; l < 16; l++)
-                        acc = fmaf(Zm[(16 * bi + i) * LDA + 16 * m + l], Xm[(16 * m + l) * LDA + 16 * bj + jj], acc);
-                }
-                Xm[(16 * bi + i) * LDA + 16 * bj + jj] = -acc;
-            }
-        }
-        __syncthreads();
+    if (ok && tid < 128) {   // X21 = -X2 Y
+        const int o1 = tid < 64 ? 0 : 32, o2 = o1 + 16;
+        block_mm(Xm + o2 * LDA + o2, LDA, Ym + (o1 >> 1), LDY, Xm + o2 * LDA + o1, LDA, 16, -1.f, tid & 63, 64);
     }
+    __syncthreads();
+    if (ok) block_mm(Am + 32 * LDA, LDA, Xm, LDA, Ym, LDY, 32, 1.f, tid, NT);   // size 32 -> 64
+    __syncthreads();
+    if (ok) block_mm(Xm + 32 * LDA + 32, LDA, Ym, LDY, Xm + 32 * LDA, LDA, 32, -1.f, tid, NT);
+    __syncthreads();
     if (ok) {   // T = X diag(beta) -> the record; T' = T diag(e^g) -> shared memory
         const int c = tid >> 2, jq = (tid & 3) * 16;
         uint32_t tp[8], tq[8];
@@ -283,7 +315,7 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             const float x0 = jj <= c ? Xm[c * LDA + jj] * s_b[jj] : 0.f;
             const float x1 = jj + 1 <= c ? Xm[c * LDA + jj + 1] * s_b[jj + 1] : 0.f;
             tp[i] = pack_half2(x0, x1);
-            tq[i] = pack_half2(x0 * __expf(s_g[jj]), x1 * __expf(s_g[jj + 1]));
+            tq[i] = pack_half2(x0 * s_eg[jj], x1 * s_eg[jj + 1]);
         }
 #pragma unroll
         for (int c2 = 0; c2 < 2; c2++) {

@@ -13,16 +13,19 @@
 //
 // Products (tcgen05.mma kind::f16, fp16 operands, fp32 accumulators in TMEM,
 // M = 128 = d_v always, the chunk is the N side):
-//   (c) V^T T^T           -> U^T accumulator            [A: V, MN-major]
-//   (d) S (-W)^T          accumulated into (c)           [B: -W, MN-major]
-//   (e) S Q^T             -> O1^T                        [double-buffered]
-//   (f) U^T P^T           -> O2^T                        [double-buffered]
-//   (g) U^T K~            -> state increment, K~ = diag(e^{g_C - g}) K [B: MN-major]
-// The chain per chunk is (c,d,e) -> U^T to fp16 -> (f,g) -> state update -> S to
-// fp16.  The output tile of chunk c-1 is formed and stored (one bulk copy)
-// while (c,d,e) of chunk c are on the tensor cores.  q^, k^, v^ tiles arrive by
-// TMA and a chunk's record by one bulk copy, issued a chunk or more ahead.  One
-// thread waits on each mbarrier; the others meet it at the CTA barrier.
+//   (c) V^T T^T           -> U^T accumulator        [A: V in shared memory, MN-major]
+//   (d) S (-W)^T          accumulated into (c)       [A: S in TMEM; B: -W, MN-major]
+//   (e) S Q~^T            -> O^T (Q~ = diag(e^g) Q)  [A: S in TMEM]
+//   (f) U^T P^T           accumulated into (e)       [A: U^T in TMEM]
+//   (g) U^T K~            -> state increment, K~ = diag(e^{g_C - g}) K [A: U^T in TMEM]
+// S and U^T live in TMEM as fp16 A operands (written with tcgen05.st), so the
+// tensor cores read only the B tiles from shared memory.  The chain per chunk is
+// (c,d) -> U^T to fp16 -> (e,f,g) -> state update -> S to fp16.  The o tile of
+// chunk c-1 (O double-buffered in TMEM) is formed and stored (one bulk copy)
+// while (c,d) of chunk c run.  q^, k^, v^ tiles (double-buffered) arrive by TMA
+// a chunk ahead, a chunk's record by one bulk copy two chunks ahead.  One
+// thread issues every MMA and waits on the tensor-core mbarrier; the others
+// meet it at the CTA barrier.
 #pragma once
 #include "device.cuh"
 #include "intra.cuh"
@@ -34,21 +37,22 @@ constexpr int C = 64;
 constexpr int NT = 512;   // 16 warps: 4 per TMEM lane quadrant
 constexpr uint32_t REC_COPY = intra::REC_G + 256;   // bytes of a record brought in
 
-constexpr uint32_t OFF_REC = 0;               // two record buffers of REC_BYTES
-constexpr uint32_t OFF_QK = 2 * intra::REC_BYTES;   // [Q;K] 128 rows x d_k, halves of 16384
-constexpr uint32_t OFF_V = OFF_QK + 32768;    // V: 64 rows x d_v, halves of 8192
-constexpr uint32_t OFF_OST = OFF_V + 16384;   // o tile staging: [64][128] out dtype (<= 32 KiB)
-constexpr uint32_t OFF_S16 = OFF_OST + 32768; // S (fp16): 128 d_v rows x d_k, halves of 16384
-constexpr uint32_t OFF_UT = OFF_S16 + 32768;  // U^T: 128 d_v rows x 64 chunk columns
-constexpr uint32_t OFF_KT = OFF_UT + 16384;   // K~: 64 rows x d_k, halves of 8192
-constexpr uint32_t OFF_EG = OFF_KT + 16384;   // e^g [2][64]
-constexpr uint32_t OFF_KS = OFF_EG + 512;     // e^{g_C - g} [64]
-constexpr uint32_t OFF_BAR = OFF_KS + 256;    // mbarriers, TMEM address, abort flag
+constexpr uint32_t OFF_REC = 0;                     // two record buffers of REC_BYTES
+constexpr uint32_t OFF_QKV = 2 * intra::REC_BYTES;  // two buffers of QKV_STRIDE:
+constexpr uint32_t QKV_STRIDE = 49152;              //   [Q;K] 128 rows x d_k (halves of 16384), V
+constexpr uint32_t QKV_V = 32768;                   //   V: 64 rows x d_v, halves of 8192
+constexpr uint32_t OFF_OST = OFF_QKV + 2 * QKV_STRIDE;   // o tile staging: 32 KiB
+constexpr uint32_t OFF_KT = OFF_OST + 32768;        // K~: 64 rows x d_k, halves of 8192
+constexpr uint32_t OFF_EG = OFF_KT + 16384;         // e^g [2][64]
+constexpr uint32_t OFF_KS = OFF_EG + 512;           // e^{g_C - g} [64]
+constexpr uint32_t OFF_BAR = OFF_KS + 256;          // mbarriers, TMEM address, abort flag
 constexpr uint32_t SMEM_USED = OFF_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-constexpr uint32_t ACC_U = 0, ACC_O1 = 64, ACC_O2 = 192, ACC_SI = 320, TMEM_COLS = 512;
+// Tensor memory: U^T (64), O^T x2 (128), increment (128), S fp16 A operand (64
+// columns of packed pairs), U^T fp16 A operand (32).
+constexpr uint32_t ACC_U = 0, ACC_O = 64, ACC_SI = 192, TA_S = 320, TA_U = 384, TMEM_COLS = 512;
 constexpr uint32_t QKV_BYTES = 6 * 8192;
 
 struct Args {
@@ -83,14 +87,16 @@ __global__ void __launch_bounds__(NT, 1)
 gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                 const __grid_constant__ CUtensorMap tm_v, Args p) {
     constexpr uint32_t O_BYTES = C * 128 * sizeof(TO);
+    constexpr int kOBufs = O_BYTES <= 16384 ? 2 : 1;   // staging buffers for the o tiles
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sb = (raw + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (sb - raw);
     float* s_eg = reinterpret_cast<float*>(smem + OFF_EG);
     float* s_ks = reinterpret_cast<float*>(smem + OFF_KS);
-    const uint32_t bar = sb + OFF_BAR, bar_qkv = sb + OFF_BAR + 8;
-    const uint32_t bar_rec0 = sb + OFF_BAR + 16, bar_rec1 = sb + OFF_BAR + 24;
+    const uint32_t bar = sb + OFF_BAR;
+    const uint32_t bar_qkv0 = sb + OFF_BAR + 8, bar_qkv1 = sb + OFF_BAR + 16;
+    const uint32_t bar_rec0 = sb + OFF_BAR + 24, bar_rec1 = sb + OFF_BAR + 32;
     volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 40);
     volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 44);
 
@@ -109,36 +115,51 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint8_t* otile0 = static_cast<uint8_t*>(p.o) + first * O_BYTES;
     const int64_t o_stride = (int64_t)Hv * O_BYTES;
 
-    // TMA / bulk loads issued (by thread 0) and waited for, for the abort path
-    int qkv_issued = 0, qkv_ok = 0, rec0_issued = 0, rec0_ok = 0, rec1_issued = 0, rec1_ok = 0;
+    // TMA / bulk loads issued (thread 0) and completed waits on them (each thread
+    // counts its own), for the abort path
+    int qkv_issued[2] = {0, 0}, qkv_ok[2] = {0, 0}, rec_issued[2] = {0, 0}, rec_ok[2] = {0, 0};
     auto issue_qkv = [&](int ci) {
         const int t = (int)(s0 + (int64_t)ci * C);
-        qkv_issued++;
-        mbar_arrive_expect_tx(bar_qkv, QKV_BYTES);
+        const uint32_t bb = (ci & 1) ? bar_qkv1 : bar_qkv0;
+        const uint32_t base = sb + OFF_QKV + (ci & 1) * QKV_STRIDE;
+        if (ci & 1) qkv_issued[1]++; else qkv_issued[0]++;
+        mbar_arrive_expect_tx(bb, QKV_BYTES);
 #pragma unroll
         for (int hf = 0; hf < 2; hf++) {
-            tma_load_3d(sb + OFF_QK + hf * 16384, &tm_q, 64 * hf, j, t, bar_qkv);
-            tma_load_3d(sb + OFF_QK + hf * 16384 + C * 128, &tm_k, 64 * hf, j, t, bar_qkv);
-            tma_load_3d(sb + OFF_V + hf * 8192, &tm_v, 64 * hf, h, t, bar_qkv);
+            tma_load_3d(base + hf * 16384, &tm_q, 64 * hf, j, t, bb);
+            tma_load_3d(base + hf * 16384 + C * 128, &tm_k, 64 * hf, j, t, bb);
+            tma_load_3d(base + QKV_V + hf * 8192, &tm_v, 64 * hf, h, t, bb);
         }
     };
     auto issue_rec = [&](int ci) {
         const uint32_t bb = (ci & 1) ? bar_rec1 : bar_rec0;
-        if (ci & 1) rec1_issued++; else rec0_issued++;
+        if (ci & 1) rec_issued[1]++; else rec_issued[0]++;
         mbar_arrive_expect_tx(bb, REC_COPY);
         bulk_g2s(sb + OFF_REC + (ci & 1) * intra::REC_BYTES, rec0 + ci * rec_stride, REC_COPY, bb);
+    };
+    auto wait_buf = [&](uint32_t b0, uint32_t b1, int (&ok)[2], int ci) {
+        const uint32_t bb = (ci & 1) ? b1 : b0;
+        if (mbar_wait_bounded(bb, (ci >> 1) & 1)) {
+            if (ci & 1) ok[1]++; else ok[0]++;
+        } else {
+            atomicOr((unsigned*)s_abort, 2u);
+        }
     };
 
     if (tid == 0) {
         mbar_init(bar, 1);
-        mbar_init(bar_qkv, 1);
+        mbar_init(bar_qkv0, 1);
+        mbar_init(bar_qkv1, 1);
         mbar_init(bar_rec0, 1);
         mbar_init(bar_rec1, 1);
         fence_mbar_init();
         *s_abort = 0;
         issue_qkv(0);
         issue_rec(0);
-        if (nchunks > 1) issue_rec(1);
+        if (nchunks > 1) {
+            issue_qkv(1);
+            issue_rec(1);
+        }
     }
     if (warp == 0) {
         tmem_alloc(sb + OFF_BAR + 40, TMEM_COLS);
@@ -154,15 +175,6 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const int col = 32 * cs + i;
         S[i] = (dv_r < dv && col < dk) ? gstate[(int64_t)dv_r * dk + col] : 0.f;
     }
-    auto write_s16 = [&]() {
-#pragma unroll
-        for (int c4 = 0; c4 < 4; c4++)
-            sts128(sb + OFF_S16 + (cs >> 1) * 16384 + swz128(dv_r, (cs & 1) * 4 + c4),
-                   pack_half2(S[8 * c4 + 0], S[8 * c4 + 1]), pack_half2(S[8 * c4 + 2], S[8 * c4 + 3]),
-                   pack_half2(S[8 * c4 + 4], S[8 * c4 + 5]), pack_half2(S[8 * c4 + 6], S[8 * c4 + 7]));
-    };
-    write_s16();
-    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -171,59 +183,50 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const float inv_sqrt_dk = rsqrtf((float)dk);
     uint32_t mphase = 0;
 
-    // Staging for the o tiles: two buffers when a tile is 16 KiB (bf16), one when 32 KiB.
-    constexpr int kOBufs = O_BYTES <= 16384 ? 2 : 1;
-    // o = (e^{g_r} O1 + O2) / sqrt(d_k) of chunk ce -> staging buffer; tid 0 stores it
-    // with one bulk copy after the next CTA barrier (issue_o).
+    // S -> fp16 A operand in TMEM: this thread's 32 columns of d_k = 16 packed columns
+    auto write_sa = [&]() {
+        uint32_t r[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++) r[i] = pack_half2(S[2 * i], S[2 * i + 1]);
+        tmem_st16(tl + TA_S + 16 * cs, r);
+    };
+    // o = O / sqrt(d_k) of chunk ce -> staging buffer; tid 0 stores it with one bulk
+    // copy after the next CTA barrier (issue_o).
     auto stage_o = [&](int ce) {
-        const int be = ce & 1;
-        uint32_t o1[16], o2[16];
-        tmem_ld16(tl + ACC_O1 + 64 * be + 16 * cs, o1);
-        tmem_ld16(tl + ACC_O2 + 64 * be + 16 * cs, o2);
+        uint32_t o[16];
+        tmem_ld16(tl + ACC_O + 64 * (ce & 1) + 16 * cs, o);
         TO* st = reinterpret_cast<TO*>(smem + OFF_OST + (ce % kOBufs) * 16384);
 #pragma unroll
-        for (int i = 0; i < 16; i++) {
-            const int r = 16 * cs + i;
-            const float o = (s_eg[64 * be + r] * __uint_as_float(o1[i]) + __uint_as_float(o2[i])) * inv_sqrt_dk;
-            from_f32(o, st + r * 128 + dv_r);
-        }
+        for (int i = 0; i < 16; i++) from_f32(__uint_as_float(o[i]) * inv_sqrt_dk, st + (16 * cs + i) * 128 + dv_r);
         fence_async_smem();
     };
-    auto issue_o = [&](int ce) {   // tid 0, after a CTA barrier that follows stage_o(ce)
+    auto issue_o = [&](int ce) {
         bulk_s2g(otile0 + ce * o_stride, sb + OFF_OST + (ce % kOBufs) * 16384, O_BYTES);
         bulk_commit();
     };
-    // Record-derived per-chunk vectors of chunk ce: e^g and e^{g_C - g} (zero past the end).
-    // Threads 0..63 only; they first wait for the record.
+    // e^g and e^{g_C - g} (zero past the chunk's end) of chunk ce, threads 0..63
     auto chunk_vectors = [&](int ce) {
-        const int be = ce & 1;
-        if (mbar_wait_bounded(be ? bar_rec1 : bar_rec0, (ce >> 1) & 1)) {
-            if (be) rec1_ok++; else rec0_ok++;
-        } else {
-            atomicOr((unsigned*)s_abort, 2u);
-        }
-        const float* rg = reinterpret_cast<const float*>(smem + OFF_REC + be * intra::REC_BYTES + intra::REC_G);
+        wait_buf(bar_rec0, bar_rec1, rec_ok, ce);
+        const float* rg = reinterpret_cast<const float*>(smem + OFF_REC + (ce & 1) * intra::REC_BYTES + intra::REC_G);
         const float g = rg[tid], gl = rg[C - 1];
-        const int64_t te = s0 + (int64_t)ce * C;
-        s_eg[64 * be + tid] = __expf(g);
-        s_ks[tid] = te + tid < s1 ? __expf(gl - g) : 0.f;
+        s_eg[64 * (ce & 1) + tid] = __expf(g);
+        s_ks[tid] = s0 + (int64_t)ce * C + tid < s1 ? __expf(gl - g) : 0.f;
     };
 
-    // Shared-memory descriptors (thread 0 issues every MMA); per-step offsets are
-    // added to the start-address field (addresses stay below 256 KiB).
-    const uint64_t dV = sdesc(sb + OFF_V, 8192, 1024);
-    const uint64_t dS = sdesc(sb + OFF_S16, 16, 1024);
-    const uint64_t dQ = sdesc(sb + OFF_QK, 16, 1024);
-    const uint64_t dUT = sdesc(sb + OFF_UT, 16, 1024);
+    // Shared-memory descriptors; per-step offsets are added to the start-address field.
+    const uint64_t dV0 = sdesc(sb + OFF_QKV + QKV_V, 8192, 1024);
+    const uint64_t dQ0 = sdesc(sb + OFF_QKV, 16, 1024);
     const uint64_t dKT = sdesc(sb + OFF_KT, 8192, 1024);
     const uint64_t dT0 = sdesc(sb + OFF_REC + intra::REC_T, 16, 1024);
     const uint64_t dW0 = sdesc(sb + OFF_REC + intra::REC_W, 8192, 1024);
     const uint64_t dP0 = sdesc(sb + OFF_REC + intra::REC_P, 16, 1024);
-    constexpr uint64_t kRecStep = intra::REC_BYTES >> 4;
+    constexpr uint64_t kRecStep = intra::REC_BYTES >> 4, kQkvStep = QKV_STRIDE >> 4;
     constexpr uint32_t ID_MK = idesc_f16(128, 64, 1, 0), ID_KM = idesc_f16(128, 64, 0, 1);
     constexpr uint32_t ID_KK = idesc_f16(128, 64, 0, 0), ID_KM128 = idesc_f16(128, 128, 0, 1);
 
+    write_sa();
     if (tid < C) chunk_vectors(0);
+    tc_fence_before();
     __syncthreads();
     if (*s_abort) goto abort_;
 
@@ -238,79 +241,79 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     for (int ci = 0; ci < nchunks; ci++) {
         const int b = ci & 1;
-        const uint64_t rs = b ? kRecStep : 0;
+        const uint64_t rs = b ? kRecStep : 0, qs = b ? kQkvStep : 0;
+        const uint32_t qkv = sb + OFF_QKV + b * QKV_STRIDE;
 
-        // ---- (c) U^T = V^T T^T, (d) U^T += S (-W)^T, (e) O1^T = S Q^T ----
+        // ---- (c) U^T = V^T T^T, (d) U^T += S (-W)^T ----
+        wait_buf(bar_qkv0, bar_qkv1, qkv_ok, ci);   // every thread reads the q, k rows below
         if (tid == 0) {
-            if (mbar_wait_bounded(bar_qkv, ci & 1)) qkv_ok++; else atomicOr((unsigned*)s_abort, 2u);
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 4; ks++)
-                mma_f16(tmem + ACC_U, dV + ks * 128, dT0 + rs + ks * 2, ID_MK, ks > 0);
+            for (int ks = 0; ks < 4; ks++) mma_f16(tmem + ACC_U, dV0 + qs + ks * 128, dT0 + rs + ks * 2, ID_MK, ks > 0);
 #pragma unroll
-            for (int ks = 0; ks < 8; ks++)
-                mma_f16(tmem + ACC_U, dS + (ks >> 2) * 1024 + (ks & 3) * 2, dW0 + rs + ks * 128, ID_KM, 1);
-#pragma unroll
-            for (int ks = 0; ks < 8; ks++)
-                mma_f16(tmem + ACC_O1 + 64 * b, dS + (ks >> 2) * 1024 + (ks & 3) * 2,
-                        dQ + (ks >> 2) * 1024 + (ks & 3) * 2, ID_KK, ks > 0);
+            for (int ks = 0; ks < 8; ks++) mma_f16_ta(tmem + ACC_U, tmem + TA_S + ks * 8, dW0 + rs + ks * 128, ID_KM, 1);
             mma_commit(bar);
         }
-        // ---- the previous chunk's o tile, while (c, d, e) run ----
+        // ---- while they run: the previous o tile; Q~ = diag(e^g) Q in place, K~ ----
         if (ci > 0) stage_o(ci - 1);
+        for (int idx = tid; idx < 2 * C * 16; idx += NT) {
+            const int isk = idx >= C * 16;
+            const int r = (idx & (C * 16 - 1)) >> 4, c16 = idx & 15;
+            const int hf = c16 >> 3, cc = c16 & 7;
+            const uint32_t src = qkv + hf * 16384 + swz128(isk * C + r, cc);
+            const uint4 x = scale8(lds128(src), isk ? s_ks[r] : s_eg[64 * b + r]);
+            const uint32_t dst = isk ? sb + OFF_KT + hf * 8192 + swz128(r, cc) : src;
+            sts128(dst, x.x, x.y, x.z, x.w);
+        }
+        fence_async_smem();
         GDN_MMA_WAIT();
         if (tid == 0 && ci > 0) issue_o(ci - 1);
 
-        // ---- K~ = diag(e^{g_C - g}) K, and U^T -> fp16 ----
-        for (int idx = tid; idx < C * 16; idx += NT) {
-            const int r = idx >> 4, c16 = idx & 15;
-            const int hf = c16 >> 3, cc = c16 & 7;
-            const uint4 kt = scale8(lds128(sb + OFF_QK + hf * 16384 + swz128(C + r, cc)), s_ks[r]);
-            sts128(sb + OFF_KT + hf * 8192 + swz128(r, cc), kt.x, kt.y, kt.z, kt.w);
-        }
+        // ---- U^T -> fp16 A operand in TMEM ----
         {
-            uint32_t r16[16];
+            uint32_t r16[16], u[8];
             tmem_ld16(tl + ACC_U + 16 * cs, r16);
-            uint32_t u[8];
 #pragma unroll
             for (int i = 0; i < 8; i++) u[i] = pack_half2(__uint_as_float(r16[2 * i]), __uint_as_float(r16[2 * i + 1]));
-            sts128(sb + OFF_UT + swz128(dv_r, 2 * cs), u[0], u[1], u[2], u[3]);
-            sts128(sb + OFF_UT + swz128(dv_r, 2 * cs + 1), u[4], u[5], u[6], u[7]);
+            tmem_st8(tl + TA_U + 8 * cs, u);
         }
-        fence_async_smem();
         tc_fence_before();
         __syncthreads();
 
-        // ---- (f) O2^T = U^T P^T, (g) increment = U^T K~ ----
+        // ---- (e) O^T = S Q~^T, (f) O^T += U^T P^T, (g) increment = U^T K~ ----
         if (tid == 0) {
             tc_fence_after();
+            const uint32_t dO = tmem + ACC_O + 64 * b;
+#pragma unroll
+            for (int ks = 0; ks < 8; ks++)
+                mma_f16_ta(dO, tmem + TA_S + ks * 8, dQ0 + qs + (ks >> 2) * 1024 + (ks & 3) * 2, ID_KK, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ks++) mma_f16_ta(dO, tmem + TA_U + ks * 8, dP0 + rs + ks * 2, ID_KK, 1);
 #pragma unroll
             for (int ks = 0; ks < 4; ks++)
-                mma_f16(tmem + ACC_O2 + 64 * b, dUT + ks * 2, dP0 + rs + ks * 2, ID_KK, ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ks++)
-                mma_f16(tmem + ACC_SI, dUT + ks * 2, dKT + ks * 128, ID_KM128, ks > 0);
+                mma_f16_ta(tmem + ACC_SI, tmem + TA_U + ks * 8, dKT + ks * 128, ID_KM128, ks > 0);
             mma_commit(bar);
-            if (ci + 1 < nchunks) issue_qkv(ci + 1);   // q, k, v tiles consumed: fetch the next chunk's
         }
         GDN_MMA_WAIT();
-        if (tid == 0 && ci + 2 < nchunks) issue_rec(ci + 2);   // record buffer b consumed
+        if (tid == 0) {   // buffers of chunk ci consumed: fetch chunk ci + 2's tiles and record
+            if (ci + 2 < nchunks) {
+                fence_async_smem();
+                issue_qkv(ci + 2);
+                issue_rec(ci + 2);
+            }
+            if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();   // next staging buffer read
+        }
 
-        // ---- S <- e^{g_C} S + U^T K~ and its fp16 copy; next chunk's vectors ----
+        // ---- S <- e^{g_C} S + U^T K~ and its fp16 A operand; next chunk's vectors ----
         {
             const float eg = s_eg[64 * b + C - 1];
             uint32_t r32[32];
             tmem_ld32(tl + ACC_SI + 32 * cs, r32);
 #pragma unroll
             for (int i = 0; i < 32; i++) S[i] = fmaf(eg, S[i], __uint_as_float(r32[i]));
-            write_s16();
+            write_sa();
         }
         if (tid < C && ci + 1 < nchunks) chunk_vectors(ci + 1);
-        // the staging buffer the next chunk writes has been read by its last bulk store
-        if (tid == 0) {
-            if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();
-        }
-        fence_async_smem();
         tc_fence_before();
         __syncthreads();
         if (*s_abort) goto abort_;
@@ -341,9 +344,10 @@ abort_:
     // recurrent state is left as it was.
     if (tid == 0) {
         record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));
-        for (int k = qkv_ok; k < qkv_issued; k++) mbar_wait_bounded(bar_qkv, k & 1);
-        for (int k = rec0_ok; k < rec0_issued; k++) mbar_wait_bounded(bar_rec0, k & 1);
-        for (int k = rec1_ok; k < rec1_issued; k++) mbar_wait_bounded(bar_rec1, k & 1);
+        for (int bb = 0; bb < 2; bb++) {
+            for (int k = qkv_ok[bb]; k < qkv_issued[bb]; k++) mbar_wait_bounded(bb ? bar_qkv1 : bar_qkv0, k & 1);
+            for (int k = rec_ok[bb]; k < rec_issued[bb]; k++) mbar_wait_bounded(bb ? bar_rec1 : bar_rec0, k & 1);
+        }
         bulk_wait<0>();
     }
     if (warp == 0) {

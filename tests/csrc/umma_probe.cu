@@ -6,6 +6,9 @@
 //   variant 1: A MN-major (M=128, K=64),  B K-major  (N=64,  K=64)
 //   variant 2: A K-major  (M=128, K=128), B MN-major (N=64,  K=128)
 //   variant 3: A K-major  (M=128, K=64),  B MN-major (N=128, K=64)
+//   variant 4: A in TMEM  (M=128, K=128), B K-major  (N=64,  K=128)
+//   variant 5: A in TMEM  (M=128, K=64),  B MN-major (N=128, K=64)
+//   variant 6: A in TMEM  (M=128, K=128), B MN-major (N=64,  K=128)
 #include "../../hybrid_linear_attention_mixer_b200/csrc/device.cuh"
 
 using namespace gdn;
@@ -19,13 +22,14 @@ __global__ void __launch_bounds__(128, 1) umma_probe_kernel(int variant, const f
     const uint32_t sb = (r0 + 1023u) & ~1023u;
     uint8_t* sm = raw + (sb - r0);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int K = (variant == 0 || variant == 2) ? 128 : 64;
-    const int N = variant == 3 ? 128 : 64;
-    const int a_mn = variant == 1, b_mn = variant >= 2;
+    const int K = (variant == 0 || variant == 2 || variant == 4 || variant == 6) ? 128 : 64;
+    const int N = (variant == 3 || variant == 5) ? 128 : 64;
+    const int a_tm = variant >= 4;
+    const int a_mn = variant == 1, b_mn = variant == 2 || variant == 3 || variant == 5 || variant == 6;
     const uint32_t lbo_a = 8192;            // MN-major A: 64 K-rows x 128 B per MN half
     const uint32_t lbo_b = (uint32_t)K * 128;  // MN-major B: K rows x 128 B per MN half
     const uint32_t half_b = (uint32_t)N * 128; // K-major B: N rows x 128 B per K half
-    for (int idx = tid; idx < 128 * K; idx += 128) {
+    for (int idx = tid; idx < 128 * K && !a_tm; idx += 128) {
         const int m = idx / K, k = idx % K;
         const uint32_t off = a_mn ? (m / 64) * lbo_a + swz128(k, (m % 64) / 8) + (m % 8) * 2
                                   : (k / 64) * 16384 + swz128(m, (k % 64) / 8) + (k % 8) * 2;
@@ -44,7 +48,7 @@ __global__ void __launch_bounds__(128, 1) umma_probe_kernel(int variant, const f
         fence_mbar_init();
     }
     if (warp == 0) {
-        tmem_alloc(sb + BAR_OFF + 8, 128);
+        tmem_alloc(sb + BAR_OFF + 8, 256);
         tmem_relinquish();
     }
     fence_async_smem();
@@ -52,12 +56,30 @@ __global__ void __launch_bounds__(128, 1) umma_probe_kernel(int variant, const f
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *slot;
+    const uint32_t a_col = 128;   // A operand columns start here when it lives in TMEM
+    if (a_tm) {   // row m = lane m (thread m); columns hold fp16 pairs (k even in the low half)
+        const uint32_t lane_addr = tmem + ((uint32_t)(32 * warp) << 16) + a_col;
+        const int row = 32 * warp + lane;
+        for (int c0 = 0; c0 < K / 2; c0 += 16) {
+            uint32_t r[16];
+            for (int i = 0; i < 16; i++)
+                r[i] = pack_half2(A[row * K + 2 * (c0 + i)], A[row * K + 2 * (c0 + i) + 1]);
+            tmem_st16(lane_addr + c0, r);
+        }
+        tc_fence_before();
+        __syncthreads();
+        tc_fence_after();
+    }
     if (tid == 0) {
         for (int ks = 0; ks < K / 16; ks++) {
             const uint32_t aa = a_mn ? sb + A_OFF + ks * 2048 : sb + A_OFF + (ks >> 2) * 16384 + (ks & 3) * 32;
             const uint32_t ba = b_mn ? sb + B_OFF + ks * 2048 : sb + B_OFF + (ks >> 2) * half_b + (ks & 3) * 32;
-            mma_f16(tmem, sdesc(aa, a_mn ? lbo_a : 16, 1024), sdesc(ba, b_mn ? lbo_b : 16, 1024),
-                    idesc_f16(128, N, a_mn, b_mn), ks > 0);
+            if (a_tm)
+                mma_f16_ta(tmem, tmem + a_col + ks * 8, sdesc(ba, b_mn ? lbo_b : 16, 1024),
+                           idesc_f16(128, N, 0, b_mn), ks > 0);
+            else
+                mma_f16(tmem, sdesc(aa, a_mn ? lbo_a : 16, 1024), sdesc(ba, b_mn ? lbo_b : 16, 1024),
+                        idesc_f16(128, N, a_mn, b_mn), ks > 0);
         }
         mma_commit(bar);
     }
@@ -77,13 +99,13 @@ __global__ void __launch_bounds__(128, 1) umma_probe_kernel(int variant, const f
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
-        tmem_dealloc(tmem, 128);
+        tmem_dealloc(tmem, 256);
     }
 }
 }  // namespace
 
 extern "C" int umma_probe(int variant, const float* A, const float* B, float* D) {
-    if (variant < 0 || variant > 3) return 1;
+    if (variant < 0 || variant > 6) return 1;
     const int smem = 65536 + 64 + 1024;
     if (cudaFuncSetAttribute(umma_probe_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
         return 2;

@@ -39,9 +39,11 @@ def _probe():
     return lib
 
 
-@pytest.mark.parametrize("variant,K,N", [(0, 128, 64), (1, 64, 64), (2, 128, 64), (3, 64, 128)])
+@pytest.mark.parametrize("variant,K,N", [(0, 128, 64), (1, 64, 64), (2, 128, 64), (3, 64, 128),
+                                         (4, 128, 64), (5, 64, 128), (6, 128, 64)])
 def test_tcgen05_operand_layouts(variant, K, N):
-    """Each K-major / MN-major operand form used by the prefill kernel multiplies correctly."""
+    """Each operand form the prefill kernels use multiplies correctly: K-major and
+    MN-major shared-memory tiles, and A read from tensor memory."""
     lib = _probe()
     rng = np.random.default_rng(variant)
     A = rng.normal(size=(128, K)).astype(np.float32)
