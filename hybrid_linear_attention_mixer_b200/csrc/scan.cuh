@@ -13,19 +13,22 @@
 //
 // Products (tcgen05.mma kind::f16, fp16 operands, fp32 accumulators in TMEM,
 // M = 128 = d_v always, the chunk is the N side):
-//   (c) V^T T^T           -> U^T accumulator        [A: V in shared memory, MN-major]
-//   (d) S (-W)^T          accumulated into (c)       [A: S in TMEM; B: -W, MN-major]
+//   (c) V^T T^T           -> U1^T                    [A: V in shared memory, MN-major]
+//   (d) S (-W)^T          -> U2^T, U^T = U1^T + U2^T [A: S in TMEM; B: -W, MN-major]
 //   (e) S Q~^T            -> O^T (Q~ = diag(e^g) Q)  [A: S in TMEM]
 //   (f) U^T P^T           accumulated into (e)       [A: U^T in TMEM]
 //   (g) U^T K~            -> state increment, K~ = diag(e^{g_C - g}) K [A: U^T in TMEM]
 // S and U^T live in TMEM as fp16 A operands (written with tcgen05.st), so the
-// tensor cores read only the B tiles from shared memory.  The chain per chunk is
-// (c,d) -> U^T to fp16 -> (e,f,g) -> state update -> S to fp16.  The o tile of
-// chunk c-1 (O double-buffered in TMEM) is formed and stored (one bulk copy)
-// while (c,d) of chunk c run.  q^, k^, v^ tiles (double-buffered) arrive by TMA
-// a chunk ahead, a chunk's record by one bulk copy two chunks ahead.  One
-// thread issues every MMA and waits on the tensor-core mbarrier; the others
-// meet it at the CTA barrier.
+// tensor cores read only B tiles from shared memory.  MMAs that accumulate into
+// one TMEM accumulator run back to back; (c), (d), (e) and then (f), (g) are
+// issued interleaved across separate accumulators so that they overlap.  The
+// chain per chunk is (c,d,e) -> U^T to fp16 -> (f,g) -> state update -> S to
+// fp16, with the next chunk's Q~ and K~ prepared beside the state update and
+// the o tile of chunk c-1 (O double-buffered in TMEM) formed and stored (one
+// bulk copy) while (c,d,e) of chunk c run.  q^, k^, v^ tiles (double-buffered)
+// and a chunk's record (one bulk copy) are fetched two chunks ahead.  One thread
+// issues every MMA and waits on the tensor-core mbarrier; the others meet it at
+// the CTA barrier.
 #pragma once
 #include "device.cuh"
 #include "intra.cuh"
@@ -44,15 +47,15 @@ constexpr uint32_t QKV_V = 32768;                   //   V: 64 rows x d_v, halve
 constexpr uint32_t OFF_OST = OFF_QKV + 2 * QKV_STRIDE;   // o tile staging: 32 KiB
 constexpr uint32_t OFF_KT = OFF_OST + 32768;        // K~: 64 rows x d_k, halves of 8192
 constexpr uint32_t OFF_EG = OFF_KT + 16384;         // e^g [2][64]
-constexpr uint32_t OFF_KS = OFF_EG + 512;           // e^{g_C - g} [64]
-constexpr uint32_t OFF_BAR = OFF_KS + 256;          // mbarriers, TMEM address, abort flag
+constexpr uint32_t OFF_KS = OFF_EG + 512;           // e^{g_C - g} [2][64]
+constexpr uint32_t OFF_BAR = OFF_KS + 512;          // mbarriers, TMEM address, abort flag
 constexpr uint32_t SMEM_USED = OFF_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// Tensor memory: U^T (64), O^T x2 (128), increment (128), S fp16 A operand (64
-// columns of packed pairs), U^T fp16 A operand (32).
-constexpr uint32_t ACC_U = 0, ACC_O = 64, ACC_SI = 192, TA_S = 320, TA_U = 384, TMEM_COLS = 512;
+// Tensor memory: U1^T, U2^T (64 each), O^T x2 (128), increment (128), S fp16 A
+// operand (64 columns of packed pairs), U^T fp16 A operand (32).
+constexpr uint32_t ACC_U1 = 0, ACC_U2 = 64, ACC_O = 128, ACC_SI = 256, TA_S = 384, TA_U = 448, TMEM_COLS = 512;
 constexpr uint32_t QKV_BYTES = 6 * 8192;
 
 struct Args {
@@ -210,7 +213,24 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         const float* rg = reinterpret_cast<const float*>(smem + OFF_REC + (ce & 1) * intra::REC_BYTES + intra::REC_G);
         const float g = rg[tid], gl = rg[C - 1];
         s_eg[64 * (ce & 1) + tid] = __expf(g);
-        s_ks[tid] = s0 + (int64_t)ce * C + tid < s1 ? __expf(gl - g) : 0.f;
+        s_ks[64 * (ce & 1) + tid] = s0 + (int64_t)ce * C + tid < s1 ? __expf(gl - g) : 0.f;
+    };
+    // Q~ = diag(e^g) Q in place and K~ = diag(e^{g_C - g}) K of chunk ce (all threads)
+    auto scale_qk = [&](int ce) {
+        wait_buf(bar_qkv0, bar_qkv1, qkv_ok, ce);
+        const uint32_t qkv = sb + OFF_QKV + (ce & 1) * QKV_STRIDE;
+        const float* eg = s_eg + 64 * (ce & 1);
+        const float* ks = s_ks + 64 * (ce & 1);
+        for (int idx = tid; idx < 2 * C * 16; idx += NT) {
+            const int isk = idx >= C * 16;
+            const int r = (idx & (C * 16 - 1)) >> 4, c16 = idx & 15;
+            const int hf = c16 >> 3, cc = c16 & 7;
+            const uint32_t src = qkv + hf * 16384 + swz128(isk * C + r, cc);
+            const uint4 x = scale8(lds128(src), isk ? ks[r] : eg[r]);
+            const uint32_t dst = isk ? sb + OFF_KT + hf * 8192 + swz128(r, cc) : src;
+            sts128(dst, x.x, x.y, x.z, x.w);
+        }
+        fence_async_smem();
     };
 
     // Shared-memory descriptors; per-step offsets are added to the start-address field.
@@ -229,6 +249,9 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     tc_fence_before();
     __syncthreads();
     if (*s_abort) goto abort_;
+    scale_qk(0);
+    __syncthreads();
+    if (*s_abort) goto abort_;
 
 #define GDN_MMA_WAIT()                                                                        \
     do {                                                                                      \
@@ -242,56 +265,48 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int ci = 0; ci < nchunks; ci++) {
         const int b = ci & 1;
         const uint64_t rs = b ? kRecStep : 0, qs = b ? kQkvStep : 0;
-        const uint32_t qkv = sb + OFF_QKV + b * QKV_STRIDE;
 
-        // ---- (c) U^T = V^T T^T, (d) U^T += S (-W)^T ----
-        wait_buf(bar_qkv0, bar_qkv1, qkv_ok, ci);   // every thread reads the q, k rows below
+        // ---- (c) U1^T = V^T T^T, (d) U2^T = S (-W)^T, (e) O^T = S Q~^T, interleaved ----
         if (tid == 0) {
             tc_fence_after();
+            const uint32_t dO = tmem + ACC_O + 64 * b;
 #pragma unroll
-            for (int ks = 0; ks < 4; ks++) mma_f16(tmem + ACC_U, dV0 + qs + ks * 128, dT0 + rs + ks * 2, ID_MK, ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 8; ks++) mma_f16_ta(tmem + ACC_U, tmem + TA_S + ks * 8, dW0 + rs + ks * 128, ID_KM, 1);
+            for (int ks = 0; ks < 8; ks++) {
+                if (ks < 4) mma_f16(tmem + ACC_U1, dV0 + qs + ks * 128, dT0 + rs + ks * 2, ID_MK, ks > 0);
+                mma_f16_ta(tmem + ACC_U2, tmem + TA_S + ks * 8, dW0 + rs + ks * 128, ID_KM, ks > 0);
+                mma_f16_ta(dO, tmem + TA_S + ks * 8, dQ0 + qs + (ks >> 2) * 1024 + (ks & 3) * 2, ID_KK, ks > 0);
+            }
             mma_commit(bar);
         }
-        // ---- while they run: the previous o tile; Q~ = diag(e^g) Q in place, K~ ----
+        // ---- while they run: the previous o tile; the next chunk's e^g, e^{g_C - g} ----
         if (ci > 0) stage_o(ci - 1);
-        for (int idx = tid; idx < 2 * C * 16; idx += NT) {
-            const int isk = idx >= C * 16;
-            const int r = (idx & (C * 16 - 1)) >> 4, c16 = idx & 15;
-            const int hf = c16 >> 3, cc = c16 & 7;
-            const uint32_t src = qkv + hf * 16384 + swz128(isk * C + r, cc);
-            const uint4 x = scale8(lds128(src), isk ? s_ks[r] : s_eg[64 * b + r]);
-            const uint32_t dst = isk ? sb + OFF_KT + hf * 8192 + swz128(r, cc) : src;
-            sts128(dst, x.x, x.y, x.z, x.w);
-        }
-        fence_async_smem();
+        if (tid < C && ci + 1 < nchunks) chunk_vectors(ci + 1);
         GDN_MMA_WAIT();
         if (tid == 0 && ci > 0) issue_o(ci - 1);
 
-        // ---- U^T -> fp16 A operand in TMEM ----
+        // ---- U^T = U1^T + U2^T -> fp16 A operand in TMEM ----
         {
-            uint32_t r16[16], u[8];
-            tmem_ld16(tl + ACC_U + 16 * cs, r16);
+            uint32_t r1[16], r2[16], u[8];
+            tmem_ld16(tl + ACC_U1 + 16 * cs, r1);
+            tmem_ld16(tl + ACC_U2 + 16 * cs, r2);
 #pragma unroll
-            for (int i = 0; i < 8; i++) u[i] = pack_half2(__uint_as_float(r16[2 * i]), __uint_as_float(r16[2 * i + 1]));
+            for (int i = 0; i < 8; i++)
+                u[i] = pack_half2(__uint_as_float(r1[2 * i]) + __uint_as_float(r2[2 * i]),
+                                  __uint_as_float(r1[2 * i + 1]) + __uint_as_float(r2[2 * i + 1]));
             tmem_st8(tl + TA_U + 8 * cs, u);
         }
         tc_fence_before();
         __syncthreads();
 
-        // ---- (e) O^T = S Q~^T, (f) O^T += U^T P^T, (g) increment = U^T K~ ----
+        // ---- (f) O^T += U^T P^T, (g) increment = U^T K~, interleaved ----
         if (tid == 0) {
             tc_fence_after();
             const uint32_t dO = tmem + ACC_O + 64 * b;
 #pragma unroll
-            for (int ks = 0; ks < 8; ks++)
-                mma_f16_ta(dO, tmem + TA_S + ks * 8, dQ0 + qs + (ks >> 2) * 1024 + (ks & 3) * 2, ID_KK, ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ks++) mma_f16_ta(dO, tmem + TA_U + ks * 8, dP0 + rs + ks * 2, ID_KK, 1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ks++)
+            for (int ks = 0; ks < 4; ks++) {
+                mma_f16_ta(dO, tmem + TA_U + ks * 8, dP0 + rs + ks * 2, ID_KK, 1);
                 mma_f16_ta(tmem + ACC_SI, tmem + TA_U + ks * 8, dKT + ks * 128, ID_KM128, ks > 0);
+            }
             mma_commit(bar);
         }
         GDN_MMA_WAIT();
@@ -304,7 +319,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();   // next staging buffer read
         }
 
-        // ---- S <- e^{g_C} S + U^T K~ and its fp16 A operand; next chunk's vectors ----
+        // ---- S <- e^{g_C} S + U^T K~ and its fp16 A operand; the next chunk's Q~, K~ ----
         {
             const float eg = s_eg[64 * b + C - 1];
             uint32_t r32[32];
@@ -313,7 +328,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             for (int i = 0; i < 32; i++) S[i] = fmaf(eg, S[i], __uint_as_float(r32[i]));
             write_sa();
         }
-        if (tid < C && ci + 1 < nchunks) chunk_vectors(ci + 1);
+        if (ci + 1 < nchunks) scale_qk(ci + 1);
         tc_fence_before();
         __syncthreads();
         if (*s_abort) goto abort_;
