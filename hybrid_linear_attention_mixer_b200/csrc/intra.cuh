@@ -15,7 +15,7 @@
 // Each (chunk, value head) record written to the workspace holds the operand
 // tiles exactly as the scan kernel's tensor cores read them (128-byte swizzled
 // shared-memory images), so the scan brings a whole record in with one bulk copy:
-//     +0      -W   MN-major [d_k rows][64 chunk columns] fp16   16384 B
+//     +0      -W   K-major  [64 rows c][d_k columns], two 64-wide halves of 8192 B
 //     +16384  T    K-major  [64 rows c][64 columns j]    fp16    8192 B
 //     +24576  P    K-major  [64 rows r][64 columns j]    fp16    8192 B
 //     +32768  g    [64] fp32 (rows past the sequence end repeat the last g)
@@ -339,18 +339,28 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     if (ok && !mbar_wait_bounded(bar, 1)) atomicOr((unsigned*)s_abort, 1u);
     __syncthreads();
     ok = *s_abort == 0;
-    if (ok) {   // -W^T -> the record (row d_k, chunk columns)
+    if (ok) {   // -W^T from TMEM -> fp16 rows [d_k][c] in shared memory (reusing A)
         tc_fence_after();
         uint32_t r32[32];
         tmem_ld32(tl + ACC_W + 32 * half, r32);
         const int row = 32 * qd + lane;
+        uint32_t* wt = reinterpret_cast<uint32_t*>(smem + OFF_A) + row * 33 + 16 * half;   // 132-byte rows
 #pragma unroll
-        for (int c4 = 0; c4 < 4; c4++) {
+        for (int i = 0; i < 16; i++)
+            wt[i] = pack_half2(-__uint_as_float(r32[2 * i]), -__uint_as_float(r32[2 * i + 1]));
+    }
+    __syncthreads();
+    if (ok) {   // -> the record, K-major: 16-byte piece (c, d_k 8q..8q+7) gathers 8 rows of -W^T
+        const __half* wt = reinterpret_cast<const __half*>(smem + OFF_A);
+        for (int idx = tid; idx < C * 16; idx += NT) {
+            const int c = idx >> 4, q8 = idx & 15;
             uint32_t w4[4];
 #pragma unroll
-            for (int i = 0; i < 4; i++)
-                w4[i] = pack_half2(-__uint_as_float(r32[8 * c4 + 2 * i]), -__uint_as_float(r32[8 * c4 + 2 * i + 1]));
-            stg128(rec + REC_W + swz128(row, 4 * half + c4), w4[0], w4[1], w4[2], w4[3]);
+            for (int i = 0; i < 4; i++) {
+                const __half lo = wt[(8 * q8 + 2 * i) * 66 + c], hi = wt[(8 * q8 + 2 * i + 1) * 66 + c];
+                w4[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+            }
+            stg128(rec + REC_W + (q8 >> 3) * 8192 + swz128(c, q8 & 7), w4[0], w4[1], w4[2], w4[3]);
         }
     } else if (tid == 0) {
         record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));

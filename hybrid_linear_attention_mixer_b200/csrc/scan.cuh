@@ -1,34 +1,28 @@
 // State chain of the chunked gated delta rule on the sm_100a tensor cores.
 //
 // One CTA (512 threads) walks one (sequence, value head) chain chunk by chunk
-// (C = 64 tokens) and carries the d_v x d_k fp32 state in registers (row = TMEM
-// lane, a quarter of d_k per warp).  The state-independent factors of every
-// chunk come from the intra-chunk kernel's records (intra.cuh: -W, T, P, g).
-// With S0 the state at the chunk start:
+// (C = 64 tokens).  The state-independent factors of every chunk come from the
+// intra-chunk kernel's records (intra.cuh: -W, T, P, g).  With S0 the state at
+// the chunk start:
 //     U   = T V - W S0^T                                    (exact per-token updates)
 //     O   = (diag(e^g) Q S0^T + P U) / sqrt(d_k)
 //     S_C = e^{g_C} S0 + U^T diag(e^{g_C - g}) K
 // o goes out as [chunk][head][64][128] tiles; the gated RMSNorm that follows
 // runs in norm.cuh, in parallel over all tiles.
 //
-// Products (tcgen05.mma kind::f16, fp16 operands, fp32 accumulators in TMEM,
-// M = 128 = d_v always, the chunk is the N side):
-//   (c) V^T T^T           -> U1^T                    [A: V in shared memory, MN-major]
-//   (d) S (-W)^T          -> U2^T, U^T = U1^T + U2^T [A: S in TMEM; B: -W, MN-major]
-//   (e) S Q~^T            -> O^T (Q~ = diag(e^g) Q)  [A: S in TMEM]
-//   (f) U^T P^T           accumulated into (e)       [A: U^T in TMEM]
-//   (g) U^T K~            -> state increment, K~ = diag(e^{g_C - g}) K [A: U^T in TMEM]
-// S and U^T live in TMEM as fp16 A operands (written with tcgen05.st), so the
-// tensor cores read only B tiles from shared memory.  MMAs that accumulate into
-// one TMEM accumulator run back to back; (c), (d), (e) and then (f), (g) are
-// issued interleaved across separate accumulators so that they overlap.  The
-// chain per chunk is (c,d,e) -> U^T to fp16 -> (f,g) -> state update -> S to
-// fp16, with the next chunk's Q~ and K~ prepared beside the state update and
-// the o tile of chunk c-1 (O double-buffered in TMEM) formed and stored (one
-// bulk copy) while (c,d,e) of chunk c run.  q^, k^, v^ tiles (double-buffered)
-// and a chunk's record (one bulk copy) are fetched two chunks ahead.  One thread
-// issues every MMA and waits on the tensor-core mbarrier; the others meet it at
-// the CTA barrier.
+// A tcgen05.mma costs about the same whatever its N up to 128, so products that
+// share an A operand are fused into one wide-N MMA, and A operands live in TMEM:
+//   MMA1  (c) V^T T^T                   -> U1^T            [A: V, shared memory]
+//         (d,e) S [-W ; Q~]^T, N = 128  -> [U2^T | O^T]     [A: S, TMEM]
+//   MMA2  (f,g) U^T [P ; K~^T]^T, N=192 -> [O^T | S]  (+=)  [A: U^T = U1^T + U2^T, TMEM]
+// with Q~ = diag(e^g) Q and K~ = diag(e^{g_C - g}) K.  The fp32 state S lives in
+// TMEM as an accumulator: before MMA2 it holds e^{g_C} S0, so MMA2 leaves S_C.
+// Per chunk: MMA1 -> U^T to fp16 -> MMA2 -> (new S: its fp16 A copy and the
+// next chunk's decayed accumulator; this chunk's o tile; the next chunk's Q~,
+// K~^T).  Loads are double-buffered and issued two chunks ahead (q, k, v by
+// TMA; -W, T, g of the record by bulk copies); P goes one chunk ahead.  One
+// thread issues every MMA and waits on the tensor-core mbarrier; the others
+// meet it at the CTA barrier.
 #pragma once
 #include "device.cuh"
 #include "intra.cuh"
@@ -38,25 +32,27 @@ namespace scan {
 
 constexpr int C = 64;
 constexpr int NT = 512;   // 16 warps: 4 per TMEM lane quadrant
-constexpr uint32_t REC_COPY = intra::REC_G + 256;   // bytes of a record brought in
 
-constexpr uint32_t OFF_REC = 0;                     // two record buffers of REC_BYTES
-constexpr uint32_t OFF_QKV = 2 * intra::REC_BYTES;  // two buffers of QKV_STRIDE:
-constexpr uint32_t QKV_STRIDE = 49152;              //   [Q;K] 128 rows x d_k (halves of 16384), V
-constexpr uint32_t QKV_V = 32768;                   //   V: 64 rows x d_v, halves of 8192
-constexpr uint32_t OFF_OST = OFF_QKV + 2 * QKV_STRIDE;   // o tile staging: 32 KiB
-constexpr uint32_t OFF_KT = OFF_OST + 32768;        // K~: 64 rows x d_k, halves of 8192
-constexpr uint32_t OFF_EG = OFF_KT + 16384;         // e^g [2][64]
-constexpr uint32_t OFF_KS = OFF_EG + 512;           // e^{g_C - g} [2][64]
-constexpr uint32_t OFF_BAR = OFF_KS + 512;          // mbarriers, TMEM address, abort flag
-constexpr uint32_t SMEM_USED = OFF_BAR + 64;
+// Shared memory (bytes from a 1024-aligned base).  Buffer pairs are indexed by
+// chunk parity.
+constexpr uint32_t OFF_B1 = 0;        // [-W ; Q] x2: per 64-wide d_k half, 64 W rows then 64 Q rows
+constexpr uint32_t B1_STRIDE = 32768;
+constexpr uint32_t OFF_K = OFF_B1 + 2 * B1_STRIDE;   // K x2: 64 token rows x d_k, halves of 8192
+constexpr uint32_t OFF_V = OFF_K + 2 * 16384;        // V x2: 64 token rows x d_v, halves of 8192
+constexpr uint32_t OFF_T = OFF_V + 2 * 16384;        // T x2: 64 x 64
+constexpr uint32_t OFF_B2 = OFF_T + 2 * 8192;        // [P ; K~^T]: 64 P rows then 128 K~^T rows
+constexpr uint32_t OFF_OST = OFF_B2 + 24576;         // o tile staging: 2 x 16 KiB (or 1 x 32 KiB)
+constexpr uint32_t OFF_G = OFF_OST + 32768;          // g [2][64]
+constexpr uint32_t OFF_EG = OFF_G + 512;             // e^g [2][64]
+constexpr uint32_t OFF_KS = OFF_EG + 512;            // e^{g_C - g} [2][64]
+constexpr uint32_t OFF_BAR = OFF_KS + 512;           // mbarriers, TMEM address, abort flag
+constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// Tensor memory: U1^T, U2^T (64 each), O^T x2 (128), increment (128), S fp16 A
-// operand (64 columns of packed pairs), U^T fp16 A operand (32).
-constexpr uint32_t ACC_U1 = 0, ACC_U2 = 64, ACC_O = 128, ACC_SI = 256, TA_S = 384, TA_U = 448, TMEM_COLS = 512;
-constexpr uint32_t QKV_BYTES = 6 * 8192;
+// Tensor memory: U1^T (64) | U2^T (64) | O^T (64) | S (128) | S fp16 A (64) | U^T fp16 A (32)
+constexpr uint32_t ACC_U1 = 0, ACC_U2 = 64, ACC_O = 128, ACC_S = 192, TA_S = 320, TA_U = 384, TMEM_COLS = 512;
+constexpr uint32_t QKV_BYTES = 6 * 8192, REC_BYTES_IN = 2 * 8192 + 8192 + 256;
 
 struct Args {
     float* rec_state;           // [N][Hv][dv][dk] in/out
@@ -70,6 +66,9 @@ struct Args {
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w)
                  : "memory");
+}
+__device__ __forceinline__ void sts16(uint32_t addr, uint16_t x) {
+    asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(x) : "memory");
 }
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
@@ -95,13 +94,15 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sb = (raw + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (sb - raw);
+    float* s_g = reinterpret_cast<float*>(smem + OFF_G);
     float* s_eg = reinterpret_cast<float*>(smem + OFF_EG);
     float* s_ks = reinterpret_cast<float*>(smem + OFF_KS);
-    const uint32_t bar = sb + OFF_BAR;
-    const uint32_t bar_qkv0 = sb + OFF_BAR + 8, bar_qkv1 = sb + OFF_BAR + 16;
-    const uint32_t bar_rec0 = sb + OFF_BAR + 24, bar_rec1 = sb + OFF_BAR + 32;
-    volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 40);
-    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 44);
+    const uint32_t bar = sb + OFF_BAR;                    // tensor-core commits
+    const uint32_t bar_qkv0 = sb + OFF_BAR + 8;           // +8 per parity: q, k, v tiles
+    const uint32_t bar_rec0 = sb + OFF_BAR + 24;          // +8 per parity: -W, T, g
+    const uint32_t bar_p = sb + OFF_BAR + 40;             // P into B2
+    volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 48);
+    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 52);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qd = warp & 3;      // TMEM lane quadrant
@@ -118,66 +119,58 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint8_t* otile0 = static_cast<uint8_t*>(p.o) + first * O_BYTES;
     const int64_t o_stride = (int64_t)Hv * O_BYTES;
 
-    // TMA / bulk loads issued (thread 0) and completed waits on them (each thread
-    // counts its own), for the abort path
+    // Loads issued (thread 0) and completed waits on them (per thread), for the abort path.
     int qkv_issued[2] = {0, 0}, qkv_ok[2] = {0, 0}, rec_issued[2] = {0, 0}, rec_ok[2] = {0, 0};
-    auto issue_qkv = [&](int ci) {
+    int p_issued = 0, p_ok = 0;
+    auto issue_chunk = [&](int ci) {   // q, k, v tiles and -W, T, g of chunk ci into buffer ci & 1
+        const int bb = ci & 1;
         const int t = (int)(s0 + (int64_t)ci * C);
-        const uint32_t bb = (ci & 1) ? bar_qkv1 : bar_qkv0;
-        const uint32_t base = sb + OFF_QKV + (ci & 1) * QKV_STRIDE;
-        if (ci & 1) qkv_issued[1]++; else qkv_issued[0]++;
-        mbar_arrive_expect_tx(bb, QKV_BYTES);
+        const uint32_t b1 = sb + OFF_B1 + bb * B1_STRIDE;
+        qkv_issued[bb]++;
+        mbar_arrive_expect_tx(bar_qkv0 + 8 * bb, QKV_BYTES);
 #pragma unroll
         for (int hf = 0; hf < 2; hf++) {
-            tma_load_3d(base + hf * 16384, &tm_q, 64 * hf, j, t, bb);
-            tma_load_3d(base + hf * 16384 + C * 128, &tm_k, 64 * hf, j, t, bb);
-            tma_load_3d(base + QKV_V + hf * 8192, &tm_v, 64 * hf, h, t, bb);
+            tma_load_3d(b1 + hf * 16384 + C * 128, &tm_q, 64 * hf, j, t, bar_qkv0 + 8 * bb);
+            tma_load_3d(sb + OFF_K + bb * 16384 + hf * 8192, &tm_k, 64 * hf, j, t, bar_qkv0 + 8 * bb);
+            tma_load_3d(sb + OFF_V + bb * 16384 + hf * 8192, &tm_v, 64 * hf, h, t, bar_qkv0 + 8 * bb);
         }
+        const uint8_t* r = rec0 + ci * rec_stride;
+        rec_issued[bb]++;
+        mbar_arrive_expect_tx(bar_rec0 + 8 * bb, REC_BYTES_IN);
+        bulk_g2s(b1, r + intra::REC_W, 8192, bar_rec0 + 8 * bb);
+        bulk_g2s(b1 + 16384, r + intra::REC_W + 8192, 8192, bar_rec0 + 8 * bb);
+        bulk_g2s(sb + OFF_T + bb * 8192, r + intra::REC_T, 8192, bar_rec0 + 8 * bb);
+        bulk_g2s(sb + OFF_G + bb * 256, r + intra::REC_G, 256, bar_rec0 + 8 * bb);
     };
-    auto issue_rec = [&](int ci) {
-        const uint32_t bb = (ci & 1) ? bar_rec1 : bar_rec0;
-        if (ci & 1) rec_issued[1]++; else rec_issued[0]++;
-        mbar_arrive_expect_tx(bb, REC_COPY);
-        bulk_g2s(sb + OFF_REC + (ci & 1) * intra::REC_BYTES, rec0 + ci * rec_stride, REC_COPY, bb);
+    auto issue_p = [&](int ci) {   // P of chunk ci into B2
+        p_issued++;
+        mbar_arrive_expect_tx(bar_p, 8192);
+        bulk_g2s(sb + OFF_B2, rec0 + ci * rec_stride + intra::REC_P, 8192, bar_p);
     };
-    auto wait_buf = [&](uint32_t b0, uint32_t b1, int (&ok)[2], int ci) {
-        const uint32_t bb = (ci & 1) ? b1 : b0;
-        if (mbar_wait_bounded(bb, (ci >> 1) & 1)) {
-            if (ci & 1) ok[1]++; else ok[0]++;
-        } else {
-            atomicOr((unsigned*)s_abort, 2u);
-        }
+    auto wait_par = [&](uint32_t bar0, int (&ok)[2], int ci) {
+        if (mbar_wait_bounded(bar0 + 8 * (ci & 1), (ci >> 1) & 1)) ok[ci & 1]++;
+        else atomicOr((unsigned*)s_abort, 2u);
     };
 
     if (tid == 0) {
         mbar_init(bar, 1);
         mbar_init(bar_qkv0, 1);
-        mbar_init(bar_qkv1, 1);
+        mbar_init(bar_qkv0 + 8, 1);
         mbar_init(bar_rec0, 1);
-        mbar_init(bar_rec1, 1);
+        mbar_init(bar_rec0 + 8, 1);
+        mbar_init(bar_p, 1);
         fence_mbar_init();
         *s_abort = 0;
-        issue_qkv(0);
-        issue_rec(0);
-        if (nchunks > 1) {
-            issue_qkv(1);
-            issue_rec(1);
-        }
+        issue_chunk(0);
+        if (nchunks > 1) issue_chunk(1);
+        issue_p(0);
     }
     if (warp == 0) {
-        tmem_alloc(sb + OFF_BAR + 40, TMEM_COLS);
+        tmem_alloc(sb + OFF_BAR + 48, TMEM_COLS);
         tmem_relinquish();
     }
-
-    // fp32 state: row dv_r, columns [32 cs, 32 cs + 32)
-    const int dv_r = 32 * qd + lane;
-    float S[32];
+    const int dv_r = 32 * qd + lane;   // this thread's state row; columns [32 cs, 32 cs + 32)
     float* gstate = p.rec_state + ((int64_t)seq * Hv + h) * dv * dk;
-#pragma unroll
-    for (int i = 0; i < 32; i++) {
-        const int col = 32 * cs + i;
-        S[i] = (dv_r < dv && col < dk) ? gstate[(int64_t)dv_r * dk + col] : 0.f;
-    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -186,18 +179,56 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const float inv_sqrt_dk = rsqrtf((float)dk);
     uint32_t mphase = 0;
 
-    // S -> fp16 A operand in TMEM: this thread's 32 columns of d_k = 16 packed columns
-    auto write_sa = [&]() {
-        uint32_t r[16];
-#pragma unroll
-        for (int i = 0; i < 16; i++) r[i] = pack_half2(S[2 * i], S[2 * i + 1]);
-        tmem_st16(tl + TA_S + 16 * cs, r);
+    // e^g and e^{g_C - g} (zero past the chunk's end) of chunk ce, threads 0..63
+    auto chunk_vectors = [&](int ce) {
+        wait_par(bar_rec0, rec_ok, ce);
+        const float* rg = s_g + 64 * (ce & 1);
+        const float g = rg[tid], gl = rg[C - 1];
+        s_eg[64 * (ce & 1) + tid] = __expf(g);
+        s_ks[64 * (ce & 1) + tid] = s0 + (int64_t)ce * C + tid < s1 ? __expf(gl - g) : 0.f;
     };
-    // o = O / sqrt(d_k) of chunk ce -> staging buffer; tid 0 stores it with one bulk
-    // copy after the next CTA barrier (issue_o).
+    // New state -> its fp16 A operand and the decayed accumulator (decay * S) of the next chunk
+    auto put_state = [&](const float (&Sv)[32], float decay) {
+        uint32_t h16[16], d0[16], d1[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            h16[i] = pack_half2(Sv[2 * i], Sv[2 * i + 1]);
+            d0[i] = __float_as_uint(decay * Sv[i]);
+            d1[i] = __float_as_uint(decay * Sv[16 + i]);
+        }
+        tmem_st16(tl + TA_S + 16 * cs, h16);
+        tmem_st16(tl + ACC_S + 32 * cs, d0);
+        tmem_st16(tl + ACC_S + 32 * cs + 16, d1);
+    };
+    // Q~ = diag(e^g) Q in place (B1) and K~^T (B2) of chunk ce, all threads
+    auto scale_qk = [&](int ce) {
+        wait_par(bar_qkv0, qkv_ok, ce);
+        const int bb = ce & 1;
+        const float* eg = s_eg + 64 * bb;
+        const float* ks = s_ks + 64 * bb;
+        for (int idx = tid; idx < C * 16; idx += NT) {   // Q rows: 16-byte pieces, in place
+            const int r = idx >> 4, c16 = idx & 15;
+            const uint32_t a = sb + OFF_B1 + bb * B1_STRIDE + (c16 >> 3) * 16384 + swz128(C + r, c16 & 7);
+            const uint4 x = scale8(lds128(a), eg[r]);
+            sts128(a, x.x, x.y, x.z, x.w);
+        }
+        for (int idx = tid; idx < C * 16; idx += NT) {   // K~^T: row d_k, column c (rows 64..191 of B2)
+            const int c = idx >> 4, c16 = idx & 15;
+            const uint4 x = scale8(lds128(sb + OFF_K + bb * 16384 + (c16 >> 3) * 8192 + swz128(c, c16 & 7)), ks[c]);
+            const uint32_t v[4] = {x.x, x.y, x.z, x.w};
+#pragma unroll
+            for (int e = 0; e < 8; e++) {
+                const int d = 8 * c16 + e;
+                const uint16_t hv = (uint16_t)(v[e >> 1] >> (16 * (e & 1)));
+                sts16(sb + OFF_B2 + swz128(C + d, c >> 3) + (c & 7) * 2, hv);
+            }
+        }
+        fence_async_smem();
+    };
+    // o = O / sqrt(d_k) of chunk ce -> staging; tid 0 stores it after the next barrier
     auto stage_o = [&](int ce) {
         uint32_t o[16];
-        tmem_ld16(tl + ACC_O + 64 * (ce & 1) + 16 * cs, o);
+        tmem_ld16(tl + ACC_O + 16 * cs, o);
         TO* st = reinterpret_cast<TO*>(smem + OFF_OST + (ce % kOBufs) * 16384);
 #pragma unroll
         for (int i = 0; i < 16; i++) from_f32(__uint_as_float(o[i]) * inv_sqrt_dk, st + (16 * cs + i) * 128 + dv_r);
@@ -207,49 +238,35 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         bulk_s2g(otile0 + ce * o_stride, sb + OFF_OST + (ce % kOBufs) * 16384, O_BYTES);
         bulk_commit();
     };
-    // e^g and e^{g_C - g} (zero past the chunk's end) of chunk ce, threads 0..63
-    auto chunk_vectors = [&](int ce) {
-        wait_buf(bar_rec0, bar_rec1, rec_ok, ce);
-        const float* rg = reinterpret_cast<const float*>(smem + OFF_REC + (ce & 1) * intra::REC_BYTES + intra::REC_G);
-        const float g = rg[tid], gl = rg[C - 1];
-        s_eg[64 * (ce & 1) + tid] = __expf(g);
-        s_ks[64 * (ce & 1) + tid] = s0 + (int64_t)ce * C + tid < s1 ? __expf(gl - g) : 0.f;
-    };
-    // Q~ = diag(e^g) Q in place and K~ = diag(e^{g_C - g}) K of chunk ce (all threads)
-    auto scale_qk = [&](int ce) {
-        wait_buf(bar_qkv0, bar_qkv1, qkv_ok, ce);
-        const uint32_t qkv = sb + OFF_QKV + (ce & 1) * QKV_STRIDE;
-        const float* eg = s_eg + 64 * (ce & 1);
-        const float* ks = s_ks + 64 * (ce & 1);
-        for (int idx = tid; idx < 2 * C * 16; idx += NT) {
-            const int isk = idx >= C * 16;
-            const int r = (idx & (C * 16 - 1)) >> 4, c16 = idx & 15;
-            const int hf = c16 >> 3, cc = c16 & 7;
-            const uint32_t src = qkv + hf * 16384 + swz128(isk * C + r, cc);
-            const uint4 x = scale8(lds128(src), isk ? ks[r] : eg[r]);
-            const uint32_t dst = isk ? sb + OFF_KT + hf * 8192 + swz128(r, cc) : src;
-            sts128(dst, x.x, x.y, x.z, x.w);
-        }
-        fence_async_smem();
-    };
 
     // Shared-memory descriptors; per-step offsets are added to the start-address field.
-    const uint64_t dV0 = sdesc(sb + OFF_QKV + QKV_V, 8192, 1024);
-    const uint64_t dQ0 = sdesc(sb + OFF_QKV, 16, 1024);
-    const uint64_t dKT = sdesc(sb + OFF_KT, 8192, 1024);
-    const uint64_t dT0 = sdesc(sb + OFF_REC + intra::REC_T, 16, 1024);
-    const uint64_t dW0 = sdesc(sb + OFF_REC + intra::REC_W, 8192, 1024);
-    const uint64_t dP0 = sdesc(sb + OFF_REC + intra::REC_P, 16, 1024);
-    constexpr uint64_t kRecStep = intra::REC_BYTES >> 4, kQkvStep = QKV_STRIDE >> 4;
-    constexpr uint32_t ID_MK = idesc_f16(128, 64, 1, 0), ID_KM = idesc_f16(128, 64, 0, 1);
-    constexpr uint32_t ID_KK = idesc_f16(128, 64, 0, 0), ID_KM128 = idesc_f16(128, 128, 0, 1);
+    const uint64_t dV0 = sdesc(sb + OFF_V, 8192, 1024);
+    const uint64_t dT0 = sdesc(sb + OFF_T, 16, 1024);
+    const uint64_t dB10 = sdesc(sb + OFF_B1, 16, 1024);
+    const uint64_t dB2 = sdesc(sb + OFF_B2, 16, 1024);
+    constexpr uint32_t ID_MK = idesc_f16(128, 64, 1, 0);     // (c)
+    constexpr uint32_t ID_DE = idesc_f16(128, 128, 0, 0);    // (d,e)
+    constexpr uint32_t ID_FG = idesc_f16(128, 192, 0, 0);    // (f,g)
 
-    write_sa();
+    // ---- prologue: initial state, chunk 0's vectors and scaled q, k ----
     if (tid < C) chunk_vectors(0);
-    tc_fence_before();
     __syncthreads();
     if (*s_abort) goto abort_;
+    {
+        float Sv[32];
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+            const int col = 32 * cs + i;
+            Sv[i] = (dv_r < dv && col < dk) ? gstate[(int64_t)dv_r * dk + col] : 0.f;
+        }
+        put_state(Sv, s_eg[C - 1]);
+    }
+    if (tid == 0) {   // P(0) must be in B2 before K~^T joins it
+        if (mbar_wait_bounded(bar_p, 0)) p_ok++; else atomicOr((unsigned*)s_abort, 2u);
+    }
+    __syncthreads();
     scale_qk(0);
+    tc_fence_before();
     __syncthreads();
     if (*s_abort) goto abort_;
 
@@ -264,27 +281,23 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     for (int ci = 0; ci < nchunks; ci++) {
         const int b = ci & 1;
-        const uint64_t rs = b ? kRecStep : 0, qs = b ? kQkvStep : 0;
 
-        // ---- (c) U1^T = V^T T^T, (d) U2^T = S (-W)^T, (e) O^T = S Q~^T, interleaved ----
+        // ---- MMA1: (c) U1^T = V^T T^T; (d,e) [U2^T | O^T] = S [-W ; Q~]^T ----
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t dO = tmem + ACC_O + 64 * b;
 #pragma unroll
             for (int ks = 0; ks < 8; ks++) {
-                if (ks < 4) mma_f16(tmem + ACC_U1, dV0 + qs + ks * 128, dT0 + rs + ks * 2, ID_MK, ks > 0);
-                mma_f16_ta(tmem + ACC_U2, tmem + TA_S + ks * 8, dW0 + rs + ks * 128, ID_KM, ks > 0);
-                mma_f16_ta(dO, tmem + TA_S + ks * 8, dQ0 + qs + (ks >> 2) * 1024 + (ks & 3) * 2, ID_KK, ks > 0);
+                if (ks < 4)
+                    mma_f16(tmem + ACC_U1, dV0 + b * 1024 + ks * 128, dT0 + b * 512 + ks * 2, ID_MK, ks > 0);
+                mma_f16_ta(tmem + ACC_U2, tmem + TA_S + ks * 8,
+                           dB10 + b * 2048 + (ks >> 2) * 1024 + (ks & 3) * 2, ID_DE, ks > 0);
             }
             mma_commit(bar);
         }
-        // ---- while they run: the previous o tile; the next chunk's e^g, e^{g_C - g} ----
-        if (ci > 0) stage_o(ci - 1);
-        if (tid < C && ci + 1 < nchunks) chunk_vectors(ci + 1);
+        if (tid < C && ci + 1 < nchunks) chunk_vectors(ci + 1);   // while MMA1 runs
         GDN_MMA_WAIT();
-        if (tid == 0 && ci > 0) issue_o(ci - 1);
 
-        // ---- U^T = U1^T + U2^T -> fp16 A operand in TMEM ----
+        // ---- U^T = U1^T + U2^T -> fp16 A operand ----
         {
             uint32_t r1[16], r2[16], u[8];
             tmem_ld16(tl + ACC_U1 + 16 * cs, r1);
@@ -298,52 +311,52 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tc_fence_before();
         __syncthreads();
 
-        // ---- (f) O^T += U^T P^T, (g) increment = U^T K~, interleaved ----
+        // ---- MMA2: [O^T | S] += U^T [P ; K~^T]^T ----
         if (tid == 0) {
             tc_fence_after();
-            const uint32_t dO = tmem + ACC_O + 64 * b;
 #pragma unroll
-            for (int ks = 0; ks < 4; ks++) {
-                mma_f16_ta(dO, tmem + TA_U + ks * 8, dP0 + rs + ks * 2, ID_KK, 1);
-                mma_f16_ta(tmem + ACC_SI, tmem + TA_U + ks * 8, dKT + ks * 128, ID_KM128, ks > 0);
-            }
+            for (int ks = 0; ks < 4; ks++) mma_f16_ta(tmem + ACC_O, tmem + TA_U + ks * 8, dB2 + ks * 2, ID_FG, 1);
             mma_commit(bar);
+            if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();   // staging buffer of stage_o(ci)
         }
         GDN_MMA_WAIT();
-        if (tid == 0) {   // buffers of chunk ci consumed: fetch chunk ci + 2's tiles and record
-            if (ci + 2 < nchunks) {
-                fence_async_smem();
-                issue_qkv(ci + 2);
-                issue_rec(ci + 2);
-            }
-            if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();   // next staging buffer read
+        if (tid == 0) {   // buffers of chunk ci consumed: fetch chunk ci + 2's; P of chunk ci + 1
+            fence_async_smem();
+            if (ci + 2 < nchunks) issue_chunk(ci + 2);
+            if (ci + 1 < nchunks) issue_p(ci + 1);
         }
 
-        // ---- S <- e^{g_C} S + U^T K~ and its fp16 A operand; the next chunk's Q~, K~ ----
+        // ---- new state: fp16 A operand and the next chunk's decayed accumulator; o tile ----
         {
-            const float eg = s_eg[64 * b + C - 1];
             uint32_t r32[32];
-            tmem_ld32(tl + ACC_SI + 32 * cs, r32);
+            tmem_ld32(tl + ACC_S + 32 * cs, r32);
+            float Sv[32];
 #pragma unroll
-            for (int i = 0; i < 32; i++) S[i] = fmaf(eg, S[i], __uint_as_float(r32[i]));
-            write_sa();
+            for (int i = 0; i < 32; i++) Sv[i] = __uint_as_float(r32[i]);
+            if (ci + 1 < nchunks) {
+                put_state(Sv, s_eg[64 * (b ^ 1) + C - 1]);
+            } else {   // the final state
+#pragma unroll
+                for (int i = 0; i < 32; i++) {
+                    const int col = 32 * cs + i;
+                    if (dv_r < dv && col < dk) gstate[(int64_t)dv_r * dk + col] = Sv[i];
+                }
+            }
         }
-        if (ci + 1 < nchunks) scale_qk(ci + 1);
+        stage_o(ci);
+        if (ci + 1 < nchunks) {
+            if (tid == 0) {   // P of chunk ci + 1 must be in B2 before K~^T joins it
+                if (mbar_wait_bounded(bar_p, (ci + 1) & 1)) p_ok++; else atomicOr((unsigned*)s_abort, 2u);
+            }
+            __syncthreads();
+            scale_qk(ci + 1);
+        }
         tc_fence_before();
         __syncthreads();
         if (*s_abort) goto abort_;
+        if (tid == 0) issue_o(ci);
     }
-    stage_o(nchunks - 1);
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0) issue_o(nchunks - 1);
 
-    // ---- final state ----
-#pragma unroll
-    for (int i = 0; i < 32; i++) {
-        const int col = 32 * cs + i;
-        if (dv_r < dv && col < dk) gstate[(int64_t)dv_r * dk + col] = S[i];
-    }
     if (tid == 0) bulk_wait<0>();   // every o tile has reached global memory
     tc_fence_before();
     __syncthreads();
@@ -360,9 +373,10 @@ abort_:
     if (tid == 0) {
         record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));
         for (int bb = 0; bb < 2; bb++) {
-            for (int k = qkv_ok[bb]; k < qkv_issued[bb]; k++) mbar_wait_bounded(bb ? bar_qkv1 : bar_qkv0, k & 1);
-            for (int k = rec_ok[bb]; k < rec_issued[bb]; k++) mbar_wait_bounded(bb ? bar_rec1 : bar_rec0, k & 1);
+            for (int k = qkv_ok[bb]; k < qkv_issued[bb]; k++) mbar_wait_bounded(bar_qkv0 + 8 * bb, k & 1);
+            for (int k = rec_ok[bb]; k < rec_issued[bb]; k++) mbar_wait_bounded(bar_rec0 + 8 * bb, k & 1);
         }
+        for (int k = p_ok; k < p_issued; k++) mbar_wait_bounded(bar_p, k & 1);
         bulk_wait<0>();
     }
     if (warp == 0) {
