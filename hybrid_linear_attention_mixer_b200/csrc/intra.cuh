@@ -17,7 +17,7 @@
 // shared-memory images), so the scan brings a whole record in with one bulk copy:
 //     +0      -W   K-major  [64 rows c][d_k columns], two 64-wide halves of 8192 B
 //     +16384  T    K-major  [64 rows c][64 columns j]    fp16    8192 B
-//     +24576  P    K-major  [64 rows r][64 columns j]    fp16    8192 B
+//     +24576  P^T  MN-major [64 rows j][64 columns r]    fp16    8192 B
 //     +32768  g    [64] fp32 (rows past the sequence end repeat the last g)
 #pragma once
 #include "device.cuh"
@@ -201,8 +201,7 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     tc_fence_after();
     if (tid >= 32 && tid < C) s_g[tid] += s_g[31];
-    for (int i = tid; i < 64 * LDA / 4; i += NT)   // X starts as zero above its diagonal blocks
-        reinterpret_cast<float4*>(Xm)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+
     const uint32_t tmem = *s_tmem;
     const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
     if (!mbar_wait_bounded(bar_ld, 0)) atomicOr((unsigned*)s_abort, 2u);
@@ -232,21 +231,18 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         uint32_t r32[32];
         tmem_ld32(tl + ACC_QK + 32 * half, r32);
         const int j0 = 32 * half;
-        if (qd < 2) {   // P rows -> the record
+        if (qd < 2) {   // P rows -> fp16 rows [r][j] in shared memory (the X region, 132-byte rows)
             const int r = 32 * qd + lane;
             const float gr = s_g[r];
-            uint32_t pk[16];
+            uint32_t* pr = reinterpret_cast<uint32_t*>(Xm) + r * 33 + j0 / 2;
 #pragma unroll
             for (int i = 0; i < 16; i++) {
                 const int jj = j0 + 2 * i;
                 const float e0 = __expf(fminf(gr - s_g[jj], 0.f));
                 const float e1 = __expf(fminf(gr - s_g[jj + 1], 0.f));
-                pk[i] = pack_half2(jj <= r ? __uint_as_float(r32[2 * i]) * e0 : 0.f,
+                pr[i] = pack_half2(jj <= r ? __uint_as_float(r32[2 * i]) * e0 : 0.f,
                                    jj + 1 <= r ? __uint_as_float(r32[2 * i + 1]) * e1 : 0.f);
             }
-#pragma unroll
-            for (int c4 = 0; c4 < 4; c4++)
-                stg128(rec + REC_P + swz128(r, j0 / 8 + c4), pk[4 * c4], pk[4 * c4 + 1], pk[4 * c4 + 2], pk[4 * c4 + 3]);
         } else {        // A rows -> shared memory
             const int r = 32 * (qd - 2) + lane;
             const float gr = s_g[r], br = s_b[r];
@@ -264,6 +260,24 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
     }
     tc_fence_before();
+    __syncthreads();
+
+    if (ok) {   // P^T -> the record (MN-major B image: row j holds P[0..63][j])
+        const __half* pr = reinterpret_cast<const __half*>(Xm);
+        for (int idx = tid; idx < C * 8; idx += NT) {
+            const int jj = idx >> 3, q8 = idx & 7;
+            uint32_t w4[4];
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                const __half lo = pr[(8 * q8 + 2 * i) * 66 + jj], hi = pr[(8 * q8 + 2 * i + 1) * 66 + jj];
+                w4[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
+            }
+            stg128(rec + REC_P + swz128(jj, q8), w4[0], w4[1], w4[2], w4[3]);
+        }
+    }
+    __syncthreads();
+    for (int i = tid; i < 64 * LDA / 4; i += NT)   // X starts as zero above its diagonal blocks
+        reinterpret_cast<float4*>(Xm)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncthreads();
 
     // ---- X = (I + A)^-1, unit lower triangular, fp32 ----

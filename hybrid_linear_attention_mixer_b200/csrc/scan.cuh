@@ -14,12 +14,13 @@
 // share an A operand are fused into one wide-N MMA, and A operands live in TMEM:
 //   MMA1  (c) V^T T^T                   -> U1^T            [A: V, shared memory]
 //         (d,e) S [-W ; Q~]^T, N = 128  -> [U2^T | O^T]     [A: S, TMEM]
-//   MMA2  (f,g) U^T [P ; K~^T]^T, N=192 -> [O^T | S]  (+=)  [A: U^T = U1^T + U2^T, TMEM]
+//   MMA2  (f,g) U^T [P ; K~^T]^T, N=192 -> [O^T | S]  (+=)  [A: U^T = U1^T + U2^T, TMEM;
+//                                                          B: [P^T | K~] MN-major]
 // with Q~ = diag(e^g) Q and K~ = diag(e^{g_C - g}) K.  The fp32 state S lives in
 // TMEM as an accumulator: before MMA2 it holds e^{g_C} S0, so MMA2 leaves S_C.
 // Per chunk: MMA1 -> U^T to fp16 -> MMA2 -> (new S: its fp16 A copy and the
 // next chunk's decayed accumulator; this chunk's o tile; the next chunk's Q~,
-// K~^T).  Loads are double-buffered and issued two chunks ahead (q, k, v by
+// K~).  Loads are double-buffered and issued two chunks ahead (q, k, v by
 // TMA; -W, T, g of the record by bulk copies); P goes one chunk ahead.  One
 // thread issues every MMA and waits on the tensor-core mbarrier; the others
 // meet it at the CTA barrier.
@@ -40,7 +41,7 @@ constexpr uint32_t B1_STRIDE = 32768;
 constexpr uint32_t OFF_K = OFF_B1 + 2 * B1_STRIDE;   // K x2: 64 token rows x d_k, halves of 8192
 constexpr uint32_t OFF_V = OFF_K + 2 * 16384;        // V x2: 64 token rows x d_v, halves of 8192
 constexpr uint32_t OFF_T = OFF_V + 2 * 16384;        // T x2: 64 x 64
-constexpr uint32_t OFF_B2 = OFF_T + 2 * 8192;        // [P ; K~^T]: 64 P rows then 128 K~^T rows
+constexpr uint32_t OFF_B2 = OFF_T + 2 * 8192;        // MN-major [P^T | K~ half 0 | K~ half 1], 8 KiB each
 constexpr uint32_t OFF_OST = OFF_B2 + 24576;         // o tile staging: 2 x 16 KiB (or 1 x 32 KiB)
 constexpr uint32_t OFF_G = OFF_OST + 32768;          // g [2][64]
 constexpr uint32_t OFF_EG = OFF_G + 512;             // e^g [2][64]
@@ -50,8 +51,9 @@ constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// Tensor memory: U1^T (64) | U2^T (64) | O^T (64) | S (128) | S fp16 A (64) | U^T fp16 A (32)
-constexpr uint32_t ACC_U1 = 0, ACC_U2 = 64, ACC_O = 128, ACC_S = 192, TA_S = 320, TA_U = 384, TMEM_COLS = 512;
+// Tensor memory: U1^T (64) | S fp16 A (64) | U^T fp16 A (32) | - | U2^T (64) | O^T (64) | S (128);
+// [U2^T | O^T | S] sits in one 256-column half so that neither MMA's D crosses it.
+constexpr uint32_t ACC_U1 = 0, TA_S = 64, TA_U = 128, ACC_U2 = 256, ACC_O = 320, ACC_S = 384, TMEM_COLS = 512;
 constexpr uint32_t QKV_BYTES = 6 * 8192, REC_BYTES_IN = 2 * 8192 + 8192 + 256;
 
 struct Args {
@@ -200,7 +202,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_st16(tl + ACC_S + 32 * cs, d0);
         tmem_st16(tl + ACC_S + 32 * cs + 16, d1);
     };
-    // Q~ = diag(e^g) Q in place (B1) and K~^T (B2) of chunk ce, all threads
+    // Q~ = diag(e^g) Q in place (B1) and K~ (B2) of chunk ce, all threads
     auto scale_qk = [&](int ce) {
         wait_par(bar_qkv0, qkv_ok, ce);
         const int bb = ce & 1;
@@ -212,16 +214,11 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const uint4 x = scale8(lds128(a), eg[r]);
             sts128(a, x.x, x.y, x.z, x.w);
         }
-        for (int idx = tid; idx < C * 16; idx += NT) {   // K~^T: row d_k, column c (rows 64..191 of B2)
+        for (int idx = tid; idx < C * 16; idx += NT) {   // K~ rows: 16-byte pieces into B2's K~ halves
             const int c = idx >> 4, c16 = idx & 15;
-            const uint4 x = scale8(lds128(sb + OFF_K + bb * 16384 + (c16 >> 3) * 8192 + swz128(c, c16 & 7)), ks[c]);
-            const uint32_t v[4] = {x.x, x.y, x.z, x.w};
-#pragma unroll
-            for (int e = 0; e < 8; e++) {
-                const int d = 8 * c16 + e;
-                const uint16_t hv = (uint16_t)(v[e >> 1] >> (16 * (e & 1)));
-                sts16(sb + OFF_B2 + swz128(C + d, c >> 3) + (c & 7) * 2, hv);
-            }
+            const uint32_t off = (c16 >> 3) * 8192 + swz128(c, c16 & 7);
+            const uint4 x = scale8(lds128(sb + OFF_K + bb * 16384 + off), ks[c]);
+            sts128(sb + OFF_B2 + 8192 + off, x.x, x.y, x.z, x.w);
         }
         fence_async_smem();
     };
@@ -243,10 +240,10 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint64_t dV0 = sdesc(sb + OFF_V, 8192, 1024);
     const uint64_t dT0 = sdesc(sb + OFF_T, 16, 1024);
     const uint64_t dB10 = sdesc(sb + OFF_B1, 16, 1024);
-    const uint64_t dB2 = sdesc(sb + OFF_B2, 16, 1024);
+    const uint64_t dB2 = sdesc(sb + OFF_B2, 8192, 1024);
     constexpr uint32_t ID_MK = idesc_f16(128, 64, 1, 0);     // (c)
     constexpr uint32_t ID_DE = idesc_f16(128, 128, 0, 0);    // (d,e)
-    constexpr uint32_t ID_FG = idesc_f16(128, 192, 0, 0);    // (f,g)
+    constexpr uint32_t ID_FG = idesc_f16(128, 192, 0, 1);    // (f,g)
 
     // ---- prologue: initial state, chunk 0's vectors and scaled q, k ----
     if (tid < C) chunk_vectors(0);
@@ -261,7 +258,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         put_state(Sv, s_eg[C - 1]);
     }
-    if (tid == 0) {   // P(0) must be in B2 before K~^T joins it
+    if (tid == 0) {   // P(0) must be in B2 before K~ joins it
         if (mbar_wait_bounded(bar_p, 0)) p_ok++; else atomicOr((unsigned*)s_abort, 2u);
     }
     __syncthreads();
@@ -315,7 +312,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         if (tid == 0) {
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 4; ks++) mma_f16_ta(tmem + ACC_O, tmem + TA_U + ks * 8, dB2 + ks * 2, ID_FG, 1);
+            for (int ks = 0; ks < 4; ks++) mma_f16_ta(tmem + ACC_O, tmem + TA_U + ks * 8, dB2 + ks * 128, ID_FG, 1);
             mma_commit(bar);
             if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();   // staging buffer of stage_o(ci)
         }
@@ -345,7 +342,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         stage_o(ci);
         if (ci + 1 < nchunks) {
-            if (tid == 0) {   // P of chunk ci + 1 must be in B2 before K~^T joins it
+            if (tid == 0) {   // P of chunk ci + 1 must be in B2 before K~ joins it
                 if (mbar_wait_bounded(bar_p, (ci + 1) & 1)) p_ok++; else atomicOr((unsigned*)s_abort, 2u);
             }
             __syncthreads();
