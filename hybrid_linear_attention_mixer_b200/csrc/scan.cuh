@@ -20,10 +20,11 @@
 // TMEM as an accumulator: before MMA2 it holds e^{g_C} S0, so MMA2 leaves S_C.
 // Per chunk: MMA1 -> U^T to fp16 -> MMA2 -> (new S: its fp16 A copy and the
 // next chunk's decayed accumulator; this chunk's o tile; the next chunk's Q~,
-// K~).  Loads are double-buffered and issued two chunks ahead (q, k, v by
-// TMA; -W, T, g of the record by bulk copies); P goes one chunk ahead.  One
-// thread issues every MMA and waits on the tensor-core mbarrier; the others
-// meet it at the CTA barrier.
+// K~).  Loads are double-buffered: q, k, v (TMA) and -W, T, g of the record
+// (bulk copies) two chunks ahead, issued while MMA2 runs; P one chunk ahead,
+// issued while MMA1 runs.  Thread 0 issues every MMA and waits on the
+// tensor-core mbarrier; thread 32 issues the loads; the others meet them at the
+// CTA barrier.
 #pragma once
 #include "device.cuh"
 #include "intra.cuh"
@@ -41,8 +42,9 @@ constexpr uint32_t B1_STRIDE = 32768;
 constexpr uint32_t OFF_K = OFF_B1 + 2 * B1_STRIDE;   // K x2: 64 token rows x d_k, halves of 8192
 constexpr uint32_t OFF_V = OFF_K + 2 * 16384;        // V x2: 64 token rows x d_v, halves of 8192
 constexpr uint32_t OFF_T = OFF_V + 2 * 16384;        // T x2: 64 x 64
-constexpr uint32_t OFF_B2 = OFF_T + 2 * 8192;        // MN-major [P^T | K~ half 0 | K~ half 1], 8 KiB each
-constexpr uint32_t OFF_OST = OFF_B2 + 24576;         // o tile staging: 2 x 16 KiB (or 1 x 32 KiB)
+constexpr uint32_t OFF_B2 = OFF_T + 2 * 8192;        // x2: MN-major [P^T | K~ half 0 | K~ half 1], 8 KiB each
+constexpr uint32_t B2_STRIDE = 24576;
+constexpr uint32_t OFF_OST = OFF_B2 + 2 * B2_STRIDE; // o tile staging: 2 x 16 KiB (or 1 x 32 KiB)
 constexpr uint32_t OFF_G = OFF_OST + 32768;          // g [2][64]
 constexpr uint32_t OFF_EG = OFF_G + 512;             // e^g [2][64]
 constexpr uint32_t OFF_KS = OFF_EG + 512;            // e^{g_C - g} [2][64]
@@ -102,9 +104,9 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t bar = sb + OFF_BAR;                    // tensor-core commits
     const uint32_t bar_qkv0 = sb + OFF_BAR + 8;           // +8 per parity: q, k, v tiles
     const uint32_t bar_rec0 = sb + OFF_BAR + 24;          // +8 per parity: -W, T, g
-    const uint32_t bar_p = sb + OFF_BAR + 40;             // P into B2
-    volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 48);
-    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 52);
+    const uint32_t bar_p0 = sb + OFF_BAR + 40;            // +8 per parity: P into B2
+    volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 56);
+    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 60);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qd = warp & 3;      // TMEM lane quadrant
@@ -121,14 +123,14 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint8_t* otile0 = static_cast<uint8_t*>(p.o) + first * O_BYTES;
     const int64_t o_stride = (int64_t)Hv * O_BYTES;
 
-    // Loads issued (thread 0) and completed waits on them (per thread), for the abort path.
-    int qkv_issued[2] = {0, 0}, qkv_ok[2] = {0, 0}, rec_issued[2] = {0, 0}, rec_ok[2] = {0, 0};
-    int p_issued = 0, p_ok = 0;
+    // Loads issued per barrier (qkv x2, record x2, P x2), kept in shared memory: the
+    // abort path waits for the last phase issued on each.
+    volatile int* s_issued = reinterpret_cast<volatile int*>(smem + OFF_BAR + 64);
     auto issue_chunk = [&](int ci) {   // q, k, v tiles and -W, T, g of chunk ci into buffer ci & 1
         const int bb = ci & 1;
         const int t = (int)(s0 + (int64_t)ci * C);
         const uint32_t b1 = sb + OFF_B1 + bb * B1_STRIDE;
-        qkv_issued[bb]++;
+        s_issued[bb]++;
         mbar_arrive_expect_tx(bar_qkv0 + 8 * bb, QKV_BYTES);
 #pragma unroll
         for (int hf = 0; hf < 2; hf++) {
@@ -137,21 +139,21 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             tma_load_3d(sb + OFF_V + bb * 16384 + hf * 8192, &tm_v, 64 * hf, h, t, bar_qkv0 + 8 * bb);
         }
         const uint8_t* r = rec0 + ci * rec_stride;
-        rec_issued[bb]++;
+        s_issued[2 + bb]++;
         mbar_arrive_expect_tx(bar_rec0 + 8 * bb, REC_BYTES_IN);
         bulk_g2s(b1, r + intra::REC_W, 8192, bar_rec0 + 8 * bb);
         bulk_g2s(b1 + 16384, r + intra::REC_W + 8192, 8192, bar_rec0 + 8 * bb);
         bulk_g2s(sb + OFF_T + bb * 8192, r + intra::REC_T, 8192, bar_rec0 + 8 * bb);
         bulk_g2s(sb + OFF_G + bb * 256, r + intra::REC_G, 256, bar_rec0 + 8 * bb);
     };
-    auto issue_p = [&](int ci) {   // P of chunk ci into B2
-        p_issued++;
-        mbar_arrive_expect_tx(bar_p, 8192);
-        bulk_g2s(sb + OFF_B2, rec0 + ci * rec_stride + intra::REC_P, 8192, bar_p);
+    auto issue_p = [&](int ci) {   // P of chunk ci into B2 buffer ci & 1
+        const int bb = ci & 1;
+        s_issued[4 + bb]++;
+        mbar_arrive_expect_tx(bar_p0 + 8 * bb, 8192);
+        bulk_g2s(sb + OFF_B2 + bb * B2_STRIDE, rec0 + ci * rec_stride + intra::REC_P, 8192, bar_p0 + 8 * bb);
     };
-    auto wait_par = [&](uint32_t bar0, int (&ok)[2], int ci) {
-        if (mbar_wait_bounded(bar0 + 8 * (ci & 1), (ci >> 1) & 1)) ok[ci & 1]++;
-        else atomicOr((unsigned*)s_abort, 2u);
+    auto wait_par = [&](uint32_t bar0, int ci) {
+        if (!mbar_wait_bounded(bar0 + 8 * (ci & 1), (ci >> 1) & 1)) atomicOr((unsigned*)s_abort, 2u);
     };
 
     if (tid == 0) {
@@ -160,15 +162,17 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         mbar_init(bar_qkv0 + 8, 1);
         mbar_init(bar_rec0, 1);
         mbar_init(bar_rec0 + 8, 1);
-        mbar_init(bar_p, 1);
+        mbar_init(bar_p0, 1);
+        mbar_init(bar_p0 + 8, 1);
         fence_mbar_init();
         *s_abort = 0;
+        for (int i = 0; i < 6; i++) s_issued[i] = 0;
         issue_chunk(0);
         if (nchunks > 1) issue_chunk(1);
         issue_p(0);
     }
     if (warp == 0) {
-        tmem_alloc(sb + OFF_BAR + 48, TMEM_COLS);
+        tmem_alloc(sb + OFF_BAR + 56, TMEM_COLS);
         tmem_relinquish();
     }
     const int dv_r = 32 * qd + lane;   // this thread's state row; columns [32 cs, 32 cs + 32)
@@ -181,13 +185,14 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const float inv_sqrt_dk = rsqrtf((float)dk);
     uint32_t mphase = 0;
 
-    // e^g and e^{g_C - g} (zero past the chunk's end) of chunk ce, threads 0..63
-    auto chunk_vectors = [&](int ce) {
-        wait_par(bar_rec0, rec_ok, ce);
+    // e^g and e^{g_C - g} (zero past the chunk's end) of chunk ce, by threads r0..r0+63
+    auto chunk_vectors = [&](int ce, int r0) {
+        wait_par(bar_rec0, ce);
+        const int r = tid - r0;
         const float* rg = s_g + 64 * (ce & 1);
-        const float g = rg[tid], gl = rg[C - 1];
-        s_eg[64 * (ce & 1) + tid] = __expf(g);
-        s_ks[64 * (ce & 1) + tid] = s0 + (int64_t)ce * C + tid < s1 ? __expf(gl - g) : 0.f;
+        const float g = rg[r], gl = rg[C - 1];
+        s_eg[64 * (ce & 1) + r] = __expf(g);
+        s_ks[64 * (ce & 1) + r] = s0 + (int64_t)ce * C + r < s1 ? __expf(gl - g) : 0.f;
     };
     // New state -> its fp16 A operand and the decayed accumulator (decay * S) of the next chunk
     auto put_state = [&](const float (&Sv)[32], float decay) {
@@ -204,7 +209,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     };
     // Q~ = diag(e^g) Q in place (B1) and K~ (B2) of chunk ce, all threads
     auto scale_qk = [&](int ce) {
-        wait_par(bar_qkv0, qkv_ok, ce);
+        wait_par(bar_qkv0, ce);
         const int bb = ce & 1;
         const float* eg = s_eg + 64 * bb;
         const float* ks = s_ks + 64 * bb;
@@ -218,7 +223,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int c = idx >> 4, c16 = idx & 15;
             const uint32_t off = (c16 >> 3) * 8192 + swz128(c, c16 & 7);
             const uint4 x = scale8(lds128(sb + OFF_K + bb * 16384 + off), ks[c]);
-            sts128(sb + OFF_B2 + 8192 + off, x.x, x.y, x.z, x.w);
+            sts128(sb + OFF_B2 + bb * B2_STRIDE + 8192 + off, x.x, x.y, x.z, x.w);
         }
         fence_async_smem();
     };
@@ -246,7 +251,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     constexpr uint32_t ID_FG = idesc_f16(128, 192, 0, 1);    // (f,g)
 
     // ---- prologue: initial state, chunk 0's vectors and scaled q, k ----
-    if (tid < C) chunk_vectors(0);
+    if (tid < C) chunk_vectors(0, 0);
     __syncthreads();
     if (*s_abort) goto abort_;
     {
@@ -258,10 +263,6 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         put_state(Sv, s_eg[C - 1]);
     }
-    if (tid == 0) {   // P(0) must be in B2 before K~ joins it
-        if (mbar_wait_bounded(bar_p, 0)) p_ok++; else atomicOr((unsigned*)s_abort, 2u);
-    }
-    __syncthreads();
     scale_qk(0);
     tc_fence_before();
     __syncthreads();
@@ -291,7 +292,10 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
             mma_commit(bar);
         }
-        if (tid < C && ci + 1 < nchunks) chunk_vectors(ci + 1);   // while MMA1 runs
+        // while MMA1 runs: P of chunk ci + 1 (its B2 buffer was freed by MMA2 of chunk ci - 1);
+        // e^g, e^{g_C - g} of chunk ci + 1
+        if (tid == 32 && ci + 1 < nchunks) issue_p(ci + 1);
+        if (tid >= 64 && tid < 64 + C && ci + 1 < nchunks) chunk_vectors(ci + 1, 64);
         GDN_MMA_WAIT();
 
         // ---- U^T = U1^T + U2^T -> fp16 A operand ----
@@ -310,18 +314,19 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
         // ---- MMA2: [O^T | S] += U^T [P ; K~^T]^T ----
         if (tid == 0) {
+            if (!mbar_wait_bounded(bar_p0 + 8 * b, (ci >> 1) & 1)) atomicOr((unsigned*)s_abort, 2u);
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < 4; ks++) mma_f16_ta(tmem + ACC_O, tmem + TA_U + ks * 8, dB2 + ks * 128, ID_FG, 1);
+            for (int ks = 0; ks < 4; ks++)
+                mma_f16_ta(tmem + ACC_O, tmem + TA_U + ks * 8, dB2 + b * (B2_STRIDE >> 4) + ks * 128, ID_FG, 1);
             mma_commit(bar);
             if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();   // staging buffer of stage_o(ci)
         }
-        GDN_MMA_WAIT();
-        if (tid == 0) {   // buffers of chunk ci consumed: fetch chunk ci + 2's; P of chunk ci + 1
+        if (tid == 32 && ci + 2 < nchunks) {   // MMA1 of chunk ci is done with buffer b: fetch chunk ci + 2's
             fence_async_smem();
-            if (ci + 2 < nchunks) issue_chunk(ci + 2);
-            if (ci + 1 < nchunks) issue_p(ci + 1);
+            issue_chunk(ci + 2);
         }
+        GDN_MMA_WAIT();
 
         // ---- new state: fp16 A operand and the next chunk's decayed accumulator; o tile ----
         {
@@ -341,13 +346,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             }
         }
         stage_o(ci);
-        if (ci + 1 < nchunks) {
-            if (tid == 0) {   // P of chunk ci + 1 must be in B2 before K~ joins it
-                if (mbar_wait_bounded(bar_p, (ci + 1) & 1)) p_ok++; else atomicOr((unsigned*)s_abort, 2u);
-            }
-            __syncthreads();
-            scale_qk(ci + 1);
-        }
+        if (ci + 1 < nchunks) scale_qk(ci + 1);
         tc_fence_before();
         __syncthreads();
         if (*s_abort) goto abort_;
@@ -369,11 +368,9 @@ abort_:
     // recurrent state is left as it was.
     if (tid == 0) {
         record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));
-        for (int bb = 0; bb < 2; bb++) {
-            for (int k = qkv_ok[bb]; k < qkv_issued[bb]; k++) mbar_wait_bounded(bar_qkv0 + 8 * bb, k & 1);
-            for (int k = rec_ok[bb]; k < rec_issued[bb]; k++) mbar_wait_bounded(bar_rec0 + 8 * bb, k & 1);
-        }
-        for (int k = p_ok; k < p_issued; k++) mbar_wait_bounded(bar_p, k & 1);
+        const uint32_t bars[6] = {bar_qkv0, bar_qkv0 + 8, bar_rec0, bar_rec0 + 8, bar_p0, bar_p0 + 8};
+        for (int i = 0; i < 6; i++)   // the last phase issued on each barrier (returns at once if complete)
+            if (s_issued[i] > 0) mbar_wait_bounded(bars[i], (uint32_t)(s_issued[i] - 1) & 1u);
         bulk_wait<0>();
     }
     if (warp == 0) {
