@@ -19,6 +19,7 @@
 //     +16384  T    K-major  [64 rows c][64 columns j]    fp16    8192 B
 //     +24576  P^T  MN-major [64 rows j][64 columns r]    fp16    8192 B
 //     +32768  g    [64] fp32 (rows past the sequence end repeat the last g)
+//     +33792  Q~   K-major  [64 rows r][d_k columns] = diag(e^g) Q, two halves of 8192 B
 #pragma once
 #include "device.cuh"
 
@@ -27,8 +28,8 @@ namespace intra {
 
 constexpr int C = 64;
 constexpr int NT = 256;
-constexpr uint32_t REC_W = 0, REC_T = 16384, REC_P = 24576, REC_G = 32768;
-constexpr uint32_t REC_BYTES = 33792;   // 33 x 1024: keeps every tile of a record 1024-aligned
+constexpr uint32_t REC_W = 0, REC_T = 16384, REC_P = 24576, REC_G = 32768, REC_Q = 33792;
+constexpr uint32_t REC_BYTES = 50176;   // 49 x 1024: keeps every tile of a record 1024-aligned
 
 constexpr uint32_t OFF_QK = 0;          // [Q;K]: 128 token rows x d_k, halves of 16384
 constexpr int LDA = 68;                 // fp32 64 x 64 work matrices: 16-byte aligned rows
@@ -211,6 +212,21 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         s_eg[tid] = __expf(s_g[tid]);
     }
     bool ok = *s_abort == 0;
+    __syncthreads();   // e^g
+    if (ok) {   // Q~ = diag(e^g) Q -> the record (same swizzled image as the Q rows here)
+        for (int idx = tid; idx < C * 16; idx += NT) {
+            const int r = idx >> 4, c16 = idx & 15;
+            const uint32_t off = (c16 >> 3) * 16384 + swz128(r, c16 & 7);
+            uint4 v;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(sb + OFF_QK + off));
+            const float e = s_eg[r];
+            const float2 a0 = unpack_half2(v.x), a1 = unpack_half2(v.y), a2 = unpack_half2(v.z), a3 = unpack_half2(v.w);
+            stg128(rec + REC_Q + (c16 >> 3) * 8192 + swz128(r, c16 & 7), pack_half2(a0.x * e, a0.y * e),
+                   pack_half2(a1.x * e, a1.y * e), pack_half2(a2.x * e, a2.y * e), pack_half2(a3.x * e, a3.y * e));
+        }
+    }
 
     // ---- [Q;K] K^T ----
     if (ok && tid == 0) {

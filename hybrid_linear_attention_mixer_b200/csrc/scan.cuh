@@ -2,8 +2,8 @@
 //
 // One CTA (512 threads) walks one (sequence, value head) chain chunk by chunk
 // (C = 64 tokens).  The state-independent factors of every chunk come from the
-// intra-chunk kernel's records (intra.cuh: -W, T, P, g).  With S0 the state at
-// the chunk start:
+// intra-chunk kernel's records (intra.cuh: -W, T, P, g, Q~).  With S0 the state
+// at the chunk start:
 //     U   = T V - W S0^T                                    (exact per-token updates)
 //     O   = (diag(e^g) Q S0^T + P U) / sqrt(d_k)
 //     S_C = e^{g_C} S0 + U^T diag(e^{g_C - g}) K
@@ -12,17 +12,21 @@
 //
 // A tcgen05.mma costs about the same whatever its N up to 128, so products that
 // share an A operand are fused into one wide-N MMA, and A operands live in TMEM:
-//   MMA1  (c) V^T T^T                   -> U1^T            [A: V, shared memory]
-//         (d,e) S [-W ; Q~]^T, N = 128  -> [U2^T | O^T]     [A: S, TMEM]
-//   MMA2  (f,g) U^T [P ; K~^T]^T, N=192 -> [O^T | S]  (+=)  [A: U^T = U1^T + U2^T, TMEM;
-//                                                          B: [P^T | K~] MN-major]
+//   MMA1  (d,e) S [-W ; Q~]^T, N = 128  -> [U2^T | O^T]      [A: S, TMEM]
+//         (c)   V^T T^T,         N = 64  -> U^T += (into U2^T) [A: V, shared memory]
+//   MMA2  (f,g) U^T [P ; K~^T]^T, N=192 -> [O^T | S]  (+=)   [A: U^T, TMEM; B MN-major]
 // with Q~ = diag(e^g) Q and K~ = diag(e^{g_C - g}) K.  The fp32 state S lives in
 // TMEM as an accumulator: before MMA2 it holds e^{g_C} S0, so MMA2 leaves S_C.
-// Per chunk: MMA1 -> U^T to fp16 -> MMA2 -> (new S: its fp16 A copy and the
-// next chunk's decayed accumulator; this chunk's o tile; the next chunk's Q~,
-// K~).  Loads are double-buffered: q, k, v (TMA) and -W, T, g of the record
-// (bulk copies) two chunks ahead, issued while MMA2 runs; P one chunk ahead,
-// issued while MMA1 runs.  Thread 0 issues every MMA and waits on the
+// The operand tiles and the U, O accumulators alternate with chunk parity so
+// that O is double-buffered while both fused MMAs keep contiguous outputs:
+//   parity 0: B1 = [-W ; Q~], B2 = [P^T | K~], TMEM [U2 | O0 | S]
+//   parity 1: B1 = [Q~ ; -W], B2 = [K~ | P^T], TMEM [S | O1 | U2']
+// Per chunk, the critical chain is MMA1 -> U^T to fp16 -> MMA2 -> new S (its
+// fp16 A copy and the next chunk's decayed accumulator).  While MMA1 runs the
+// other threads build K~, write the previous chunk's o tile, and prepare the
+// next chunk's gate vectors.  Loads are double-buffered: k, v (TMA) and the
+// record (bulk copies) two chunks ahead, issued while MMA2 runs; P one chunk
+// ahead, issued while MMA1 runs.  Thread 0 issues every MMA and waits on the
 // tensor-core mbarrier; thread 32 issues the loads; the others meet them at the
 // CTA barrier.
 #pragma once
@@ -35,28 +39,30 @@ namespace scan {
 constexpr int C = 64;
 constexpr int NT = 512;   // 16 warps: 4 per TMEM lane quadrant
 
-// Shared memory (bytes from a 1024-aligned base).  Buffer pairs are indexed by
-// chunk parity.
-constexpr uint32_t OFF_B1 = 0;        // [-W ; Q] x2: per 64-wide d_k half, 64 W rows then 64 Q rows
+// Shared memory (bytes from a 1024-aligned base); pairs are indexed by chunk parity.
+constexpr uint32_t OFF_B1 = 0;          // x2: per 64-wide d_k half (16 KiB), 64 + 64 rows of -W / Q~
 constexpr uint32_t B1_STRIDE = 32768;
 constexpr uint32_t OFF_K = OFF_B1 + 2 * B1_STRIDE;   // K x2: 64 token rows x d_k, halves of 8192
 constexpr uint32_t OFF_V = OFF_K + 2 * 16384;        // V x2: 64 token rows x d_v, halves of 8192
 constexpr uint32_t OFF_T = OFF_V + 2 * 16384;        // T x2: 64 x 64
-constexpr uint32_t OFF_B2 = OFF_T + 2 * 8192;        // x2: MN-major [P^T | K~ half 0 | K~ half 1], 8 KiB each
+constexpr uint32_t OFF_B2 = OFF_T + 2 * 8192;        // x2: three MN-major 8 KiB atoms of P^T and K~
 constexpr uint32_t B2_STRIDE = 24576;
 constexpr uint32_t OFF_OST = OFF_B2 + 2 * B2_STRIDE; // o tile staging: 2 x 16 KiB (or 1 x 32 KiB)
 constexpr uint32_t OFF_G = OFF_OST + 32768;          // g [2][64]
-constexpr uint32_t OFF_EG = OFF_G + 512;             // e^g [2][64]
-constexpr uint32_t OFF_KS = OFF_EG + 512;            // e^{g_C - g} [2][64]
-constexpr uint32_t OFF_BAR = OFF_KS + 512;           // mbarriers, TMEM address, abort flag
+constexpr uint32_t OFF_KS = OFF_G + 512;             // e^{g_C - g} [2][64]
+constexpr uint32_t OFF_BAR = OFF_KS + 512;           // mbarriers, TMEM address, abort flag, counters
 constexpr uint32_t SMEM_USED = OFF_BAR + 128;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 
-// Tensor memory: U1^T (64) | S fp16 A (64) | U^T fp16 A (32) | - | U2^T (64) | O^T (64) | S (128);
-// [U2^T | O^T | S] sits in one 256-column half so that neither MMA's D crosses it.
-constexpr uint32_t ACC_U1 = 0, TA_S = 64, TA_U = 128, ACC_U2 = 256, ACC_O = 320, ACC_S = 384, TMEM_COLS = 512;
-constexpr uint32_t QKV_BYTES = 6 * 8192, REC_BYTES_IN = 2 * 8192 + 8192 + 256;
+// Tensor memory: U2 | O0 | S (128) | O1 | U2' | S fp16 A (64) | U^T fp16 A (32)
+constexpr uint32_t ACC_U0 = 0, ACC_O0 = 64, ACC_S = 128, ACC_O1 = 256, ACC_U1 = 320;
+constexpr uint32_t TA_S = 384, TA_U = 448, TMEM_COLS = 512;
+__host__ __device__ constexpr uint32_t acc_u(int b) { return b ? ACC_U1 : ACC_U0; }
+__host__ __device__ constexpr uint32_t acc_o(int b) { return b ? ACC_O1 : ACC_O0; }
+
+constexpr uint32_t KV_BYTES = 4 * 8192;
+constexpr uint32_t REC_BYTES_IN = 4 * 8192 + 8192 + 256;   // -W, Q~ (two halves each), T, g
 
 struct Args {
     float* rec_state;           // [N][Hv][dv][dk] in/out
@@ -70,9 +76,6 @@ struct Args {
 __device__ __forceinline__ void sts128(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w)
                  : "memory");
-}
-__device__ __forceinline__ void sts16(uint32_t addr, uint16_t x) {
-    asm volatile("st.shared.b16 [%0], %1;" ::"r"(addr), "h"(x) : "memory");
 }
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
@@ -90,8 +93,7 @@ __device__ __forceinline__ uint4 scale8(uint4 v, float s) {
 
 template <typename TO>
 __global__ void __launch_bounds__(NT, 1)
-gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                const __grid_constant__ CUtensorMap tm_v, Args p) {
+gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, Args p) {
     constexpr uint32_t O_BYTES = C * 128 * sizeof(TO);
     constexpr int kOBufs = O_BYTES <= 16384 ? 2 : 1;   // staging buffers for the o tiles
     extern __shared__ uint8_t smem_raw[];
@@ -99,14 +101,15 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint32_t sb = (raw + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (sb - raw);
     float* s_g = reinterpret_cast<float*>(smem + OFF_G);
-    float* s_eg = reinterpret_cast<float*>(smem + OFF_EG);
     float* s_ks = reinterpret_cast<float*>(smem + OFF_KS);
     const uint32_t bar = sb + OFF_BAR;                    // tensor-core commits
-    const uint32_t bar_qkv0 = sb + OFF_BAR + 8;           // +8 per parity: q, k, v tiles
-    const uint32_t bar_rec0 = sb + OFF_BAR + 24;          // +8 per parity: -W, T, g
+    const uint32_t bar_kv0 = sb + OFF_BAR + 8;            // +8 per parity: k, v tiles
+    const uint32_t bar_rec0 = sb + OFF_BAR + 24;          // +8 per parity: -W, Q~, T, g
     const uint32_t bar_p0 = sb + OFF_BAR + 40;            // +8 per parity: P into B2
     volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 56);
     volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 60);
+    // loads issued per barrier (kv x2, record x2, P x2): the abort path waits for the last phase of each
+    volatile int* s_issued = reinterpret_cast<volatile int*>(smem + OFF_BAR + 64);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qd = warp & 3;      // TMEM lane quadrant
@@ -123,34 +126,36 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     uint8_t* otile0 = static_cast<uint8_t*>(p.o) + first * O_BYTES;
     const int64_t o_stride = (int64_t)Hv * O_BYTES;
 
-    // Loads issued per barrier (qkv x2, record x2, P x2), kept in shared memory: the
-    // abort path waits for the last phase issued on each.
-    volatile int* s_issued = reinterpret_cast<volatile int*>(smem + OFF_BAR + 64);
-    auto issue_chunk = [&](int ci) {   // q, k, v tiles and -W, T, g of chunk ci into buffer ci & 1
+    // k, v tiles and the record (-W, Q~, T, g) of chunk ci into buffer ci & 1
+    auto issue_chunk = [&](int ci) {
         const int bb = ci & 1;
         const int t = (int)(s0 + (int64_t)ci * C);
-        const uint32_t b1 = sb + OFF_B1 + bb * B1_STRIDE;
         s_issued[bb]++;
-        mbar_arrive_expect_tx(bar_qkv0 + 8 * bb, QKV_BYTES);
+        mbar_arrive_expect_tx(bar_kv0 + 8 * bb, KV_BYTES);
 #pragma unroll
         for (int hf = 0; hf < 2; hf++) {
-            tma_load_3d(b1 + hf * 16384 + C * 128, &tm_q, 64 * hf, j, t, bar_qkv0 + 8 * bb);
-            tma_load_3d(sb + OFF_K + bb * 16384 + hf * 8192, &tm_k, 64 * hf, j, t, bar_qkv0 + 8 * bb);
-            tma_load_3d(sb + OFF_V + bb * 16384 + hf * 8192, &tm_v, 64 * hf, h, t, bar_qkv0 + 8 * bb);
+            tma_load_3d(sb + OFF_K + bb * 16384 + hf * 8192, &tm_k, 64 * hf, j, t, bar_kv0 + 8 * bb);
+            tma_load_3d(sb + OFF_V + bb * 16384 + hf * 8192, &tm_v, 64 * hf, h, t, bar_kv0 + 8 * bb);
         }
         const uint8_t* r = rec0 + ci * rec_stride;
+        const uint32_t b1 = sb + OFF_B1 + bb * B1_STRIDE;
+        const uint32_t wslot = bb ? 8192 : 0, qslot = bb ? 0 : 8192;   // row order of B1 by parity
         s_issued[2 + bb]++;
         mbar_arrive_expect_tx(bar_rec0 + 8 * bb, REC_BYTES_IN);
-        bulk_g2s(b1, r + intra::REC_W, 8192, bar_rec0 + 8 * bb);
-        bulk_g2s(b1 + 16384, r + intra::REC_W + 8192, 8192, bar_rec0 + 8 * bb);
+#pragma unroll
+        for (int hf = 0; hf < 2; hf++) {
+            bulk_g2s(b1 + hf * 16384 + wslot, r + intra::REC_W + hf * 8192, 8192, bar_rec0 + 8 * bb);
+            bulk_g2s(b1 + hf * 16384 + qslot, r + intra::REC_Q + hf * 8192, 8192, bar_rec0 + 8 * bb);
+        }
         bulk_g2s(sb + OFF_T + bb * 8192, r + intra::REC_T, 8192, bar_rec0 + 8 * bb);
         bulk_g2s(sb + OFF_G + bb * 256, r + intra::REC_G, 256, bar_rec0 + 8 * bb);
     };
-    auto issue_p = [&](int ci) {   // P of chunk ci into B2 buffer ci & 1
+    auto issue_p = [&](int ci) {   // P^T of chunk ci into its B2 atom (first at parity 0, last at 1)
         const int bb = ci & 1;
         s_issued[4 + bb]++;
         mbar_arrive_expect_tx(bar_p0 + 8 * bb, 8192);
-        bulk_g2s(sb + OFF_B2 + bb * B2_STRIDE, rec0 + ci * rec_stride + intra::REC_P, 8192, bar_p0 + 8 * bb);
+        bulk_g2s(sb + OFF_B2 + bb * B2_STRIDE + (bb ? 16384 : 0), rec0 + ci * rec_stride + intra::REC_P, 8192,
+                 bar_p0 + 8 * bb);
     };
     auto wait_par = [&](uint32_t bar0, int ci) {
         if (!mbar_wait_bounded(bar0 + 8 * (ci & 1), (ci >> 1) & 1)) atomicOr((unsigned*)s_abort, 2u);
@@ -158,12 +163,8 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 
     if (tid == 0) {
         mbar_init(bar, 1);
-        mbar_init(bar_qkv0, 1);
-        mbar_init(bar_qkv0 + 8, 1);
-        mbar_init(bar_rec0, 1);
-        mbar_init(bar_rec0 + 8, 1);
-        mbar_init(bar_p0, 1);
-        mbar_init(bar_p0 + 8, 1);
+#pragma unroll
+        for (int i = 0; i < 6; i++) mbar_init(bar_kv0 + 8 * i, 1);   // kv x2, rec x2, P x2
         fence_mbar_init();
         *s_abort = 0;
         for (int i = 0; i < 6; i++) s_issued[i] = 0;
@@ -185,14 +186,12 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const float inv_sqrt_dk = rsqrtf((float)dk);
     uint32_t mphase = 0;
 
-    // e^g and e^{g_C - g} (zero past the chunk's end) of chunk ce, by threads r0..r0+63
+    // e^{g_C - g} (zero past the chunk's end) of chunk ce, by threads r0..r0+63
     auto chunk_vectors = [&](int ce, int r0) {
         wait_par(bar_rec0, ce);
         const int r = tid - r0;
         const float* rg = s_g + 64 * (ce & 1);
-        const float g = rg[r], gl = rg[C - 1];
-        s_eg[64 * (ce & 1) + r] = __expf(g);
-        s_ks[64 * (ce & 1) + r] = s0 + (int64_t)ce * C + r < s1 ? __expf(gl - g) : 0.f;
+        s_ks[64 * (ce & 1) + r] = s0 + (int64_t)ce * C + r < s1 ? __expf(rg[C - 1] - rg[r]) : 0.f;
     };
     // New state -> its fp16 A operand and the decayed accumulator (decay * S) of the next chunk
     auto put_state = [&](const float (&Sv)[32], float decay) {
@@ -207,30 +206,24 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         tmem_st16(tl + ACC_S + 32 * cs, d0);
         tmem_st16(tl + ACC_S + 32 * cs + 16, d1);
     };
-    // Q~ = diag(e^g) Q in place (B1) and K~ (B2) of chunk ce, all threads
-    auto scale_qk = [&](int ce) {
-        wait_par(bar_qkv0, ce);
+    // K~ = diag(e^{g_C - g}) K of chunk ce into its two B2 atoms (last two at parity 0, first two at 1)
+    auto build_kt = [&](int ce) {
+        wait_par(bar_kv0, ce);
         const int bb = ce & 1;
-        const float* eg = s_eg + 64 * bb;
         const float* ks = s_ks + 64 * bb;
-        for (int idx = tid; idx < C * 16; idx += NT) {   // Q rows: 16-byte pieces, in place
-            const int r = idx >> 4, c16 = idx & 15;
-            const uint32_t a = sb + OFF_B1 + bb * B1_STRIDE + (c16 >> 3) * 16384 + swz128(C + r, c16 & 7);
-            const uint4 x = scale8(lds128(a), eg[r]);
-            sts128(a, x.x, x.y, x.z, x.w);
-        }
-        for (int idx = tid; idx < C * 16; idx += NT) {   // K~ rows: 16-byte pieces into B2's K~ halves
+        const uint32_t dst = sb + OFF_B2 + bb * B2_STRIDE + (bb ? 0 : 8192);
+        for (int idx = tid; idx < C * 16; idx += NT) {
             const int c = idx >> 4, c16 = idx & 15;
             const uint32_t off = (c16 >> 3) * 8192 + swz128(c, c16 & 7);
             const uint4 x = scale8(lds128(sb + OFF_K + bb * 16384 + off), ks[c]);
-            sts128(sb + OFF_B2 + bb * B2_STRIDE + 8192 + off, x.x, x.y, x.z, x.w);
+            sts128(dst + off, x.x, x.y, x.z, x.w);
         }
         fence_async_smem();
     };
     // o = O / sqrt(d_k) of chunk ce -> staging; tid 0 stores it after the next barrier
     auto stage_o = [&](int ce) {
         uint32_t o[16];
-        tmem_ld16(tl + ACC_O + 16 * cs, o);
+        tmem_ld16(tl + acc_o(ce & 1) + 16 * cs, o);
         TO* st = reinterpret_cast<TO*>(smem + OFF_OST + (ce % kOBufs) * 16384);
 #pragma unroll
         for (int i = 0; i < 16; i++) from_f32(__uint_as_float(o[i]) * inv_sqrt_dk, st + (16 * cs + i) * 128 + dv_r);
@@ -245,15 +238,16 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     const uint64_t dV0 = sdesc(sb + OFF_V, 8192, 1024);
     const uint64_t dT0 = sdesc(sb + OFF_T, 16, 1024);
     const uint64_t dB10 = sdesc(sb + OFF_B1, 16, 1024);
-    const uint64_t dB2 = sdesc(sb + OFF_B2, 8192, 1024);
-    constexpr uint32_t ID_MK = idesc_f16(128, 64, 1, 0);     // (c)
+    const uint64_t dB20 = sdesc(sb + OFF_B2, 8192, 1024);
+    constexpr uint32_t ID_C = idesc_f16(128, 64, 1, 0);      // (c)
     constexpr uint32_t ID_DE = idesc_f16(128, 128, 0, 0);    // (d,e)
     constexpr uint32_t ID_FG = idesc_f16(128, 192, 0, 1);    // (f,g)
 
-    // ---- prologue: initial state, chunk 0's vectors and scaled q, k ----
+    // ---- prologue: chunk 0's vectors and K~, the initial state ----
     if (tid < C) chunk_vectors(0, 0);
     __syncthreads();
     if (*s_abort) goto abort_;
+    build_kt(0);
     {
         float Sv[32];
 #pragma unroll
@@ -261,9 +255,8 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
             const int col = 32 * cs + i;
             Sv[i] = (dv_r < dv && col < dk) ? gstate[(int64_t)dv_r * dk + col] : 0.f;
         }
-        put_state(Sv, s_eg[C - 1]);
+        put_state(Sv, __expf(s_g[C - 1]));
     }
-    scale_qk(0);
     tc_fence_before();
     __syncthreads();
     if (*s_abort) goto abort_;
@@ -280,45 +273,47 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
     for (int ci = 0; ci < nchunks; ci++) {
         const int b = ci & 1;
 
-        // ---- MMA1: (c) U1^T = V^T T^T; (d,e) [U2^T | O^T] = S [-W ; Q~]^T ----
+        // ---- MMA1: (d,e) [U2^T | O^T] = S [-W ; Q~]^T, then (c) U2^T += V^T T^T ----
         if (tid == 0) {
+            wait_par(bar_rec0, ci);
+            wait_par(bar_kv0, ci);
             tc_fence_after();
+            const uint32_t d1 = tmem + (b ? ACC_O1 : ACC_U0);
 #pragma unroll
-            for (int ks = 0; ks < 8; ks++) {
-                if (ks < 4)
-                    mma_f16(tmem + ACC_U1, dV0 + b * 1024 + ks * 128, dT0 + b * 512 + ks * 2, ID_MK, ks > 0);
-                mma_f16_ta(tmem + ACC_U2, tmem + TA_S + ks * 8,
-                           dB10 + b * 2048 + (ks >> 2) * 1024 + (ks & 3) * 2, ID_DE, ks > 0);
-            }
+            for (int ks = 0; ks < 8; ks++)
+                mma_f16_ta(d1, tmem + TA_S + ks * 8, dB10 + b * 2048 + (ks >> 2) * 1024 + (ks & 3) * 2, ID_DE, ks > 0);
+#pragma unroll
+            for (int ks = 0; ks < 4; ks++)
+                mma_f16(tmem + acc_u(b), dV0 + b * 1024 + ks * 128, dT0 + b * 512 + ks * 2, ID_C, 1);
             mma_commit(bar);
         }
-        // while MMA1 runs: P of chunk ci + 1 (its B2 buffer was freed by MMA2 of chunk ci - 1);
-        // e^g, e^{g_C - g} of chunk ci + 1
-        if (tid == 32 && ci + 1 < nchunks) issue_p(ci + 1);
+        // ---- while MMA1 runs: K~ of this chunk, the previous o tile, P and e^{g_C - g} of the next ----
+        if (tid == 32 && ci + 1 < nchunks) issue_p(ci + 1);   // its B2 atom was freed by MMA2 of chunk ci - 1
         if (tid >= 64 && tid < 64 + C && ci + 1 < nchunks) chunk_vectors(ci + 1, 64);
+        if (ci > 0) build_kt(ci);
+        if (ci > 0) stage_o(ci - 1);
         GDN_MMA_WAIT();
+        if (tid == 0 && ci > 0) issue_o(ci - 1);
 
-        // ---- U^T = U1^T + U2^T -> fp16 A operand ----
+        // ---- U^T -> fp16 A operand ----
         {
-            uint32_t r1[16], r2[16], u[8];
-            tmem_ld16(tl + ACC_U1 + 16 * cs, r1);
-            tmem_ld16(tl + ACC_U2 + 16 * cs, r2);
+            uint32_t r16[16], u[8];
+            tmem_ld16(tl + acc_u(b) + 16 * cs, r16);
 #pragma unroll
-            for (int i = 0; i < 8; i++)
-                u[i] = pack_half2(__uint_as_float(r1[2 * i]) + __uint_as_float(r2[2 * i]),
-                                  __uint_as_float(r1[2 * i + 1]) + __uint_as_float(r2[2 * i + 1]));
+            for (int i = 0; i < 8; i++) u[i] = pack_half2(__uint_as_float(r16[2 * i]), __uint_as_float(r16[2 * i + 1]));
             tmem_st8(tl + TA_U + 8 * cs, u);
         }
         tc_fence_before();
         __syncthreads();
 
-        // ---- MMA2: [O^T | S] += U^T [P ; K~^T]^T ----
+        // ---- MMA2: [O^T | S] (parity 0) or [S | O^T] (parity 1) += U^T [P ; K~^T]^T ----
         if (tid == 0) {
-            if (!mbar_wait_bounded(bar_p0 + 8 * b, (ci >> 1) & 1)) atomicOr((unsigned*)s_abort, 2u);
+            wait_par(bar_p0, ci);
             tc_fence_after();
+            const uint32_t d2 = tmem + (b ? ACC_S : ACC_O0);
 #pragma unroll
             for (int ks = 0; ks < 4; ks++)
-                mma_f16_ta(tmem + ACC_O, tmem + TA_U + ks * 8, dB2 + b * (B2_STRIDE >> 4) + ks * 128, ID_FG, 1);
+                mma_f16_ta(d2, tmem + TA_U + ks * 8, dB20 + b * (B2_STRIDE >> 4) + ks * 128, ID_FG, 1);
             mma_commit(bar);
             if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();   // staging buffer of stage_o(ci)
         }
@@ -328,7 +323,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
         }
         GDN_MMA_WAIT();
 
-        // ---- new state: fp16 A operand and the next chunk's decayed accumulator; o tile ----
+        // ---- new state: fp16 A operand and the next chunk's decayed accumulator ----
         {
             uint32_t r32[32];
             tmem_ld32(tl + ACC_S + 32 * cs, r32);
@@ -336,7 +331,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
 #pragma unroll
             for (int i = 0; i < 32; i++) Sv[i] = __uint_as_float(r32[i]);
             if (ci + 1 < nchunks) {
-                put_state(Sv, s_eg[64 * (b ^ 1) + C - 1]);
+                put_state(Sv, __expf(s_g[64 * (b ^ 1) + C - 1]));
             } else {   // the final state
 #pragma unroll
                 for (int i = 0; i < 32; i++) {
@@ -345,16 +340,17 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant_
                 }
             }
         }
-        stage_o(ci);
-        if (ci + 1 < nchunks) scale_qk(ci + 1);
         tc_fence_before();
         __syncthreads();
         if (*s_abort) goto abort_;
-        if (tid == 0) issue_o(ci);
     }
-
-    if (tid == 0) bulk_wait<0>();   // every o tile has reached global memory
+    stage_o(nchunks - 1);
     tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+        issue_o(nchunks - 1);
+        bulk_wait<0>();   // every o tile has reached global memory
+    }
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();
@@ -368,9 +364,8 @@ abort_:
     // recurrent state is left as it was.
     if (tid == 0) {
         record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));
-        const uint32_t bars[6] = {bar_qkv0, bar_qkv0 + 8, bar_rec0, bar_rec0 + 8, bar_p0, bar_p0 + 8};
         for (int i = 0; i < 6; i++)   // the last phase issued on each barrier (returns at once if complete)
-            if (s_issued[i] > 0) mbar_wait_bounded(bars[i], (uint32_t)(s_issued[i] - 1) & 1u);
+            if (s_issued[i] > 0) mbar_wait_bounded(bar_kv0 + 8 * i, (uint32_t)(s_issued[i] - 1) & 1u);
         bulk_wait<0>();
     }
     if (warp == 0) {

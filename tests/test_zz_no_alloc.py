@@ -82,7 +82,7 @@ def test_noalloc_rejects_requests_beyond_its_scratch():
     fits = 1
     while gdn.workspace_size(cfg, fits + 1, 1) <= SCRATCH_BYTES:   # largest single sequence that fits
         fits += 1
-    assert fits > 1000
+    assert fits >= 896   # the limit include/gdn.h states for one sequence
     cc, cw = cfg.c(), gdn._weights(L.weights_on(c, DEV), torch.device(DEV))
     dummy = torch.zeros(16, device=DEV)
     P = ctypes.c_void_p(dummy.data_ptr())
