@@ -1,6 +1,6 @@
 // State chain of the chunked gated delta rule on the sm_100a tensor cores.
 //
-// One CTA (512 threads) walks one (sequence, value head) chain chunk by chunk
+// One CTA (17 warps) walks one (sequence, value head) chain chunk by chunk
 // (C = 64 tokens).  The state-independent factors of every chunk come from the
 // intra-chunk kernel's records (intra.cuh: -W, T, P, g, Q~).  With S0 the state
 // at the chunk start:
@@ -12,23 +12,24 @@
 //
 // A tcgen05.mma costs about the same whatever its N up to 128, so products that
 // share an A operand are fused into one wide-N MMA, and A operands live in TMEM:
-//   MMA1  (d,e) S [-W ; Q~]^T, N = 128  -> [U2^T | O^T]      [A: S, TMEM]
-//         (c)   V^T T^T,         N = 64  -> U^T += (into U2^T) [A: V, shared memory]
-//   MMA2  (f,g) U^T [P ; K~^T]^T, N=192 -> [O^T | S]  (+=)   [A: U^T, TMEM; B MN-major]
-// with Q~ = diag(e^g) Q and K~ = diag(e^{g_C - g}) K.  The fp32 state S lives in
-// TMEM as an accumulator: before MMA2 it holds e^{g_C} S0, so MMA2 leaves S_C.
-// The operand tiles and the U, O accumulators alternate with chunk parity so
-// that O is double-buffered while both fused MMAs keep contiguous outputs:
+//   (c)   V^T T^T,             N = 64  -> U2^T           [A: V, shared memory]
+//   MMA1  (d,e) S [-W ; Q~]^T, N = 128 -> [U2^T | O^T] += [A: S, TMEM]
+//   MMA2  (f,g) U^T [P ; K~^T]^T, N=192 -> [O^T | S]  += [A: U^T, TMEM; B MN-major]
+// with Q~ = diag(e^g) Q and K~ = diag(e^{g_C - g}) K.  (c) does not depend on the
+// state, so its k-steps are issued right after MMA1 and MMA2 of the previous
+// chunk and run while U^T and the new state are converted.  The fp32 state S lives in TMEM as an
+// accumulator: before MMA2 it holds e^{g_C} S0, so MMA2 leaves S_C.  The operand
+// tiles and the U, O accumulators alternate with chunk parity so that O is
+// double-buffered while both fused MMAs keep contiguous outputs:
 //   parity 0: B1 = [-W ; Q~], B2 = [P^T | K~], TMEM [U2 | O0 | S]
 //   parity 1: B1 = [Q~ ; -W], B2 = [K~ | P^T], TMEM [S | O1 | U2']
-// Per chunk, the critical chain is MMA1 -> U^T to fp16 -> MMA2 -> new S (its
-// fp16 A copy and the next chunk's decayed accumulator).  While MMA1 runs the
-// other threads build K~, write the previous chunk's o tile, and prepare the
-// next chunk's gate vectors.  Loads are double-buffered: k, v (TMA) and the
-// record (bulk copies) two chunks ahead, issued while MMA2 runs; P one chunk
-// ahead, issued while MMA1 runs.  Thread 0 issues every MMA and waits on the
-// tensor-core mbarrier; thread 32 issues the loads; the others meet them at the
-// CTA barrier.
+// Per chunk, the critical chain is MMA1 -> U^T to fp16 -> MMA2 -> the fp16 copy
+// of the new state.  While MMA1 runs, the 16 worker warps write the decayed state
+// accumulator, build K~ and prepare the next chunk's gate vectors; while MMA2
+// runs, they write the previous chunk's o tile (and zero its accumulator for the
+// chunk after next).  A 17th warp issues every MMA and every copy, so that its
+// waits on the tensor pipe delay no other work.  Loads are double-buffered: k, v (TMA)
+// and the record (bulk copies) two chunks ahead, P one chunk ahead.
 #pragma once
 #include "device.cuh"
 #include "intra.cuh"
@@ -37,7 +38,9 @@ namespace gdn {
 namespace scan {
 
 constexpr int C = 64;
-constexpr int NT = 512;   // 16 warps: 4 per TMEM lane quadrant
+constexpr int NW = 512;               // 16 worker warps: 4 per TMEM lane quadrant
+constexpr int NT = NW + 32;           // + the issuing warp
+constexpr int ISSUER = NW;            // lane 0 of warp 16: every MMA, load and store
 
 // Shared memory (bytes from a 1024-aligned base); pairs are indexed by chunk parity.
 constexpr uint32_t OFF_B1 = 0;          // x2: per 64-wide d_k half (16 KiB), 64 + 64 rows of -W / Q~
@@ -110,10 +113,12 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 60);
     // loads issued per barrier (kv x2, record x2, P x2): the abort path waits for the last phase of each
     volatile int* s_issued = reinterpret_cast<volatile int*>(smem + OFF_BAR + 64);
+    const uint32_t bar_fin = sb + OFF_BAR + 96;           // abort path: every MMA issued so far
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const bool worker = tid < NW;
     const int qd = warp & 3;      // TMEM lane quadrant
-    const int cs = warp >> 2;     // column slice 0..3
+    const int cs = warp >> 2;     // column slice 0..3 (worker warps)
     const int Hv = p.Hv, dk = p.dk, dv = p.dv;
     const int seq = blockIdx.x / Hv, h = blockIdx.x % Hv;
     const int j = h / (Hv / p.Hk);
@@ -161,10 +166,11 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         if (!mbar_wait_bounded(bar0 + 8 * (ci & 1), (ci >> 1) & 1)) atomicOr((unsigned*)s_abort, 2u);
     };
 
-    if (tid == 0) {
+    if (tid == ISSUER) {
         mbar_init(bar, 1);
 #pragma unroll
         for (int i = 0; i < 6; i++) mbar_init(bar_kv0 + 8 * i, 1);   // kv x2, rec x2, P x2
+        mbar_init(bar_fin, 1);
         fence_mbar_init();
         *s_abort = 0;
         for (int i = 0; i < 6; i++) s_issued[i] = 0;
@@ -176,8 +182,16 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         tmem_alloc(sb + OFF_BAR + 56, TMEM_COLS);
         tmem_relinquish();
     }
-    const int dv_r = 32 * qd + lane;   // this thread's state row; columns [32 cs, 32 cs + 32)
+    const int dv_r = 32 * qd + lane;   // this worker's state row; columns [32 cs, 32 cs + 32)
     float* gstate = p.rec_state + ((int64_t)seq * Hv + h) * dv * dk;
+    float Sv[32];   // this worker's slice of the state at the start of the current chunk
+    if (worker) {
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+            const int col = 32 * cs + i;
+            Sv[i] = (dv_r < dv && col < dk) ? gstate[(int64_t)dv_r * dk + col] : 0.f;
+        }
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -185,54 +199,6 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
     const float inv_sqrt_dk = rsqrtf((float)dk);
     uint32_t mphase = 0;
-
-    // e^{g_C - g} (zero past the chunk's end) of chunk ce, by threads r0..r0+63
-    auto chunk_vectors = [&](int ce, int r0) {
-        wait_par(bar_rec0, ce);
-        const int r = tid - r0;
-        const float* rg = s_g + 64 * (ce & 1);
-        s_ks[64 * (ce & 1) + r] = s0 + (int64_t)ce * C + r < s1 ? __expf(rg[C - 1] - rg[r]) : 0.f;
-    };
-    // New state -> its fp16 A operand and the decayed accumulator (decay * S) of the next chunk
-    auto put_state = [&](const float (&Sv)[32], float decay) {
-        uint32_t h16[16], d0[16], d1[16];
-#pragma unroll
-        for (int i = 0; i < 16; i++) {
-            h16[i] = pack_half2(Sv[2 * i], Sv[2 * i + 1]);
-            d0[i] = __float_as_uint(decay * Sv[i]);
-            d1[i] = __float_as_uint(decay * Sv[16 + i]);
-        }
-        tmem_st16(tl + TA_S + 16 * cs, h16);
-        tmem_st16(tl + ACC_S + 32 * cs, d0);
-        tmem_st16(tl + ACC_S + 32 * cs + 16, d1);
-    };
-    // K~ = diag(e^{g_C - g}) K of chunk ce into its two B2 atoms (last two at parity 0, first two at 1)
-    auto build_kt = [&](int ce) {
-        wait_par(bar_kv0, ce);
-        const int bb = ce & 1;
-        const float* ks = s_ks + 64 * bb;
-        const uint32_t dst = sb + OFF_B2 + bb * B2_STRIDE + (bb ? 0 : 8192);
-        for (int idx = tid; idx < C * 16; idx += NT) {
-            const int c = idx >> 4, c16 = idx & 15;
-            const uint32_t off = (c16 >> 3) * 8192 + swz128(c, c16 & 7);
-            const uint4 x = scale8(lds128(sb + OFF_K + bb * 16384 + off), ks[c]);
-            sts128(dst + off, x.x, x.y, x.z, x.w);
-        }
-        fence_async_smem();
-    };
-    // o = O / sqrt(d_k) of chunk ce -> staging; tid 0 stores it after the next barrier
-    auto stage_o = [&](int ce) {
-        uint32_t o[16];
-        tmem_ld16(tl + acc_o(ce & 1) + 16 * cs, o);
-        TO* st = reinterpret_cast<TO*>(smem + OFF_OST + (ce % kOBufs) * 16384);
-#pragma unroll
-        for (int i = 0; i < 16; i++) from_f32(__uint_as_float(o[i]) * inv_sqrt_dk, st + (16 * cs + i) * 128 + dv_r);
-        fence_async_smem();
-    };
-    auto issue_o = [&](int ce) {
-        bulk_s2g(otile0 + ce * o_stride, sb + OFF_OST + (ce % kOBufs) * 16384, O_BYTES);
-        bulk_commit();
-    };
 
     // Shared-memory descriptors; per-step offsets are added to the start-address field.
     const uint64_t dV0 = sdesc(sb + OFF_V, 8192, 1024);
@@ -243,60 +209,125 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
     constexpr uint32_t ID_DE = idesc_f16(128, 128, 0, 0);    // (d,e)
     constexpr uint32_t ID_FG = idesc_f16(128, 192, 0, 1);    // (f,g)
 
-    // ---- prologue: chunk 0's vectors and K~, the initial state ----
-    if (tid < C) chunk_vectors(0, 0);
-    __syncthreads();
-    if (*s_abort) goto abort_;
-    build_kt(0);
-    {
-        float Sv[32];
+    // (c) of chunk ce, k-steps [k0, k1): U2^T = V^T T^T into its U accumulator (issuer; the
+    // steps run in the tensor pipe's idle windows and are committed with the next MMA)
+    auto issue_c = [&](int ce, int k0, int k1) {
+        wait_par(bar_rec0, ce);
+        wait_par(bar_kv0, ce);
+        tc_fence_after();
+        const int bb = ce & 1;
+        for (int ks = k0; ks < k1; ks++)
+            mma_f16(tmem + acc_u(bb), dV0 + bb * 1024 + ks * 128, dT0 + bb * 512 + ks * 2, ID_C, ks > 0);
+    };
+    // e^{g_C - g} (zero past the chunk's end) of chunk ce, by threads r0..r0+63
+    auto chunk_vectors = [&](int ce, int r0) {
+        wait_par(bar_rec0, ce);
+        const int r = tid - r0;
+        const float* rg = s_g + 64 * (ce & 1);
+        s_ks[64 * (ce & 1) + r] = s0 + (int64_t)ce * C + r < s1 ? __expf(rg[C - 1] - rg[r]) : 0.f;
+    };
+    // fp16 copy of the state: the A operand of MMA1
+    auto put_state_a = [&]() {
+        uint32_t h16[16];
 #pragma unroll
-        for (int i = 0; i < 32; i++) {
-            const int col = 32 * cs + i;
-            Sv[i] = (dv_r < dv && col < dk) ? gstate[(int64_t)dv_r * dk + col] : 0.f;
+        for (int i = 0; i < 16; i++) h16[i] = pack_half2(Sv[2 * i], Sv[2 * i + 1]);
+        tmem_st16(tl + TA_S + 16 * cs, h16);
+    };
+    // decayed state e^{g_C} S: the accumulator that MMA2 completes
+    auto put_state_acc = [&](float decay) {
+        uint32_t d[32];
+#pragma unroll
+        for (int i = 0; i < 32; i++) d[i] = __float_as_uint(decay * Sv[i]);
+        tmem_st32(tl + ACC_S + 32 * cs, d);
+    };
+    // K~ = diag(e^{g_C - g}) K of chunk ce into its two B2 atoms (last two at parity 0, first two at 1)
+    auto build_kt = [&](int ce) {
+        wait_par(bar_kv0, ce);
+        const int bb = ce & 1;
+        const float* ks = s_ks + 64 * bb;
+        const uint32_t dst = sb + OFF_B2 + bb * B2_STRIDE + (bb ? 0 : 8192);
+        for (int idx = tid; idx < C * 16; idx += NW) {
+            const int c = idx >> 4, c16 = idx & 15;
+            const uint32_t off = (c16 >> 3) * 8192 + swz128(c, c16 & 7);
+            const uint4 x = scale8(lds128(sb + OFF_K + bb * 16384 + off), ks[c]);
+            sts128(dst + off, x.x, x.y, x.z, x.w);
         }
-        put_state(Sv, __expf(s_g[C - 1]));
+        fence_async_smem();
+    };
+    // o = O / sqrt(d_k) of chunk ce -> staging, and its accumulator zeroed for chunk ce + 2;
+    // the issuer stores the tile after the next barrier (its buffer is free: see bulk_wait_read)
+    auto stage_o = [&](int ce) {
+        uint32_t o[16];
+        tmem_ld16(tl + acc_o(ce & 1) + 16 * cs, o);
+        TO* st = reinterpret_cast<TO*>(smem + OFF_OST + (ce % kOBufs) * 16384);
+#pragma unroll
+        for (int i = 0; i < 16; i++) from_f32(__uint_as_float(o[i]) * inv_sqrt_dk, st + (16 * cs + i) * 128 + dv_r);
+        fence_async_smem();
+#pragma unroll
+        for (int i = 0; i < 16; i++) o[i] = 0u;
+        tmem_st16(tl + acc_o(ce & 1) + 16 * cs, o);
+    };
+    auto issue_o = [&](int ce) {
+        bulk_s2g(otile0 + ce * o_stride, sb + OFF_OST + (ce % kOBufs) * 16384, O_BYTES);
+        bulk_commit();
+    };
+
+    // ---- prologue: zero O accumulators, fp16 S0, (c) and e^{g_C - g} of chunk 0 ----
+    if (tid == ISSUER) issue_c(0, 0, 4);
+    if (worker) {
+        uint32_t z[16];
+#pragma unroll
+        for (int i = 0; i < 16; i++) z[i] = 0u;
+        tmem_st16(tl + ACC_O0 + 16 * cs, z);
+        tmem_st16(tl + ACC_O1 + 16 * cs, z);
+        put_state_a();
+        if (tid < C) chunk_vectors(0, 0);
     }
     tc_fence_before();
     __syncthreads();
     if (*s_abort) goto abort_;
 
-#define GDN_MMA_WAIT()                                                                        \
-    do {                                                                                      \
-        if (tid == 0 && !mbar_wait_bounded(bar, mphase)) atomicOr((unsigned*)s_abort, 1u);  \
-        mphase ^= 1u;                                                                         \
-        __syncthreads();                                                                      \
-        if (*s_abort) goto abort_;                                                            \
-        tc_fence_after();                                                                     \
+#define GDN_MMA_WAIT()                                                                               \
+    do {                                                                                             \
+        if (tid == ISSUER && !mbar_wait_bounded(bar, mphase)) atomicOr((unsigned*)s_abort, 1u);    \
+        mphase ^= 1u;                                                                                \
+        __syncthreads();                                                                             \
+        if (*s_abort) goto abort_;                                                                   \
+        tc_fence_after();                                                                            \
     } while (0)
 
     for (int ci = 0; ci < nchunks; ci++) {
         const int b = ci & 1;
 
-        // ---- MMA1: (d,e) [U2^T | O^T] = S [-W ; Q~]^T, then (c) U2^T += V^T T^T ----
-        if (tid == 0) {
+        // ---- MMA1: (d,e) [U2^T | O^T] += S [-W ; Q~]^T ((c) and zeroed O are already there) ----
+        if (tid == ISSUER) {
             wait_par(bar_rec0, ci);
-            wait_par(bar_kv0, ci);
             tc_fence_after();
             const uint32_t d1 = tmem + (b ? ACC_O1 : ACC_U0);
 #pragma unroll
             for (int ks = 0; ks < 8; ks++)
-                mma_f16_ta(d1, tmem + TA_S + ks * 8, dB10 + b * 2048 + (ks >> 2) * 1024 + (ks & 3) * 2, ID_DE, ks > 0);
-#pragma unroll
-            for (int ks = 0; ks < 4; ks++)
-                mma_f16(tmem + acc_u(b), dV0 + b * 1024 + ks * 128, dT0 + b * 512 + ks * 2, ID_C, 1);
+                mma_f16_ta(d1, tmem + TA_S + ks * 8, dB10 + b * 2048 + (ks >> 2) * 1024 + (ks & 3) * 2, ID_DE, 1);
             mma_commit(bar);
+            if (ci + 1 < nchunks) issue_c(ci + 1, 0, 2);   // runs while U^T is converted
         }
-        // ---- while MMA1 runs: K~ of this chunk, the previous o tile, P and e^{g_C - g} of the next ----
-        if (tid == 32 && ci + 1 < nchunks) issue_p(ci + 1);   // its B2 atom was freed by MMA2 of chunk ci - 1
-        if (tid >= 64 && tid < 64 + C && ci + 1 < nchunks) chunk_vectors(ci + 1, 64);
-        if (ci > 0) build_kt(ci);
-        if (ci > 0) stage_o(ci - 1);
+        // ---- workers, while MMA1 runs: decayed state, next e^{g_C - g}, K~ ----
+        if (worker) {
+            put_state_acc(__expf(s_g[64 * b + C - 1]));
+            if (tid >= 64 && tid < 64 + C && ci + 1 < nchunks) chunk_vectors(ci + 1, 64);
+            build_kt(ci);
+        }
         GDN_MMA_WAIT();
-        if (tid == 0 && ci > 0) issue_o(ci - 1);
 
-        // ---- U^T -> fp16 A operand ----
-        {
+        // ---- U^T -> fp16 A operand; the issuer queues loads ----
+        if (tid == ISSUER) {
+            if (ci + 1 < nchunks) issue_p(ci + 1);   // its B2 atom was freed by MMA2 of chunk ci - 1
+            if (ci + 2 < nchunks) {   // MMA1, (c) and K~ of chunk ci are done with buffer b
+                fence_async_smem();
+                issue_chunk(ci + 2);
+            }
+            if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();   // staging buffer of stage_o(ci - 1)
+        }
+        if (worker) {
             uint32_t r16[16], u[8];
             tmem_ld16(tl + acc_u(b) + 16 * cs, r16);
 #pragma unroll
@@ -307,7 +338,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         __syncthreads();
 
         // ---- MMA2: [O^T | S] (parity 0) or [S | O^T] (parity 1) += U^T [P ; K~^T]^T ----
-        if (tid == 0) {
+        if (tid == ISSUER) {
             wait_par(bar_p0, ci);
             tc_fence_after();
             const uint32_t d2 = tmem + (b ? ACC_S : ACC_O0);
@@ -315,24 +346,22 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
             for (int ks = 0; ks < 4; ks++)
                 mma_f16_ta(d2, tmem + TA_U + ks * 8, dB20 + b * (B2_STRIDE >> 4) + ks * 128, ID_FG, 1);
             mma_commit(bar);
-            if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();   // staging buffer of stage_o(ci)
+            if (ci + 1 < nchunks) issue_c(ci + 1, 2, 4);   // runs while the new state is converted
         }
-        if (tid == 32 && ci + 2 < nchunks) {   // MMA1 of chunk ci is done with buffer b: fetch chunk ci + 2's
-            fence_async_smem();
-            issue_chunk(ci + 2);
-        }
+        // ---- workers, while MMA2 runs: the previous chunk's o tile ----
+        if (worker && ci > 0) stage_o(ci - 1);
         GDN_MMA_WAIT();
 
-        // ---- new state: fp16 A operand and the next chunk's decayed accumulator ----
-        {
+        // ---- new state: its fp16 copy for the next MMA1, or the final state ----
+        if (tid == ISSUER && ci > 0) issue_o(ci - 1);
+        if (worker) {
             uint32_t r32[32];
             tmem_ld32(tl + ACC_S + 32 * cs, r32);
-            float Sv[32];
 #pragma unroll
             for (int i = 0; i < 32; i++) Sv[i] = __uint_as_float(r32[i]);
             if (ci + 1 < nchunks) {
-                put_state(Sv, __expf(s_g[64 * (b ^ 1) + C - 1]));
-            } else {   // the final state
+                put_state_a();
+            } else {
 #pragma unroll
                 for (int i = 0; i < 32; i++) {
                     const int col = 32 * cs + i;
@@ -344,10 +373,14 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant_
         __syncthreads();
         if (*s_abort) goto abort_;
     }
-    stage_o(nchunks - 1);
+    if (tid == ISSUER) {
+        if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();
+    }
+    __syncthreads();
+    if (worker) stage_o(nchunks - 1);
     tc_fence_before();
     __syncthreads();
-    if (tid == 0) {
+    if (tid == ISSUER) {
         issue_o(nchunks - 1);
         bulk_wait<0>();   // every o tile has reached global memory
     }
@@ -362,15 +395,17 @@ abort_:
     // A tensor-core commit or a copy never arrived: report it, give whatever is
     // still in flight one more bounded wait, free tensor memory and return.  The
     // recurrent state is left as it was.
-    if (tid == 0) {
+    if (tid == ISSUER) {
         record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));
+        mma_commit(bar_fin);   // tracks every MMA this thread has issued
+        mbar_wait_bounded(bar_fin, 0);
         for (int i = 0; i < 6; i++)   // the last phase issued on each barrier (returns at once if complete)
             if (s_issued[i] > 0) mbar_wait_bounded(bar_kv0 + 8 * i, (uint32_t)(s_issued[i] - 1) & 1u);
         bulk_wait<0>();
     }
+    tc_fence_before();
+    __syncthreads();
     if (warp == 0) {
-        mbar_wait_bounded(bar, mphase ^ 1u);
-        __syncwarp();
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
