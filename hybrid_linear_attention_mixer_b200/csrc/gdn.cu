@@ -169,7 +169,7 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     sa.cu = cu; sa.chunk_off = chunk_off; sa.rec = recs;
     sa.o = otiles;
     sa.Hk = Hk; sa.Hv = Hv; sa.dk = c->d_k; sa.dv = c->d_v;
-    k_scan<<<(unsigned)n_seqs * Hv, gdn::scan::NT, gdn::scan::SMEM_BYTES, st>>>(tm_k, tm_v, sa);
+    k_scan<<<(unsigned)n_seqs * Hv, gdn::scan::NT, gdn::scan::SMEM_BYTES, st>>>(tm_v, sa);
 
     gdn::norm::Args na;
     na.o = otiles; na.z = z; na.norm_w = w->norm_weight;

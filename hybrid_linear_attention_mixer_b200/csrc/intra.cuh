@@ -14,12 +14,17 @@
 //
 // Each (chunk, value head) record written to the workspace holds the operand
 // tiles exactly as the scan kernel's tensor cores read them (128-byte swizzled
-// shared-memory images), so the scan brings a whole record in with one bulk copy:
-//     +0      -W   K-major  [64 rows c][d_k columns], two 64-wide halves of 8192 B
-//     +16384  T    K-major  [64 rows c][64 columns j]    fp16    8192 B
-//     +24576  P^T  MN-major [64 rows j][64 columns r]    fp16    8192 B
-//     +32768  g    [64] fp32 (rows past the sequence end repeat the last g)
-//     +33792  Q~   K-major  [64 rows r][d_k columns] = diag(e^g) Q, two halves of 8192 B
+// shared-memory images), so the scan brings a record in with two bulk copies.
+// Q~ = diag(e^g) Q and K~ = diag(e^{g_C - g}) K (zero past the sequence end).
+// The order of the tiles inside the two images alternates with the parity p of
+// the chunk within its sequence, to match the scan's alternating TMEM layout:
+//     +0      B1 image, two 64-wide d_k halves of 16384 B, each [X rows | Y rows]
+//             (64 rows each, K-major): X, Y = -W, Q~ (p = 0) or Q~, -W (p = 1)
+//     +32768  T    K-major  [64 rows c][64 columns j]    fp16    8192 B
+//     +40960  g    [64] fp32 (rows past the sequence end repeat the last g)
+//     +41984  B2 image, three MN-major atoms of 8192 B:
+//             [P^T | K~ half 0 | K~ half 1] (p = 0) or [K~ half 0 | K~ half 1 | P^T] (p = 1)
+//             (P^T: row j holds P[0..63][j]; K~: row c holds 64 d_k values)
 #pragma once
 #include "device.cuh"
 
@@ -28,8 +33,14 @@ namespace intra {
 
 constexpr int C = 64;
 constexpr int NT = 256;
-constexpr uint32_t REC_W = 0, REC_T = 16384, REC_P = 24576, REC_G = 32768, REC_Q = 33792;
-constexpr uint32_t REC_BYTES = 50176;   // 49 x 1024: keeps every tile of a record 1024-aligned
+constexpr uint32_t REC_B1 = 0, REC_T = 32768, REC_G = 40960, REC_B2 = 41984;
+constexpr uint32_t REC_B1_BYTES = REC_G + 256 - REC_B1;   // B1, T and g: one copy
+constexpr uint32_t REC_B2_BYTES = 24576;
+constexpr uint32_t REC_BYTES = 66560;   // 65 x 1024: keeps every tile of a record 1024-aligned
+__host__ __device__ constexpr uint32_t rec_w(int par, int hf) { return REC_B1 + hf * 16384 + (par ? 8192 : 0); }
+__host__ __device__ constexpr uint32_t rec_q(int par, int hf) { return REC_B1 + hf * 16384 + (par ? 0 : 8192); }
+__host__ __device__ constexpr uint32_t rec_p(int par) { return REC_B2 + (par ? 16384 : 0); }
+__host__ __device__ constexpr uint32_t rec_kt(int par, int hf) { return REC_B2 + (par ? 0 : 8192) + hf * 8192; }
 
 constexpr uint32_t OFF_QK = 0;          // [Q;K]: 128 token rows x d_k, halves of 16384
 constexpr int LDA = 68;                 // fp32 64 x 64 work matrices: 16-byte aligned rows
@@ -162,6 +173,7 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int64_t rem = (int64_t)p.cu[seq + 1] - t0;
     const int n = (int)(rem < C ? rem : C);
     const int j = h / (Hv / p.Hk);
+    const int par = (gc - p.chunk_off[seq]) & 1;   // parity of the chunk within its sequence
     uint8_t* rec = p.rec + ((int64_t)gc * Hv + h) * REC_BYTES;
 
     if (tid == 0) {
@@ -207,26 +219,7 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
     if (!mbar_wait_bounded(bar_ld, 0)) atomicOr((unsigned*)s_abort, 2u);
     __syncthreads();
-    if (tid < C) {
-        reinterpret_cast<float*>(rec + REC_G)[tid] = s_g[tid];
-        s_eg[tid] = __expf(s_g[tid]);
-    }
     bool ok = *s_abort == 0;
-    __syncthreads();   // e^g
-    if (ok) {   // Q~ = diag(e^g) Q -> the record (same swizzled image as the Q rows here)
-        for (int idx = tid; idx < C * 16; idx += NT) {
-            const int r = idx >> 4, c16 = idx & 15;
-            const uint32_t off = (c16 >> 3) * 16384 + swz128(r, c16 & 7);
-            uint4 v;
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                         : "r"(sb + OFF_QK + off));
-            const float e = s_eg[r];
-            const float2 a0 = unpack_half2(v.x), a1 = unpack_half2(v.y), a2 = unpack_half2(v.z), a3 = unpack_half2(v.w);
-            stg128(rec + REC_Q + (c16 >> 3) * 8192 + swz128(r, c16 & 7), pack_half2(a0.x * e, a0.y * e),
-                   pack_half2(a1.x * e, a1.y * e), pack_half2(a2.x * e, a2.y * e), pack_half2(a3.x * e, a3.y * e));
-        }
-    }
 
     // ---- [Q;K] K^T ----
     if (ok && tid == 0) {
@@ -238,6 +231,26 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                     idesc_f16(128, 64, 0, 0), ks > 0);
         }
         mma_commit(bar);
+    }
+    if (tid < C) {
+        reinterpret_cast<float*>(rec + REC_G)[tid] = s_g[tid];
+        s_eg[tid] = __expf(s_g[tid]);
+    }
+    __syncthreads();   // e^g
+    if (ok) {   // Q~ and K~ -> the record (same swizzled rows as the Q and K tiles here)
+        const float gC = s_g[C - 1];
+        for (int idx = tid; idx < 2 * C * 16; idx += NT) {
+            const int kk = idx >= C * 16, r = (idx >> 4) & (C - 1), c16 = idx & 15, hf = c16 >> 3;
+            const uint32_t sw = swz128(r, c16 & 7);
+            uint4 v;
+            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                         : "r"(sb + OFF_QK + hf * 16384 + kk * (C * 128) + sw));
+            const float e = kk ? (r < n ? __expf(gC - s_g[r]) : 0.f) : s_eg[r];
+            const float2 a0 = unpack_half2(v.x), a1 = unpack_half2(v.y), a2 = unpack_half2(v.z), a3 = unpack_half2(v.w);
+            stg128(rec + (kk ? rec_kt(par, hf) : rec_q(par, hf)) + sw, pack_half2(a0.x * e, a0.y * e),
+                   pack_half2(a1.x * e, a1.y * e), pack_half2(a2.x * e, a2.y * e), pack_half2(a3.x * e, a3.y * e));
+        }
     }
     if (ok && !mbar_wait_bounded(bar, 0)) atomicOr((unsigned*)s_abort, 1u);
     __syncthreads();
@@ -288,7 +301,7 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const __half lo = pr[(8 * q8 + 2 * i) * 66 + jj], hi = pr[(8 * q8 + 2 * i + 1) * 66 + jj];
                 w4[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
             }
-            stg128(rec + REC_P + swz128(jj, q8), w4[0], w4[1], w4[2], w4[3]);
+            stg128(rec + rec_p(par) + swz128(jj, q8), w4[0], w4[1], w4[2], w4[3]);
         }
     }
     __syncthreads();
@@ -390,7 +403,7 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
                 const __half lo = wt[(8 * q8 + 2 * i) * 66 + c], hi = wt[(8 * q8 + 2 * i + 1) * 66 + c];
                 w4[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
             }
-            stg128(rec + REC_W + (q8 >> 3) * 8192 + swz128(c, q8 & 7), w4[0], w4[1], w4[2], w4[3]);
+            stg128(rec + rec_w(par, q8 >> 3) + swz128(c, q8 & 7), w4[0], w4[1], w4[2], w4[3]);
         }
     } else if (tid == 0) {
         record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));
