@@ -71,7 +71,7 @@ Layout workspace_layout(const gdn_config* c, int64_t T, int64_t n_seqs) {
 // Opt in to > 48 KiB of dynamic shared memory, once per device and kernel.
 template <typename K>
 cudaError_t ensure_smem(K kernel, int variant, size_t bytes) {
-    static bool done[64][8];
+    static bool done[64][16];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -110,6 +110,48 @@ bool head_tile_map(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D map over a row-major [T][C] bf16 activation: boxes of 64 channels x 35
+// tokens (the conv tile), no swizzle; rows outside [0, T) read as zero.
+bool conv_tile_map(CUtensorMap* m, const void* base, int C, int64_t T) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)C, (cuuint64_t)T};
+    cuuint64_t strides[1] = {(cuuint64_t)C * 2};
+    cuuint32_t box[2] = {(cuuint32_t)gdn::ctile::BOXW, (cuuint32_t)gdn::ctile::ROWS};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// 2-D map over z as [T][Hv * dv] (bf16 or fp32): boxes of d_v channels x 64
+// tokens (one chunk of one head), no swizzle; rows past T read as zero.
+bool z_rows_map(CUtensorMap* m, const void* base, bool bf16, int width, int dv, int64_t T) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    const int eb = bf16 ? 2 : 4;
+    cuuint64_t dims[2] = {(cuuint64_t)width, (cuuint64_t)T};
+    cuuint64_t strides[1] = {(cuuint64_t)width * eb};
+    cuuint32_t box[2] = {(cuuint32_t)dv, (cuuint32_t)gdn::norm::C};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+               const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+               CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Streaming multiprocessors of the current device (cached per device).
+int sm_count() {
+    static int count[64];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (dev < 64 && count[dev]) return count[dev];
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    if (dev < 64) count[dev] = n;
+    return n;
+}
+
 template <typename TA, typename TO>
 cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void* q, const void* k,
                            const void* v, const void* a, const void* b, const void* z, void* conv_state,
@@ -137,22 +179,46 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     if (e != cudaSuccess) return e;
     e = ensure_smem(k_scan, 6 + (sizeof(TO) == 2 ? 0 : 1), gdn::scan::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    CUtensorMap tm_q, tm_k, tm_v;
+    e = ensure_smem(gdn::norm::gdn_gated_norm_kernel<TA, TO>, 8 + (sizeof(TA) == 4 ? 2 : 0) + (sizeof(TO) == 4 ? 1 : 0),
+                    gdn::norm::smem_bytes<TA, TO>());
+    if (e != cudaSuccess) return e;
+    CUtensorMap tm_q, tm_k, tm_v, tm_z;
     const int Hk = c->n_k_heads, Hv = c->n_v_heads;
+    if (!z_rows_map(&tm_z, z, sizeof(TA) == 2, Hv * c->d_v, c->d_v, T)) return cudaErrorInvalidValue;
     if (!head_tile_map(&tm_q, ca.qh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, Hk, T) ||
         !head_tile_map(&tm_k, ca.kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, Hk, T) ||
         !head_tile_map(&tm_v, ca.vh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_v, Hv, T))
         return cudaErrorInvalidValue;
     const int Ctot = 2 * c->n_k_heads * c->d_k + c->n_v_heads * c->d_v;
     const int cblocks = (Ctot / 8 + gdn::kConvThreads - 1) / gdn::kConvThreads;
-    const int64_t tblocks = (T + gdn::conv_tokens<TA>() - 1) / gdn::conv_tokens<TA>();
+    const int64_t tblocks = (T + gdn::kConvRun - 1) / gdn::kConvRun;
     const int64_t max_chunks = (T + gdn::intra::C - 1) / gdn::intra::C + n_seqs;
     if (tblocks > 0x7fffffff || max_chunks * Hv > 0x7fffffff) return cudaErrorInvalidValue;
     int32_t* chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off);
     uint8_t* recs = wsb + L.rec_off;
     void* otiles = wsb + L.o_off;
 
-    gdn::conv_silu_norm_kernel<TA><<<dim3((unsigned)tblocks, cblocks), gdn::kConvThreads, 0, st>>>(ca);
+    // the tiled conv for bf16 activations whose q, k and v widths are multiples of its slice
+    const int Cq = c->n_k_heads * c->d_k, Cv = c->n_v_heads * c->d_v;
+    bool tiled = sizeof(TA) == 2 && Cq % gdn::ctile::CH == 0 && Cv % gdn::ctile::CH == 0;
+    CUtensorMap tm_cq, tm_ck, tm_cv;
+    auto k_conv = c->d_k == 32 ? gdn::conv_tile_kernel<4> : c->d_k == 64 ? gdn::conv_tile_kernel<8>
+                                                                           : gdn::conv_tile_kernel<16>;
+    if (tiled) {
+        tiled = conv_tile_map(&tm_cq, q, Cq, T) && conv_tile_map(&tm_ck, k, Cq, T) && conv_tile_map(&tm_cv, v, Cv, T);
+        e = ensure_smem(k_conv, 12 + (c->d_k == 32 ? 0 : c->d_k == 64 ? 1 : 2), gdn::ctile::SMEM_BYTES);
+        if (e != cudaSuccess) return e;
+    }
+    if (tiled) {
+        const int n_slices = Ctot / gdn::ctile::CH;
+        const int64_t n_tiles = (T + gdn::ctile::TOK - 1) / gdn::ctile::TOK;
+        int64_t parts = (int64_t)2 * sm_count() / n_slices;
+        parts = parts < 1 ? 1 : parts > n_tiles ? n_tiles : parts;
+        k_conv<<<(unsigned)(n_slices * parts), gdn::ctile::NT, gdn::ctile::SMEM_BYTES, st>>>(
+            tm_cq, tm_ck, tm_cv, ca, (int)parts);
+    } else {
+        gdn::conv_silu_norm_kernel<TA><<<dim3((unsigned)tblocks, cblocks), gdn::kConvThreads, 0, st>>>(ca);
+    }
     gdn::conv_state_update_kernel<TA><<<dim3(n_seqs, (Ctot + 255) / 256), 256, 0, st>>>(ca, conv_state);
     gdn::intra::chunk_offsets_kernel<<<1, 1024, 0, st>>>(cu, n_seqs, chunk_off);
 
@@ -172,10 +238,13 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     k_scan<<<(unsigned)n_seqs * Hv, gdn::scan::NT, gdn::scan::SMEM_BYTES, st>>>(tm_v, sa);
 
     gdn::norm::Args na;
-    na.o = otiles; na.z = z; na.norm_w = w->norm_weight;
+    na.o = otiles; na.norm_w = w->norm_weight;
     na.cu = cu; na.chunk_off = chunk_off; na.out = out;
     na.n_seqs = n_seqs; na.Hv = Hv; na.dv = c->d_v; na.eps = c->norm_eps;
-    gdn::norm::gdn_gated_norm_kernel<TA, TO><<<(unsigned)(max_chunks * Hv), gdn::norm::NT, 0, st>>>(na);
+    int64_t norm_ctas = (int64_t)sm_count() * (232448 / (int64_t)gdn::norm::smem_bytes<TA, TO>());
+    norm_ctas = norm_ctas < max_chunks * Hv ? norm_ctas : max_chunks * Hv;
+    gdn::norm::gdn_gated_norm_kernel<TA, TO>
+        <<<(unsigned)norm_ctas, gdn::norm::NT, gdn::norm::smem_bytes<TA, TO>(), st>>>(tm_z, na);
     return cudaGetLastError();
 }
 

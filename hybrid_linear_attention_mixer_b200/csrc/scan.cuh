@@ -1,6 +1,6 @@
 // State chain of the chunked gated delta rule on the sm_100a tensor cores.
 //
-// One CTA (17 warps) walks one (sequence, value head) chain chunk by chunk
+// One CTA (18 warps) walks one (sequence, value head) chain chunk by chunk
 // (C = 64 tokens).  The state-independent factors of every chunk come from the
 // intra-chunk kernel's records (intra.cuh: -W, Q~, T, g, P, K~), whose tiles are
 // already the shared-memory images the tensor cores read.  With S0 the state
@@ -17,8 +17,8 @@
 //   MMA1  (d,e) S [-W ; Q~]^T, N = 128 -> [U2^T | O^T] += [A: S, TMEM]
 //   MMA2  (f,g) U^T [P ; K~^T]^T, N=192 -> [O^T | S]  += [A: U^T, TMEM; B MN-major]
 // with Q~ = diag(e^g) Q and K~ = diag(e^{g_C - g}) K.  (c) does not depend on the
-// state, so its k-steps are issued once MMA1 and MMA2 of the previous chunk have
-// completed and run while U^T and the new state are converted.  The fp32 state S lives in TMEM as an
+// state: the loading warp issues it once MMA2 of the previous chunk has completed,
+// so it runs while that chunk's new state is converted.  The fp32 state S lives in TMEM as an
 // accumulator: before MMA2 it holds e^{g_C} S0, so MMA2 leaves S_C.  The operand
 // tiles and the U, O accumulators alternate with chunk parity so that O is
 // double-buffered while both fused MMAs keep contiguous outputs:
@@ -28,10 +28,14 @@
 // of the new state.  While MMA1 runs, the 16 worker warps write the decayed state
 // accumulator; while MMA2
 // runs, they write the previous chunk's o tile (and zero its accumulator for the
-// chunk after next).  A 17th warp issues every MMA and every copy, so that its
-// waits on the tensor pipe delay no other work.  Loads are double-buffered: v
-// (TMA) and the record's B1 image, T and g (one bulk copy) two chunks ahead, its
-// B2 image (one bulk copy) one chunk ahead.
+// chunk after next).  A 17th warp issues the chain's MMAs, so that its waits on
+// the tensor pipe delay no other work, and an 18th issues every copy and (c): a bulk copy
+// holds its issuing thread for about as long as the copy engine takes to walk
+// its bytes, so copies stay off the MMA chain.  The loader meets the others
+// only through mbarriers (buffer released, o tile staged, staging buffer free),
+// never at a CTA barrier.  Loads are double-buffered two chunks ahead: v (TMA),
+// the record's B1 image with T and g (one bulk copy) and its B2 image (one
+// bulk copy).
 #pragma once
 #include "device.cuh"
 #include "intra.cuh"
@@ -41,8 +45,10 @@ namespace scan {
 
 constexpr int C = 64;
 constexpr int NW = 512;               // 16 worker warps: 4 per TMEM lane quadrant
-constexpr int NT = NW + 32;           // + the issuing warp
-constexpr int IW = NW / 32;           // the issuing warp: every MMA, load and store
+constexpr int IW = NW / 32;           // the issuing warp: every MMA
+constexpr int LW = IW + 1;            // the loading warp: every copy
+constexpr int NMAIN = NW + 32;        // workers + issuer: they meet at named barrier 1
+constexpr int NT = NMAIN + 32;
 
 // Shared memory (bytes from a 1024-aligned base); pairs are indexed by chunk parity.
 constexpr uint32_t OFF_R = 0;           // x2: the record's B1 image (32 KiB), T (8 KiB), g (256 B)
@@ -53,7 +59,7 @@ constexpr uint32_t OFF_B2 = OFF_V + 2 * 16384;       // x2: the record's B2 imag
 constexpr uint32_t B2_STRIDE = 24576;
 constexpr uint32_t OFF_OST = OFF_B2 + 2 * B2_STRIDE; // o tile staging: 2 x 16 KiB (or 1 x 32 KiB)
 constexpr uint32_t OFF_BAR = OFF_OST + 32768;        // mbarriers, TMEM address, abort flag, counters
-constexpr uint32_t SMEM_USED = OFF_BAR + 128;
+constexpr uint32_t SMEM_USED = OFF_BAR + 192;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 static_assert(R_STRIDE % 1024 == 0 && R_STRIDE >= intra::REC_B1_BYTES, "record slot");
@@ -76,6 +82,11 @@ struct Args {
     int Hk, Hv, dk, dv;
 };
 
+__device__ __forceinline__ void main_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NMAIN) : "memory"); }
+__device__ __forceinline__ void mbar_arrive(uint32_t bar) {
+    asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
 template <typename TO>
 __global__ void __launch_bounds__(NT, 1)
 gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
@@ -85,14 +96,21 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sb = (raw + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (sb - raw);
-    const uint32_t bar = sb + OFF_BAR;                    // tensor-core commits
-    const uint32_t bar_ld0 = sb + OFF_BAR + 8;            // +8 per parity: v, B1, T, g
-    const uint32_t bar_b20 = sb + OFF_BAR + 24;           // +8 per parity: B2
+    const uint32_t bar = sb + OFF_BAR;                    // tensor-core commits (issuer)
+    const uint32_t bar_ld0 = sb + OFF_BAR + 8;            // [2] v, B1, T, g arrived
+    const uint32_t bar_b20 = sb + OFF_BAR + 24;           // [2] B2 arrived
     const uint32_t bar_fin = sb + OFF_BAR + 40;           // abort path: every MMA issued so far
-    volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 48);
-    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 52);
-    // loads issued per barrier (ld x2, B2 x2): the abort path waits for the last phase of each
-    volatile int* s_issued = reinterpret_cast<volatile int*>(smem + OFF_BAR + 64);
+    const uint32_t ev10 = sb + OFF_BAR + 48;              // [2] MMA1 of a chunk done: its v/record buffer is free
+    const uint32_t ev20 = sb + OFF_BAR + 64;              // [2] MMA2 done, previous o tile staged
+    const uint32_t evo = sb + OFF_BAR + 80;               // a staging buffer is free again
+    const uint32_t ev_end = sb + OFF_BAR + 88;            // the last o tile is staged
+    const uint32_t evc0 = sb + OFF_BAR + 96;              // [2] (c) of a chunk is in its U accumulator
+    const uint32_t bar_lfin = sb + OFF_BAR + 112;         // the loading warp's own MMAs (drain)
+    const uint32_t ev_ldone = sb + OFF_BAR + 120;         // the loading warp has drained everything
+    volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 128);
+    volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 132);
+    // loads issued per barrier (ld x2, B2 x2): the loader's drain waits for the last phase of each
+    volatile int* s_issued = reinterpret_cast<volatile int*>(smem + OFF_BAR + 136);
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool worker = tid < NW;
@@ -109,8 +127,8 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
     uint8_t* otile0 = static_cast<uint8_t*>(p.o) + first * O_BYTES;
     const int64_t o_stride = (int64_t)Hv * O_BYTES;
 
-    // v tile and the record's B1 image, T and g of chunk ci into buffer ci & 1
-    auto issue_chunk = [&](int ci) {
+    // ---- the loading warp's copies ----
+    auto issue_chunk = [&](int ci) {   // v tile and the record's B1 image, T and g of chunk ci
         const int bb = ci & 1;
         if (lane == 0) s_issued[bb]++;
         mbar_arrive_expect_tx_w(bar_ld0 + 8 * bb, LD_BYTES);
@@ -128,26 +146,28 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         bulk_g2s_w(sb + OFF_B2 + bb * B2_STRIDE, rec0 + ci * rec_stride + intra::REC_B2, intra::REC_B2_BYTES,
                    bar_b20 + 8 * bb);
     };
+    auto issue_o = [&](int ce) {
+        bulk_s2g_commit_w(otile0 + ce * o_stride, sb + OFF_OST + (ce % kOBufs) * 16384, O_BYTES);
+    };
     auto wait_par = [&](uint32_t bar0, int ci) {
         if (!mbar_wait_bounded(bar0 + 8 * (ci & 1), (ci >> 1) & 1)) atomicOr((unsigned*)s_abort, 2u);
     };
 
-    if (warp == IW) {
+    if (warp == LW) {
         if (lane == 0) {
             mbar_init(bar, 1);
 #pragma unroll
-            for (int i = 0; i < 5; i++) mbar_init(bar_ld0 + 8 * i, 1);   // ld x2, B2 x2, fin
+            for (int i = 0; i < 15; i++) mbar_init(bar_ld0 + 8 * i, 1);   // ld, B2, fin, ev1, ev2, evo, end, evc, lfin, ldone
             fence_mbar_init();
             *s_abort = 0;
             for (int i = 0; i < 4; i++) s_issued[i] = 0;
         }
         __syncwarp();
-        issue_chunk(0);
-        if (nchunks > 1) issue_chunk(1);
+        issue_chunk(0);   // chunk 1's loads follow once the chain can start
         issue_b2(0);
     }
     if (warp == 0) {
-        tmem_alloc(sb + OFF_BAR + 48, TMEM_COLS);
+        tmem_alloc(sb + OFF_BAR + 128, TMEM_COLS);
         tmem_relinquish();
     }
     const int dv_r = 32 * qd + lane;   // this worker's state row; columns [32 cs, 32 cs + 32)
@@ -155,38 +175,97 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
     float Sv[32];   // this worker's slice of the state at the start of the current chunk
     if (worker) {
 #pragma unroll
-        for (int i = 0; i < 32; i++) {
-            const int col = 32 * cs + i;
-            Sv[i] = (dv_r < dv && col < dk) ? gstate[(int64_t)dv_r * dk + col] : 0.f;
+        for (int i4 = 0; i4 < 8; i4++) {   // 16-byte loads (d_k and the slice start are multiples of 4)
+            const int col = 32 * cs + 4 * i4;
+            float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+            if (dv_r < dv && col < dk) v = *reinterpret_cast<const float4*>(gstate + (int64_t)dv_r * dk + col);
+            Sv[4 * i4] = v.x; Sv[4 * i4 + 1] = v.y; Sv[4 * i4 + 2] = v.z; Sv[4 * i4 + 3] = v.w;
         }
     }
     tc_fence_before();
-    __syncthreads();
+    __syncthreads();   // every warp: barriers initialised, TMEM allocated
     tc_fence_after();
     const uint32_t tmem = *s_tmem;
+
+    if (warp == LW) {
+        // (c) of chunk ce: U2^T = V^T T^T into its U accumulator, committed to evc[ce & 1].  It
+        // is issued once MMA2 of the chunk before has completed, so it runs while that chunk's
+        // new state is converted, and MMA1 of chunk ce accumulates onto it.
+        const uint64_t dV0 = sdesc(sb + OFF_V, 8192, 1024);
+        const uint64_t dT0 = sdesc(sb + OFF_R + R_T, 16, 1024);
+        constexpr uint32_t ID_C = idesc_f16(128, 64, 1, 0);
+        int c_issued = 0;
+        auto issue_c = [&](int ce) {
+            const int bb = ce & 1;
+            tc_fence_after();
+#pragma unroll
+            for (int ks = 0; ks < 4; ks++)
+                mma_f16_w(tmem + acc_u(bb), dV0 + bb * 1024 + ks * 128, dT0 + bb * (R_STRIDE >> 4) + ks * 2, ID_C,
+                          ks > 0);
+            mma_commit_w(evc0 + 8 * bb);
+            c_issued++;
+        };
+        // Waits for an event of the other warps; gives up on their abort or after the time limit.
+        auto lwait = [&](uint32_t b, uint32_t parity) -> bool {
+            if (mbar_try_wait(b, parity)) return true;
+            const unsigned long long t0 = global_ns();
+            while (!mbar_try_wait(b, parity)) {
+                if (*s_abort) return false;
+                if (global_ns() - t0 > kWaitLimitNs) {
+                    atomicOr((unsigned*)s_abort, 2u);
+                    return false;
+                }
+            }
+            return true;
+        };
+        bool ok = lwait(bar_ld0, 0);
+        if (ok) issue_c(0);
+        if (ok && nchunks > 1) {
+            issue_chunk(1);
+            issue_b2(1);
+        }
+        for (int ci = 0; ci < nchunks && ok; ci++) {
+            ok = lwait(ev10 + 8 * (ci & 1), (ci >> 1) & 1);         // MMA1 of chunk ci is done with buffer ci & 1
+            if (!ok) break;
+            if (ci + 2 < nchunks) {
+                fence_async_smem();
+                issue_chunk(ci + 2);
+            }
+            ok = lwait(ev20 + 8 * (ci & 1), (ci >> 1) & 1);         // MMA2 of chunk ci done; o of chunk ci - 1 staged
+            if (!ok) break;
+            if (ci + 1 < nchunks) {   // U accumulator (ci + 1) & 1 was read by the U conversion of chunk ci - 1
+                ok = lwait(bar_ld0 + 8 * ((ci + 1) & 1), ((ci + 1) >> 1) & 1);
+                if (!ok) break;
+                issue_c(ci + 1);      // first: the next MMA1 waits for it
+            }
+            if (ci + 2 < nchunks) issue_b2(ci + 2);
+            if (ci > 0) issue_o(ci - 1);
+            if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();   // the staging buffer of o(ci) is free
+            if (lane == 0) mbar_arrive(evo);
+        }
+        if (ok && lwait(ev_end, 0)) issue_o(nchunks - 1);
+        // drain: every copy this warp issued completes before the CTA may exit
+        bulk_wait<0>();
+        if (lane == 0)
+            for (int i = 0; i < 4; i++)   // the last phase issued on each load barrier (returns at once if complete)
+                if (s_issued[i] > 0) mbar_wait_bounded(bar_ld0 + 8 * i, (uint32_t)(s_issued[i] - 1) & 1u);
+        if (c_issued > 0) {   // every MMA of this warp has completed
+            mma_commit_w(bar_lfin);
+            mbar_wait_bounded(bar_lfin, 0);
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(ev_ldone);
+        return;
+    }
+
+    // ---- workers and the issuer ----
     const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
     const float inv_sqrt_dk = rsqrtf((float)dk);
     uint32_t mphase = 0;
-
-    // Shared-memory descriptors; per-step offsets are added to the start-address field.
-    const uint64_t dV0 = sdesc(sb + OFF_V, 8192, 1024);
-    const uint64_t dT0 = sdesc(sb + OFF_R + R_T, 16, 1024);
     const uint64_t dB10 = sdesc(sb + OFF_R, 16, 1024);
     const uint64_t dB20 = sdesc(sb + OFF_B2, 8192, 1024);
-    constexpr uint32_t ID_C = idesc_f16(128, 64, 1, 0);      // (c)
     constexpr uint32_t ID_DE = idesc_f16(128, 128, 0, 0);    // (d,e)
     constexpr uint32_t ID_FG = idesc_f16(128, 192, 0, 1);    // (f,g)
-
-    // (c) of chunk ce, k-steps [k0, k1): U2^T = V^T T^T into its U accumulator (issuer; the
-    // steps run in the tensor pipe's idle windows and are committed with the next MMA)
-    auto issue_c = [&](int ce, int k0, int k1) {
-        wait_par(bar_ld0, ce);
-        tc_fence_after();
-        const int bb = ce & 1;
-        for (int ks = k0; ks < k1; ks++)
-            mma_f16_w(tmem + acc_u(bb), dV0 + bb * 1024 + ks * 128, dT0 + bb * (R_STRIDE >> 4) + ks * 2, ID_C,
-                      ks > 0);
-    };
     // fp16 copy of the state: the A operand of MMA1
     auto put_state_a = [&]() {
         uint32_t h16[16];
@@ -201,8 +280,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         for (int i = 0; i < 32; i++) d[i] = __float_as_uint(decay * Sv[i]);
         tmem_st32(tl + ACC_S + 32 * cs, d);
     };
-    // o = O / sqrt(d_k) of chunk ce -> staging, and its accumulator zeroed for chunk ce + 2;
-    // the issuer stores the tile after the next barrier (its buffer is free: see bulk_wait_read)
+    // o = O / sqrt(d_k) of chunk ce -> staging, and its accumulator zeroed for chunk ce + 2
     auto stage_o = [&](int ce) {
         uint32_t o[16];
         tmem_ld16(tl + acc_o(ce & 1) + 16 * cs, o);
@@ -214,12 +292,8 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         for (int i = 0; i < 16; i++) o[i] = 0u;
         tmem_st16(tl + acc_o(ce & 1) + 16 * cs, o);
     };
-    auto issue_o = [&](int ce) {
-        bulk_s2g_commit_w(otile0 + ce * o_stride, sb + OFF_OST + (ce % kOBufs) * 16384, O_BYTES);
-    };
 
-    // ---- prologue: zero O accumulators, fp16 S0, (c) of chunk 0 ----
-    if (warp == IW) issue_c(0, 0, 4);
+    // ---- prologue: zero O accumulators, fp16 S0 ----
     if (worker) {
         uint32_t z[16];
 #pragma unroll
@@ -229,14 +303,14 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         put_state_a();
     }
     tc_fence_before();
-    __syncthreads();
+    main_sync();
     if (*s_abort) goto abort_;
 
 #define GDN_MMA_WAIT()                                                                               \
     do {                                                                                             \
         if (warp == IW && !mbar_wait_bounded(bar, mphase)) atomicOr((unsigned*)s_abort, 1u);       \
         mphase ^= 1u;                                                                                \
-        __syncthreads();                                                                             \
+        main_sync();                                                                                 \
         if (*s_abort) goto abort_;                                                                   \
         tc_fence_after();                                                                            \
     } while (0)
@@ -247,6 +321,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         // ---- MMA1: (d,e) [U2^T | O^T] += S [-W ; Q~]^T ((c) and zeroed O are already there) ----
         if (warp == IW) {
             wait_par(bar_ld0, ci);
+            wait_par(evc0, ci);   // (c) of chunk ci
             tc_fence_after();
             const uint32_t d1 = tmem + (b ? ACC_O1 : ACC_U0);
 #pragma unroll
@@ -254,8 +329,6 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
                 mma_f16_ta_w(d1, tmem + TA_S + ks * 8, dB10 + b * (R_STRIDE >> 4) + (ks >> 2) * 1024 + (ks & 3) * 2,
                              ID_DE, 1);
             mma_commit_w(bar);
-            if (ci + 1 < nchunks) issue_b2(ci + 1);   // its buffer was freed by MMA2 of chunk ci - 1
-            if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();   // staging buffer of stage_o(ci - 1)
         }
         // ---- workers, while MMA1 runs: the decayed state accumulator ----
         if (worker) {
@@ -263,9 +336,11 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
             put_state_acc(__expf(reinterpret_cast<const float*>(smem + OFF_R + b * R_STRIDE + R_G)[C - 1]));
         }
         GDN_MMA_WAIT();
+        if (warp == IW && lane == 0) mbar_arrive(ev10 + 8 * b);   // MMA1, (c) and the decay are done with buffer b
 
-        // ---- U^T -> fp16 A operand; (c) of the next chunk starts in the tensor pipe ----
-        if (warp == IW && ci + 1 < nchunks) issue_c(ci + 1, 0, 2);
+        // ---- U^T -> fp16 A operand ----
+        if (warp == IW && ci > 0 && !mbar_wait_bounded(evo, (ci - 1) & 1))   // staging buffer for o(ci - 1)
+            atomicOr((unsigned*)s_abort, 2u);
         if (worker) {
             uint32_t r16[16], u[8];
             tmem_ld16(tl + acc_u(b) + 16 * cs, r16);
@@ -274,7 +349,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
             tmem_st8(tl + TA_U + 8 * cs, u);
         }
         tc_fence_before();
-        __syncthreads();
+        main_sync();
 
         // ---- MMA2: [O^T | S] (parity 0) or [S | O^T] (parity 1) += U^T [P ; K~^T]^T ----
         if (warp == IW) {
@@ -285,20 +360,13 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
             for (int ks = 0; ks < 4; ks++)
                 mma_f16_ta_w(d2, tmem + TA_U + ks * 8, dB20 + b * (B2_STRIDE >> 4) + ks * 128, ID_FG, 1);
             mma_commit_w(bar);
-            if (ci + 2 < nchunks) {   // MMA1, (c) and the decay of chunk ci are done with buffer b
-                fence_async_smem();
-                issue_chunk(ci + 2);
-            }
         }
         // ---- workers, while MMA2 runs: the previous chunk's o tile ----
         if (worker && ci > 0) stage_o(ci - 1);
         GDN_MMA_WAIT();
+        if (warp == IW && lane == 0) mbar_arrive(ev20 + 8 * b);   // B2 buffer b free; o(ci - 1) staged
 
-        // ---- new state: its fp16 copy for the next MMA1, or the final state; the rest of (c) ----
-        if (warp == IW) {
-            if (ci > 0) issue_o(ci - 1);
-            if (ci + 1 < nchunks) issue_c(ci + 1, 2, 4);
-        }
+        // ---- new state: its fp16 copy for the next MMA1, or the final state ----
         if (worker) {
             uint32_t r32[32];
             tmem_ld32(tl + ACC_S + 32 * cs, r32);
@@ -308,50 +376,46 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
                 put_state_a();
             } else {
 #pragma unroll
-                for (int i = 0; i < 32; i++) {
-                    const int col = 32 * cs + i;
-                    if (dv_r < dv && col < dk) gstate[(int64_t)dv_r * dk + col] = Sv[i];
+                for (int i4 = 0; i4 < 8; i4++) {
+                    const int col = 32 * cs + 4 * i4;
+                    if (dv_r < dv && col < dk)
+                        *reinterpret_cast<float4*>(gstate + (int64_t)dv_r * dk + col) =
+                            make_float4(Sv[4 * i4], Sv[4 * i4 + 1], Sv[4 * i4 + 2], Sv[4 * i4 + 3]);
                 }
             }
         }
         tc_fence_before();
-        __syncthreads();
+        main_sync();
         if (*s_abort) goto abort_;
     }
-    if (warp == IW) {
-        if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();
-    }
-    __syncthreads();
+    if (warp == IW && !mbar_wait_bounded(evo, (nchunks - 1) & 1)) atomicOr((unsigned*)s_abort, 2u);
+    main_sync();
+    if (*s_abort) goto abort_;
     if (worker) stage_o(nchunks - 1);
     tc_fence_before();
-    __syncthreads();
-    if (warp == IW) {
-        issue_o(nchunks - 1);
-        bulk_wait<0>();   // every o tile has reached global memory
-    }
-    __syncthreads();
+    main_sync();
+    if (warp == IW && lane == 0) mbar_arrive(ev_end);   // the loader stores the last tile
     if (warp == 0) {
+        mbar_wait_bounded(ev_ldone, 0);   // the loading warp's MMAs and copies are done
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
     return;
 
 abort_:
-    // A tensor-core commit or a copy never arrived: report it, give whatever is
-    // still in flight one more bounded wait, free tensor memory and return.  The
-    // recurrent state is left as it was.
+    // A tensor-core commit or a copy never arrived: report it, give the MMAs still in
+    // flight one more bounded wait, free tensor memory and return (the loading warp
+    // sees the flag and drains its own copies).  The recurrent state is left as it was.
     if (warp == IW) {
         if (lane == 0)
             record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));
         mma_commit_w(bar_fin);   // tracks every MMA the issuing lane has issued
         mbar_wait_bounded(bar_fin, 0);
-        for (int i = 0; i < 4; i++)   // the last phase issued on each barrier (returns at once if complete)
-            if (s_issued[i] > 0) mbar_wait_bounded(bar_ld0 + 8 * i, (uint32_t)(s_issued[i] - 1) & 1u);
-        bulk_wait<0>();
     }
     tc_fence_before();
-    __syncthreads();
+    main_sync();
     if (warp == 0) {
+        mbar_wait_bounded(ev_ldone, 0);   // the loading warp sees the flag and drains its MMAs and copies
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }

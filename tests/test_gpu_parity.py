@@ -110,6 +110,27 @@ def test_ragged_varlen_with_states():
     np.testing.assert_array_equal(g["rec_state"][4], c.rec_state[4].astype(np.float64))
 
 
+def test_bf16_small_heads_ragged_streaming_conv():
+    """bf16 activations at 2 key / 6 value heads of 64: q, k, v widths that are not
+    multiples of 512 channels take the streaming conv kernel (the tiled one needs
+    whole 512-channel slices); ragged lengths, an empty sequence, nonzero states."""
+    Hk, Hv, d, K = 2, 6, 64, 4
+    lens = [1, 63, 70, 0, 130, 2, 40]
+    T, N = sum(lens), len(lens)
+    w = inputs._weights(7, Hk, Hv, d, d, K)
+    acts = inputs._acts(7, T, Hk, Hv, d, d, True, "model")
+    rng = np.random.default_rng(7)
+    C = 2 * Hk * d + Hv * d
+    cs = inputs.f32_to_bf16_bits(rng.normal(size=(N, C, K - 1)).astype(np.float32))
+    rs = (0.05 * rng.normal(size=(N, Hv, d, d))).astype(np.float32)
+    cu = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    c = inputs.Case("small_bf16", Hk, Hv, d, d, K, 64, True, cu, w, acts, cs, rs)
+    g = L.gpu_prefill(c)
+    L.assert_parity(g, L.oracle_run(c))
+    np.testing.assert_array_equal(L.conv_state_bits(c, g["conv_state_t"]),
+                                  L.expected_conv_state(c, c.acts, c.conv_state, c.cu_seqlens))
+
+
 def test_varlen_8_full_size_sampled_heads():
     """The 8-sequence packed workload at full size; oracle on sampled value heads."""
     c = inputs.make_case("varlen_8")
