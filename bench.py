@@ -47,8 +47,8 @@ DECODE_BYTES_PER_STEP = (2 * DECODE_N * H_V * D * D * 4 + 2 * DECODE_N * C_CONV 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu DRAM bytes (read + write) per decode launch at batch 256, taken on the
 # decode kernel whose source hashes to DECODE_SRC_SHA; null once it changes.
-DECODE_TRAFFIC = None
-DECODE_SRC_SHA = None
+DECODE_TRAFFIC = 1593586090          # profiles/decode_256_launches.md (mean of 3 launches)
+DECODE_SRC_SHA = "9c863bc17a82d5f8"
 
 
 def peaks():
@@ -319,13 +319,14 @@ def main():
             "roofline": {"kernel": "gdn_decode_kernel", "bound": "hbm", "achieved": dec_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / pk["hbm_gbs"],
                          "traffic": traffic, "peak_source": src},
-            "prefill_roofline": {"kernels": "conv + chunk (whole prefill call)", "bound": "tensor",
+            "prefill_roofline": {"kernels": "whole prefill call (conv, conv state, chunk offsets, intra, scan, norm)", "bound": "tensor",
                                  "achieved": pre_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
                                  "frac": pre_tflops / pk["bf16_tflops"], "peak_source": src},
             "clocks": clocks.summary(),
             "e2e": {"value": PREFILL_T * world * K / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": K * (3 + args.decode_steps),
+            # per prefill call: conv, conv-state update, chunk offsets, intra-chunk, scan, gated norm
+            "gpu_launches": K * (6 + args.decode_steps),
             "context": {"pages_cost_model": "6.05 GiB KV+state at 256K tokens and 13.3 GFLOP/token "
                                             "decode at 4K (whole model, no hardware stated)"},
         }
