@@ -47,7 +47,7 @@ DECODE_BYTES_PER_STEP = (2 * DECODE_N * H_V * D * D * 4 + 2 * DECODE_N * C_CONV 
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu DRAM bytes (read + write) per decode launch at batch 256, taken on the
 # decode kernel whose source hashes to DECODE_SRC_SHA; null once it changes.
-DECODE_TRAFFIC = 1593586090          # profiles/decode_256_launches.md (mean of 3 launches)
+DECODE_TRAFFIC = 1593586090          # mean of 3 launches at batch 256
 DECODE_SRC_SHA = "9c863bc17a82d5f8"
 
 
