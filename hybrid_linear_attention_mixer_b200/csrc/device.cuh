@@ -86,6 +86,35 @@ __device__ __forceinline__ uint32_t swz128(uint32_t row, uint32_t chunk16) {
     return row * 128u + ((chunk16 ^ (row & 7u)) << 4);
 }
 
+// 16-byte shared-memory accesses by address, and fp16 x8 scaling
+__device__ __forceinline__ void sts128(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
+    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w)
+                 : "memory");
+}
+__device__ __forceinline__ uint4 lds128(uint32_t addr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(addr)
+                 : "memory");
+    return v;
+}
+// the same with packed half2 multiplies (the factor rounded to fp16 first)
+__device__ __forceinline__ uint4 scale8_h2(uint4 v, float s) {
+    const __half2 f = __float2half2_rn(s);
+    uint4 r;
+    const __half2* in = reinterpret_cast<const __half2*>(&v);
+    __half2* out = reinterpret_cast<__half2*>(&r);
+#pragma unroll
+    for (int i = 0; i < 4; i++) out[i] = __hmul2(in[i], f);
+    return r;
+}
+__device__ __forceinline__ uint4 scale8(uint4 v, float s) {
+    const float2 a = unpack_half2(v.x), b = unpack_half2(v.y), c = unpack_half2(v.z), d = unpack_half2(v.w);
+    return make_uint4(pack_half2(a.x * s, a.y * s), pack_half2(b.x * s, b.y * s),
+                      pack_half2(c.x * s, c.y * s), pack_half2(d.x * s, d.y * s));
+}
+
 // ---------------------------------------------------------------------------
 // mbarrier
 // ---------------------------------------------------------------------------

@@ -8,9 +8,13 @@
 //     P_rj = q_r.k_j e^{g_r - g_j}          (j <= r)
 //     W    = T diag(e^g) K
 // These are the state-independent factors of the chunk's update (see scan.cuh
-// for the state chain that consumes them).  [Q;K] K^T and K^T (T diag(e^g))^T
-// run as tcgen05 MMAs (fp16 operands, fp32 accumulators in TMEM); the
-// triangular solve runs in fp32 on the CUDA cores.
+// for the state chain that consumes them).  The chunk's k rows are stacked on
+// its q rows, so one tcgen05 MMA chain of the tile with itself gives K K^T and
+// K Q^T = P^T (before masks) with the chunk position j on the TMEM lanes: P^T
+// rows and A columns come straight out of TMEM.  W = T diag(e^g) K is a second
+// MMA with the chunk position on the lanes again.  fp16 operands, fp32
+// accumulators in TMEM; the triangular solve runs in fp32 on the CUDA cores.
+// Warps with nothing to take out of TMEM scale Q and K into Q~ and K~ in place.
 //
 // Each (chunk, value head) record written to the workspace holds the operand
 // tiles exactly as the scan kernel's tensor cores read them (128-byte swizzled
@@ -25,6 +29,7 @@
 //     +41984  B2 image, three MN-major atoms of 8192 B:
 //             [P^T | K~ half 0 | K~ half 1] (p = 0) or [K~ half 0 | K~ half 1 | P^T] (p = 1)
 //             (P^T: row j holds P[0..63][j]; K~: row c holds 64 d_k values)
+// Every tile is built in shared memory and written with a bulk copy.
 #pragma once
 #include "device.cuh"
 
@@ -42,7 +47,7 @@ __host__ __device__ constexpr uint32_t rec_q(int par, int hf) { return REC_B1 + 
 __host__ __device__ constexpr uint32_t rec_p(int par) { return REC_B2 + (par ? 16384 : 0); }
 __host__ __device__ constexpr uint32_t rec_kt(int par, int hf) { return REC_B2 + (par ? 0 : 8192) + hf * 8192; }
 
-constexpr uint32_t OFF_QK = 0;          // [Q;K]: 128 token rows x d_k, halves of 16384
+constexpr uint32_t OFF_QK = 0;          // [K;Q]: 128 token rows x d_k, halves of 16384 (k rows first)
 constexpr int LDA = 68;                 // fp32 64 x 64 work matrices: 16-byte aligned rows
 constexpr int LDY = 36;
 constexpr uint32_t OFF_A = 32768;       // A; after the solve, T' = T diag(e^g) (fp16 tile)
@@ -57,7 +62,7 @@ constexpr uint32_t SMEM_USED = OFF_BAR + 64;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(3 * SMEM_BYTES <= 232448, "three CTAs per SM");
 static_assert(OFF_A % 1024 == 0, "T' tile alignment");
-constexpr uint32_t ACC_QK = 0, ACC_W = 64, TMEM_COLS = 128;
+constexpr uint32_t ACC_D = 0, TMEM_COLS = 128;   // [K K^T | K Q^T], later W
 
 struct Args {
     const void* a;            // [T][Hv] act dtype
@@ -73,10 +78,6 @@ struct Args {
 
 __device__ __forceinline__ void stg128(void* p, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
     *reinterpret_cast<uint4*>(p) = make_uint4(x, y, z, w);
-}
-__device__ __forceinline__ void sts128(uint32_t addr, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w)
-                 : "memory");
 }
 
 // chunk_off[s] = sum_{i<s} ceil(len_i / C) (one CTA, any number of sequences)
@@ -117,14 +118,18 @@ __global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int32_t* cu, 
 }
 
 // C = sgn * L R for n x n blocks (n = 16 or 32; rows 16-byte aligned), 1 x 4
-// register tiles: thread t of nt takes tiles t, t + nt, ...
+// register tiles: thread t of nt takes tiles t, t + nt, ...  LTRI_L / LTRI_R: L or
+// R is lower triangular, so the products it zeroes are skipped.
+template <bool LTRI_L, bool LTRI_R>
 __device__ __forceinline__ void block_mm(const float* L, int ldl, const float* R, int ldr, float* Cm, int ldc,
                                          int n, float sgn, int t, int nt) {
     const int tpr = n >> 2;
     for (int tile = t; tile < n * tpr; tile += nt) {
         const int i = tile / tpr, j0 = (tile % tpr) * 4;
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int l0 = 0; l0 < n; l0 += 4) {
+        const int l_begin = LTRI_R ? j0 : 0;                 // R[l][j] = 0 for l < j
+        const int l_end = LTRI_L ? ((i >> 2) + 1) * 4 : n;   // L[i][l] = 0 for l > i
+        for (int l0 = l_begin; l0 < l_end; l0 += 4) {
             const float4 a = *reinterpret_cast<const float4*>(L + i * ldl + l0);
             const float av[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
@@ -156,6 +161,10 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const uint32_t bar = sb + OFF_BAR, bar_ld = sb + OFF_BAR + 8;
     volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 16);
     volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 20);
+    // staging of the record tiles in regions that are free by then
+    const uint32_t st_p = sb + OFF_X;                   // P^T: X (written only from the solve on)
+    const uint32_t st_t = sb + OFF_QK + 16384 + 8192;   // T: q rows of half 1 (Q~ is stored by then)
+    const uint32_t st_w = sb + OFF_X;                   // -W: X (dead once T is formed), 16 KiB
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int qd = warp & 3, half = warp >> 2;
@@ -184,8 +193,8 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         mbar_arrive_expect_tx(bar_ld, 4 * 8192);
 #pragma unroll
         for (int hf = 0; hf < 2; hf++) {
-            tma_load_3d(sb + OFF_QK + hf * 16384, &tm_q, 64 * hf, j, (int)t0, bar_ld);
-            tma_load_3d(sb + OFF_QK + hf * 16384 + C * 128, &tm_k, 64 * hf, j, (int)t0, bar_ld);
+            tma_load_3d(sb + OFF_QK + hf * 16384, &tm_k, 64 * hf, j, (int)t0, bar_ld);
+            tma_load_3d(sb + OFF_QK + hf * 16384 + C * 128, &tm_q, 64 * hf, j, (int)t0, bar_ld);
         }
     }
     if (warp == 0) {
@@ -221,14 +230,14 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     bool ok = *s_abort == 0;
 
-    // ---- [Q;K] K^T ----
+    // ---- [K;Q] [K;Q]^T: lanes 0-63 hold row j of [K K^T | K Q^T] ----
     if (ok && tid == 0) {
         tc_fence_after();
+        constexpr uint32_t ID = idesc_f16(128, 128, 0, 0);
 #pragma unroll
         for (int ks = 0; ks < 8; ks++) {
-            const uint32_t o = (ks >> 2) * 16384 + (ks & 3) * 32;
-            mma_f16(tmem + ACC_QK, sdesc(sb + OFF_QK + o, 16, 1024), sdesc(sb + OFF_QK + o + C * 128, 16, 1024),
-                    idesc_f16(128, 64, 0, 0), ks > 0);
+            const uint64_t d = sdesc(sb + OFF_QK + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024);
+            mma_f16(tmem + ACC_D, d, d, ID, ks > 0);
         }
         mma_commit(bar);
     }
@@ -236,77 +245,65 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         reinterpret_cast<float*>(rec + REC_G)[tid] = s_g[tid];
         s_eg[tid] = __expf(s_g[tid]);
     }
-    __syncthreads();   // e^g
-    if (ok) {   // Q~ and K~ -> the record (same swizzled rows as the Q and K tiles here)
-        const float gC = s_g[C - 1];
-        for (int idx = tid; idx < 2 * C * 16; idx += NT) {
-            const int kk = idx >= C * 16, r = (idx >> 4) & (C - 1), c16 = idx & 15, hf = c16 >> 3;
-            const uint32_t sw = swz128(r, c16 & 7);
-            uint4 v;
-            asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"
-                         : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                         : "r"(sb + OFF_QK + hf * 16384 + kk * (C * 128) + sw));
-            const float e = kk ? (r < n ? __expf(gC - s_g[r]) : 0.f) : s_eg[r];
-            const float2 a0 = unpack_half2(v.x), a1 = unpack_half2(v.y), a2 = unpack_half2(v.z), a3 = unpack_half2(v.w);
-            stg128(rec + (kk ? rec_kt(par, hf) : rec_q(par, hf)) + sw, pack_half2(a0.x * e, a0.y * e),
-                   pack_half2(a1.x * e, a1.y * e), pack_half2(a2.x * e, a2.y * e), pack_half2(a3.x * e, a3.y * e));
-        }
-    }
     if (ok && !mbar_wait_bounded(bar, 0)) atomicOr((unsigned*)s_abort, 1u);
     __syncthreads();
     ok = *s_abort == 0;
-    if (ok) {
+    if (ok && qd < 2) {
         tc_fence_after();
+        const int jr = 32 * qd + lane;     // chunk position j of this lane
+        const float gj = s_g[jr];
         uint32_t r32[32];
-        tmem_ld32(tl + ACC_QK + 32 * half, r32);
-        const int j0 = 32 * half;
-        if (qd < 2) {   // P rows -> fp16 rows [r][j] in shared memory (the X region, 132-byte rows)
-            const int r = 32 * qd + lane;
-            const float gr = s_g[r];
-            uint32_t* pr = reinterpret_cast<uint32_t*>(Xm) + r * 33 + j0 / 2;
+        if (half == 0) {
+            // column j of A: A[r][j] = beta_r e^{g_r - g_j} k_r.k_j for r > j
 #pragma unroll
-            for (int i = 0; i < 16; i++) {
-                const int jj = j0 + 2 * i;
-                const float e0 = __expf(fminf(gr - s_g[jj], 0.f));
-                const float e1 = __expf(fminf(gr - s_g[jj + 1], 0.f));
-                pr[i] = pack_half2(jj <= r ? __uint_as_float(r32[2 * i]) * e0 : 0.f,
-                                   jj + 1 <= r ? __uint_as_float(r32[2 * i + 1]) * e1 : 0.f);
-            }
-        } else {        // A rows -> shared memory
-            const int r = 32 * (qd - 2) + lane;
-            const float gr = s_g[r], br = s_b[r];
+            for (int c2 = 0; c2 < 2; c2++) {
+                tmem_ld32(tl + ACC_D + 32 * c2, r32);
 #pragma unroll
-            for (int i4 = 0; i4 < 8; i4++) {
-                float a4[4];
-#pragma unroll
-                for (int u = 0; u < 4; u++) {
-                    const int jj = j0 + 4 * i4 + u;
-                    const float e = __expf(fminf(gr - s_g[jj], 0.f));
-                    a4[u] = jj < r ? br * __uint_as_float(r32[4 * i4 + u]) * e : 0.f;
+                for (int i = 0; i < 32; i++) {
+                    const int r = 32 * c2 + i;
+                    const float e = __expf(fminf(s_g[r] - gj, 0.f));
+                    Am[r * LDA + jr] = r > jr ? s_b[r] * __uint_as_float(r32[i]) * e : 0.f;
                 }
-                *reinterpret_cast<float4*>(Am + r * LDA + j0 + 4 * i4) = make_float4(a4[0], a4[1], a4[2], a4[3]);
             }
+        } else {
+            // row j of P^T: P[r][j] = e^{g_r - g_j} q_r.k_j for r >= j -> fp16, MN-major image
+#pragma unroll
+            for (int c2 = 0; c2 < 2; c2++) {
+                tmem_ld32(tl + ACC_D + 64 + 32 * c2, r32);
+                uint32_t w[16];
+#pragma unroll
+                for (int i = 0; i < 16; i++) {
+                    const int r = 32 * c2 + 2 * i;
+                    const float e0 = __expf(fminf(s_g[r] - gj, 0.f)), e1 = __expf(fminf(s_g[r + 1] - gj, 0.f));
+                    w[i] = pack_half2(r >= jr ? __uint_as_float(r32[2 * i]) * e0 : 0.f,
+                                      r + 1 >= jr ? __uint_as_float(r32[2 * i + 1]) * e1 : 0.f);
+                }
+#pragma unroll
+                for (int q4 = 0; q4 < 4; q4++)
+                    sts128(st_p + swz128(jr, 4 * c2 + q4), w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2], w[4 * q4 + 3]);
+            }
+            fence_async_smem();
         }
+    } else if (ok) {   // Q~ = diag(e^g) Q in place (the q rows are dead after the first MMA); Q~ feeds
+                       // only the output, so packed half2 products are precise enough
+        const int t = tid - 64 * (tid >= 128 ? 1 : 0) - 64;   // 0..127 over warps 2, 3, 6, 7
+        for (int idx = t; idx < 2 * C * 8; idx += 128) {
+            const int hf = idx >> 9, r = (idx >> 3) & 63, ch = idx & 7;
+            const uint32_t a = sb + OFF_QK + hf * 16384 + 8192 + swz128(r, ch);
+            const uint4 x = scale8_h2(lds128(a), s_eg[r]);
+            sts128(a, x.x, x.y, x.z, x.w);
+        }
+        fence_async_smem();
     }
     tc_fence_before();
     __syncthreads();
-
-    if (ok) {   // P^T -> the record (MN-major B image: row j holds P[0..63][j])
-        const __half* pr = reinterpret_cast<const __half*>(Xm);
-        for (int idx = tid; idx < C * 8; idx += NT) {
-            const int jj = idx >> 3, q8 = idx & 7;
-            uint32_t w4[4];
-#pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const __half lo = pr[(8 * q8 + 2 * i) * 66 + jj], hi = pr[(8 * q8 + 2 * i + 1) * 66 + jj];
-                w4[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
-            }
-            stg128(rec + rec_p(par) + swz128(jj, q8), w4[0], w4[1], w4[2], w4[3]);
-        }
+    if (ok && tid == 0) {
+        bulk_s2g(rec + rec_p(par), st_p, 8192);
+        bulk_s2g(rec + rec_q(par, 0), sb + OFF_QK + 8192, 8192);
+        bulk_s2g(rec + rec_q(par, 1), sb + OFF_QK + 16384 + 8192, 8192);
+        bulk_commit();
+        bulk_wait_read<0>();   // the solve writes X, where P^T was staged
     }
-    __syncthreads();
-    for (int i = tid; i < 64 * LDA / 4; i += NT)   // X starts as zero above its diagonal blocks
-        reinterpret_cast<float4*>(Xm)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     __syncthreads();
 
     // ---- X = (I + A)^-1, unit lower triangular, fp32 ----
@@ -337,19 +334,21 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __syncthreads();
     if (ok && tid < 128) {   // size 16 -> 32: Y = A21 X1 for the block pairs (0,1) and (2,3)
         const int o1 = tid < 64 ? 0 : 32, o2 = o1 + 16;
-        block_mm(Am + o2 * LDA + o1, LDA, Xm + o1 * LDA + o1, LDA, Ym + (o1 >> 1), LDY, 16, 1.f, tid & 63, 64);
+        block_mm<false, true>(Am + o2 * LDA + o1, LDA, Xm + o1 * LDA + o1, LDA, Ym + (o1 >> 1), LDY, 16, 1.f,
+                              tid & 63, 64);
     }
     __syncthreads();
     if (ok && tid < 128) {   // X21 = -X2 Y
         const int o1 = tid < 64 ? 0 : 32, o2 = o1 + 16;
-        block_mm(Xm + o2 * LDA + o2, LDA, Ym + (o1 >> 1), LDY, Xm + o2 * LDA + o1, LDA, 16, -1.f, tid & 63, 64);
+        block_mm<true, false>(Xm + o2 * LDA + o2, LDA, Ym + (o1 >> 1), LDY, Xm + o2 * LDA + o1, LDA, 16, -1.f,
+                              tid & 63, 64);
     }
     __syncthreads();
-    if (ok) block_mm(Am + 32 * LDA, LDA, Xm, LDA, Ym, LDY, 32, 1.f, tid, NT);   // size 32 -> 64
+    if (ok) block_mm<false, true>(Am + 32 * LDA, LDA, Xm, LDA, Ym, LDY, 32, 1.f, tid, NT);   // size 32 -> 64
     __syncthreads();
-    if (ok) block_mm(Xm + 32 * LDA + 32, LDA, Ym, LDY, Xm + 32 * LDA, LDA, 32, -1.f, tid, NT);
+    if (ok) block_mm<true, false>(Xm + 32 * LDA + 32, LDA, Ym, LDY, Xm + 32 * LDA, LDA, 32, -1.f, tid, NT);
     __syncthreads();
-    if (ok) {   // T = X diag(beta) -> the record; T' = T diag(e^g) -> shared memory
+    if (ok) {   // T = X diag(beta) -> staged for the record; T' = T diag(e^g) -> the W MMA's operand
         const int c = tid >> 2, jq = (tid & 3) * 16;
         uint32_t tp[8], tq[8];
 #pragma unroll
@@ -362,7 +361,7 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         }
 #pragma unroll
         for (int c2 = 0; c2 < 2; c2++) {
-            stg128(rec + REC_T + swz128(c, jq / 8 + c2), tp[4 * c2], tp[4 * c2 + 1], tp[4 * c2 + 2], tp[4 * c2 + 3]);
+            sts128(st_t + swz128(c, jq / 8 + c2), tp[4 * c2], tp[4 * c2 + 1], tp[4 * c2 + 2], tp[4 * c2 + 3]);
             sts128(sb + OFF_TP + swz128(c, jq / 8 + c2), tq[4 * c2], tq[4 * c2 + 1], tq[4 * c2 + 2], tq[4 * c2 + 3]);
         }
     }
@@ -370,49 +369,67 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     tc_fence_before();
     __syncthreads();
 
-    // ---- W^T = K^T T'^T (M = d_k, N = 64 chunk columns, K = 64 tokens) ----
+    // ---- W = T' K (M = 128 with the chunk's 64 rows first, N = d_k, K = 64 tokens) ----
     if (ok && tid == 0) {
+        bulk_s2g(rec + REC_T, st_t, 8192);
+        bulk_commit();
         tc_fence_after();
+        constexpr uint32_t ID = idesc_f16(128, 128, 0, 1);
 #pragma unroll
         for (int ks = 0; ks < 4; ks++)
-            mma_f16(tmem + ACC_W, sdesc(sb + OFF_QK + C * 128 + ks * 2048, 16384, 1024),
-                    sdesc(sb + OFF_TP + ks * 32, 16, 1024), idesc_f16(128, 64, 1, 0), ks > 0);
+            mma_f16(tmem + ACC_D, sdesc(sb + OFF_TP + ks * 32, 16, 1024), sdesc(sb + OFF_QK + ks * 2048, 16384, 1024),
+                    ID, ks > 0);
         mma_commit(bar);
     }
     if (ok && !mbar_wait_bounded(bar, 1)) atomicOr((unsigned*)s_abort, 1u);
     __syncthreads();
     ok = *s_abort == 0;
-    if (ok) {   // -W^T from TMEM -> fp16 rows [d_k][c] in shared memory (reusing A)
+    if (ok && qd < 2) {   // row c of -W, one 64-wide d_k half per warp half -> K-major image
         tc_fence_after();
+        const int c = 32 * qd + lane;
         uint32_t r32[32];
-        tmem_ld32(tl + ACC_W + 32 * half, r32);
-        const int row = 32 * qd + lane;
-        uint32_t* wt = reinterpret_cast<uint32_t*>(smem + OFF_A) + row * 33 + 16 * half;   // 132-byte rows
 #pragma unroll
-        for (int i = 0; i < 16; i++)
-            wt[i] = pack_half2(-__uint_as_float(r32[2 * i]), -__uint_as_float(r32[2 * i + 1]));
-    }
-    __syncthreads();
-    if (ok) {   // -> the record, K-major: 16-byte piece (c, d_k 8q..8q+7) gathers 8 rows of -W^T
-        const __half* wt = reinterpret_cast<const __half*>(smem + OFF_A);
-        for (int idx = tid; idx < C * 16; idx += NT) {
-            const int c = idx >> 4, q8 = idx & 15;
-            uint32_t w4[4];
+        for (int c2 = 0; c2 < 2; c2++) {
+            tmem_ld32(tl + ACC_D + 64 * half + 32 * c2, r32);
+            uint32_t w[16];
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                const __half lo = wt[(8 * q8 + 2 * i) * 66 + c], hi = wt[(8 * q8 + 2 * i + 1) * 66 + c];
-                w4[i] = (uint32_t)__half_as_ushort(lo) | ((uint32_t)__half_as_ushort(hi) << 16);
-            }
-            stg128(rec + rec_w(par, q8 >> 3) + swz128(c, q8 & 7), w4[0], w4[1], w4[2], w4[3]);
+            for (int i = 0; i < 16; i++)
+                w[i] = pack_half2(-__uint_as_float(r32[2 * i]), -__uint_as_float(r32[2 * i + 1]));
+#pragma unroll
+            for (int q4 = 0; q4 < 4; q4++)
+                sts128(st_w + half * 8192 + swz128(c, 4 * c2 + q4), w[4 * q4], w[4 * q4 + 1], w[4 * q4 + 2],
+                       w[4 * q4 + 3]);
         }
-    } else if (tid == 0) {
-        record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));
-        // one more bounded wait for whatever may still be in flight
-        mbar_wait_bounded(bar_ld, 0);
-        mbar_wait_bounded(bar, 0);
-        mbar_wait_bounded(bar, 1);
+        fence_async_smem();
+    } else if (ok) {   // K~ = diag(e^{g_C - g}) K in place (the W MMA is done with K); zero past the end
+        const int t = tid - 64 * (tid >= 128 ? 1 : 0) - 64;
+        const float gC = s_g[C - 1];
+        for (int idx = t; idx < 2 * C * 8; idx += 128) {
+            const int hf = idx >> 9, r = (idx >> 3) & 63, ch = idx & 7;
+            const uint32_t a = sb + OFF_QK + hf * 16384 + swz128(r, ch);
+            const uint4 x = scale8(lds128(a), r < n ? __expf(gC - s_g[r]) : 0.f);   // fp32: K~ feeds the state
+            sts128(a, x.x, x.y, x.z, x.w);
+        }
+        fence_async_smem();
     }
     tc_fence_before();
+    __syncthreads();
+    if (tid == 0) {
+        if (ok) {
+            bulk_s2g(rec + rec_w(par, 0), st_w, 8192);
+            bulk_s2g(rec + rec_w(par, 1), st_w + 8192, 8192);
+            bulk_s2g(rec + rec_kt(par, 0), sb + OFF_QK, 8192);
+            bulk_s2g(rec + rec_kt(par, 1), sb + OFF_QK + 16384, 8192);
+            bulk_commit();
+        } else {
+            record_error((*s_abort & 1u ? kErrMmaTimeout : 0u) | (*s_abort & 2u ? kErrCopyTimeout : 0u));
+            // one more bounded wait for whatever may still be in flight
+            mbar_wait_bounded(bar_ld, 0);
+            mbar_wait_bounded(bar, 0);
+            mbar_wait_bounded(bar, 1);
+        }
+        bulk_wait<0>();   // the record's bulk stores have read their staging
+    }
     __syncthreads();
     if (warp == 0) {
         tc_fence_after();

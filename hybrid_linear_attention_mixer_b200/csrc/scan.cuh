@@ -111,6 +111,9 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
     volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 132);
     // loads issued per barrier (ld x2, B2 x2): the loader's drain waits for the last phase of each
     volatile int* s_issued = reinterpret_cast<volatile int*>(smem + OFF_BAR + 136);
+    // the issuer has issued MMA1 (phase parity 0) or MMA2 (parity 1) of the current chunk: the
+    // workers' TMEM traffic waits for it so that it does not slow the issue down
+    const uint32_t ev_iss = sb + OFF_BAR + 152;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool worker = tid < NW;
@@ -158,6 +161,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
             mbar_init(bar, 1);
 #pragma unroll
             for (int i = 0; i < 15; i++) mbar_init(bar_ld0 + 8 * i, 1);   // ld, B2, fin, ev1, ev2, evo, end, evc, lfin, ldone
+            mbar_init(ev_iss, 1);
             fence_mbar_init();
             *s_abort = 0;
             for (int i = 0; i < 4; i++) s_issued[i] = 0;
@@ -329,11 +333,14 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
                 mma_f16_ta_w(d1, tmem + TA_S + ks * 8, dB10 + b * (R_STRIDE >> 4) + (ks >> 2) * 1024 + (ks & 3) * 2,
                              ID_DE, 1);
             mma_commit_w(bar);
+            if (lane == 0) mbar_arrive(ev_iss);
         }
         // ---- workers, while MMA1 runs: the decayed state accumulator ----
         if (worker) {
             wait_par(bar_ld0, ci);   // g
-            put_state_acc(__expf(reinterpret_cast<const float*>(smem + OFF_R + b * R_STRIDE + R_G)[C - 1]));
+            const float decay = __expf(reinterpret_cast<const float*>(smem + OFF_R + b * R_STRIDE + R_G)[C - 1]);
+            if (!mbar_wait_bounded(ev_iss, 0)) atomicOr((unsigned*)s_abort, 1u);
+            put_state_acc(decay);
         }
         GDN_MMA_WAIT();
         if (warp == IW && lane == 0) mbar_arrive(ev10 + 8 * b);   // MMA1, (c) and the decay are done with buffer b
@@ -360,9 +367,13 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
             for (int ks = 0; ks < 4; ks++)
                 mma_f16_ta_w(d2, tmem + TA_U + ks * 8, dB20 + b * (B2_STRIDE >> 4) + ks * 128, ID_FG, 1);
             mma_commit_w(bar);
+            if (lane == 0) mbar_arrive(ev_iss);
         }
         // ---- workers, while MMA2 runs: the previous chunk's o tile ----
-        if (worker && ci > 0) stage_o(ci - 1);
+        if (worker && ci > 0) {
+            if (!mbar_wait_bounded(ev_iss, 1)) atomicOr((unsigned*)s_abort, 1u);
+            stage_o(ci - 1);
+        }
         GDN_MMA_WAIT();
         if (warp == IW && lane == 0) mbar_arrive(ev20 + 8 * b);   // B2 buffer b free; o(ci - 1) staged
 
