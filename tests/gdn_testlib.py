@@ -86,6 +86,7 @@ def assert_parity(gpu: dict, ref: dict, heads=None, out_tol=OUT_TOL, state_tol=S
         g_out, r_out = g_out[rows], r_out[rows]
     eo = rel_err(g_out, r_out)
     es = rel_err(g_rs, ref["rec_state"])
+    print("parity: out rel err %.3e (tol %.0e), state rel err %.3e (tol %.0e)" % (eo, out_tol, es, state_tol))
     assert np.isfinite(g_out).all() and np.isfinite(g_rs).all()
     assert eo <= out_tol, "out rel err %.3e > %.1e" % (eo, out_tol)
     assert es <= state_tol, "state rel err %.3e > %.1e" % (es, state_tol)
