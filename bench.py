@@ -44,6 +44,11 @@ PREFILL_FLOP_PER_TOKEN = H_K * 4 * 64 * D + H_V * (6 * 64 * D + 6 * D * D)
 DECODE_BYTES_PER_STEP = (2 * DECODE_N * H_V * D * D * 4 + 2 * DECODE_N * C_CONV * 3 * 2
                          + DECODE_N * (2 * H_K * D + 2 * H_V * D + 2 * H_V) * 2
                          + DECODE_N * H_V * D * 2 + (C_CONV * 4 + 2 * H_V + D) * 4)
+#   multi-token decode bytes per call: the state and conv state once, inputs and outputs per token
+MULTI_TOK = 4
+MULTI_BYTES_PER_CALL = (2 * DECODE_N * H_V * D * D * 4 + 2 * DECODE_N * C_CONV * 3 * 2
+                        + MULTI_TOK * DECODE_N * (2 * H_K * D + 2 * H_V * D + 2 * H_V) * 2
+                        + MULTI_TOK * DECODE_N * H_V * D * 2 + (C_CONV * 4 + 2 * H_V + D) * 4)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu DRAM bytes (read + write) per decode launch at batch 256, taken on the
 # decode kernel whose source hashes to DECODE_SRC_SHA; null once it changes.
@@ -274,6 +279,32 @@ def main():
         dist.all_reduce(t, op=dist.ReduceOp.MAX)
     pre_ms, dec_ms = float(t[0]), float(t[1])
 
+    # ---- multi-token decode (draft verification): MULTI_TOK tokens per sequence, one pass ----
+    mt = MULTI_TOK
+    m_in = {n: torch.stack([st[n] for st in steps[:mt]], dim=1).reshape(DECODE_N * mt, -1).contiguous()
+            for n in "qkvabz"}
+    m_out = torch.empty((DECODE_N * mt, H_V * D), dtype=torch.bfloat16, device=dev)
+
+    def decode_multi():
+        gdn.decode_multi(cfg, dw, m_in["q"], m_in["k"], m_in["v"], m_in["a"], m_in["b"], m_in["z"],
+                         d_cs, d_rs, mt, out=m_out, stream=stream)
+
+    m_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    for i in range(-args.warmup, args.steps):
+        flush.zero_()
+        if i >= 0:
+            m_ev[i][0].record(stream)
+        decode_multi()
+        if i >= 0:
+            m_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    gdn.check_device_error(stream)
+    tm = torch.tensor([sum(a.elapsed_time(b) for a, b in m_ev)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tm, op=dist.ReduceOp.MAX)
+    multi_ms = float(tm[0])
+
     # ---- end to end through the public API with host buffers ----
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
@@ -315,6 +346,10 @@ def main():
             "decode": {"value": dec_gbs, "unit": "GB/s", "us_per_step": dec_launch_s * 1e6,
                        "tokens_per_s": DECODE_N * world / dec_launch_s,
                        "bytes_per_step": DECODE_BYTES_PER_STEP},
+            "decode_multi": {"tokens_per_seq": MULTI_TOK, "value": MULTI_BYTES_PER_CALL / (multi_ms / 1e3 / K) / 1e9,
+                             "unit": "GB/s", "us_per_call": multi_ms * 1e3 / K,
+                             "tokens_per_s": DECODE_N * MULTI_TOK * world / (multi_ms / 1e3 / K),
+                             "bytes_per_call": MULTI_BYTES_PER_CALL},
             "prefill_ms": pre_ms / K,
             "roofline": {"kernel": "gdn_decode_kernel", "bound": "hbm", "achieved": dec_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / pk["hbm_gbs"],

@@ -169,5 +169,205 @@ __global__ void __launch_bounds__(NT) gdn_decode_kernel(Args p) {
     }
 }
 
+// ---------------------------------------------------------------------------
+// Multi-token decode (draft verification): n_tok consecutive tokens of each
+// sequence in one pass over its state.  Multi-token prediction drafts several
+// future tokens ("Qwen3.8-Flash-Next", "Architecture concepts": Multi-Token
+// Prediction; table "Every architecture field", row mtp_layers); checking a
+// draft runs the recurrence over the drafted tokens.  Row r of S takes the
+// n_tok updates one after another, exactly as n_tok decode steps would (same
+// operations in the same order, so the results are bit-identical to n_tok calls
+// of the one-token kernel), while the state is read and written once.
+// Optionally the state after every token is written out (snapshots), so that
+// a caller who accepts only the first j drafted tokens can restore the state
+// after token j; the conv state after every token can be written out likewise.
+// Inputs and outputs are token-major within each sequence: row seq*n_tok + t.
+// ---------------------------------------------------------------------------
+constexpr int kMaxTok = 16;
+
+struct MultiArgs {
+    Args a;
+    int n_tok;
+    float* state_snap;   // [n_tok][N][Hv][dv][dk] or null
+    void* conv_snap;     // [n_tok][N][Ctot][3] act dtype, or null
+    int n_seqs;
+};
+
+__host__ __device__ constexpr size_t smem_floats_multi(int dk, int G, int dv, int n_tok) {
+    return (size_t)n_tok * (2 * dk + 2 * G * dv + 2 * G);
+}
+
+template <typename TA, typename TO, int DK>
+__global__ void __launch_bounds__(NT) gdn_decode_multi_kernel(MultiArgs m) {
+    constexpr int LPR = DK / 4;        // lanes per state row (4 fp32 each)
+    constexpr int RPP = 32 / LPR;      // rows per warp pass
+    constexpr int U = DK == 128 ? 4 : 2;   // passes in flight per warp
+    const Args& p = m.a;
+    const int NTK = m.n_tok;
+    extern __shared__ float sm[];
+    const int Hk = p.Hk, Hv = p.Hv, dv = p.dv, G = Hv / Hk;
+    const int Cq = Hk * DK, Cv = Hv * dv, Ctot = 2 * Cq + Cv;
+    const int seq = blockIdx.x / Hk, j = blockIdx.x % Hk;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nch = 2 * DK + G * dv;   // this CTA's channels: q, k of key head j, v of its value heads
+    float* sfeat = sm;                      // [NTK][nch]: q^ | k^ | v^ per token
+    float* so = sfeat + NTK * nch;          // [NTK][G*dv]
+    float* s_al = so + NTK * G * dv;        // [NTK][G]
+    float* s_be = s_al + NTK * G;           // [NTK][G]
+
+    // ---- conv + SiLU of every token, with the conv-state roll ----
+    const TA* pq = static_cast<const TA*>(p.q);
+    const TA* pk = static_cast<const TA*>(p.k);
+    const TA* pv = static_cast<const TA*>(p.v);
+    TA* cst = static_cast<TA*>(p.conv_state);
+    for (int i = tid; i < nch; i += NT) {
+        int ch;
+        const TA* src;
+        int64_t ld;
+        if (i < DK) {
+            ch = j * DK + i;
+            src = pq + ch;
+            ld = Cq;
+        } else if (i < 2 * DK) {
+            ch = Cq + j * DK + (i - DK);
+            src = pk + (ch - Cq);
+            ld = Cq;
+        } else {
+            const int vi = j * G * dv + (i - 2 * DK);
+            ch = 2 * Cq + vi;
+            src = pv + vi;
+            ld = Cv;
+        }
+        TA* st = cst + ((int64_t)seq * Ctot + ch) * 3;
+        TA h0 = st[0], h1 = st[1], h2 = st[2];
+        const float4 w = reinterpret_cast<const float4*>(p.conv_w)[ch];
+        for (int t = 0; t < NTK; t++) {
+            const TA xr = src[((int64_t)seq * NTK + t) * ld];
+            float acc = w.x * to_f32(h0);
+            acc = fmaf(w.y, to_f32(h1), acc);
+            acc = fmaf(w.z, to_f32(h2), acc);
+            acc = fmaf(w.w, to_f32(xr), acc);
+            sfeat[t * nch + i] = silu_f(acc);
+            h0 = h1;
+            h1 = h2;
+            h2 = xr;
+            if (m.conv_snap) {
+                TA* cs = static_cast<TA*>(m.conv_snap) + (((int64_t)t * m.n_seqs + seq) * Ctot + ch) * 3;
+                cs[0] = h0;
+                cs[1] = h1;
+                cs[2] = h2;
+            }
+        }
+        st[0] = h0;
+        st[1] = h1;
+        st[2] = h2;
+    }
+    for (int i = tid; i < NTK * G; i += NT) {
+        const int t = i / G, g = i % G, h = j * G + g;
+        const int64_t row = (int64_t)seq * NTK + t;
+        const float av = to_f32(static_cast<const TA*>(p.a)[row * Hv + h]);
+        const float bv = to_f32(static_cast<const TA*>(p.b)[row * Hv + h]);
+        s_al[i] = __expf(-__expf(p.A_log[h]) * softplus_f(av + p.dt_bias[h]));
+        s_be[i] = sigmoid_f(bv);
+    }
+    __syncthreads();
+    for (int vi = warp; vi < 2 * NTK; vi += NW) {   // L2 norms: q^ and k^ of every token
+        float* x = sfeat + (vi >> 1) * nch + (vi & 1) * DK;
+        float ss = 0.f;
+        for (int i = lane; i < DK; i += 32) ss = fmaf(x[i], x[i], ss);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float r = rsqrtf(ss + p.l2_eps);
+        for (int i = lane; i < DK; i += 32) x[i] *= r;
+    }
+    __syncthreads();
+
+    // ---- stream the state rows: n_tok updates per row ----
+    const int col = 4 * (lane % LPR);
+    const int sub = lane / LPR;
+    float kq[kMaxTok];   // k_t . q_t, reduced over the row's lanes as the one-token kernel does
+#pragma unroll
+    for (int t = 0; t < kMaxTok; t++) {
+        if (t < NTK) {
+            const float4 k4 = *reinterpret_cast<const float4*>(sfeat + t * nch + DK + col);
+            const float4 q4 = *reinterpret_cast<const float4*>(sfeat + t * nch + col);
+            float x = k4.x * q4.x + k4.y * q4.y + k4.z * q4.z + k4.w * q4.w;
+#pragma unroll
+            for (int off = LPR / 2; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+            kq[t] = x;
+        }
+    }
+    const float inv_sqrt_dk = rsqrtf((float)DK);
+    const int64_t blk = ((int64_t)seq * Hv + (int64_t)j * G) * dv * DK;
+    float* Sb = p.rec_state + blk;
+    const int64_t snap_stride = (int64_t)m.n_seqs * Hv * dv * DK;
+    const int rows = G * dv;
+    for (int R0 = warp * RPP * U; R0 < rows; R0 += NW * RPP * U) {
+        float4 s[U];
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const int R = R0 + u * RPP + sub;
+            s[u] = R < rows ? __ldcs(reinterpret_cast<const float4*>(Sb + (int64_t)R * DK + col))
+                            : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int t = 0; t < kMaxTok; t++) {
+            if (t >= NTK) break;
+            const float4 k4 = *reinterpret_cast<const float4*>(sfeat + t * nch + DK + col);
+            const float4 q4 = *reinterpret_cast<const float4*>(sfeat + t * nch + col);
+#pragma unroll
+            for (int u = 0; u < U; u++) {
+                const int R = R0 + u * RPP + sub;
+                const int g = min(R, rows - 1) / dv;
+                float uk = s[u].x * k4.x + s[u].y * k4.y + s[u].z * k4.z + s[u].w * k4.w;
+                float up = s[u].x * q4.x + s[u].y * q4.y + s[u].z * q4.z + s[u].w * q4.w;
+#pragma unroll
+                for (int off = LPR / 2; off >= 1; off >>= 1) {
+                    uk += __shfl_xor_sync(0xffffffffu, uk, off);
+                    up += __shfl_xor_sync(0xffffffffu, up, off);
+                }
+                if (R < rows) {
+                    const float al = s_al[t * G + g], be = s_be[t * G + g];
+                    const float d = be * (sfeat[t * nch + 2 * DK + R] - al * uk);
+                    float4 o4;
+                    o4.x = fmaf(al, s[u].x, d * k4.x);
+                    o4.y = fmaf(al, s[u].y, d * k4.y);
+                    o4.z = fmaf(al, s[u].z, d * k4.z);
+                    o4.w = fmaf(al, s[u].w, d * k4.w);
+                    s[u] = o4;
+                    if (m.state_snap)
+                        __stcs(reinterpret_cast<float4*>(m.state_snap + t * snap_stride + blk + (int64_t)R * DK + col), o4);
+                    if (lane % LPR == 0) so[t * rows + R] = (al * up + d * kq[t]) * inv_sqrt_dk;
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; u++) {
+            const int R = R0 + u * RPP + sub;
+            if (R < rows) __stcs(reinterpret_cast<float4*>(Sb + (int64_t)R * DK + col), s[u]);
+        }
+    }
+    __syncthreads();
+
+    // ---- gated RMSNorm per token and value head ----
+    const TA* pz = static_cast<const TA*>(p.z);
+    TO* po = static_cast<TO*>(p.out);
+    for (int tg = warp; tg < NTK * G; tg += NW) {
+        const int t = tg / G, g = tg % G;
+        const float* o = so + t * rows + g * dv;
+        float ss = 0.f;
+        for (int r = lane; r < dv; r += 32) ss = fmaf(o[r], o[r], ss);
+#pragma unroll
+        for (int off = 16; off >= 1; off >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
+        const float rs = rsqrtf(ss / (float)dv + p.norm_eps);
+        const int h = j * G + g;
+        for (int r = lane; r < dv; r += 32) {
+            const int64_t off = (((int64_t)seq * NTK + t) * Hv + h) * dv + r;
+            const float zz = to_f32(pz[off]);
+            from_f32(o[r] * rs * p.norm_w[r] * silu_f(zz), po + off);
+        }
+    }
+}
+
 }  // namespace dec
 }  // namespace gdn

@@ -261,6 +261,28 @@ cudaError_t launch_decode_dk(const gdn::dec::Args& a, int n_seqs, cudaStream_t s
     return cudaGetLastError();
 }
 
+template <typename TA, typename TO, int DK>
+cudaError_t launch_decode_multi_dk(const gdn::dec::MultiArgs& m, cudaStream_t st) {
+    const int G = m.a.Hv / m.a.Hk;
+    const size_t smem = gdn::dec::smem_floats_multi(DK, G, m.a.dv, m.n_tok) * sizeof(float);
+    auto kern = gdn::dec::gdn_decode_multi_kernel<TA, TO, DK>;
+    if (smem > 48 * 1024) {
+        cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+        if (e != cudaSuccess) return e;
+    }
+    kern<<<(unsigned)m.n_seqs * m.a.Hk, gdn::dec::NT, smem, st>>>(m);
+    return cudaGetLastError();
+}
+
+template <typename TA, typename TO>
+cudaError_t launch_decode_multi(const gdn::dec::MultiArgs& m, cudaStream_t st) {
+    switch (m.a.dk) {
+        case 32: return launch_decode_multi_dk<TA, TO, 32>(m, st);
+        case 64: return launch_decode_multi_dk<TA, TO, 64>(m, st);
+        default: return launch_decode_multi_dk<TA, TO, 128>(m, st);
+    }
+}
+
 template <typename TA, typename TO>
 cudaError_t launch_decode(const gdn::dec::Args& a, int n_seqs, cudaStream_t st) {
     switch (a.dk) {
@@ -357,6 +379,46 @@ gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w, const void* q
     else if (abf) e = launch_decode<__nv_bfloat16, float>(da, n_seqs, st);
     else if (obf) e = launch_decode<float, __nv_bfloat16>(da, n_seqs, st);
     else e = launch_decode<float, float>(da, n_seqs, st);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+static_assert(gdn::dec::kMaxTok == GDN_DECODE_MULTI_MAX_TOKENS, "multi-token limit");
+
+gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_weights* w, const void* q, const void* k,
+                            const void* v, const void* a, const void* b, const void* z, void* conv_state,
+                            float* rec_state, int32_t n_seqs, int32_t n_tok, void* out, float* state_snapshots,
+                            void* conv_snapshots, void* stream) {
+    gdn_status s = check_config(cfg);
+    if (s != GDN_OK) return s;
+    if ((s = check_weights(w)) != GDN_OK) return s;
+    if (n_seqs < 0 || n_tok < 0) return GDN_ERR_INVALID_ARG;
+    if (n_tok > GDN_DECODE_MULTI_MAX_TOKENS) return GDN_ERR_UNSUPPORTED;
+    if (n_seqs == 0 || n_tok == 0) return GDN_OK;
+    if (!q || !k || !v || !a || !b || !z || !conv_state || !rec_state || !out) return GDN_ERR_INVALID_ARG;
+    const void* a16[] = {q, k, v, z, out, rec_state, state_snapshots};
+    for (const void* p : a16)
+        if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;   // null snapshots pass
+    if ((int64_t)n_seqs * cfg->n_k_heads > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    gdn::dec::MultiArgs m;
+    gdn::dec::Args& da = m.a;
+    da.q = q; da.k = k; da.v = v; da.a = a; da.b = b; da.z = z;
+    da.conv_w = w->conv_weight; da.A_log = w->A_log; da.dt_bias = w->dt_bias; da.norm_w = w->norm_weight;
+    da.conv_state = conv_state;
+    da.rec_state = rec_state;
+    da.out = out;
+    da.Hk = cfg->n_k_heads; da.Hv = cfg->n_v_heads; da.dk = cfg->d_k; da.dv = cfg->d_v;
+    da.l2_eps = cfg->l2_eps; da.norm_eps = cfg->norm_eps;
+    m.n_tok = n_tok;
+    m.state_snap = state_snapshots;
+    m.conv_snap = conv_snapshots;
+    m.n_seqs = n_seqs;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    const bool abf = cfg->act_dtype == GDN_BF16, obf = cfg->out_dtype == GDN_BF16;
+    if (abf && obf) e = launch_decode_multi<__nv_bfloat16, __nv_bfloat16>(m, st);
+    else if (abf) e = launch_decode_multi<__nv_bfloat16, float>(m, st);
+    else if (obf) e = launch_decode_multi<float, __nv_bfloat16>(m, st);
+    else e = launch_decode_multi<float, float>(m, st);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -48,7 +48,8 @@ class _CWeights(ctypes.Structure):
 
 _lib = None
 EXPORTS = ("gdn_config_default", "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode",
-           "gdn_check_device_error", "gdn_status_string")
+           "gdn_decode_multi", "gdn_check_device_error", "gdn_status_string")
+DECODE_MULTI_MAX_TOKENS = 16   # GDN_DECODE_MULTI_MAX_TOKENS
 
 
 def lib() -> ctypes.CDLL:
@@ -68,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_prefill.restype = ctypes.c_int
         L.gdn_decode.argtypes = [vp, vp] + [vp] * 8 + [i32, vp, vp]
         L.gdn_decode.restype = ctypes.c_int
+        L.gdn_decode_multi.argtypes = [vp, vp] + [vp] * 8 + [i32, i32, vp, vp, vp, vp]
+        L.gdn_decode_multi.restype = ctypes.c_int
         L.gdn_check_device_error.argtypes = [vp]
         L.gdn_check_device_error.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -178,6 +181,37 @@ def decode(cfg: Config, w: dict, q, k, v, a, b, z, conv_state, rec_state, out=No
                          _stream(stream))
     if s != 0:
         raise GdnError(s, "gdn_decode")
+    return out
+
+
+def decode_multi(cfg: Config, w: dict, q, k, v, a, b, z, conv_state, rec_state, n_tok: int, out=None,
+                 state_snapshots=None, conv_snapshots=None, stream=None):
+    """n_tok consecutive tokens per sequence (rows token-major within a sequence);
+    returns out [N*n_tok, H_v*d_v].  Optional snapshots receive the recurrent state
+    [n_tok, N, H_v, d_v, d_k] (fp32) and the conv state [n_tok, N, C, K-1] after each token."""
+    dev = q.device
+    rows = q.shape[0]
+    if n_tok <= 0 or rows % n_tok:
+        raise ValueError("rows (%d) must be a positive multiple of n_tok (%d)" % (rows, n_tok))
+    N = rows // n_tok
+    for n, t in (("q", q), ("k", k), ("v", v), ("a", a), ("b", b), ("z", z),
+                 ("conv_state", conv_state)):
+        _check(t, n, cfg.act_dtype, dev)
+    _check(rec_state, "rec_state", torch.float32, dev)
+    if state_snapshots is not None:
+        _check(state_snapshots, "state_snapshots", torch.float32, dev)
+    if conv_snapshots is not None:
+        _check(conv_snapshots, "conv_snapshots", cfg.act_dtype, dev)
+    if out is None:
+        out = torch.empty((rows, cfg.n_v_heads * cfg.d_v), dtype=cfg.out_dtype, device=dev)
+    _check(out, "out", cfg.out_dtype, dev)
+    c, cw = cfg.c(), _weights(w, dev)
+    opt = lambda t: None if t is None else _ptr(t)
+    s = lib().gdn_decode_multi(ctypes.byref(c), ctypes.byref(cw), _ptr(q), _ptr(k), _ptr(v), _ptr(a),
+                               _ptr(b), _ptr(z), _ptr(conv_state), _ptr(rec_state), N, int(n_tok),
+                               _ptr(out), opt(state_snapshots), opt(conv_snapshots), _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_decode_multi")
     return out
 
 

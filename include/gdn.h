@@ -129,6 +129,37 @@ gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w,
                       void* conv_state, float* rec_state, int32_t n_seqs,
                       void* out, void* stream);
 
+/* Largest number of tokens per sequence that gdn_decode_multi takes in one call. */
+#define GDN_DECODE_MULTI_MAX_TOKENS 16
+
+/*
+ * Several decode steps at once: n_tok consecutive new tokens for each of n_seqs
+ * sequences, for checking tokens that a multi-token-prediction head drafted
+ * ("Qwen3.8-Flash-Next", section "Architecture concepts": Multi-Token
+ * Prediction drafts tokens at inference; table "Every architecture field",
+ * row mtp_layers).  The result equals n_tok consecutive gdn_decode calls, bit
+ * for bit, but each state is read and written once.
+ *   q, k [n_seqs*n_tok][H_k][d_k]; v, z [n_seqs*n_tok][H_v][d_v];
+ *   a, b [n_seqs*n_tok][H_v]  act_dtype, token-major within a sequence: row
+ *   seq*n_tok + t holds token t of sequence seq
+ *   conv_state [n_seqs][C][K-1] act_dtype in/out; rec_state
+ *   [n_seqs][H_v][d_v][d_k] float32 in/out (the state after the last token)
+ *   out [n_seqs*n_tok][H_v][d_v] out_dtype
+ *   state_snapshots  optional (may be NULL), [n_tok][n_seqs][H_v][d_v][d_k]
+ *                    float32, 16-byte aligned: the state after each token, so
+ *                    that a caller who accepts only the first j drafted tokens
+ *                    can restore the state after token j
+ *   conv_snapshots   optional (may be NULL), [n_tok][n_seqs][C][K-1] act_dtype:
+ *                    the conv state after each token
+ * 1 <= n_tok <= GDN_DECODE_MULTI_MAX_TOKENS (larger: GDN_ERR_UNSUPPORTED);
+ * n_tok == 0 or n_seqs == 0 is a no-op.  No workspace.
+ */
+gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_weights* w,
+                            const void* q, const void* k, const void* v,
+                            const void* a, const void* b, const void* z,
+                            void* conv_state, float* rec_state, int32_t n_seqs, int32_t n_tok,
+                            void* out, float* state_snapshots, void* conv_snapshots, void* stream);
+
 /* Capacity, in bytes, of the fixed scratch array used by gdn_prefill_noalloc. */
 #define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 

@@ -108,3 +108,33 @@ def expected_conv_state(case, acts, conv_state, cu) -> np.ndarray:
         hist = np.concatenate([conv_state[s].T, x[t0:t1]], axis=0)[-3:]
         out[s] = hist.T
     return out
+
+
+def decode_steps(c, steps, dev="cuda:0", snapshots=False):
+    """gdn_decode once per step; returns (outs, conv_state, rec_state[, state and conv
+    state after every step])."""
+    cfg = config_of(c)
+    w = weights_on(c, dev)
+    cs = t_act(c.conv_state, dev)
+    rs = torch.from_numpy(c.rec_state).to(dev)
+    outs, snaps, csnaps = [], [], []
+    for st in steps:
+        d = {n: t_act(st[n], dev) for n in "qkvabz"}
+        o = gdn.decode(cfg, w, d["q"], d["k"], d["v"], d["a"], d["b"], d["z"], cs, rs)
+        outs.append(to_f64(o).reshape(-1, c.n_v_heads, c.d_v))
+        if snapshots:
+            snaps.append(rs.clone())
+            csnaps.append(cs.clone())
+    gdn.check_device_error()
+    if snapshots:
+        return outs, cs, rs, snaps, csnaps
+    return outs, cs, to_f64(rs)
+
+
+def as_sequences(c, steps, seqs):
+    """Per-step one-token inputs of the chosen sequences, packed token-major within each
+    sequence (one prefill of len(steps) tokens per sequence; the multi-token decode layout)."""
+    n = len(steps)
+    acts = {k: np.concatenate([np.stack([st[k][s] for st in steps]) for s in seqs]) for k in "qkvabz"}
+    cu = np.arange(0, n * len(seqs) + 1, n, dtype=np.int32)
+    return acts, cu

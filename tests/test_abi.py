@@ -89,6 +89,20 @@ def test_argument_errors_are_synchronous_and_launch_nothing(lib):
     assert lib.gdn_decode(None, ctypes.byref(cw), *[P(0x1000)] * 8, 4, P(0x7000), None) == INVALID
 
 
+def test_decode_multi_argument_errors(lib):
+    c = gdn.Config().c()
+    cw = gdn._CWeights(0x2000, 0x3000, 0x4000, 0x5000)
+    P = ctypes.c_void_p
+    call = lambda n, k, snap=0, ptr=0x1000: lib.gdn_decode_multi(
+        ctypes.byref(c), ctypes.byref(cw), *[P(ptr)] * 8, n, k, P(0x7000), P(snap), None, None)
+    assert call(4, gdn.DECODE_MULTI_MAX_TOKENS + 1) == UNSUPPORTED
+    assert call(4, -1) == INVALID
+    assert call(-1, 2) == INVALID
+    assert call(4, 0) == OK and call(0, 3) == OK          # nothing to do
+    assert call(4, 2, snap=0x8008) == INVALID             # misaligned snapshots
+    assert call(4, 2, ptr=0) == INVALID                   # missing inputs
+
+
 def test_status_strings(lib):
     for s in range(6):
         assert gdn.status_string(s)

@@ -186,27 +186,8 @@ def test_zero_tokens_is_noop():
 # decode
 # ---------------------------------------------------------------------------
 
-def _decode_steps(c, steps, dev=DEV):
-    cfg = L.config_of(c)
-    w = L.weights_on(c, dev)
-    cs = L.t_act(c.conv_state, dev)
-    rs = torch.from_numpy(c.rec_state).to(dev)
-    outs = []
-    for st in steps:
-        d = {n: L.t_act(st[n], dev) for n in "qkvabz"}
-        o = gdn.decode(cfg, w, d["q"], d["k"], d["v"], d["a"], d["b"], d["z"], cs, rs)
-        outs.append(L.to_f64(o).reshape(-1, c.n_v_heads, c.d_v))
-    gdn.check_device_error()
-    return outs, cs, L.to_f64(rs)
-
-
-def _as_sequences(c, steps, seqs):
-    """Per-step one-token inputs of the chosen sequences, packed as one prefill of
-    len(steps) tokens per sequence (prefill-then-decode equivalence)."""
-    n = len(steps)
-    acts = {k: np.concatenate([np.stack([st[k][s] for st in steps]) for s in seqs]) for k in "qkvabz"}
-    cu = np.arange(0, n * len(seqs) + 1, n, dtype=np.int32)
-    return acts, cu
+_decode_steps = L.decode_steps
+_as_sequences = L.as_sequences
 
 
 def test_decode_batch256_four_steps_all_heads():
