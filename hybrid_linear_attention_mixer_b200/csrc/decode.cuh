@@ -169,15 +169,53 @@ __global__ void __launch_bounds__(NT) gdn_decode_kernel(Args p) {
     }
 }
 
+// Multi-token rows: a state row (d_k fp32) is spread over 8 lanes; lane l of the row
+// holds the float4s at columns 4l + 32i, i < d_k/32, so each 16-byte access of the
+// row's 8 lanes is one contiguous 128-byte piece, and a row's dot products take
+// 3 butterfly steps instead of 5.  Dot products add in one fixed order (explicit fmaf,
+// then the butterfly over the 8 lanes).
+constexpr int MLPR = 8;     // lanes per state row
+constexpr int MRPP = 32 / MLPR;
+template <int NF4>
+__device__ __forceinline__ float row_dot(const float4 (&s)[NF4], const float4 (&v)[NF4]) {
+    float x = 0.f;
+#pragma unroll
+    for (int i = 0; i < NF4; i++) {
+        x = fmaf(s[i].x, v[i].x, x);
+        x = fmaf(s[i].y, v[i].y, x);
+        x = fmaf(s[i].z, v[i].z, x);
+        x = fmaf(s[i].w, v[i].w, x);
+    }
+#pragma unroll
+    for (int off = MLPR / 2; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    return x;
+}
+template <int NF4>
+__device__ __forceinline__ void row_load(const float* base, int lane8, float4 (&v)[NF4]) {
+#pragma unroll
+    for (int i = 0; i < NF4; i++) v[i] = *reinterpret_cast<const float4*>(base + 4 * lane8 + 32 * i);
+}
+// S_r <- alpha S_r + d k
+template <int NF4>
+__device__ __forceinline__ void row_update(float4 (&s)[NF4], const float4 (&k)[NF4], float al, float d) {
+#pragma unroll
+    for (int i = 0; i < NF4; i++) {
+        s[i].x = fmaf(al, s[i].x, d * k[i].x);
+        s[i].y = fmaf(al, s[i].y, d * k[i].y);
+        s[i].z = fmaf(al, s[i].z, d * k[i].z);
+        s[i].w = fmaf(al, s[i].w, d * k[i].w);
+    }
+}
+
 // ---------------------------------------------------------------------------
 // Multi-token decode (draft verification): n_tok consecutive tokens of each
 // sequence in one pass over its state.  Multi-token prediction drafts several
 // future tokens ("Qwen3.8-Flash-Next", "Architecture concepts": Multi-Token
 // Prediction; table "Every architecture field", row mtp_layers); checking a
 // draft runs the recurrence over the drafted tokens.  Row r of S takes the
-// n_tok updates one after another, exactly as n_tok decode steps would (same
-// operations in the same order, so the results are bit-identical to n_tok calls
-// of the one-token kernel), while the state is read and written once.
+// n_tok updates one after another, as n_tok decode steps would (equal to them up
+// to the order of fp32 additions inside a row's dot products), while the state is
+// read and written once.
 // Optionally the state after every token is written out (snapshots), so that
 // a caller who accepts only the first j drafted tokens can restore the state
 // after token j; the conv state after every token can be written out likewise.
@@ -194,14 +232,11 @@ struct MultiArgs {
 };
 
 __host__ __device__ constexpr size_t smem_floats_multi(int dk, int G, int dv, int n_tok) {
-    return (size_t)n_tok * (2 * dk + 2 * G * dv + 2 * G);
+    return (size_t)n_tok * (2 * dk + 2 * G * dv + 2 * G + 1);
 }
 
 template <typename TA, typename TO, int DK>
-__global__ void __launch_bounds__(NT) gdn_decode_multi_kernel(MultiArgs m) {
-    constexpr int LPR = DK / 4;        // lanes per state row (4 fp32 each)
-    constexpr int RPP = 32 / LPR;      // rows per warp pass
-    constexpr int U = DK == 128 ? 4 : 2;   // passes in flight per warp
+__global__ void __launch_bounds__(NT, 2) gdn_decode_multi_kernel(MultiArgs m) {
     const Args& p = m.a;
     const int NTK = m.n_tok;
     extern __shared__ float sm[];
@@ -214,6 +249,7 @@ __global__ void __launch_bounds__(NT) gdn_decode_multi_kernel(MultiArgs m) {
     float* so = sfeat + NTK * nch;          // [NTK][G*dv]
     float* s_al = so + NTK * G * dv;        // [NTK][G]
     float* s_be = s_al + NTK * G;           // [NTK][G]
+    float* s_kq = s_be + NTK * G;           // [NTK] k_t . q_t
 
     // ---- conv + SiLU of every token, with the conv-state roll ----
     const TA* pq = static_cast<const TA*>(p.q);
@@ -283,68 +319,74 @@ __global__ void __launch_bounds__(NT) gdn_decode_multi_kernel(MultiArgs m) {
     __syncthreads();
 
     // ---- stream the state rows: n_tok updates per row ----
-    const int col = 4 * (lane % LPR);
-    const int sub = lane / LPR;
-    float kq[kMaxTok];   // k_t . q_t, reduced over the row's lanes as the one-token kernel does
-#pragma unroll
-    for (int t = 0; t < kMaxTok; t++) {
-        if (t < NTK) {
-            const float4 k4 = *reinterpret_cast<const float4*>(sfeat + t * nch + DK + col);
-            const float4 q4 = *reinterpret_cast<const float4*>(sfeat + t * nch + col);
-            float x = k4.x * q4.x + k4.y * q4.y + k4.z * q4.z + k4.w * q4.w;
-#pragma unroll
-            for (int off = LPR / 2; off >= 1; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-            kq[t] = x;
-        }
+    constexpr int NF4 = DK / 32;
+    constexpr int U = DK == 32 ? 4 : 2;   // passes of MRPP rows in flight per warp
+    const int lane8 = lane % MLPR, sub = lane / MLPR;
+    if (warp < NTK) {   // k_t . q_t, formed as the one-token kernel forms it
+        const int t = warp;
+        float4 k4[NF4], q4[NF4];
+        row_load<NF4>(sfeat + t * nch + DK, lane8, k4);
+        row_load<NF4>(sfeat + t * nch, lane8, q4);
+        const float x = row_dot<NF4>(k4, q4);
+        if (lane == 0) s_kq[t] = x;
     }
+    for (int t = NW + warp; t < NTK; t += NW) {
+        float4 k4[NF4], q4[NF4];
+        row_load<NF4>(sfeat + t * nch + DK, lane8, k4);
+        row_load<NF4>(sfeat + t * nch, lane8, q4);
+        const float x = row_dot<NF4>(k4, q4);
+        if (lane == 0) s_kq[t] = x;
+    }
+    __syncthreads();
     const float inv_sqrt_dk = rsqrtf((float)DK);
     const int64_t blk = ((int64_t)seq * Hv + (int64_t)j * G) * dv * DK;
     float* Sb = p.rec_state + blk;
     const int64_t snap_stride = (int64_t)m.n_seqs * Hv * dv * DK;
     const int rows = G * dv;
-    for (int R0 = warp * RPP * U; R0 < rows; R0 += NW * RPP * U) {
-        float4 s[U];
+    for (int R0 = warp * MRPP * U; R0 < rows; R0 += NW * MRPP * U) {
+        float4 s[U][NF4];
 #pragma unroll
         for (int u = 0; u < U; u++) {
-            const int R = R0 + u * RPP + sub;
-            s[u] = R < rows ? __ldcs(reinterpret_cast<const float4*>(Sb + (int64_t)R * DK + col))
-                            : make_float4(0.f, 0.f, 0.f, 0.f);
+            const int R = R0 + u * MRPP + sub;
+#pragma unroll
+            for (int i = 0; i < NF4; i++)
+                s[u][i] = R < rows ? __ldcs(reinterpret_cast<const float4*>(Sb + (int64_t)R * DK + 4 * lane8 + 32 * i))
+                                   : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
         for (int t = 0; t < kMaxTok; t++) {
             if (t >= NTK) break;
-            const float4 k4 = *reinterpret_cast<const float4*>(sfeat + t * nch + DK + col);
-            const float4 q4 = *reinterpret_cast<const float4*>(sfeat + t * nch + col);
+            float4 k4[NF4], q4[NF4];
+            row_load<NF4>(sfeat + t * nch + DK, lane8, k4);
+            row_load<NF4>(sfeat + t * nch, lane8, q4);
 #pragma unroll
             for (int u = 0; u < U; u++) {
-                const int R = R0 + u * RPP + sub;
+                const int R = R0 + u * MRPP + sub;
                 const int g = min(R, rows - 1) / dv;
-                float uk = s[u].x * k4.x + s[u].y * k4.y + s[u].z * k4.z + s[u].w * k4.w;
-                float up = s[u].x * q4.x + s[u].y * q4.y + s[u].z * q4.z + s[u].w * q4.w;
-#pragma unroll
-                for (int off = LPR / 2; off >= 1; off >>= 1) {
-                    uk += __shfl_xor_sync(0xffffffffu, uk, off);
-                    up += __shfl_xor_sync(0xffffffffu, up, off);
-                }
+                const float uk = row_dot<NF4>(s[u], k4);
+                const float up = row_dot<NF4>(s[u], q4);
                 if (R < rows) {
                     const float al = s_al[t * G + g], be = s_be[t * G + g];
                     const float d = be * (sfeat[t * nch + 2 * DK + R] - al * uk);
-                    float4 o4;
-                    o4.x = fmaf(al, s[u].x, d * k4.x);
-                    o4.y = fmaf(al, s[u].y, d * k4.y);
-                    o4.z = fmaf(al, s[u].z, d * k4.z);
-                    o4.w = fmaf(al, s[u].w, d * k4.w);
-                    s[u] = o4;
-                    if (m.state_snap)
-                        __stcs(reinterpret_cast<float4*>(m.state_snap + t * snap_stride + blk + (int64_t)R * DK + col), o4);
-                    if (lane % LPR == 0) so[t * rows + R] = (al * up + d * kq[t]) * inv_sqrt_dk;
+                    row_update<NF4>(s[u], k4, al, d);
+                    if (m.state_snap) {
+#pragma unroll
+                        for (int i = 0; i < NF4; i++)
+                            __stcs(reinterpret_cast<float4*>(m.state_snap + t * snap_stride + blk + (int64_t)R * DK +
+                                                             4 * lane8 + 32 * i), s[u][i]);
+                    }
+                    if (lane8 == 0) so[t * rows + R] = (al * up + d * s_kq[t]) * inv_sqrt_dk;
                 }
             }
         }
 #pragma unroll
         for (int u = 0; u < U; u++) {
-            const int R = R0 + u * RPP + sub;
-            if (R < rows) __stcs(reinterpret_cast<float4*>(Sb + (int64_t)R * DK + col), s[u]);
+            const int R = R0 + u * MRPP + sub;
+            if (R < rows) {
+#pragma unroll
+                for (int i = 0; i < NF4; i++)
+                    __stcs(reinterpret_cast<float4*>(Sb + (int64_t)R * DK + 4 * lane8 + 32 * i), s[u][i]);
+            }
         }
     }
     __syncthreads();

@@ -137,8 +137,9 @@ gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w,
  * sequences, for checking tokens that a multi-token-prediction head drafted
  * ("Qwen3.8-Flash-Next", section "Architecture concepts": Multi-Token
  * Prediction drafts tokens at inference; table "Every architecture field",
- * row mtp_layers).  The result equals n_tok consecutive gdn_decode calls, bit
- * for bit, but each state is read and written once.
+ * row mtp_layers).  The result equals n_tok consecutive gdn_decode calls (the
+ * conv states bit for bit, the rest up to the order of fp32 additions inside a
+ * state row's dot products), but each state is read and written once.
  *   q, k [n_seqs*n_tok][H_k][d_k]; v, z [n_seqs*n_tok][H_v][d_v];
  *   a, b [n_seqs*n_tok][H_v]  act_dtype, token-major within a sequence: row
  *   seq*n_tok + t holds token t of sequence seq
