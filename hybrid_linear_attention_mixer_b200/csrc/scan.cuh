@@ -114,6 +114,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
     // the issuer has issued MMA1 (phase parity 0) or MMA2 (parity 1) of the current chunk: the
     // workers' TMEM traffic waits for it so that it does not slow the issue down
     const uint32_t ev_iss = sb + OFF_BAR + 152;
+    const uint32_t ev_m20 = sb + OFF_BAR + 160;           // [2] MMA2 of a chunk issued: (c) may queue behind it
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool worker = tid < NW;
@@ -162,6 +163,8 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
 #pragma unroll
             for (int i = 0; i < 15; i++) mbar_init(bar_ld0 + 8 * i, 1);   // ld, B2, fin, ev1, ev2, evo, end, evc, lfin, ldone
             mbar_init(ev_iss, 1);
+            mbar_init(ev_m20, 1);
+            mbar_init(ev_m20 + 8, 1);
             fence_mbar_init();
             *s_abort = 0;
             for (int i = 0; i < 4; i++) s_issued[i] = 0;
@@ -235,13 +238,14 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
                 fence_async_smem();
                 issue_chunk(ci + 2);
             }
+            if (ci + 1 < nchunks) {   // U accumulator (ci + 1) & 1 was read by the U conversion of chunk ci - 1
+                ok = lwait(ev_m20 + 8 * (ci & 1), (ci >> 1) & 1);   // queued behind MMA2 of chunk ci
+                if (ok) ok = lwait(bar_ld0 + 8 * ((ci + 1) & 1), ((ci + 1) >> 1) & 1);
+                if (!ok) break;
+                issue_c(ci + 1);      // the next MMA1 waits for it
+            }
             ok = lwait(ev20 + 8 * (ci & 1), (ci >> 1) & 1);         // MMA2 of chunk ci done; o of chunk ci - 1 staged
             if (!ok) break;
-            if (ci + 1 < nchunks) {   // U accumulator (ci + 1) & 1 was read by the U conversion of chunk ci - 1
-                ok = lwait(bar_ld0 + 8 * ((ci + 1) & 1), ((ci + 1) >> 1) & 1);
-                if (!ok) break;
-                issue_c(ci + 1);      // first: the next MMA1 waits for it
-            }
             if (ci + 2 < nchunks) issue_b2(ci + 2);
             if (ci > 0) issue_o(ci - 1);
             if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();   // the staging buffer of o(ci) is free
@@ -310,12 +314,13 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
     main_sync();
     if (*s_abort) goto abort_;
 
+// Every main thread waits for the tensor-core commit itself (no CTA barrier: the
+// barriers that follow each window order everything else).  A wait that gives up
+// raises the abort flag, which the next barrier's check turns into a uniform exit.
 #define GDN_MMA_WAIT()                                                                               \
     do {                                                                                             \
-        if (warp == IW && !mbar_wait_bounded(bar, mphase)) atomicOr((unsigned*)s_abort, 1u);       \
+        if (!mbar_wait_bounded(bar, mphase)) atomicOr((unsigned*)s_abort, 1u);                      \
         mphase ^= 1u;                                                                                \
-        main_sync();                                                                                 \
-        if (*s_abort) goto abort_;                                                                   \
         tc_fence_after();                                                                            \
     } while (0)
 
@@ -343,7 +348,6 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
             put_state_acc(decay);
         }
         GDN_MMA_WAIT();
-        if (warp == IW && lane == 0) mbar_arrive(ev10 + 8 * b);   // MMA1, (c) and the decay are done with buffer b
 
         // ---- U^T -> fp16 A operand ----
         if (warp == IW && ci > 0 && !mbar_wait_bounded(evo, (ci - 1) & 1))   // staging buffer for o(ci - 1)
@@ -357,6 +361,8 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         }
         tc_fence_before();
         main_sync();
+        if (*s_abort) goto abort_;
+        if (warp == IW && lane == 0) mbar_arrive(ev10 + 8 * b);   // MMA1, (c) and the decay are done with buffer b
 
         // ---- MMA2: [O^T | S] (parity 0) or [S | O^T] (parity 1) += U^T [P ; K~^T]^T ----
         if (warp == IW) {
@@ -367,7 +373,10 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
             for (int ks = 0; ks < 4; ks++)
                 mma_f16_ta_w(d2, tmem + TA_U + ks * 8, dB20 + b * (B2_STRIDE >> 4) + ks * 128, ID_FG, 1);
             mma_commit_w(bar);
-            if (lane == 0) mbar_arrive(ev_iss);
+            if (lane == 0) {
+                mbar_arrive(ev_iss);
+                mbar_arrive(ev_m20 + 8 * b);
+            }
         }
         // ---- workers, while MMA2 runs: the previous chunk's o tile ----
         if (worker && ci > 0) {
@@ -375,7 +384,6 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
             stage_o(ci - 1);
         }
         GDN_MMA_WAIT();
-        if (warp == IW && lane == 0) mbar_arrive(ev20 + 8 * b);   // B2 buffer b free; o(ci - 1) staged
 
         // ---- new state: its fp16 copy for the next MMA1, or the final state ----
         if (worker) {
@@ -398,6 +406,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         tc_fence_before();
         main_sync();
         if (*s_abort) goto abort_;
+        if (warp == IW && lane == 0) mbar_arrive(ev20 + 8 * b);   // B2 buffer b free; o(ci - 1) staged
     }
     if (warp == IW && !mbar_wait_bounded(evo, (nchunks - 1) & 1)) atomicOr((unsigned*)s_abort, 2u);
     main_sync();
