@@ -49,6 +49,9 @@ MULTI_TOK = 4
 MULTI_BYTES_PER_CALL = (2 * DECODE_N * H_V * D * D * 4 + 2 * DECODE_N * C_CONV * 3 * 2
                         + MULTI_TOK * DECODE_N * (2 * H_K * D + 2 * H_V * D + 2 * H_V) * 2
                         + MULTI_TOK * DECODE_N * H_V * D * 2 + (C_CONV * 4 + 2 * H_V + D) * 4)
+#   decode with a bf16 state: the state bytes halve
+BF16_BLOCK = 16
+DECODE_BF16_BYTES_PER_STEP = DECODE_BYTES_PER_STEP - DECODE_N * H_V * D * D * 4
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu DRAM bytes (read + write) per decode launch at batch 256, taken on the
 # decode kernel whose source hashes to DECODE_SRC_SHA; null once it changes.
@@ -305,6 +308,27 @@ def main():
         dist.all_reduce(tm, op=dist.ReduceOp.MAX)
     multi_ms = float(tm[0])
 
+    # ---- decode with the state stored in bf16: 16 consecutive steps per timed block ----
+    cfg_b = gdn.Config(state_dtype=torch.bfloat16)
+    b_rs = d_rs.to(torch.bfloat16)
+    b_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+            for _ in range(args.steps)]
+    for i in range(-args.warmup, args.steps):
+        flush.zero_()
+        if i >= 0:
+            b_ev[i][0].record(stream)
+        for st in steps[:BF16_BLOCK]:
+            gdn.decode(cfg_b, dw, st["q"], st["k"], st["v"], st["a"], st["b"], st["z"], d_cs, b_rs,
+                       out=d_out, stream=stream)
+        if i >= 0:
+            b_ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    gdn.check_device_error(stream)
+    tb = torch.tensor([sum(a.elapsed_time(b) for a, b in b_ev)], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(tb, op=dist.ReduceOp.MAX)
+    bf16_step_s = float(tb[0]) / 1e3 / (args.steps * BF16_BLOCK)
+
     # ---- end to end through the public API with host buffers ----
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
@@ -350,6 +374,9 @@ def main():
                              "unit": "GB/s", "us_per_call": multi_ms * 1e3 / K,
                              "tokens_per_s": DECODE_N * MULTI_TOK * world / (multi_ms / 1e3 / K),
                              "bytes_per_call": MULTI_BYTES_PER_CALL},
+            "decode_bf16_state": {"value": DECODE_BF16_BYTES_PER_STEP / bf16_step_s / 1e9, "unit": "GB/s",
+                                  "us_per_step": bf16_step_s * 1e6, "tokens_per_s": DECODE_N * world / bf16_step_s,
+                                  "bytes_per_step": DECODE_BF16_BYTES_PER_STEP},
             "prefill_ms": pre_ms / K,
             "roofline": {"kernel": "gdn_decode_kernel", "bound": "hbm", "achieved": dec_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / pk["hbm_gbs"],

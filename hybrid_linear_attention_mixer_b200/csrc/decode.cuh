@@ -21,6 +21,28 @@ namespace dec {
 constexpr int NT = 256;
 constexpr int NW = NT / 32;
 
+// 4 consecutive state entries: fp32 as is, or bf16 storage (read exactly, written
+// round-to-nearest-even); all arithmetic is fp32.  Streaming (evict-first) accesses.
+template <typename TS> struct State4;
+template <> struct State4<float> {
+    static __device__ __forceinline__ float4 ld(const float* p) { return __ldcs(reinterpret_cast<const float4*>(p)); }
+    static __device__ __forceinline__ void st(float* p, float4 v) { __stcs(reinterpret_cast<float4*>(p), v); }
+};
+template <> struct State4<__nv_bfloat16> {
+    static __device__ __forceinline__ float4 ld(const __nv_bfloat16* p) {
+        const uint2 u = __ldcs(reinterpret_cast<const uint2*>(p));
+        return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                           __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+    }
+    static __device__ __forceinline__ void st(__nv_bfloat16* p, float4 v) {
+        __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+        uint2 u;
+        u.x = *reinterpret_cast<uint32_t*>(&a);
+        u.y = *reinterpret_cast<uint32_t*>(&b);
+        __stcs(reinterpret_cast<uint2*>(p), u);
+    }
+};
+
 struct Args {
     const void *q, *k, *v, *a, *b, *z;   // act dtype; q,k [N][Hk*dk], v,z [N][Hv*dv], a,b [N][Hv]
     const float* conv_w;                 // [Ctot][4]
@@ -28,7 +50,7 @@ struct Args {
     const float* dt_bias;
     const float* norm_w;
     void* conv_state;                    // [N][Ctot][3] act dtype, in/out
-    float* rec_state;                    // [N][Hv][dv][dk], in/out
+    void* rec_state;                     // [N][Hv][dv][dk] state dtype (fp32 or bf16), in/out
     void* out;                           // [N][Hv][dv] out dtype
     int Hk, Hv, dk, dv;
     float l2_eps, norm_eps;
@@ -38,7 +60,7 @@ __host__ __device__ constexpr size_t smem_floats(int dk, int G, int dv) {
     return (size_t)2 * dk + (size_t)2 * G * dv + 2 * G;
 }
 
-template <typename TA, typename TO, int DK>
+template <typename TA, typename TO, typename TS, int DK>
 __global__ void __launch_bounds__(NT) gdn_decode_kernel(Args p) {
     constexpr int LPR = DK / 4;        // lanes per state row (4 fp32 each)
     constexpr int RPP = 32 / LPR;      // rows per warp pass
@@ -115,14 +137,14 @@ __global__ void __launch_bounds__(NT) gdn_decode_kernel(Args p) {
 #pragma unroll
     for (int off = LPR / 2; off >= 1; off >>= 1) kq += __shfl_xor_sync(0xffffffffu, kq, off);
     const float inv_sqrt_dk = rsqrtf((float)DK);
-    float* Sb = p.rec_state + ((int64_t)seq * Hv + (int64_t)j * G) * dv * DK;
+    TS* Sb = static_cast<TS*>(p.rec_state) + ((int64_t)seq * Hv + (int64_t)j * G) * dv * DK;
     const int rows = G * dv;
     for (int R0 = warp * RPP * U; R0 < rows; R0 += NW * RPP * U) {
         float4 s[U];
 #pragma unroll
         for (int u = 0; u < U; u++) {
             const int R = R0 + u * RPP + sub;
-            s[u] = R < rows ? __ldcs(reinterpret_cast<const float4*>(Sb + (int64_t)R * DK + col))
+            s[u] = R < rows ? State4<TS>::ld(Sb + (int64_t)R * DK + col)
                             : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
@@ -144,7 +166,7 @@ __global__ void __launch_bounds__(NT) gdn_decode_kernel(Args p) {
                 o4.y = fmaf(al, s[u].y, d * k4.y);
                 o4.z = fmaf(al, s[u].z, d * k4.z);
                 o4.w = fmaf(al, s[u].w, d * k4.w);
-                __stcs(reinterpret_cast<float4*>(Sb + (int64_t)R * DK + col), o4);
+                State4<TS>::st(Sb + (int64_t)R * DK + col, o4);
                 if (lane % LPR == 0) so[R] = (al * up + d * kq) * inv_sqrt_dk;
             }
         }
@@ -226,7 +248,7 @@ constexpr int kMaxTok = 16;
 struct MultiArgs {
     Args a;
     int n_tok;
-    float* state_snap;   // [n_tok][N][Hv][dv][dk] or null
+    void* state_snap;    // [n_tok][N][Hv][dv][dk] state dtype, or null
     void* conv_snap;     // [n_tok][N][Ctot][3] act dtype, or null
     int n_seqs;
 };
@@ -235,7 +257,7 @@ __host__ __device__ constexpr size_t smem_floats_multi(int dk, int G, int dv, in
     return (size_t)n_tok * (2 * dk + 2 * G * dv + 2 * G + 1);
 }
 
-template <typename TA, typename TO, int DK>
+template <typename TA, typename TO, typename TS, int DK>
 __global__ void __launch_bounds__(NT, 2) gdn_decode_multi_kernel(MultiArgs m) {
     const Args& p = m.a;
     const int NTK = m.n_tok;
@@ -340,7 +362,8 @@ __global__ void __launch_bounds__(NT, 2) gdn_decode_multi_kernel(MultiArgs m) {
     __syncthreads();
     const float inv_sqrt_dk = rsqrtf((float)DK);
     const int64_t blk = ((int64_t)seq * Hv + (int64_t)j * G) * dv * DK;
-    float* Sb = p.rec_state + blk;
+    TS* Sb = static_cast<TS*>(p.rec_state) + blk;
+    TS* snap0 = static_cast<TS*>(m.state_snap);
     const int64_t snap_stride = (int64_t)m.n_seqs * Hv * dv * DK;
     const int rows = G * dv;
     for (int R0 = warp * MRPP * U; R0 < rows; R0 += NW * MRPP * U) {
@@ -350,7 +373,7 @@ __global__ void __launch_bounds__(NT, 2) gdn_decode_multi_kernel(MultiArgs m) {
             const int R = R0 + u * MRPP + sub;
 #pragma unroll
             for (int i = 0; i < NF4; i++)
-                s[u][i] = R < rows ? __ldcs(reinterpret_cast<const float4*>(Sb + (int64_t)R * DK + 4 * lane8 + 32 * i))
+                s[u][i] = R < rows ? State4<TS>::ld(Sb + (int64_t)R * DK + 4 * lane8 + 32 * i)
                                    : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
@@ -369,11 +392,11 @@ __global__ void __launch_bounds__(NT, 2) gdn_decode_multi_kernel(MultiArgs m) {
                     const float al = s_al[t * G + g], be = s_be[t * G + g];
                     const float d = be * (sfeat[t * nch + 2 * DK + R] - al * uk);
                     row_update<NF4>(s[u], k4, al, d);
-                    if (m.state_snap) {
+                    if (snap0) {
 #pragma unroll
                         for (int i = 0; i < NF4; i++)
-                            __stcs(reinterpret_cast<float4*>(m.state_snap + t * snap_stride + blk + (int64_t)R * DK +
-                                                             4 * lane8 + 32 * i), s[u][i]);
+                            State4<TS>::st(snap0 + t * snap_stride + blk + (int64_t)R * DK + 4 * lane8 + 32 * i,
+                                           s[u][i]);
                     }
                     if (lane8 == 0) so[t * rows + R] = (al * up + d * s_kq[t]) * inv_sqrt_dk;
                 }
@@ -385,7 +408,7 @@ __global__ void __launch_bounds__(NT, 2) gdn_decode_multi_kernel(MultiArgs m) {
             if (R < rows) {
 #pragma unroll
                 for (int i = 0; i < NF4; i++)
-                    __stcs(reinterpret_cast<float4*>(Sb + (int64_t)R * DK + 4 * lane8 + 32 * i), s[u][i]);
+                    State4<TS>::st(Sb + (int64_t)R * DK + 4 * lane8 + 32 * i, s[u][i]);
             }
         }
     }

@@ -32,6 +32,7 @@ gdn_status check_config(const gdn_config* c) {
         return GDN_ERR_INVALID_ARG;
     if (c->act_dtype != GDN_BF16 && c->act_dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
     if (c->out_dtype != GDN_BF16 && c->out_dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
+    if (c->state_dtype != GDN_BF16 && c->state_dtype != GDN_F32) return GDN_ERR_INVALID_ARG;
     if (c->n_v_heads % c->n_k_heads != 0) return GDN_ERR_UNSUPPORTED;
     if (!dim_ok(c->d_k) || !dim_ok(c->d_v)) return GDN_ERR_UNSUPPORTED;
     if (c->conv_kernel != 4 || c->chunk != gdn::intra::C) return GDN_ERR_UNSUPPORTED;
@@ -71,7 +72,7 @@ Layout workspace_layout(const gdn_config* c, int64_t T, int64_t n_seqs) {
 // Opt in to > 48 KiB of dynamic shared memory, once per device and kernel.
 template <typename K>
 cudaError_t ensure_smem(K kernel, int variant, size_t bytes) {
-    static bool done[64][16];
+    static bool done[64][32];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -155,7 +156,7 @@ int sm_count() {
 template <typename TA, typename TO>
 cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void* q, const void* k,
                            const void* v, const void* a, const void* b, const void* z, void* conv_state,
-                           float* rec_state, const int32_t* cu, int n_seqs, int64_t T, void* out,
+                           void* rec_state, const int32_t* cu, int n_seqs, int64_t T, void* out,
                            void* ws, int variant, cudaStream_t st) {
     const Layout L = workspace_layout(c, T, n_seqs);
     uint8_t* wsb = static_cast<uint8_t*>(ws);
@@ -174,10 +175,11 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     // Set-up first: nothing is launched unless the tensor maps encode and the
     // kernels' shared-memory opt-ins succeed.
     auto k_intra = gdn::intra::gdn_intra_kernel<TA>;
-    auto k_scan = gdn::scan::gdn_scan_kernel<TO>;
+    auto k_scan = c->state_dtype == GDN_BF16 ? gdn::scan::gdn_scan_kernel<TO, __nv_bfloat16>
+                                             : gdn::scan::gdn_scan_kernel<TO, float>;
     cudaError_t e = ensure_smem(k_intra, 4 + (sizeof(TA) == 2 ? 0 : 1), gdn::intra::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = ensure_smem(k_scan, 6 + (sizeof(TO) == 2 ? 0 : 1), gdn::scan::SMEM_BYTES);
+    e = ensure_smem(k_scan, 16 + (sizeof(TO) == 2 ? 0 : 1) + (c->state_dtype == GDN_BF16 ? 2 : 0), gdn::scan::SMEM_BYTES);
     if (e != cudaSuccess) return e;
     e = ensure_smem(gdn::norm::gdn_gated_norm_kernel<TA, TO>, 8 + (sizeof(TA) == 4 ? 2 : 0) + (sizeof(TO) == 4 ? 1 : 0),
                     gdn::norm::smem_bytes<TA, TO>());
@@ -248,11 +250,11 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     return cudaGetLastError();
 }
 
-template <typename TA, typename TO, int DK>
+template <typename TA, typename TO, typename TS, int DK>
 cudaError_t launch_decode_dk(const gdn::dec::Args& a, int n_seqs, cudaStream_t st) {
     const int G = a.Hv / a.Hk;
     const size_t smem = gdn::dec::smem_floats(DK, G, a.dv) * sizeof(float);
-    auto kern = gdn::dec::gdn_decode_kernel<TA, TO, DK>;
+    auto kern = gdn::dec::gdn_decode_kernel<TA, TO, TS, DK>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
@@ -261,11 +263,11 @@ cudaError_t launch_decode_dk(const gdn::dec::Args& a, int n_seqs, cudaStream_t s
     return cudaGetLastError();
 }
 
-template <typename TA, typename TO, int DK>
+template <typename TA, typename TO, typename TS, int DK>
 cudaError_t launch_decode_multi_dk(const gdn::dec::MultiArgs& m, cudaStream_t st) {
     const int G = m.a.Hv / m.a.Hk;
     const size_t smem = gdn::dec::smem_floats_multi(DK, G, m.a.dv, m.n_tok) * sizeof(float);
-    auto kern = gdn::dec::gdn_decode_multi_kernel<TA, TO, DK>;
+    auto kern = gdn::dec::gdn_decode_multi_kernel<TA, TO, TS, DK>;
     if (smem > 48 * 1024) {
         cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         if (e != cudaSuccess) return e;
@@ -274,22 +276,32 @@ cudaError_t launch_decode_multi_dk(const gdn::dec::MultiArgs& m, cudaStream_t st
     return cudaGetLastError();
 }
 
-template <typename TA, typename TO>
-cudaError_t launch_decode_multi(const gdn::dec::MultiArgs& m, cudaStream_t st) {
+template <typename TA, typename TO, typename TS>
+cudaError_t launch_decode_multi_ts(const gdn::dec::MultiArgs& m, cudaStream_t st) {
     switch (m.a.dk) {
-        case 32: return launch_decode_multi_dk<TA, TO, 32>(m, st);
-        case 64: return launch_decode_multi_dk<TA, TO, 64>(m, st);
-        default: return launch_decode_multi_dk<TA, TO, 128>(m, st);
+        case 32: return launch_decode_multi_dk<TA, TO, TS, 32>(m, st);
+        case 64: return launch_decode_multi_dk<TA, TO, TS, 64>(m, st);
+        default: return launch_decode_multi_dk<TA, TO, TS, 128>(m, st);
     }
 }
-
 template <typename TA, typename TO>
-cudaError_t launch_decode(const gdn::dec::Args& a, int n_seqs, cudaStream_t st) {
+cudaError_t launch_decode_multi(const gdn::dec::MultiArgs& m, bool bf16_state, cudaStream_t st) {
+    return bf16_state ? launch_decode_multi_ts<TA, TO, __nv_bfloat16>(m, st)
+                      : launch_decode_multi_ts<TA, TO, float>(m, st);
+}
+
+template <typename TA, typename TO, typename TS>
+cudaError_t launch_decode_ts(const gdn::dec::Args& a, int n_seqs, cudaStream_t st) {
     switch (a.dk) {
-        case 32: return launch_decode_dk<TA, TO, 32>(a, n_seqs, st);
-        case 64: return launch_decode_dk<TA, TO, 64>(a, n_seqs, st);
-        default: return launch_decode_dk<TA, TO, 128>(a, n_seqs, st);
+        case 32: return launch_decode_dk<TA, TO, TS, 32>(a, n_seqs, st);
+        case 64: return launch_decode_dk<TA, TO, TS, 64>(a, n_seqs, st);
+        default: return launch_decode_dk<TA, TO, TS, 128>(a, n_seqs, st);
     }
+}
+template <typename TA, typename TO>
+cudaError_t launch_decode(const gdn::dec::Args& a, int n_seqs, bool bf16_state, cudaStream_t st) {
+    return bf16_state ? launch_decode_ts<TA, TO, __nv_bfloat16>(a, n_seqs, st)
+                      : launch_decode_ts<TA, TO, float>(a, n_seqs, st);
 }
 
 }  // namespace
@@ -308,6 +320,7 @@ void gdn_config_default(gdn_config* cfg) {
     cfg->norm_eps = 1e-6f;
     cfg->act_dtype = GDN_BF16;
     cfg->out_dtype = GDN_BF16;
+    cfg->state_dtype = GDN_F32;
 }
 
 size_t gdn_prefill_workspace_size(const gdn_config* cfg, int64_t T_total, int32_t n_seqs) {
@@ -317,7 +330,7 @@ size_t gdn_prefill_workspace_size(const gdn_config* cfg, int64_t T_total, int32_
 
 gdn_status gdn_prefill(const gdn_config* cfg, const gdn_weights* w, const void* q, const void* k,
                        const void* v, const void* a, const void* b, const void* z, void* conv_state,
-                       float* rec_state, const int32_t* cu_seqlens, int32_t n_seqs, int64_t T_total,
+                       void* rec_state, const int32_t* cu_seqlens, int32_t n_seqs, int64_t T_total,
                        void* out, void* workspace, size_t workspace_bytes, void* stream) {
     gdn_status s = check_config(cfg);
     if (s != GDN_OK) return s;
@@ -353,7 +366,7 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_weights* w, const void* 
 
 gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w, const void* q, const void* k,
                       const void* v, const void* a, const void* b, const void* z, void* conv_state,
-                      float* rec_state, int32_t n_seqs, void* out, void* stream) {
+                      void* rec_state, int32_t n_seqs, void* out, void* stream) {
     gdn_status s = check_config(cfg);
     if (s != GDN_OK) return s;
     if ((s = check_weights(w)) != GDN_OK) return s;
@@ -375,10 +388,11 @@ gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w, const void* q
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     const bool abf = cfg->act_dtype == GDN_BF16, obf = cfg->out_dtype == GDN_BF16;
-    if (abf && obf) e = launch_decode<__nv_bfloat16, __nv_bfloat16>(da, n_seqs, st);
-    else if (abf) e = launch_decode<__nv_bfloat16, float>(da, n_seqs, st);
-    else if (obf) e = launch_decode<float, __nv_bfloat16>(da, n_seqs, st);
-    else e = launch_decode<float, float>(da, n_seqs, st);
+    const bool sbf = cfg->state_dtype == GDN_BF16;
+    if (abf && obf) e = launch_decode<__nv_bfloat16, __nv_bfloat16>(da, n_seqs, sbf, st);
+    else if (abf) e = launch_decode<__nv_bfloat16, float>(da, n_seqs, sbf, st);
+    else if (obf) e = launch_decode<float, __nv_bfloat16>(da, n_seqs, sbf, st);
+    else e = launch_decode<float, float>(da, n_seqs, sbf, st);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -386,7 +400,7 @@ static_assert(gdn::dec::kMaxTok == GDN_DECODE_MULTI_MAX_TOKENS, "multi-token lim
 
 gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_weights* w, const void* q, const void* k,
                             const void* v, const void* a, const void* b, const void* z, void* conv_state,
-                            float* rec_state, int32_t n_seqs, int32_t n_tok, void* out, float* state_snapshots,
+                            void* rec_state, int32_t n_seqs, int32_t n_tok, void* out, void* state_snapshots,
                             void* conv_snapshots, void* stream) {
     gdn_status s = check_config(cfg);
     if (s != GDN_OK) return s;
@@ -415,10 +429,11 @@ gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_weights* w, const v
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;
     const bool abf = cfg->act_dtype == GDN_BF16, obf = cfg->out_dtype == GDN_BF16;
-    if (abf && obf) e = launch_decode_multi<__nv_bfloat16, __nv_bfloat16>(m, st);
-    else if (abf) e = launch_decode_multi<__nv_bfloat16, float>(m, st);
-    else if (obf) e = launch_decode_multi<float, __nv_bfloat16>(m, st);
-    else e = launch_decode_multi<float, float>(m, st);
+    const bool sbf = cfg->state_dtype == GDN_BF16;
+    if (abf && obf) e = launch_decode_multi<__nv_bfloat16, __nv_bfloat16>(m, sbf, st);
+    else if (abf) e = launch_decode_multi<__nv_bfloat16, float>(m, sbf, st);
+    else if (obf) e = launch_decode_multi<float, __nv_bfloat16>(m, sbf, st);
+    else e = launch_decode_multi<float, float>(m, sbf, st);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -463,7 +478,7 @@ void* g_noalloc_addr[64];   // device address of g_noalloc_scratch, per device
 
 extern "C" gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const gdn_weights* w, const void* q,
                                           const void* k, const void* v, const void* a, const void* b,
-                                          const void* z, void* conv_state, float* rec_state,
+                                          const void* z, void* conv_state, void* rec_state,
                                           const int32_t* cu_seqlens, int32_t n_seqs, int64_t T_total,
                                           void* out, void* stream) {
     gdn_status s = check_config(cfg);

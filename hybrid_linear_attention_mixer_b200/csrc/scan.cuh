@@ -74,7 +74,7 @@ __host__ __device__ constexpr uint32_t acc_o(int b) { return b ? ACC_O1 : ACC_O0
 constexpr uint32_t LD_BYTES = 2 * 8192 + intra::REC_B1_BYTES;   // v halves + B1, T, g
 
 struct Args {
-    float* rec_state;           // [N][Hv][dv][dk] in/out
+    void* rec_state;            // [N][Hv][dv][dk] state dtype (fp32 or bf16), in/out
     const int32_t* cu;          // [N+1]
     const int32_t* chunk_off;   // [N+1]
     const uint8_t* rec;         // intra-chunk records
@@ -82,12 +82,26 @@ struct Args {
     int Hk, Hv, dk, dv;
 };
 
+// 4 consecutive state entries: fp32, or bf16 storage (read exactly, written
+// round-to-nearest-even); the chain itself always runs in fp32
+__device__ __forceinline__ float4 ld_state4(const float* p) { return *reinterpret_cast<const float4*>(p); }
+__device__ __forceinline__ float4 ld_state4(const __nv_bfloat16* p) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u), __uint_as_float(u.y << 16),
+                       __uint_as_float(u.y & 0xffff0000u));
+}
+__device__ __forceinline__ void st_state4(float* p, float4 v) { *reinterpret_cast<float4*>(p) = v; }
+__device__ __forceinline__ void st_state4(__nv_bfloat16* p, float4 v) {
+    __nv_bfloat162 a = __floats2bfloat162_rn(v.x, v.y), b = __floats2bfloat162_rn(v.z, v.w);
+    *reinterpret_cast<uint2*>(p) = make_uint2(*reinterpret_cast<uint32_t*>(&a), *reinterpret_cast<uint32_t*>(&b));
+}
+
 __device__ __forceinline__ void main_sync() { asm volatile("bar.sync 1, %0;" ::"n"(NMAIN) : "memory"); }
 __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
 }
 
-template <typename TO>
+template <typename TO, typename TS>
 __global__ void __launch_bounds__(NT, 1)
 gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
     constexpr uint32_t O_BYTES = C * 128 * sizeof(TO);
@@ -178,14 +192,14 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         tmem_relinquish();
     }
     const int dv_r = 32 * qd + lane;   // this worker's state row; columns [32 cs, 32 cs + 32)
-    float* gstate = p.rec_state + ((int64_t)seq * Hv + h) * dv * dk;
+    TS* gstate = static_cast<TS*>(p.rec_state) + ((int64_t)seq * Hv + h) * dv * dk;
     float Sv[32];   // this worker's slice of the state at the start of the current chunk
     if (worker) {
 #pragma unroll
         for (int i4 = 0; i4 < 8; i4++) {   // 16-byte loads (d_k and the slice start are multiples of 4)
             const int col = 32 * cs + 4 * i4;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (dv_r < dv && col < dk) v = *reinterpret_cast<const float4*>(gstate + (int64_t)dv_r * dk + col);
+            if (dv_r < dv && col < dk) v = ld_state4(gstate + (int64_t)dv_r * dk + col);
             Sv[4 * i4] = v.x; Sv[4 * i4 + 1] = v.y; Sv[4 * i4 + 2] = v.z; Sv[4 * i4 + 3] = v.w;
         }
     }
@@ -398,8 +412,8 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
                 for (int i4 = 0; i4 < 8; i4++) {
                     const int col = 32 * cs + 4 * i4;
                     if (dv_r < dv && col < dk)
-                        *reinterpret_cast<float4*>(gstate + (int64_t)dv_r * dk + col) =
-                            make_float4(Sv[4 * i4], Sv[4 * i4 + 1], Sv[4 * i4 + 2], Sv[4 * i4 + 3]);
+                        st_state4(gstate + (int64_t)dv_r * dk + col,
+                                  make_float4(Sv[4 * i4], Sv[4 * i4 + 1], Sv[4 * i4 + 2], Sv[4 * i4 + 3]));
                 }
             }
         }

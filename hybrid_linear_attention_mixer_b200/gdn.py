@@ -38,7 +38,8 @@ class _CConfig(ctypes.Structure):
                 ("d_k", ctypes.c_int32), ("d_v", ctypes.c_int32),
                 ("conv_kernel", ctypes.c_int32), ("chunk", ctypes.c_int32),
                 ("l2_eps", ctypes.c_float), ("norm_eps", ctypes.c_float),
-                ("act_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32)]
+                ("act_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
+                ("state_dtype", ctypes.c_int32)]
 
 
 class _CWeights(ctypes.Structure):
@@ -96,6 +97,7 @@ class Config:
     norm_eps: float = 1e-6
     act_dtype: torch.dtype = torch.bfloat16
     out_dtype: torch.dtype = torch.bfloat16
+    state_dtype: torch.dtype = torch.float32   # bf16: the recurrent state stored in bf16
 
     @property
     def channels(self) -> int:
@@ -104,7 +106,7 @@ class Config:
     def c(self) -> _CConfig:
         return _CConfig(self.n_k_heads, self.n_v_heads, self.d_k, self.d_v, self.conv_kernel,
                         self.chunk, self.l2_eps, self.norm_eps, _DT[self.act_dtype],
-                        _DT[self.out_dtype])
+                        _DT[self.out_dtype], _DT[self.state_dtype])
 
 
 def _ptr(t):
@@ -146,7 +148,7 @@ def prefill(cfg: Config, w: dict, q, k, v, a, b, z, conv_state, rec_state, cu_se
     for n, t in (("q", q), ("k", k), ("v", v), ("a", a), ("b", b), ("z", z),
                  ("conv_state", conv_state)):
         _check(t, n, cfg.act_dtype, dev)
-    _check(rec_state, "rec_state", torch.float32, dev)
+    _check(rec_state, "rec_state", cfg.state_dtype, dev)
     _check(cu_seqlens, "cu_seqlens", torch.int32, dev)
     n_seqs = cu_seqlens.shape[0] - 1
     if out is None:
@@ -171,7 +173,7 @@ def decode(cfg: Config, w: dict, q, k, v, a, b, z, conv_state, rec_state, out=No
     for n, t in (("q", q), ("k", k), ("v", v), ("a", a), ("b", b), ("z", z),
                  ("conv_state", conv_state)):
         _check(t, n, cfg.act_dtype, dev)
-    _check(rec_state, "rec_state", torch.float32, dev)
+    _check(rec_state, "rec_state", cfg.state_dtype, dev)
     if out is None:
         out = torch.empty((N, cfg.n_v_heads * cfg.d_v), dtype=cfg.out_dtype, device=dev)
     _check(out, "out", cfg.out_dtype, dev)
@@ -188,7 +190,7 @@ def decode_multi(cfg: Config, w: dict, q, k, v, a, b, z, conv_state, rec_state, 
                  state_snapshots=None, conv_snapshots=None, stream=None):
     """n_tok consecutive tokens per sequence (rows token-major within a sequence);
     returns out [N*n_tok, H_v*d_v].  Optional snapshots receive the recurrent state
-    [n_tok, N, H_v, d_v, d_k] (fp32) and the conv state [n_tok, N, C, K-1] after each token."""
+    [n_tok, N, H_v, d_v, d_k] (state dtype) and the conv state [n_tok, N, C, K-1] after each token."""
     dev = q.device
     rows = q.shape[0]
     if n_tok <= 0 or rows % n_tok:
@@ -197,9 +199,9 @@ def decode_multi(cfg: Config, w: dict, q, k, v, a, b, z, conv_state, rec_state, 
     for n, t in (("q", q), ("k", k), ("v", v), ("a", a), ("b", b), ("z", z),
                  ("conv_state", conv_state)):
         _check(t, n, cfg.act_dtype, dev)
-    _check(rec_state, "rec_state", torch.float32, dev)
+    _check(rec_state, "rec_state", cfg.state_dtype, dev)
     if state_snapshots is not None:
-        _check(state_snapshots, "state_snapshots", torch.float32, dev)
+        _check(state_snapshots, "state_snapshots", cfg.state_dtype, dev)
     if conv_snapshots is not None:
         _check(conv_snapshots, "conv_snapshots", cfg.act_dtype, dev)
     if out is None:

@@ -76,6 +76,10 @@ typedef struct {
     float norm_eps;       /* default 1e-6     */
     int32_t act_dtype;    /* gdn_dtype of q, k, v, a, b, z, conv_state; default GDN_BF16 */
     int32_t out_dtype;    /* gdn_dtype of out; default GDN_BF16 */
+    int32_t state_dtype;  /* gdn_dtype of rec_state and of state snapshots; default GDN_F32
+                             (the layer's fp32 state).  GDN_BF16 stores the state in bf16
+                             (half the bytes a decode step moves); every step still
+                             computes in fp32 and rounds the stored state to nearest even */
 } gdn_config;
 
 typedef struct {
@@ -87,7 +91,7 @@ typedef struct {
 } gdn_weights;
 
 /* Fills *cfg with the layer's published shape (16/48 heads of 128, K = 4,
- * chunk 64, eps 1e-6, bf16 activations and output). */
+ * chunk 64, eps 1e-6, bf16 activations and output, fp32 state). */
 void gdn_config_default(gdn_config* cfg);
 
 /* Bytes of device workspace gdn_prefill needs for T_total packed tokens.
@@ -100,7 +104,7 @@ size_t gdn_prefill_workspace_size(const gdn_config* cfg, int64_t T_total, int32_
  *   v, z        [T_total][H_v][d_v]    act_dtype
  *   a, b        [T_total][H_v]         act_dtype
  *   conv_state  [n_seqs][2*H_k*d_k + H_v*d_v][K-1]  act_dtype, in/out, oldest first
- *   rec_state   [n_seqs][H_v][d_v][d_k] float32, in/out
+ *   rec_state   [n_seqs][H_v][d_v][d_k] state_dtype (float32 by default), in/out
  *   cu_seqlens  [n_seqs + 1] int32 device, cu_seqlens[0] = 0, non-decreasing,
  *               cu_seqlens[n_seqs] = T_total (not checked on the host: it is
  *               device memory and reading it would synchronise)
@@ -112,7 +116,7 @@ size_t gdn_prefill_workspace_size(const gdn_config* cfg, int64_t T_total, int32_
 gdn_status gdn_prefill(const gdn_config* cfg, const gdn_weights* w,
                        const void* q, const void* k, const void* v,
                        const void* a, const void* b, const void* z,
-                       void* conv_state, float* rec_state,
+                       void* conv_state, void* rec_state,
                        const int32_t* cu_seqlens, int32_t n_seqs, int64_t T_total,
                        void* out, void* workspace, size_t workspace_bytes, void* stream);
 
@@ -120,13 +124,13 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_weights* w,
  * One decode step: one new token for each of n_seqs sequences.
  *   q, k [n_seqs][H_k][d_k]; v, z [n_seqs][H_v][d_v]; a, b [n_seqs][H_v]  act_dtype
  *   conv_state [n_seqs][C][K-1] act_dtype in/out; rec_state [n_seqs][H_v][d_v][d_k]
- *   float32 in/out; out [n_seqs][H_v][d_v] out_dtype.  No workspace.
+ *   state_dtype in/out; out [n_seqs][H_v][d_v] out_dtype.  No workspace.
  * Equal to gdn_prefill with every sequence of length 1.
  */
 gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w,
                       const void* q, const void* k, const void* v,
                       const void* a, const void* b, const void* z,
-                      void* conv_state, float* rec_state, int32_t n_seqs,
+                      void* conv_state, void* rec_state, int32_t n_seqs,
                       void* out, void* stream);
 
 /* Largest number of tokens per sequence that gdn_decode_multi takes in one call. */
@@ -144,10 +148,10 @@ gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w,
  *   a, b [n_seqs*n_tok][H_v]  act_dtype, token-major within a sequence: row
  *   seq*n_tok + t holds token t of sequence seq
  *   conv_state [n_seqs][C][K-1] act_dtype in/out; rec_state
- *   [n_seqs][H_v][d_v][d_k] float32 in/out (the state after the last token)
+ *   [n_seqs][H_v][d_v][d_k] state_dtype in/out (the state after the last token)
  *   out [n_seqs*n_tok][H_v][d_v] out_dtype
  *   state_snapshots  optional (may be NULL), [n_tok][n_seqs][H_v][d_v][d_k]
- *                    float32, 16-byte aligned: the state after each token, so
+ *                    state_dtype, 16-byte aligned: the state after each token, so
  *                    that a caller who accepts only the first j drafted tokens
  *                    can restore the state after token j
  *   conv_snapshots   optional (may be NULL), [n_tok][n_seqs][C][K-1] act_dtype:
@@ -158,8 +162,8 @@ gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w,
 gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_weights* w,
                             const void* q, const void* k, const void* v,
                             const void* a, const void* b, const void* z,
-                            void* conv_state, float* rec_state, int32_t n_seqs, int32_t n_tok,
-                            void* out, float* state_snapshots, void* conv_snapshots, void* stream);
+                            void* conv_state, void* rec_state, int32_t n_seqs, int32_t n_tok,
+                            void* out, void* state_snapshots, void* conv_snapshots, void* stream);
 
 /* Capacity, in bytes, of the fixed scratch array used by gdn_prefill_noalloc. */
 #define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
@@ -200,7 +204,7 @@ gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_weights* w,
 gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const gdn_weights* w,
                                const void* q, const void* k, const void* v,
                                const void* a, const void* b, const void* z,
-                               void* conv_state, float* rec_state,
+                               void* conv_state, void* rec_state,
                                const int32_t* cu_seqlens, int32_t n_seqs, int64_t T_total,
                                void* out, void* stream);
 

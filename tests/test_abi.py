@@ -41,7 +41,7 @@ def test_default_config_is_the_published_shape(lib):
     lib.gdn_config_default(ctypes.byref(c))
     assert (c.n_k_heads, c.n_v_heads, c.d_k, c.d_v, c.conv_kernel, c.chunk) == (16, 48, 128, 128, 4, 64)
     assert abs(c.norm_eps - 1e-6) < 1e-12 and abs(c.l2_eps - 1e-6) < 1e-12
-    assert c.act_dtype == 0 and c.out_dtype == 0
+    assert c.act_dtype == 0 and c.out_dtype == 0 and c.state_dtype == 1   # bf16 I/O, fp32 state
 
 
 def test_workspace_size(lib):
@@ -76,6 +76,9 @@ def test_argument_errors_are_synchronous_and_launch_nothing(lib):
     assert _call_prefill(lib, gdn.Config(n_k_heads=5)) == UNSUPPORTED
     assert _call_prefill(lib, gdn.Config(conv_kernel=3)) == UNSUPPORTED
     assert _call_prefill(lib, gdn.Config(chunk=32)) == UNSUPPORTED
+    bad = gdn.Config().c()
+    bad.state_dtype = 7
+    assert lib.gdn_prefill_workspace_size(ctypes.byref(bad), 16, 1) == 0   # invalid config
     assert _call_prefill(lib, cfg, ptr=0x1001) == INVALID          # misaligned activation
     assert _call_prefill(lib, cfg, ws=0x100010) == INVALID         # workspace not 256-aligned
     assert _call_prefill(lib, cfg, ws_bytes=1000) == WORKSPACE
