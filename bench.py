@@ -52,11 +52,16 @@ MULTI_BYTES_PER_CALL = (2 * DECODE_N * H_V * D * D * 4 + 2 * DECODE_N * C_CONV *
 #   decode with a bf16 state: the state bytes halve
 BF16_BLOCK = 16
 DECODE_BF16_BYTES_PER_STEP = DECODE_BYTES_PER_STEP - DECODE_N * H_V * D * D * 4
+#   projections around the mixer (hidden size 2,560): dense FLOPs per call at PREFILL_T tokens
+D_MODEL = 2560
+PROJ_IN_N = 2 * H_K * D + 2 * H_V * D + 2 * H_V
+PROJ_IN_FLOP = 2 * PREFILL_T * D_MODEL * PROJ_IN_N
+PROJ_OUT_FLOP = 2 * PREFILL_T * H_V * D * D_MODEL
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu DRAM bytes (read + write) per decode launch at batch 256, taken on the
 # decode kernel whose source hashes to DECODE_SRC_SHA; null once it changes.
-DECODE_TRAFFIC = 1593586090          # mean of 3 launches at batch 256
-DECODE_SRC_SHA = "9c863bc17a82d5f8"
+DECODE_TRAFFIC = 1593363968          # mean of 3 launches at batch 256
+DECODE_SRC_SHA = "1ad3fb952dfab07f"
 
 
 def peaks():
@@ -329,6 +334,35 @@ def main():
         dist.all_reduce(tb, op=dist.ReduceOp.MAX)
     bf16_step_s = float(tb[0]) / 1e3 / (args.steps * BF16_BLOCK)
 
+    # ---- projections around the mixer at the prefill workload's 4096 tokens ----
+    pj = inputs.make_proj_case(PREFILL_T, seed=5 + rank)
+    hid, w_in, w_out = (act(x).to(dev) for x in (pj.hidden, pj.w_in, pj.w_out))
+    pj_out = gdn.in_proj(cfg, hid, w_in, stream=stream)
+    y_out = torch.empty((PREFILL_T, D_MODEL), dtype=torch.bfloat16, device=dev)
+
+    def timed(fn):
+        evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
+        for i in range(-args.warmup, args.steps):
+            flush.zero_()
+            if i >= 0:
+                evs[i][0].record(stream)
+            fn()
+            if i >= 0:
+                evs[i][1].record(stream)
+        torch.cuda.synchronize()
+        tt = torch.tensor([sum(a.elapsed_time(b) for a, b in evs)], dtype=torch.float64, device=dev)
+        if world > 1:
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        return float(tt[0]) / args.steps / 1e3          # seconds per call
+
+    in_s = timed(lambda: gdn.in_proj(cfg, hid, w_in, out=pj_out, stream=stream))
+    out_s = timed(lambda: gdn.out_proj(cfg, p_out, w_out, y=y_out, stream=stream))
+    gdn.check_device_error(stream)
+    # cuBLAS on the same shapes, for context only (not part of the product path)
+    in_cublas_s = timed(lambda: torch.nn.functional.linear(hid, w_in))
+    out_cublas_s = timed(lambda: torch.nn.functional.linear(p_out, w_out))
+
     # ---- end to end through the public API with host buffers ----
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
@@ -377,6 +411,14 @@ def main():
             "decode_bf16_state": {"value": DECODE_BF16_BYTES_PER_STEP / bf16_step_s / 1e9, "unit": "GB/s",
                                   "us_per_step": bf16_step_s * 1e6, "tokens_per_s": DECODE_N * world / bf16_step_s,
                                   "bytes_per_step": DECODE_BF16_BYTES_PER_STEP},
+            "projections": {
+                "tokens": PREFILL_T, "d_model": D_MODEL, "unit": "TFLOP/s", "peak": pk["bf16_tflops"],
+                "in": {"shape": [PREFILL_T, PROJ_IN_N, D_MODEL], "us": in_s * 1e6,
+                       "value": PROJ_IN_FLOP / in_s / 1e12, "frac": PROJ_IN_FLOP / in_s / 1e12 / pk["bf16_tflops"],
+                       "cublas_value": PROJ_IN_FLOP / in_cublas_s / 1e12},
+                "out": {"shape": [PREFILL_T, D_MODEL, H_V * D], "us": out_s * 1e6,
+                        "value": PROJ_OUT_FLOP / out_s / 1e12, "frac": PROJ_OUT_FLOP / out_s / 1e12 / pk["bf16_tflops"],
+                        "cublas_value": PROJ_OUT_FLOP / out_cublas_s / 1e12}},
             "prefill_ms": pre_ms / K,
             "roofline": {"kernel": "gdn_decode_kernel", "bound": "hbm", "achieved": dec_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / pk["hbm_gbs"],

@@ -4,6 +4,7 @@
 
 #include <cudaTypedefs.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstring>
 #include <mutex>
@@ -11,6 +12,7 @@
 #include "conv.cuh"
 #include "decode.cuh"
 #include "device.cuh"
+#include "gemm.cuh"
 #include "intra.cuh"
 #include "norm.cuh"
 #include "scan.cuh"
@@ -151,6 +153,90 @@ int sm_count() {
     if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
     if (dev < 64) count[dev] = n;
     return n;
+}
+
+// 2-D map over a row-major [rows][K] bf16 matrix for the projections: boxes of
+// 64 (K) x box_rows, 128-byte swizzle; elements past K or rows read as zero.
+bool kmajor_map(CUtensorMap* m, const void* base, int64_t rows, int K, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+    cuuint32_t box[2] = {(cuuint32_t)gdn::gemm::BK, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int BN>
+cudaError_t launch_linear(const void* x, const void* w, gdn::gemm::Args a, int variant, cudaStream_t st) {
+    using S = gdn::gemm::Shape<BN>;
+    CUtensorMap tm_x, tm_w;
+    if (!kmajor_map(&tm_x, x, a.M, a.K, gdn::gemm::BM) || !kmajor_map(&tm_w, w, a.N, a.K, BN))
+        return cudaErrorInvalidValue;
+    a.n_blocks = (a.N + BN - 1) / BN;
+    a.tiles = (int64_t)a.m_blocks * a.n_blocks;
+    cudaError_t e = ensure_smem(gdn::gemm::linear_kernel<BN>, variant, S::SMEM);
+    if (e != cudaSuccess) return e;
+    const int grid = (int)std::min<int64_t>(a.tiles, sm_count());
+    gdn::gemm::linear_kernel<BN><<<grid, gdn::gemm::NT, S::SMEM, st>>>(tm_x, tm_w, a);
+    return cudaGetLastError();
+}
+
+// Tile width: fewest (waves x (BN + a fixed per-tile cost)) over the MMA widths
+// that keep a stage ring of at least 4; ties go to the wider tile.
+int pick_bn(int64_t M, int N, int sms) {
+    static const int cand[] = {256, 224, 192, 160, 128};
+    const int64_t mb = (M + gdn::gemm::BM - 1) / gdn::gemm::BM;
+    int best = 256;
+    int64_t best_cost = -1;
+    for (int bn : cand) {
+        const int64_t tiles = mb * ((N + bn - 1) / bn);
+        const int64_t cost = (tiles + sms - 1) / sms * (bn + 32);
+        if (best_cost < 0 || cost < best_cost) {
+            best = bn;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+gdn_status run_linear(const void* x, const void* w, int64_t M, int32_t N, int32_t K, const gdn_out_segment* segs,
+                      int32_t n_segs, void* stream) {
+    if (M < 0 || N <= 0 || K <= 0 || !segs || n_segs <= 0) return GDN_ERR_INVALID_ARG;
+    if (n_segs > GDN_LINEAR_MAX_SEGMENTS) return GDN_ERR_UNSUPPORTED;
+    if (N % 8 != 0 || K % 8 != 0) return GDN_ERR_UNSUPPORTED;
+    if (M == 0) return GDN_OK;
+    if (!x || !w || !aligned(x, 16) || !aligned(w, 16)) return GDN_ERR_INVALID_ARG;
+    if ((M + gdn::gemm::BM - 1) / gdn::gemm::BM > 0x7fffffffLL) return GDN_ERR_UNSUPPORTED;
+    gdn::gemm::Args a;
+    a.M = M;
+    a.N = N;
+    a.K = K;
+    a.m_blocks = (int)((M + gdn::gemm::BM - 1) / gdn::gemm::BM);
+    a.n_segs = n_segs;
+    int n0 = 0;
+    for (int i = 0; i < n_segs; ++i) {
+        const gdn_out_segment& g = segs[i];
+        if (!g.dst || !aligned(g.dst, 16) || g.width <= 0 || g.width % 8 != 0) return GDN_ERR_INVALID_ARG;
+        a.seg[i].dst = static_cast<__nv_bfloat16*>(g.dst);
+        a.seg[i].n0 = n0;
+        a.seg[i].width = g.width;
+        n0 += g.width;
+        if (n0 > N) return GDN_ERR_INVALID_ARG;
+    }
+    if (n0 != N) return GDN_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaError_t e;
+    switch (pick_bn(M, N, sm_count())) {
+        case 256: e = launch_linear<256>(x, w, a, 20, st); break;
+        case 224: e = launch_linear<224>(x, w, a, 21, st); break;
+        case 192: e = launch_linear<192>(x, w, a, 22, st); break;
+        case 160: e = launch_linear<160>(x, w, a, 23, st); break;
+        default: e = launch_linear<128>(x, w, a, 24, st); break;
+    }
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 template <typename TA, typename TO>
@@ -435,6 +521,31 @@ gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_weights* w, const v
     else if (obf) e = launch_decode_multi<float, __nv_bfloat16>(m, sbf, st);
     else e = launch_decode_multi<float, float>(m, sbf, st);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_linear(const void* x, const void* w, int64_t M, int32_t N, int32_t K, const gdn_out_segment* segs,
+                      int32_t n_segs, void* stream) {
+    return run_linear(x, w, M, N, K, segs, n_segs, stream);
+}
+
+gdn_status gdn_in_proj(const gdn_config* cfg, const void* hidden, const void* w_in, int64_t T, int32_t d_model,
+                       void* q, void* k, void* v, void* z, void* a, void* b, void* stream) {
+    gdn_status s = check_config(cfg);
+    if (s != GDN_OK) return s;
+    if (T < 0 || d_model <= 0) return GDN_ERR_INVALID_ARG;
+    const int qk = cfg->n_k_heads * cfg->d_k, vz = cfg->n_v_heads * cfg->d_v, ab = cfg->n_v_heads;
+    if (ab % 8 != 0) return GDN_ERR_UNSUPPORTED;
+    const gdn_out_segment segs[6] = {{q, qk}, {k, qk}, {v, vz}, {z, vz}, {a, ab}, {b, ab}};
+    return run_linear(hidden, w_in, T, 2 * qk + 2 * vz + 2 * ab, d_model, segs, 6, stream);
+}
+
+gdn_status gdn_out_proj(const gdn_config* cfg, const void* o, const void* w_out, int64_t T, int32_t d_model, void* y,
+                        void* stream) {
+    gdn_status s = check_config(cfg);
+    if (s != GDN_OK) return s;
+    if (T < 0 || d_model <= 0) return GDN_ERR_INVALID_ARG;
+    const gdn_out_segment seg = {y, d_model};
+    return run_linear(o, w_out, T, d_model, cfg->n_v_heads * cfg->d_v, &seg, 1, stream);
 }
 
 gdn_status gdn_check_device_error(void* stream) {

@@ -42,6 +42,10 @@ class _CConfig(ctypes.Structure):
                 ("state_dtype", ctypes.c_int32)]
 
 
+class _CSegment(ctypes.Structure):
+    _fields_ = [("dst", ctypes.c_void_p), ("width", ctypes.c_int32)]
+
+
 class _CWeights(ctypes.Structure):
     _fields_ = [("conv_weight", ctypes.c_void_p), ("A_log", ctypes.c_void_p),
                 ("dt_bias", ctypes.c_void_p), ("norm_weight", ctypes.c_void_p)]
@@ -49,8 +53,10 @@ class _CWeights(ctypes.Structure):
 
 _lib = None
 EXPORTS = ("gdn_config_default", "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode",
-           "gdn_decode_multi", "gdn_check_device_error", "gdn_status_string")
+           "gdn_decode_multi", "gdn_linear", "gdn_in_proj", "gdn_out_proj", "gdn_check_device_error",
+           "gdn_status_string")
 DECODE_MULTI_MAX_TOKENS = 16   # GDN_DECODE_MULTI_MAX_TOKENS
+LINEAR_MAX_SEGMENTS = 8        # GDN_LINEAR_MAX_SEGMENTS
 
 
 def lib() -> ctypes.CDLL:
@@ -72,6 +78,12 @@ def lib() -> ctypes.CDLL:
         L.gdn_decode.restype = ctypes.c_int
         L.gdn_decode_multi.argtypes = [vp, vp] + [vp] * 8 + [i32, i32, vp, vp, vp, vp]
         L.gdn_decode_multi.restype = ctypes.c_int
+        L.gdn_linear.argtypes = [vp, vp, i64, i32, i32, vp, i32, vp]
+        L.gdn_linear.restype = ctypes.c_int
+        L.gdn_in_proj.argtypes = [vp, vp, vp, i64, i32] + [vp] * 6 + [vp]
+        L.gdn_in_proj.restype = ctypes.c_int
+        L.gdn_out_proj.argtypes = [vp, vp, vp, i64, i32, vp, vp]
+        L.gdn_out_proj.restype = ctypes.c_int
         L.gdn_check_device_error.argtypes = [vp]
         L.gdn_check_device_error.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -215,6 +227,80 @@ def decode_multi(cfg: Config, w: dict, q, k, v, a, b, z, conv_state, rec_state, 
     if s != 0:
         raise GdnError(s, "gdn_decode_multi")
     return out
+
+
+def linear(x, w, outs=None, stream=None):
+    """y = x . w^T on the tensor cores: x [M, K] and w [N, K] bf16, fp32 accumulation.
+    ``outs`` (optional) is a list of bf16 [M, width] tensors that receive consecutive
+    column ranges of y (widths adding up to N); default one [M, N] tensor.  Returns
+    the list of outputs."""
+    dev = x.device
+    if x.dim() != 2 or w.dim() != 2 or x.shape[1] != w.shape[1]:
+        raise ValueError("x [M, K] and w [N, K] expected, got %s and %s" % (tuple(x.shape), tuple(w.shape)))
+    M, K = x.shape
+    N = w.shape[0]
+    _check(x, "x", torch.bfloat16, dev)
+    _check(w, "w", torch.bfloat16, dev)
+    if outs is None:
+        outs = [torch.empty((M, N), dtype=torch.bfloat16, device=dev)]
+    if not 1 <= len(outs) <= LINEAR_MAX_SEGMENTS:
+        raise ValueError("1..%d output segments" % LINEAR_MAX_SEGMENTS)
+    for i, o in enumerate(outs):
+        _check(o, "outs[%d]" % i, torch.bfloat16, dev)
+        if o.dim() != 2 or o.shape[0] != M:
+            raise ValueError("outs[%d] must be [M, width]" % i)
+    segs = (_CSegment * len(outs))(*[_CSegment(o.data_ptr(), o.shape[1]) for o in outs])
+    s = lib().gdn_linear(_ptr(x), _ptr(w), M, N, K, segs, len(outs), _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_linear")
+    return outs
+
+
+def in_proj(cfg: Config, hidden, w_in, out: dict | None = None, stream=None) -> dict:
+    """The mixer's input projection: hidden [T, d_model] bf16, w_in [16,480, d_model]
+    bf16 at the published shape (channels q | k | v | z | a | b).  Returns q, k
+    [T, H_k*d_k], v, z [T, H_v*d_v], a, b [T, H_v], all bf16 (written into ``out``'s
+    tensors when given)."""
+    dev = hidden.device
+    T, D = hidden.shape
+    _check(hidden, "hidden", torch.bfloat16, dev)
+    _check(w_in, "w_in", torch.bfloat16, dev)
+    qk, vz, ab = cfg.n_k_heads * cfg.d_k, cfg.n_v_heads * cfg.d_v, cfg.n_v_heads
+    if tuple(w_in.shape) != (2 * qk + 2 * vz + 2 * ab, D):
+        raise ValueError("w_in shape %s, expected %s" % (tuple(w_in.shape), (2 * qk + 2 * vz + 2 * ab, D)))
+    widths = (("q", qk), ("k", qk), ("v", vz), ("z", vz), ("a", ab), ("b", ab))
+    o = out if out is not None else {n: torch.empty((T, wd), dtype=torch.bfloat16, device=dev) for n, wd in widths}
+    for n, wd in widths:
+        _check(o[n], n, torch.bfloat16, dev)
+        if o[n].numel() != T * wd:
+            raise ValueError("%s must hold [T, %d]" % (n, wd))
+    c = cfg.c()
+    s = lib().gdn_in_proj(ctypes.byref(c), _ptr(hidden), _ptr(w_in), T, D, _ptr(o["q"]), _ptr(o["k"]),
+                          _ptr(o["v"]), _ptr(o["z"]), _ptr(o["a"]), _ptr(o["b"]), _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_in_proj")
+    return o
+
+
+def out_proj(cfg: Config, o, w_out, y=None, stream=None):
+    """The mixer's output projection: o [T, H_v*d_v] bf16 (the layer's output),
+    w_out [d_model, H_v*d_v] bf16 -> y [T, d_model] bf16."""
+    dev = o.device
+    o2 = o.reshape(o.shape[0], -1)
+    T = o2.shape[0]
+    D = w_out.shape[0]
+    _check(o2, "o", torch.bfloat16, dev)
+    _check(w_out, "w_out", torch.bfloat16, dev)
+    if w_out.shape[1] != cfg.n_v_heads * cfg.d_v or o2.shape[1] != w_out.shape[1]:
+        raise ValueError("w_out must be [d_model, H_v*d_v] and o [T, H_v*d_v]")
+    if y is None:
+        y = torch.empty((T, D), dtype=torch.bfloat16, device=dev)
+    _check(y, "y", torch.bfloat16, dev)
+    c = cfg.c()
+    s = lib().gdn_out_proj(ctypes.byref(c), _ptr(o2), _ptr(w_out), T, D, _ptr(y), _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_out_proj")
+    return y
 
 
 def check_device_error(stream=None) -> None:

@@ -22,6 +22,12 @@ Workloads (head shape of the layer: 16 key heads, 48 value heads, d_k = d_v =
 * ``decode_256``  256 sequences x 1 token, fp32 state ~ N(0, 0.02) (std),
                   bf16 conv state; 64 consecutive steps.
 * ``prefill_256k`` 1 sequence, T = 262144, -log alpha ~ U(1e-4, 0.1).
+
+Projections around the mixer (``make_proj_case``): hidden states [T, 2560]
+bf16 ~ N(0, 1) (hidden size 2,560: "Qwen3.8-Flash-Next" (llm-atlas-9r2), "Key
+facts"); random-init bf16 weights w_in [16480, 2560] ~ N(0, 1/2560) and w_out
+[2560, 6144] ~ N(0, 1/6144), so that every projected channel is ~ N(0, 1) like
+the mixer's own synthetic inputs.
 """
 from __future__ import annotations
 
@@ -221,3 +227,23 @@ def make_case(name: str, seed: int | None = None, T: int | None = None,
 
 
 CASES = ("tiny", "prefill_4k", "varlen_8", "decode_256", "prefill_256k")
+
+
+@dataclass
+class ProjCase:
+    """Inputs of the mixer's two projections (bf16 bit patterns)."""
+    hidden: np.ndarray      # [T, d_model]
+    w_in: np.ndarray        # [2*Hk*dk + 2*Hv*dv + 2*Hv, d_model]
+    w_out: np.ndarray       # [d_model, Hv*dv]
+    o: np.ndarray           # [T, Hv*dv], a stand-in layer output for the out projection alone
+
+
+def make_proj_case(T: int, d_model: int = 2560, Hk: int = 16, Hv: int = 48, dk: int = 128, dv: int = 128,
+                   seed: int = 0) -> ProjCase:
+    n_in = 2 * Hk * dk + 2 * Hv * dv + 2 * Hv
+    return ProjCase(
+        hidden=_normal_rows(seed, "proj.hidden", T, d_model),
+        w_in=_normal_rows(seed, "proj.w_in", n_in, d_model, std=float(d_model) ** -0.5),
+        w_out=_normal_rows(seed, "proj.w_out", d_model, Hv * dv, std=float(Hv * dv) ** -0.5),
+        o=_normal_rows(seed, "proj.o", T, Hv * dv),
+    )

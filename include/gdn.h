@@ -165,6 +165,57 @@ gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_weights* w,
                             void* conv_state, void* rec_state, int32_t n_seqs, int32_t n_tok,
                             void* out, void* state_snapshots, void* conv_snapshots, void* stream);
 
+/* Largest number of output segments one gdn_linear call writes. */
+#define GDN_LINEAR_MAX_SEGMENTS 8
+
+/* One output segment of a projection: the next `width` columns of y go to
+ * dst, a row-major [M][width] bf16 matrix (device pointer, 16-byte aligned,
+ * width a multiple of 8). */
+typedef struct {
+    void* dst;
+    int32_t width;
+} gdn_out_segment;
+
+/*
+ * Dense projection on the tensor cores: y[M][N] = x[M][K] . w[N][K]^T, bf16
+ * operands, fp32 accumulation, each output rounded once to bf16 (nearest even).
+ * No bias.  w is laid out as a linear layer's weight (one row per output
+ * column).  The columns of y are split, in order, over segs[0..n_segs): the
+ * widths must add up to N.  This serves the projections around the mixer,
+ * whose widths come from the hidden size 2,560 ("Qwen3.8-Flash-Next"
+ * (llm-atlas-9r2), "Key facts"; (llm-architectures-explained), "Every
+ * architecture field", row d_model) and the head shapes above.
+ *   x  [M][K] bf16, 16-byte aligned; w [N][K] bf16, 16-byte aligned
+ *   N, K multiples of 8 (else GDN_ERR_UNSUPPORTED); M == 0 is a no-op;
+ *   1 <= n_segs <= GDN_LINEAR_MAX_SEGMENTS (more: GDN_ERR_UNSUPPORTED)
+ * No workspace.  Asynchronous on `stream`.
+ */
+gdn_status gdn_linear(const void* x, const void* w, int64_t M, int32_t N, int32_t K,
+                      const gdn_out_segment* segs, int32_t n_segs, void* stream);
+
+/*
+ * The mixer's input projection.  The pages do not print the projection layout;
+ * the reading taken is one bias-free linear map from the hidden state to all of
+ * the mixer's inputs, its output channels in the order
+ *   q (H_k*d_k) | k (H_k*d_k) | v (H_v*d_v) | z (H_v*d_v) | a (H_v) | b (H_v)
+ * (16,480 channels at the published shape).
+ *   hidden [T][d_model] bf16; w_in [2*H_k*d_k + 2*H_v*d_v + 2*H_v][d_model] bf16
+ *   q, k [T][H_k][d_k]; v, z [T][H_v][d_v]; a, b [T][H_v]: bf16 outputs, 16-byte
+ *   aligned, ready for gdn_prefill / gdn_decode with act_dtype GDN_BF16.
+ * H_v must be a multiple of 8 and d_model of 8 (else GDN_ERR_UNSUPPORTED).
+ */
+gdn_status gdn_in_proj(const gdn_config* cfg, const void* hidden, const void* w_in, int64_t T,
+                       int32_t d_model, void* q, void* k, void* v, void* z, void* a, void* b,
+                       void* stream);
+
+/*
+ * The mixer's output projection: y[T][d_model] = o[T][H_v*d_v] . w_out^T, with
+ * o the bf16 output of gdn_prefill / gdn_decode and w_out [d_model][H_v*d_v]
+ * bf16.  d_model must be a multiple of 8.
+ */
+gdn_status gdn_out_proj(const gdn_config* cfg, const void* o, const void* w_out, int64_t T,
+                        int32_t d_model, void* y, void* stream);
+
 /* Capacity, in bytes, of the fixed scratch array used by gdn_prefill_noalloc. */
 #define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 

@@ -159,6 +159,45 @@ def forward(shape: Shape, w: dict, q, k, v, a, b, z, conv_state, rec_state, cu_s
 
 
 # ---------------------------------------------------------------------------
+# Projections around the mixer
+# ---------------------------------------------------------------------------
+# The hidden size is 2,560 ("Qwen3.8-Flash-Next" (llm-atlas-9r2), "Key facts";
+# (llm-architectures-explained), "Every architecture field", row d_model).  The
+# pages do not print how the mixer's inputs are projected from it; the reading
+# taken is one bias-free linear map per side, the input map's output channels
+# in the order q | k | v | z | a | b, the output map from the 6,144 channels of
+# the layer's output back to the hidden size.
+
+def linear(x, w) -> np.ndarray:
+    """y = x . w^T in fp64, x [M, K], w [N, K] (bf16 bit patterns or floats).
+    The plain definition; numpy's matmul is the one step."""
+    return act_to_f64(x) @ act_to_f64(w).T
+
+
+def in_proj_widths(shape: Shape):
+    """(name, width) of the input projection's output channels, in order."""
+    qk, vz = shape.n_k_heads * shape.d_k, shape.n_v_heads * shape.d_v
+    return (("q", qk), ("k", qk), ("v", vz), ("z", vz), ("a", shape.n_v_heads), ("b", shape.n_v_heads))
+
+
+def in_proj(shape: Shape, hidden, w_in) -> dict:
+    """hidden [T, d_model] -> {q, k, v, z, a, b} fp64, split in the order above."""
+    y = linear(hidden, w_in)
+    out, c = {}, 0
+    for name, wd in in_proj_widths(shape):
+        out[name] = y[:, c:c + wd]
+        c += wd
+    assert c == y.shape[1], "w_in has %d rows, the split needs %d" % (y.shape[1], c)
+    return out
+
+
+def out_proj(o, w_out) -> np.ndarray:
+    """o [T, H_v*d_v] -> y [T, d_model] fp64."""
+    o = np.asarray(o)
+    return linear(o.reshape(o.shape[0], -1), w_out)
+
+
+# ---------------------------------------------------------------------------
 # Pure-numpy formulations (small inputs only)
 # ---------------------------------------------------------------------------
 

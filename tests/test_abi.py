@@ -106,6 +106,34 @@ def test_decode_multi_argument_errors(lib):
     assert call(4, 2, ptr=0) == INVALID                   # missing inputs
 
 
+def test_linear_argument_errors(lib):
+    P = ctypes.c_void_p
+
+    def segs(*widths, ptr=0x10000):
+        return (gdn._CSegment * len(widths))(*[gdn._CSegment(ptr, w) for w in widths])
+
+    call = lambda M, N, K, sg, n=None, x=0x1000, w=0x2000: lib.gdn_linear(
+        P(x), P(w), M, N, K, sg, len(sg) if n is None else n, None)
+    assert call(-1, 64, 64, segs(64)) == INVALID
+    assert call(4, 0, 64, segs(64)) == INVALID
+    assert call(4, 64, 64, segs(8, 8, 8, 8, 8, 8, 8, 8, 8), n=9) == UNSUPPORTED
+    assert call(4, 12, 64, segs(12)) == UNSUPPORTED       # N not a multiple of 8
+    assert call(4, 64, 20, segs(64)) == UNSUPPORTED       # K not a multiple of 8
+    assert call(0, 64, 64, segs(64)) == OK                # nothing to do
+    assert call(4, 64, 64, segs(32, 16)) == INVALID       # widths do not add up to N
+    assert call(4, 64, 64, segs(60, 4)) == INVALID        # width not a multiple of 8
+    assert call(4, 64, 64, segs(64, ptr=0x10008)) == INVALID   # misaligned output
+    assert call(4, 64, 64, segs(64), x=0x1004) == INVALID       # misaligned x
+    assert call(4, 64, 64, segs(64), w=0) == INVALID
+    c = gdn.Config(n_k_heads=2, n_v_heads=6, d_k=32, d_v=32).c()
+    assert lib.gdn_in_proj(ctypes.byref(c), P(0x1000), P(0x2000), 4, 64, *[P(0x3000)] * 6, None) == UNSUPPORTED
+    c = gdn.Config().c()
+    assert lib.gdn_in_proj(ctypes.byref(c), P(0x1000), P(0x2000), 0, 2560, *[P(0x3000)] * 6, None) == OK
+    assert lib.gdn_in_proj(ctypes.byref(c), P(0x1000), P(0x2000), 4, 2564, *[P(0x3000)] * 6, None) == UNSUPPORTED
+    assert lib.gdn_out_proj(ctypes.byref(c), P(0x1000), P(0x2000), 0, 2560, P(0x3000), None) == OK
+    assert lib.gdn_out_proj(ctypes.byref(c), P(0x1000), P(0x2000), -1, 2560, P(0x3000), None) == INVALID
+
+
 def test_status_strings(lib):
     for s in range(6):
         assert gdn.status_string(s)

@@ -308,3 +308,64 @@ def test_bf16_inputs_are_read_exactly():
     np.testing.assert_array_equal(r1["rec_state"], r2["rec_state"])
     assert inputs.bf16_bits_to_f32(inputs.f32_to_bf16_bits(np.array([1.0, -2.5, 1 + 2 ** -9],
                                                                      np.float32))).tolist() == [1.0, -2.5, 1.0]
+
+
+# ---------------------------------------------------------------------------
+# Projections around the mixer
+# ---------------------------------------------------------------------------
+
+def test_linear_brute_force_sums():
+    """y[i, j] = sum_k x[i, k] w[j, k], summed term by term with exact rounding."""
+    rng = np.random.default_rng(20)
+    x, w = rng.normal(size=(5, 7)), rng.normal(size=(3, 7))
+    y = oracle.linear(x, w)
+    assert y.shape == (5, 3)
+    for i in range(5):
+        for j in range(3):
+            assert abs(y[i, j] - math.fsum(x[i, k] * w[j, k] for k in range(7))) <= 1e-14
+
+
+def test_linear_cyclic_permutation_picks_columns():
+    """w = a cyclic shift P (not its own inverse): row j of w is e_{(j+1) mod K},
+    so y[:, j] = x[:, j+1].  A transposed w would give x[:, j-1]."""
+    rng = np.random.default_rng(21)
+    K = 6
+    x = rng.normal(size=(4, K))
+    w = np.zeros((K, K))
+    for j in range(K):
+        w[j, (j + 1) % K] = 1.0
+    np.testing.assert_array_equal(oracle.linear(x, w), x[:, (np.arange(K) + 1) % K])
+
+
+def test_in_proj_channel_order_and_out_proj():
+    """With an identity w_in the projection's outputs are the hidden columns,
+    split q | k | v | z | a | b in that order and width; out_proj with a basis
+    w_out selects the chosen channels of o."""
+    shape = oracle.Shape(2, 8, 8, 8)
+    widths = dict(oracle.in_proj_widths(shape))
+    assert list(widths) == ["q", "k", "v", "z", "a", "b"]
+    assert list(widths.values()) == [16, 16, 64, 64, 8, 8]
+    N = sum(widths.values())
+    rng = np.random.default_rng(22)
+    h = rng.normal(size=(3, N))
+    parts = oracle.in_proj(shape, h, np.eye(N))
+    c = 0
+    for name, wd in widths.items():
+        np.testing.assert_array_equal(parts[name], h[:, c:c + wd])
+        c += wd
+    with pytest.raises(AssertionError):
+        oracle.in_proj(shape, h[:, :N - 8], np.eye(N - 8))
+    o = rng.normal(size=(3, 8, 8))
+    pick = [5, 60, 0]
+    w_out = np.zeros((3, 64))
+    w_out[np.arange(3), pick] = 1.0
+    np.testing.assert_array_equal(oracle.out_proj(o, w_out), o.reshape(3, 64)[:, pick])
+
+
+def test_linear_reads_bf16_exactly():
+    rng = np.random.default_rng(23)
+    x, w = rng.normal(size=(4, 16)).astype(np.float32), rng.normal(size=(5, 16)).astype(np.float32)
+    xb, wb = inputs.f32_to_bf16_bits(x), inputs.f32_to_bf16_bits(w)
+    np.testing.assert_array_equal(oracle.linear(xb, wb),
+                                  inputs.bf16_bits_to_f32(xb).astype(np.float64)
+                                  @ inputs.bf16_bits_to_f32(wb).astype(np.float64).T)
