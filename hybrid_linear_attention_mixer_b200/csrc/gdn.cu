@@ -184,16 +184,71 @@ cudaError_t launch_linear(const void* x, const void* w, gdn::gemm::Args a, int v
     return cudaGetLastError();
 }
 
-// Tile width: fewest (waves x (BN + a fixed per-tile cost)) over the MMA widths
-// that keep a stage ring of at least 4; ties go to the wider tile.
+// Tile width of the one-CTA form: fewest (waves x (BN + a fixed per-tile cost));
+// ties go to the wider tile.
 int pick_bn(int64_t M, int N, int sms) {
-    static const int cand[] = {256, 224, 192, 160, 128};
+    static const int cand[] = {256, 128};
     const int64_t mb = (M + gdn::gemm::BM - 1) / gdn::gemm::BM;
     int best = 256;
     int64_t best_cost = -1;
     for (int bn : cand) {
         const int64_t tiles = mb * ((N + bn - 1) / bn);
         const int64_t cost = (tiles + sms - 1) / sms * (bn + 32);
+        if (best_cost < 0 || cost < best_cost) {
+            best = bn;
+            best_cost = cost;
+        }
+    }
+    return best;
+}
+
+// Pair form (2-CTA clusters, M = 256 pair tiles).  The number of clusters that
+// fit at once is asked of the runtime once per device and width.
+template <int BN>
+cudaError_t launch_linear_pair(const void* x, const void* w, gdn::gemm::Args a, int variant, cudaStream_t st) {
+    using S = gdn::gemm::Shape2<BN>;
+    CUtensorMap tm_x, tm_w;
+    if (!kmajor_map(&tm_x, x, a.M, a.K, gdn::gemm::BM) || !kmajor_map(&tm_w, w, a.N, a.K, BN / 2))
+        return cudaErrorInvalidValue;
+    a.n_blocks = (a.N + BN - 1) / BN;
+    const int64_t m_pairs = (a.M + 2 * gdn::gemm::BM - 1) / (2 * gdn::gemm::BM);
+    a.tiles = m_pairs * a.n_blocks;
+    cudaError_t e = ensure_smem(gdn::gemm::linear_pair_kernel<BN>, variant, S::SMEM);
+    if (e != cudaSuccess) return e;
+    static int clusters[64];
+    int dev = 0;
+    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    int n_cl = dev < 64 ? clusters[dev] : 0;
+    if (n_cl <= 0) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(2 * (unsigned)std::max(1, sm_count() / 2), 1, 1);
+        cfg.blockDim = dim3(gdn::gemm::NT, 1, 1);
+        cfg.dynamicSmemBytes = S::SMEM;
+        if (cudaOccupancyMaxActiveClusters(&n_cl, gdn::gemm::linear_pair_kernel<BN>, &cfg) != cudaSuccess ||
+            n_cl <= 0) {
+            (void)cudaGetLastError();
+            n_cl = std::max(1, sm_count() / 2);
+        }
+        if (dev < 64) clusters[dev] = n_cl;
+    }
+    const int pairs = (int)std::min<int64_t>(a.tiles, n_cl);
+    gdn::gemm::linear_pair_kernel<BN><<<2 * pairs, gdn::gemm::NT, S::SMEM, st>>>(tm_x, tm_w, a);
+    return cudaGetLastError();
+}
+
+// Pair tile width: fewest waves x (time of one k-block), over the MMA widths,
+// with ~74 pairs in flight on 148 SMs.  Measured on B200 the pair kernel is
+// bound by the operand bytes each SM loads from L2 per k-block (16 KiB of A plus
+// BN/2 rows of 128 B of B, ~90 GB/s per SM), and at the widest tiles by the MMA
+// rate (~2.1 x BN in the same units): time ~ max(256 + BN, 17 BN / 8).
+int pick_bn_pair(int64_t M, int N, int pairs) {
+    static const int cand[] = {256, 224, 208, 192, 160, 144, 128};
+    const int64_t mp = (M + 2 * gdn::gemm::BM - 1) / (2 * gdn::gemm::BM);
+    int best = 256;
+    int64_t best_cost = -1;
+    for (int bn : cand) {
+        const int64_t tiles = mp * ((N + bn - 1) / bn);
+        const int64_t cost = (tiles + pairs - 1) / pairs * std::max<int64_t>(256 + bn, 17 * bn / 8);
         if (best_cost < 0 || cost < best_cost) {
             best = bn;
             best_cost = cost;
@@ -229,13 +284,22 @@ gdn_status run_linear(const void* x, const void* w, int64_t M, int32_t N, int32_
     if (n0 != N) return GDN_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaError_t e;
-    switch (pick_bn(M, N, sm_count())) {
-        case 256: e = launch_linear<256>(x, w, a, 20, st); break;
-        case 224: e = launch_linear<224>(x, w, a, 21, st); break;
-        case 192: e = launch_linear<192>(x, w, a, 22, st); break;
-        case 160: e = launch_linear<160>(x, w, a, 23, st); break;
-        default: e = launch_linear<128>(x, w, a, 24, st); break;
+    if (M > gdn::gemm::BM) {
+        // pairs of CTAs once there are two 128-row halves to give them
+        switch (pick_bn_pair(M, N, std::max(1, sm_count() / 2))) {
+            case 256: e = launch_linear_pair<256>(x, w, a, 25, st); break;
+            case 224: e = launch_linear_pair<224>(x, w, a, 26, st); break;
+            case 208: e = launch_linear_pair<208>(x, w, a, 27, st); break;
+            case 192: e = launch_linear_pair<192>(x, w, a, 28, st); break;
+            case 160: e = launch_linear_pair<160>(x, w, a, 29, st); break;
+            case 144: e = launch_linear_pair<144>(x, w, a, 30, st); break;
+            default: e = launch_linear_pair<128>(x, w, a, 31, st); break;
+        }
+        return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
     }
+    // one CTA per 128-row tile for short inputs (decode-sized batches)
+    if (pick_bn(M, N, sm_count()) == 256) e = launch_linear<256>(x, w, a, 20, st);
+    else e = launch_linear<128>(x, w, a, 24, st);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 

@@ -2,6 +2,7 @@
 
     python -m hybrid_linear_attention_mixer_b200.run_case --case prefill_4k --iters 2
     python -m hybrid_linear_attention_mixer_b200.run_case --case decode_256 --batch 64 --iters 3
+    python -m hybrid_linear_attention_mixer_b200.run_case --proj --tokens 4096 --iters 1
 
 A small, fixed-size target for profilers such as ncu: it builds the seeded
 inputs of the named workload, runs the layer `iters` times on cuda:0 and checks
@@ -30,8 +31,22 @@ def main():
     ap.add_argument("--iters", type=int, default=2)
     ap.add_argument("--tokens", type=int, default=None, help="shrink a prefill workload to T tokens")
     ap.add_argument("--batch", type=int, default=None, help="decode batch (sequences)")
+    ap.add_argument("--proj", action="store_true",
+                    help="run the input and output projections (hidden 2560) at --tokens instead")
     args = ap.parse_args()
     dev = torch.device("cuda:0")
+    if args.proj:
+        T = args.tokens or 4096
+        pc = inputs.make_proj_case(T)
+        cfg = gdn.Config()
+        hid, w_in, w_out, o = (_act(x, dev) for x in (pc.hidden, pc.w_in, pc.w_out, pc.o))
+        for _ in range(args.iters):
+            gdn.in_proj(cfg, hid, w_in)
+            gdn.out_proj(cfg, o, w_out)
+        gdn.check_device_error()
+        torch.cuda.synchronize()
+        print("ok proj T=%d" % T)
+        return
     if args.case == "decode_256":
         c = inputs.make_case(args.case, n_seqs=args.batch, T=1)
     else:

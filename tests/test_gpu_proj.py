@@ -46,9 +46,12 @@ def _bound_ok(y_gpu: np.ndarray, x_bits, w_bits, y_ref: np.ndarray):
     return worst <= 1.0
 
 
-# (M, N): each shape makes the tile-width choice land on a different width
-# (128, 160, 192, 224, 256 on 148 SMs); every one has ragged M, N and K tails.
-SHAPES = [(1000, 256), (1000, 2312), (1000, 2888), (1000, 3464), (1000, 4040), (1, 8), (130, 264)]
+# (M, N): with M > 128 the CTA-pair form runs; each of the first seven shapes makes
+# its tile-width choice land on a different width (128, 144, 160, 192, 208, 224,
+# 256 with 74 pairs on 148 SMs).  M <= 128 runs the one-CTA form (widths 128 and
+# 256).  Every shape has ragged M, N and K tails.
+SHAPES = [(1000, 200), (1000, 2312), (1000, 2600), (1000, 2888), (1000, 3464), (1000, 3752), (1000, 4040),
+          (130, 264), (1, 8), (100, 264), (64, 20000)]
 
 
 @pytest.mark.parametrize("M,N", SHAPES)
