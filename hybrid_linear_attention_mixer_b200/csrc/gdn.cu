@@ -10,6 +10,7 @@
 #include <mutex>
 
 #include "conv.cuh"
+#include "cp.cuh"
 #include "decode.cuh"
 #include "device.cuh"
 #include "gemm.cuh"
@@ -68,6 +69,23 @@ Layout workspace_layout(const gdn_config* c, int64_t T, int64_t n_seqs) {
     L.rec_off = L.coff_off + cb;
     L.o_off = L.rec_off + max_chunks * c->n_v_heads * gdn::intra::REC_BYTES;
     L.total = L.o_off + max_chunks * c->n_v_heads * o_tile;
+    return L;
+}
+
+// Context-parallel workspace: the one-sequence prefill workspace of the segment,
+// then its cu_seqlens {0, T_seg}, then a zeroed 64-row v^ block whose tensor map
+// reads zeros for every later row (V = 0 for the transition's scan).
+struct CpLayout {
+    Layout pre;
+    size_t cu_off, zv_off, total;
+};
+
+CpLayout cp_layout(const gdn_config* c, int64_t T_seg) {
+    CpLayout L;
+    L.pre = workspace_layout(c, T_seg, 1);
+    L.cu_off = align_up(L.pre.total, 256);
+    L.zv_off = L.cu_off + 256;
+    L.total = L.zv_off + align_up((size_t)gdn::intra::C * c->n_v_heads * c->d_v * sizeof(__half), 256);
     return L;
 }
 
@@ -303,11 +321,17 @@ gdn_status run_linear(const void* x, const void* w, int64_t M, int32_t N, int32_
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
-template <typename TA, typename TO>
-cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void* q, const void* k,
-                           const void* v, const void* a, const void* b, const void* z, void* conv_state,
-                           void* rec_state, const int32_t* cu, int n_seqs, int64_t T, void* out,
-                           void* ws, int variant, cudaStream_t st) {
+// Prefill, split in its two stages so that context-parallel prefill can run the
+// chunk scan more than once over one set of intra-chunk records.
+//   stage A: conv + SiLU + L2 norm into the workspace, conv-state update, chunk
+//            offsets, intra-chunk records
+//   stage B: the chunk scan from rec_state (in/out), then the gated norm into out
+// Set-up first: nothing is launched unless the tensor maps encode and the
+// kernels' shared-memory opt-ins succeed.
+template <typename TA>
+cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void* q, const void* k, const void* v,
+                           const void* a, const void* b, void* conv_state, const int32_t* cu, int n_seqs,
+                           int64_t T, void* ws, cudaStream_t st) {
     const Layout L = workspace_layout(c, T, n_seqs);
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     ConvArgs ca;
@@ -322,24 +346,13 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     ca.qh = reinterpret_cast<__half*>(wsb + L.q_off);
     ca.kh = reinterpret_cast<__half*>(wsb + L.k_off);
     ca.vh = reinterpret_cast<__half*>(wsb + L.v_off);
-    // Set-up first: nothing is launched unless the tensor maps encode and the
-    // kernels' shared-memory opt-ins succeed.
     auto k_intra = gdn::intra::gdn_intra_kernel<TA>;
-    auto k_scan = c->state_dtype == GDN_BF16 ? gdn::scan::gdn_scan_kernel<TO, __nv_bfloat16>
-                                             : gdn::scan::gdn_scan_kernel<TO, float>;
     cudaError_t e = ensure_smem(k_intra, 4 + (sizeof(TA) == 2 ? 0 : 1), gdn::intra::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    e = ensure_smem(k_scan, 16 + (sizeof(TO) == 2 ? 0 : 1) + (c->state_dtype == GDN_BF16 ? 2 : 0), gdn::scan::SMEM_BYTES);
-    if (e != cudaSuccess) return e;
-    e = ensure_smem(gdn::norm::gdn_gated_norm_kernel<TA, TO>, 8 + (sizeof(TA) == 4 ? 2 : 0) + (sizeof(TO) == 4 ? 1 : 0),
-                    gdn::norm::smem_bytes<TA, TO>());
-    if (e != cudaSuccess) return e;
-    CUtensorMap tm_q, tm_k, tm_v, tm_z;
+    CUtensorMap tm_q, tm_k;
     const int Hk = c->n_k_heads, Hv = c->n_v_heads;
-    if (!z_rows_map(&tm_z, z, sizeof(TA) == 2, Hv * c->d_v, c->d_v, T)) return cudaErrorInvalidValue;
     if (!head_tile_map(&tm_q, ca.qh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, Hk, T) ||
-        !head_tile_map(&tm_k, ca.kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, Hk, T) ||
-        !head_tile_map(&tm_v, ca.vh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_v, Hv, T))
+        !head_tile_map(&tm_k, ca.kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, Hk, T))
         return cudaErrorInvalidValue;
     const int Ctot = 2 * c->n_k_heads * c->d_k + c->n_v_heads * c->d_v;
     const int cblocks = (Ctot / 8 + gdn::kConvThreads - 1) / gdn::kConvThreads;
@@ -348,7 +361,6 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     if (tblocks > 0x7fffffff || max_chunks * Hv > 0x7fffffff) return cudaErrorInvalidValue;
     int32_t* chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off);
     uint8_t* recs = wsb + L.rec_off;
-    void* otiles = wsb + L.o_off;
 
     // the tiled conv for bf16 activations whose q, k and v widths are multiples of its slice
     const int Cq = c->n_k_heads * c->d_k, Cv = c->n_v_heads * c->d_v;
@@ -381,23 +393,70 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
     ia.Hk = Hk; ia.Hv = Hv;
     ia.rec = recs;
     k_intra<<<(unsigned)(max_chunks * Hv), gdn::intra::NT, gdn::intra::SMEM_BYTES, st>>>(tm_q, tm_k, ia);
+    return cudaGetLastError();
+}
 
+// The chunk scan over the records of stage A, reading V through `v_src` (the
+// workspace's v^, or a zero block whose map reads zeros past its 64 rows).
+template <typename TO>
+cudaError_t launch_scan(const gdn_config* c, const void* v_src, int64_t v_rows, void* rec_state, const int32_t* cu,
+                        int n_seqs, int64_t T, void* ws, cudaStream_t st) {
+    const Layout L = workspace_layout(c, T, n_seqs);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    auto k_scan = c->state_dtype == GDN_BF16 ? gdn::scan::gdn_scan_kernel<TO, __nv_bfloat16>
+                                             : gdn::scan::gdn_scan_kernel<TO, float>;
+    cudaError_t e = ensure_smem(k_scan, 16 + (sizeof(TO) == 2 ? 0 : 1) + (c->state_dtype == GDN_BF16 ? 2 : 0),
+                                gdn::scan::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    CUtensorMap tm_v;
+    if (!head_tile_map(&tm_v, v_src, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_v, c->n_v_heads, v_rows))
+        return cudaErrorInvalidValue;
     gdn::scan::Args sa;
     sa.rec_state = rec_state;
-    sa.cu = cu; sa.chunk_off = chunk_off; sa.rec = recs;
-    sa.o = otiles;
-    sa.Hk = Hk; sa.Hv = Hv; sa.dk = c->d_k; sa.dv = c->d_v;
-    k_scan<<<(unsigned)n_seqs * Hv, gdn::scan::NT, gdn::scan::SMEM_BYTES, st>>>(tm_v, sa);
+    sa.cu = cu;
+    sa.chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off);
+    sa.rec = wsb + L.rec_off;
+    sa.o = wsb + L.o_off;
+    sa.Hk = c->n_k_heads; sa.Hv = c->n_v_heads; sa.dk = c->d_k; sa.dv = c->d_v;
+    k_scan<<<(unsigned)n_seqs * c->n_v_heads, gdn::scan::NT, gdn::scan::SMEM_BYTES, st>>>(tm_v, sa);
+    return cudaGetLastError();
+}
 
+template <typename TA, typename TO>
+cudaError_t launch_norm(const gdn_config* c, const gdn_weights* w, const void* z, const int32_t* cu, int n_seqs,
+                        int64_t T, void* out, void* ws, cudaStream_t st) {
+    const Layout L = workspace_layout(c, T, n_seqs);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    cudaError_t e = ensure_smem(gdn::norm::gdn_gated_norm_kernel<TA, TO>,
+                                8 + (sizeof(TA) == 4 ? 2 : 0) + (sizeof(TO) == 4 ? 1 : 0),
+                                gdn::norm::smem_bytes<TA, TO>());
+    if (e != cudaSuccess) return e;
+    CUtensorMap tm_z;
+    const int Hv = c->n_v_heads;
+    if (!z_rows_map(&tm_z, z, sizeof(TA) == 2, Hv * c->d_v, c->d_v, T)) return cudaErrorInvalidValue;
+    const int64_t max_chunks = (T + gdn::intra::C - 1) / gdn::intra::C + n_seqs;
     gdn::norm::Args na;
-    na.o = otiles; na.norm_w = w->norm_weight;
-    na.cu = cu; na.chunk_off = chunk_off; na.out = out;
+    na.o = wsb + L.o_off; na.norm_w = w->norm_weight;
+    na.cu = cu; na.chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off); na.out = out;
     na.n_seqs = n_seqs; na.Hv = Hv; na.dv = c->d_v; na.eps = c->norm_eps;
     int64_t norm_ctas = (int64_t)sm_count() * (232448 / (int64_t)gdn::norm::smem_bytes<TA, TO>());
     norm_ctas = norm_ctas < max_chunks * Hv ? norm_ctas : max_chunks * Hv;
     gdn::norm::gdn_gated_norm_kernel<TA, TO>
         <<<(unsigned)norm_ctas, gdn::norm::NT, gdn::norm::smem_bytes<TA, TO>(), st>>>(tm_z, na);
     return cudaGetLastError();
+}
+
+template <typename TA, typename TO>
+cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void* q, const void* k,
+                           const void* v, const void* a, const void* b, const void* z, void* conv_state,
+                           void* rec_state, const int32_t* cu, int n_seqs, int64_t T, void* out,
+                           void* ws, cudaStream_t st) {
+    const Layout L = workspace_layout(c, T, n_seqs);
+    cudaError_t e = launch_stage_a<TA>(c, w, q, k, v, a, b, conv_state, cu, n_seqs, T, ws, st);
+    if (e != cudaSuccess) return e;
+    e = launch_scan<TO>(c, static_cast<uint8_t*>(ws) + L.v_off, T, rec_state, cu, n_seqs, T, ws, st);
+    if (e != cudaSuccess) return e;
+    return launch_norm<TA, TO>(c, w, z, cu, n_seqs, T, out, ws, st);
 }
 
 template <typename TA, typename TO, typename TS, int DK>
@@ -501,16 +560,16 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_weights* w, const void* 
     const bool abf = cfg->act_dtype == GDN_BF16, obf = cfg->out_dtype == GDN_BF16;
     if (abf && obf)
         e = launch_prefill<__nv_bfloat16, __nv_bfloat16>(cfg, w, q, k, v, a, b, z, conv_state, rec_state,
-                                                          cu_seqlens, n_seqs, T_total, out, workspace, 0, st);
+                                                          cu_seqlens, n_seqs, T_total, out, workspace, st);
     else if (abf)
         e = launch_prefill<__nv_bfloat16, float>(cfg, w, q, k, v, a, b, z, conv_state, rec_state, cu_seqlens,
-                                                 n_seqs, T_total, out, workspace, 1, st);
+                                                 n_seqs, T_total, out, workspace, st);
     else if (obf)
         e = launch_prefill<float, __nv_bfloat16>(cfg, w, q, k, v, a, b, z, conv_state, rec_state, cu_seqlens,
-                                                 n_seqs, T_total, out, workspace, 2, st);
+                                                 n_seqs, T_total, out, workspace, st);
     else
         e = launch_prefill<float, float>(cfg, w, q, k, v, a, b, z, conv_state, rec_state, cu_seqlens, n_seqs,
-                                         T_total, out, workspace, 3, st);
+                                         T_total, out, workspace, st);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -610,6 +669,95 @@ gdn_status gdn_out_proj(const gdn_config* cfg, const void* o, const void* w_out,
     if (T < 0 || d_model <= 0) return GDN_ERR_INVALID_ARG;
     const gdn_out_segment seg = {y, d_model};
     return run_linear(o, w_out, T, d_model, cfg->n_v_heads * cfg->d_v, &seg, 1, stream);
+}
+
+// ---------------------------------------------------------------------------
+// Context-parallel prefill (see cp.cuh)
+// ---------------------------------------------------------------------------
+static gdn_status cp_check(const gdn_config* cfg, int64_t T_seg) {
+    gdn_status s = check_config(cfg);
+    if (s != GDN_OK) return s;
+    if (T_seg < 1) return GDN_ERR_INVALID_ARG;
+    if (cfg->state_dtype != GDN_F32 || cfg->d_k != cfg->d_v) return GDN_ERR_UNSUPPORTED;
+    if (T_seg > 0x7fffffffLL - 64) return GDN_ERR_UNSUPPORTED;
+    return GDN_OK;
+}
+
+size_t gdn_cp_workspace_size(const gdn_config* cfg, int64_t T_seg) {
+    if (cp_check(cfg, T_seg) != GDN_OK) return 0;
+    return cp_layout(cfg, T_seg).total;
+}
+
+gdn_status gdn_cp_local(const gdn_config* cfg, const gdn_weights* w, const void* q, const void* k, const void* v,
+                        const void* a, const void* b, void* conv_state, int64_t T_seg, void* summary,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+    gdn_status s = cp_check(cfg, T_seg);
+    if (s != GDN_OK) return s;
+    if ((s = check_weights(w)) != GDN_OK) return s;
+    if (!q || !k || !v || !a || !b || !conv_state || !summary || !workspace) return GDN_ERR_INVALID_ARG;
+    const void* a16[] = {q, k, v, summary};
+    for (const void* p : a16)
+        if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return GDN_ERR_INVALID_ARG;
+    const CpLayout L = cp_layout(cfg, T_seg);
+    if (workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    int32_t* cu = reinterpret_cast<int32_t*>(wsb + L.cu_off);
+    const int Hv = cfg->n_v_heads, d = cfg->d_k;
+    float* P = static_cast<float*>(summary);
+    float* S_loc = P + (size_t)Hv * d * d;
+    const bool abf = cfg->act_dtype == GDN_BF16, obf = cfg->out_dtype == GDN_BF16;
+    gdn::cp::segment_cu_kernel<<<1, 32, 0, st>>>(cu, (int32_t)T_seg);
+    cudaError_t e = abf ? launch_stage_a<__nv_bfloat16>(cfg, w, q, k, v, a, b, conv_state, cu, 1, T_seg, workspace, st)
+                        : launch_stage_a<float>(cfg, w, q, k, v, a, b, conv_state, cu, 1, T_seg, workspace, st);
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    // S_loc: the scan from a zero state over the real v^
+    if ((e = cudaMemsetAsync(S_loc, 0, (size_t)Hv * d * d * sizeof(float), st)) != cudaSuccess) return GDN_ERR_CUDA;
+    const void* vh = wsb + L.pre.v_off;
+    e = obf ? launch_scan<__nv_bfloat16>(cfg, vh, T_seg, S_loc, cu, 1, T_seg, workspace, st)
+            : launch_scan<float>(cfg, vh, T_seg, S_loc, cu, 1, T_seg, workspace, st);
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    // P: the scan from I with V = 0 (a zero block of 64 rows, zeros past it)
+    if ((e = cudaMemsetAsync(wsb + L.zv_off, 0, L.total - L.zv_off, st)) != cudaSuccess) return GDN_ERR_CUDA;
+    gdn::cp::identity_kernel<<<(unsigned)std::max<int64_t>(1, std::min<int64_t>((int64_t)Hv * d * d / 256, 1024)), 256, 0,
+                               st>>>(P, Hv, d);
+    e = obf ? launch_scan<__nv_bfloat16>(cfg, wsb + L.zv_off, gdn::intra::C, P, cu, 1, T_seg, workspace, st)
+            : launch_scan<float>(cfg, wsb + L.zv_off, gdn::intra::C, P, cu, 1, T_seg, workspace, st);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+gdn_status gdn_cp_finish(const gdn_config* cfg, const gdn_weights* w, const void* z, const void* summaries,
+                         int32_t n_ranks, int32_t rank, const void* state_in, int64_t T_seg, void* out,
+                         void* state_out, void* workspace, size_t workspace_bytes, void* stream) {
+    gdn_status s = cp_check(cfg, T_seg);
+    if (s != GDN_OK) return s;
+    if ((s = check_weights(w)) != GDN_OK) return s;
+    if (n_ranks < 1 || rank < 0 || rank >= n_ranks) return GDN_ERR_INVALID_ARG;
+    if (!z || !summaries || !state_in || !out || !state_out || !workspace) return GDN_ERR_INVALID_ARG;
+    const void* a16[] = {z, summaries, state_in, out, state_out};
+    for (const void* p : a16)
+        if (!aligned(p, 16)) return GDN_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return GDN_ERR_INVALID_ARG;
+    const CpLayout L = cp_layout(cfg, T_seg);
+    if (workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    const int32_t* cu = reinterpret_cast<const int32_t*>(wsb + L.cu_off);
+    const int Hv = cfg->n_v_heads, d = cfg->d_k;
+    gdn::cp::fold_kernel<<<(unsigned)(Hv * (d / gdn::cp::CR)), gdn::cp::CT, 0, st>>>(
+        static_cast<const float*>(state_in), static_cast<const float*>(summaries), rank, Hv, d,
+        static_cast<float*>(state_out));
+    const bool abf = cfg->act_dtype == GDN_BF16, obf = cfg->out_dtype == GDN_BF16;
+    const void* vh = wsb + L.pre.v_off;
+    cudaError_t e = obf ? launch_scan<__nv_bfloat16>(cfg, vh, T_seg, state_out, cu, 1, T_seg, workspace, st)
+                        : launch_scan<float>(cfg, vh, T_seg, state_out, cu, 1, T_seg, workspace, st);
+    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    if (abf && obf) e = launch_norm<__nv_bfloat16, __nv_bfloat16>(cfg, w, z, cu, 1, T_seg, out, workspace, st);
+    else if (abf) e = launch_norm<__nv_bfloat16, float>(cfg, w, z, cu, 1, T_seg, out, workspace, st);
+    else if (obf) e = launch_norm<float, __nv_bfloat16>(cfg, w, z, cu, 1, T_seg, out, workspace, st);
+    else e = launch_norm<float, float>(cfg, w, z, cu, 1, T_seg, out, workspace, st);
+    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 gdn_status gdn_check_device_error(void* stream) {

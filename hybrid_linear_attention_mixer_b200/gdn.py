@@ -53,8 +53,8 @@ class _CWeights(ctypes.Structure):
 
 _lib = None
 EXPORTS = ("gdn_config_default", "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode",
-           "gdn_decode_multi", "gdn_linear", "gdn_in_proj", "gdn_out_proj", "gdn_check_device_error",
-           "gdn_status_string")
+           "gdn_decode_multi", "gdn_linear", "gdn_in_proj", "gdn_out_proj", "gdn_cp_workspace_size",
+           "gdn_cp_local", "gdn_cp_finish", "gdn_check_device_error", "gdn_status_string")
 DECODE_MULTI_MAX_TOKENS = 16   # GDN_DECODE_MULTI_MAX_TOKENS
 LINEAR_MAX_SEGMENTS = 8        # GDN_LINEAR_MAX_SEGMENTS
 
@@ -84,6 +84,12 @@ def lib() -> ctypes.CDLL:
         L.gdn_in_proj.restype = ctypes.c_int
         L.gdn_out_proj.argtypes = [vp, vp, vp, i64, i32, vp, vp]
         L.gdn_out_proj.restype = ctypes.c_int
+        L.gdn_cp_workspace_size.argtypes = [vp, i64]
+        L.gdn_cp_workspace_size.restype = sz
+        L.gdn_cp_local.argtypes = [vp, vp] + [vp] * 5 + [vp, i64, vp, vp, sz, vp]
+        L.gdn_cp_local.restype = ctypes.c_int
+        L.gdn_cp_finish.argtypes = [vp, vp, vp, vp, i32, i32, vp, i64, vp, vp, vp, sz, vp]
+        L.gdn_cp_finish.restype = ctypes.c_int
         L.gdn_check_device_error.argtypes = [vp]
         L.gdn_check_device_error.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -301,6 +307,55 @@ def out_proj(cfg: Config, o, w_out, y=None, stream=None):
     if s != 0:
         raise GdnError(s, "gdn_out_proj")
     return y
+
+
+def cp_workspace_size(cfg: Config, T_seg: int) -> int:
+    c = cfg.c()
+    return int(lib().gdn_cp_workspace_size(ctypes.byref(c), T_seg))
+
+
+def cp_local(cfg: Config, w: dict, q, k, v, a, b, conv_state, workspace=None, summary=None, stream=None):
+    """Context-parallel phase 1 on this rank's segment: returns (summary, workspace).
+    conv_state [C, K-1] holds the K-1 input rows before the segment (updated in
+    place to the segment's last rows); summary [2, H_v, d_k, d_k] fp32 = (P, S_loc)."""
+    dev = q.device
+    T = q.shape[0]
+    for n, t in (("q", q), ("k", k), ("v", v), ("a", a), ("b", b), ("conv_state", conv_state)):
+        _check(t, n, cfg.act_dtype, dev)
+    if workspace is None:
+        workspace = torch.empty(cp_workspace_size(cfg, T), dtype=torch.uint8, device=dev)
+    if summary is None:
+        summary = torch.empty((2, cfg.n_v_heads, cfg.d_k, cfg.d_k), dtype=torch.float32, device=dev)
+    _check(summary, "summary", torch.float32, dev)
+    c, cw = cfg.c(), _weights(w, dev)
+    s = lib().gdn_cp_local(ctypes.byref(c), ctypes.byref(cw), _ptr(q), _ptr(k), _ptr(v), _ptr(a), _ptr(b),
+                           _ptr(conv_state), T, _ptr(summary), _ptr(workspace), workspace.numel(), _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_cp_local")
+    return summary, workspace
+
+
+def cp_finish(cfg: Config, w: dict, z, summaries, rank: int, state_in, workspace, out=None, state_out=None,
+              stream=None):
+    """Context-parallel phase 2: summaries [R, 2, H_v, d_k, d_k] (every rank's, in rank
+    order), state_in [H_v, d_v, d_k] the state before the whole sequence.  Returns
+    (out [T_seg, H_v*d_v], state_out [H_v, d_v, d_k]: the state after this segment)."""
+    dev = z.device
+    T = z.shape[0]
+    _check(z, "z", cfg.act_dtype, dev)
+    _check(summaries, "summaries", torch.float32, dev)
+    _check(state_in, "state_in", torch.float32, dev)
+    if out is None:
+        out = torch.empty((T, cfg.n_v_heads * cfg.d_v), dtype=cfg.out_dtype, device=dev)
+    if state_out is None:
+        state_out = torch.empty_like(state_in)
+    c, cw = cfg.c(), _weights(w, dev)
+    s = lib().gdn_cp_finish(ctypes.byref(c), ctypes.byref(cw), _ptr(z), _ptr(summaries), summaries.shape[0],
+                            rank, _ptr(state_in), T, _ptr(out), _ptr(state_out), _ptr(workspace),
+                            workspace.numel(), _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_cp_finish")
+    return out, state_out
 
 
 def check_device_error(stream=None) -> None:

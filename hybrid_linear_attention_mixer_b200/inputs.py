@@ -165,8 +165,9 @@ def _acts(seed, T, Hk, Hv, dk, dv, bf16, gates, alpha_range=None, nla_range=None
 
 
 def make_case(name: str, seed: int | None = None, T: int | None = None,
-              n_seqs: int | None = None) -> Case:
-    """Build one named workload.  ``T`` / ``n_seqs`` shrink a workload for quick runs."""
+              n_seqs: int | None = None, nla_range: tuple | None = None) -> Case:
+    """Build one named workload.  ``T`` / ``n_seqs`` shrink a workload for quick runs;
+    ``nla_range`` replaces the -log alpha range of ``prefill_256k``."""
     if name == "tiny":
         s = 0 if seed is None else seed
         Hk, Hv, d, K = 2, 6, 32, 4
@@ -219,7 +220,7 @@ def make_case(name: str, seed: int | None = None, T: int | None = None,
         s = 4 if seed is None else seed
         T = 262144 if T is None else T
         w = _weights(s, Hk, Hv, d, d, K, gates="alpha")
-        acts = _acts(s, T, Hk, Hv, d, d, True, "alpha", nla_range=(1e-4, 0.1))
+        acts = _acts(s, T, Hk, Hv, d, d, True, "alpha", nla_range=nla_range or (1e-4, 0.1))
         cu = np.array([0, T], np.int32)
         return Case(name, Hk, Hv, d, d, K, 64, True, cu, w, acts,
                     np.zeros((1, C, K - 1), np.uint16), np.zeros((1, Hv, d, d), np.float32))

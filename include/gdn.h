@@ -216,6 +216,40 @@ gdn_status gdn_in_proj(const gdn_config* cfg, const void* hidden, const void* w_
 gdn_status gdn_out_proj(const gdn_config* cfg, const void* o, const void* w_out, int64_t T,
                         int32_t d_model, void* y, void* stream);
 
+/*
+ * Context-parallel prefill: one long sequence (up to the 262,144-token context of
+ * "Qwen3.8-Flash-Next" (llm-atlas-9r2), "Key facts") cut into contiguous
+ * segments, one per rank, computing what one gdn_prefill over the whole
+ * sequence computes.  Over a segment the state map is affine,
+ * S_end = S_0 . P + S_loc, with P (d_k x d_k) the product of the segment's chunk
+ * transitions and S_loc its end state from S_0 = 0.  Each rank:
+ *   1. gdn_cp_local on its segment, with conv_state set to the K-1 input rows
+ *      (q | k | v channels) before the segment (the previous rank's last rows,
+ *      or the sequence's conv state on rank 0): writes summary = {P, S_loc};
+ *   2. the ranks exchange their summaries (an all-gather, in rank order);
+ *   3. gdn_cp_finish: folds the maps of ranks 0 .. rank-1 onto state_in (the
+ *      state before the whole sequence) to get this segment's S_0, then runs the
+ *      scan and the gated norm: out holds the segment's outputs and state_out the
+ *      state after the segment (on the last rank: the sequence's final state).
+ * The segment runs as one sequence; the caller keeps `workspace` (of
+ * gdn_cp_workspace_size bytes, 256-byte aligned) between the two calls.
+ * Requires state_dtype GDN_F32 and d_k == d_v (else GDN_ERR_UNSUPPORTED).
+ *   q, k, v, a, b, z: this segment's rows, as for gdn_prefill (T_seg >= 1)
+ *   conv_state [C][K-1] act_dtype in/out (out: the segment's last K-1 inputs)
+ *   summary    [2][H_v][d_k][d_k] fp32 out: P, then S_loc
+ *   summaries  [n_ranks][2][H_v][d_k][d_k] fp32: every rank's summary
+ *   state_in, state_out [H_v][d_v][d_k] fp32; they may alias
+ */
+size_t gdn_cp_workspace_size(const gdn_config* cfg, int64_t T_seg);
+gdn_status gdn_cp_local(const gdn_config* cfg, const gdn_weights* w,
+                        const void* q, const void* k, const void* v, const void* a, const void* b,
+                        void* conv_state, int64_t T_seg, void* summary,
+                        void* workspace, size_t workspace_bytes, void* stream);
+gdn_status gdn_cp_finish(const gdn_config* cfg, const gdn_weights* w, const void* z,
+                         const void* summaries, int32_t n_ranks, int32_t rank,
+                         const void* state_in, int64_t T_seg, void* out, void* state_out,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
 /* Capacity, in bytes, of the fixed scratch array used by gdn_prefill_noalloc. */
 #define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 

@@ -159,6 +159,40 @@ def forward(shape: Shape, w: dict, q, k, v, a, b, z, conv_state, rec_state, cu_s
 
 
 # ---------------------------------------------------------------------------
+# Segment state maps (context-parallel prefill)
+# ---------------------------------------------------------------------------
+# Over one segment the recurrence maps the initial state affinely:
+#     S_end = S_0 . P + S_loc.
+# With v = 0 every update is S <- alpha S (I - beta k k^T), linear in S, so the run
+# from S_0 = I returns P (d_v = d_k required); the run from S_0 = 0 returns S_loc.
+
+def segment_map(shape: Shape, w: dict, q, k, v, a, b, conv_state):
+    """(P [H_v, d_k, d_k], S_loc [H_v, d_v, d_k]) of one segment, fp64.
+    conv_state [C, K-1]: the inputs before the segment."""
+    assert shape.d_k == shape.d_v, "P has the state's shape only when d_k == d_v"
+    T = np.asarray(q).shape[0]
+    cu = np.array([0, T], np.int32)
+    cs = np.asarray(act_to_f64(conv_state))[None]
+    Hv, d = shape.n_v_heads, shape.d_k
+    z = np.zeros((T, Hv * shape.d_v))
+    acts = [act_to_f64(x) for x in (q, k, v, a, b)]
+    S_loc = forward(shape, w, *acts, z, cs, np.zeros((1, Hv, d, d)), cu)["rec_state"][0]
+    cs0 = cs.copy()
+    cs0[:, 2 * shape.n_k_heads * shape.d_k:] = 0.0          # the v channels of the conv window
+    eye = np.broadcast_to(np.eye(d), (1, Hv, d, d)).copy()
+    P = forward(shape, w, acts[0], acts[1], np.zeros_like(acts[2]), acts[3], acts[4], z, cs0, eye, cu)["rec_state"][0]
+    return P, S_loc
+
+
+def fold_segment_maps(state_in, maps):
+    """The state after the segments whose (P, S_loc) are listed, from state_in."""
+    S = np.asarray(state_in, dtype=np.float64)
+    for P, S_loc in maps:
+        S = S @ P + S_loc
+    return S
+
+
+# ---------------------------------------------------------------------------
 # Projections around the mixer
 # ---------------------------------------------------------------------------
 # The hidden size is 2,560 ("Qwen3.8-Flash-Next" (llm-atlas-9r2), "Key facts";

@@ -5,6 +5,7 @@ import os
 import re
 
 import pytest
+import torch
 
 from hybrid_linear_attention_mixer_b200 import build, gdn
 
@@ -132,6 +133,28 @@ def test_linear_argument_errors(lib):
     assert lib.gdn_in_proj(ctypes.byref(c), P(0x1000), P(0x2000), 4, 2564, *[P(0x3000)] * 6, None) == UNSUPPORTED
     assert lib.gdn_out_proj(ctypes.byref(c), P(0x1000), P(0x2000), 0, 2560, P(0x3000), None) == OK
     assert lib.gdn_out_proj(ctypes.byref(c), P(0x1000), P(0x2000), -1, 2560, P(0x3000), None) == INVALID
+
+
+def test_cp_argument_errors(lib):
+    P = ctypes.c_void_p
+    cw = gdn._CWeights(0x2000, 0x3000, 0x4000, 0x5000)
+    c = gdn.Config().c()
+    assert lib.gdn_cp_workspace_size(ctypes.byref(c), 4096) > gdn.workspace_size(gdn.Config(), 4096, 1)
+    assert lib.gdn_cp_workspace_size(ctypes.byref(c), 0) == 0
+    local = lambda cfg, T, ws=1 << 40, p=0x1000: lib.gdn_cp_local(
+        ctypes.byref(cfg), ctypes.byref(cw), *[P(p)] * 5, P(0x6000), T, P(0x7000), P(0x100000), ws, None)
+    assert local(c, 0) == INVALID
+    assert local(c, 64, p=0) == INVALID
+    assert local(c, 64, ws=1024) == WORKSPACE
+    cb = gdn.Config(state_dtype=torch.bfloat16).c()
+    assert local(cb, 64) == UNSUPPORTED                   # the maps need an fp32 state
+    cd = gdn.Config(d_k=64, d_v=128).c()
+    assert local(cd, 64) == UNSUPPORTED                   # P has the state's shape only when d_k == d_v
+    fin = lambda n, r, ws=1 << 40: lib.gdn_cp_finish(
+        ctypes.byref(c), ctypes.byref(cw), P(0x1000), P(0x2000), n, r, P(0x3000), 64, P(0x4000), P(0x5000),
+        P(0x100000), ws, None)
+    assert fin(2, 2) == INVALID and fin(2, -1) == INVALID and fin(0, 0) == INVALID
+    assert fin(2, 1, ws=1024) == WORKSPACE
 
 
 def test_status_strings(lib):

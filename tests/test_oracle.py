@@ -369,3 +369,34 @@ def test_linear_reads_bf16_exactly():
     np.testing.assert_array_equal(oracle.linear(xb, wb),
                                   inputs.bf16_bits_to_f32(xb).astype(np.float64)
                                   @ inputs.bf16_bits_to_f32(wb).astype(np.float64).T)
+
+
+# ---------------------------------------------------------------------------
+# Segment state maps (context-parallel prefill)
+# ---------------------------------------------------------------------------
+
+def test_segment_map_is_the_affine_state_map():
+    """For any S_0 the segment's end state is S_0 . P + S_loc, with (P, S_loc) from the
+    v = 0 run from I and the run from 0; folding two segments' maps equals one run over
+    both segments (the conv window carried across the cut)."""
+    rng = np.random.default_rng(31)
+    shape, w, acts, cs, rs, cu = _random_case(rng, Hk=1, G=2, d=4, T=9, n_seqs=1, state_std=0.5)
+    T = int(cu[-1])
+    P, S_loc = oracle.segment_map(shape, w, *[acts[n] for n in "qkvab"], cs[0])
+    for trial in range(3):
+        S0 = rng.normal(0, 0.7, (1, shape.n_v_heads, 4, 4))
+        end = _run(shape, w, acts, cs, S0, cu)["rec_state"][0]
+        np.testing.assert_allclose(end, S0[0] @ P + S_loc, rtol=0, atol=1e-12)
+    # two segments [0, c) and [c, T): maps folded in order == one run
+    c = T // 2 + 1
+    first = {n: x[:c] for n, x in acts.items()}
+    second = {n: x[c:] for n, x in acts.items()}
+    cs_mid = np.concatenate([acts["q"], acts["k"], acts["v"]], axis=1)[c - 3:c].T      # [C, 3], oldest first
+    m1 = oracle.segment_map(shape, w, *[first[n] for n in "qkvab"], cs[0])
+    m2 = oracle.segment_map(shape, w, *[second[n] for n in "qkvab"], cs_mid)
+    whole = _run(shape, w, acts, cs, rs, cu)["rec_state"][0]
+    np.testing.assert_allclose(oracle.fold_segment_maps(rs[0], [m1, m2]), whole, rtol=0, atol=1e-12)
+    # a map that decays to nothing (beta = 0, strong gate) leaves P ~ 0 and S_loc = 0
+    a0 = dict(acts, b=np.full_like(acts["b"], -60.0), a=np.full_like(acts["a"], 30.0))
+    P0, S0_loc = oracle.segment_map(shape, w, *[a0[n] for n in "qkvab"], cs[0])
+    assert np.abs(S0_loc).max() < 1e-20 and np.abs(P0).max() < 1e-6
