@@ -363,6 +363,37 @@ def main():
     in_cublas_s = timed(lambda: torch.nn.functional.linear(hid, w_in))
     out_cublas_s = timed(lambda: torch.nn.functional.linear(p_out, w_out))
 
+    # ---- context-parallel prefill: one sequence of PREFILL_T x N tokens, one segment per rank ----
+    cp_cs = act(pc.conv_state[0]).to(dev)
+    cp_rs = torch.zeros((H_V, D, D), dtype=torch.float32, device=dev)
+    cp_seg = {n: P[n] for n in "qkvabz"}
+    if world > 1:
+        from hybrid_linear_attention_mixer_b200 import cp as cp_mod
+
+        def cp_step():
+            cp_mod.prefill(cfg, w, cp_seg["q"], cp_seg["k"], cp_seg["v"], cp_seg["a"], cp_seg["b"], cp_seg["z"],
+                           cp_cs, cp_rs)
+        cp_local_s = cp_finish_s = None
+    else:
+        cp_ws = torch.empty(gdn.cp_workspace_size(cfg, PREFILL_T), dtype=torch.uint8, device=dev)
+        cp_sum = torch.empty((1, 2, H_V, D, D), dtype=torch.float32, device=dev)
+        cp_cs1 = cp_cs.clone()
+
+        def cp_local():
+            cp_cs1.copy_(cp_cs)
+            gdn.cp_local(cfg, w, cp_seg["q"], cp_seg["k"], cp_seg["v"], cp_seg["a"], cp_seg["b"], cp_cs1,
+                         workspace=cp_ws, summary=cp_sum[0], stream=stream)
+
+        def cp_finish():
+            gdn.cp_finish(cfg, w, cp_seg["z"], cp_sum, 0, cp_rs, cp_ws, out=p_out, stream=stream)
+
+        def cp_step():
+            cp_local()
+            cp_finish()
+        cp_local_s, cp_finish_s = timed(cp_local), timed(cp_finish)
+    cp_s = timed(cp_step)
+    gdn.check_device_error(stream)
+
     # ---- end to end through the public API with host buffers ----
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
@@ -419,6 +450,14 @@ def main():
                 "out": {"shape": [PREFILL_T, D_MODEL, H_V * D], "us": out_s * 1e6,
                         "value": PROJ_OUT_FLOP / out_s / 1e12, "frac": PROJ_OUT_FLOP / out_s / 1e12 / pk["bf16_tflops"],
                         "cublas_value": PROJ_OUT_FLOP / out_cublas_s / 1e12}},
+            "context_parallel": {
+                "sequence_tokens": PREFILL_T * world, "segment_tokens": PREFILL_T, "ranks": world,
+                "value": PREFILL_T * world / cp_s, "unit": "tokens/s", "us_per_call": cp_s * 1e6,
+                "local_us": None if cp_local_s is None else cp_local_s * 1e6,
+                "finish_us": None if cp_finish_s is None else cp_finish_s * 1e6,
+                "exchange_bytes_per_rank": 2 * H_V * D * D * 4,
+                "note": "one rank: phase 1 and phase 2 on one segment, no exchange"
+                        if world == 1 else "NCCL all-gathers inside the timed call"},
             "prefill_ms": pre_ms / K,
             "roofline": {"kernel": "gdn_decode_kernel", "bound": "hbm", "achieved": dec_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / pk["hbm_gbs"],

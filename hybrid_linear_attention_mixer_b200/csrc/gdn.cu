@@ -77,13 +77,16 @@ Layout workspace_layout(const gdn_config* c, int64_t T, int64_t n_seqs) {
 // reads zeros for every later row (V = 0 for the transition's scan).
 struct CpLayout {
     Layout pre;
-    size_t cu_off, zv_off, total;
+    size_t o2_off, cu_off, zv_off, total;
 };
 
+// (after the prefill workspace: a second o-tile region, for the transition's
+// scan, whose outputs are not used, so that it may run beside the other scan)
 CpLayout cp_layout(const gdn_config* c, int64_t T_seg) {
     CpLayout L;
     L.pre = workspace_layout(c, T_seg, 1);
-    L.cu_off = align_up(L.pre.total, 256);
+    L.o2_off = align_up(L.pre.total, 256);
+    L.cu_off = align_up(L.o2_off + (L.pre.total - L.pre.o_off), 256);
     L.zv_off = L.cu_off + 256;
     L.total = L.zv_off + align_up((size_t)gdn::intra::C * c->n_v_heads * c->d_v * sizeof(__half), 256);
     return L;
@@ -159,6 +162,19 @@ bool z_rows_map(CUtensorMap* m, const void* base, bool bf16, int width, int dv, 
                const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// A non-blocking stream per device for work that may overlap the caller's
+// stream (joined back to it by events).
+cudaStream_t side_stream() {
+    static cudaStream_t streams[64];
+    static std::mutex mu;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
+        streams[dev] = nullptr;
+    return streams[dev];
 }
 
 // Streaming multiprocessors of the current device (cached per device).
@@ -400,7 +416,7 @@ cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void
 // workspace's v^, or a zero block whose map reads zeros past its 64 rows).
 template <typename TO>
 cudaError_t launch_scan(const gdn_config* c, const void* v_src, int64_t v_rows, void* rec_state, const int32_t* cu,
-                        int n_seqs, int64_t T, void* ws, cudaStream_t st) {
+                        int n_seqs, int64_t T, void* ws, cudaStream_t st, void* o_dst = nullptr) {
     const Layout L = workspace_layout(c, T, n_seqs);
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     auto k_scan = c->state_dtype == GDN_BF16 ? gdn::scan::gdn_scan_kernel<TO, __nv_bfloat16>
@@ -416,7 +432,7 @@ cudaError_t launch_scan(const gdn_config* c, const void* v_src, int64_t v_rows, 
     sa.cu = cu;
     sa.chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off);
     sa.rec = wsb + L.rec_off;
-    sa.o = wsb + L.o_off;
+    sa.o = o_dst ? o_dst : wsb + L.o_off;
     sa.Hk = c->n_k_heads; sa.Hv = c->n_v_heads; sa.dk = c->d_k; sa.dv = c->d_v;
     k_scan<<<(unsigned)n_seqs * c->n_v_heads, gdn::scan::NT, gdn::scan::SMEM_BYTES, st>>>(tm_v, sa);
     return cudaGetLastError();
@@ -712,19 +728,38 @@ gdn_status gdn_cp_local(const gdn_config* cfg, const gdn_weights* w, const void*
     cudaError_t e = abf ? launch_stage_a<__nv_bfloat16>(cfg, w, q, k, v, a, b, conv_state, cu, 1, T_seg, workspace, st)
                         : launch_stage_a<float>(cfg, w, q, k, v, a, b, conv_state, cu, 1, T_seg, workspace, st);
     if (e != cudaSuccess) return GDN_ERR_CUDA;
-    // S_loc: the scan from a zero state over the real v^
+    // starting states: S_loc from zero, P from I; V = 0 for P: a zero block of 64
+    // rows whose map reads zeros past it
     if ((e = cudaMemsetAsync(S_loc, 0, (size_t)Hv * d * d * sizeof(float), st)) != cudaSuccess) return GDN_ERR_CUDA;
-    const void* vh = wsb + L.pre.v_off;
-    e = obf ? launch_scan<__nv_bfloat16>(cfg, vh, T_seg, S_loc, cu, 1, T_seg, workspace, st)
-            : launch_scan<float>(cfg, vh, T_seg, S_loc, cu, 1, T_seg, workspace, st);
-    if (e != cudaSuccess) return GDN_ERR_CUDA;
-    // P: the scan from I with V = 0 (a zero block of 64 rows, zeros past it)
     if ((e = cudaMemsetAsync(wsb + L.zv_off, 0, L.total - L.zv_off, st)) != cudaSuccess) return GDN_ERR_CUDA;
     gdn::cp::identity_kernel<<<(unsigned)std::max<int64_t>(1, std::min<int64_t>((int64_t)Hv * d * d / 256, 1024)), 256, 0,
                                st>>>(P, Hv, d);
-    e = obf ? launch_scan<__nv_bfloat16>(cfg, wsb + L.zv_off, gdn::intra::C, P, cu, 1, T_seg, workspace, st)
-            : launch_scan<float>(cfg, wsb + L.zv_off, gdn::intra::C, P, cu, 1, T_seg, workspace, st);
-    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    // The two scans read the same records and are independent, one CTA per head
+    // each: the transition's runs on a side stream, forked from and joined back
+    // to the caller's stream by events.
+    cudaStream_t side = side_stream();
+    if (!side) return GDN_ERR_CUDA;
+    cudaEvent_t fork = nullptr, join = nullptr;
+    if (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
+        cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
+        if (fork) cudaEventDestroy(fork);
+        return GDN_ERR_CUDA;
+    }
+    cudaError_t e2 = cudaEventRecord(fork, st);
+    if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(side, fork, 0);
+    if (e2 == cudaSuccess)
+        e2 = obf ? launch_scan<__nv_bfloat16>(cfg, wsb + L.zv_off, gdn::intra::C, P, cu, 1, T_seg, workspace, side,
+                                              wsb + L.o2_off)
+                 : launch_scan<float>(cfg, wsb + L.zv_off, gdn::intra::C, P, cu, 1, T_seg, workspace, side,
+                                      wsb + L.o2_off);
+    if (e2 == cudaSuccess) e2 = cudaEventRecord(join, side);
+    const void* vh = wsb + L.pre.v_off;
+    e = obf ? launch_scan<__nv_bfloat16>(cfg, vh, T_seg, S_loc, cu, 1, T_seg, workspace, st)
+            : launch_scan<float>(cfg, vh, T_seg, S_loc, cu, 1, T_seg, workspace, st);
+    if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, join, 0);
+    cudaEventDestroy(fork);
+    cudaEventDestroy(join);
+    return e == cudaSuccess && e2 == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
 gdn_status gdn_cp_finish(const gdn_config* cfg, const gdn_weights* w, const void* z, const void* summaries,
