@@ -395,13 +395,14 @@ def main():
     gdn.check_device_error(stream)
 
     # ---- end to end through the public API with host buffers ----
+    h_ws = torch.empty(gdn.prefill_host_workspace_size(cfg, PREFILL_T, 1), dtype=torch.uint8, device=dev)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
               for _ in range(args.steps)]
     for i in range(-args.warmup, args.steps):
         flush.zero_()
         if i >= 0:
             e2e_ev[i][0].record(stream)
-        gdn.prefill_host(cfg, w, host, p_cs, p_rs, stream=stream)
+        gdn.prefill_host(cfg, w, host, p_cs, p_rs, workspace=h_ws, stream=stream)
         if i >= 0:
             e2e_ev[i][1].record(stream)
     torch.cuda.synchronize()

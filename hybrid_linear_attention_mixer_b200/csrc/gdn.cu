@@ -8,6 +8,7 @@
 #include <cmath>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "conv.cuh"
 #include "cp.cuh"
@@ -92,6 +93,60 @@ CpLayout cp_layout(const gdn_config* c, int64_t T_seg) {
     return L;
 }
 
+// Prefill from host buffers: the tokens are cut into at most 8 segments of a
+// multiple of 64 rows (at least 512), which run one after another on the
+// caller's stream with the states carried on the device, while the next
+// segment's inputs come in and the previous segment's output goes out on two
+// copy streams.  Two staging slots; one prefill workspace.
+struct HostPlan {
+    int64_t seg_len;
+    int n_seg;
+};
+
+HostPlan host_plan(int64_t T) {
+    HostPlan h;
+    int64_t n = (T + 511) / 512;
+    n = n < 1 ? 1 : n > 8 ? 8 : n;
+    h.seg_len = align_up((size_t)((T + n - 1) / n), 64);
+    h.n_seg = (int)((T + h.seg_len - 1) / h.seg_len);
+    return h;
+}
+
+struct HostLayout {
+    HostPlan plan;
+    size_t row_in[6];     // bytes per token of q, k, v, a, b, z
+    size_t row_out;       // bytes per token of out
+    size_t pre_off, cu_off, seg_cu_off[2], slot_off[2], in_off[6], out_off, slot_bytes, total;
+};
+
+HostLayout host_layout(const gdn_config* c, int64_t T, int32_t n_seqs) {
+    HostLayout L;
+    L.plan = host_plan(T);
+    const size_t ab = c->act_dtype == GDN_F32 ? 4 : 2, ob = c->out_dtype == GDN_F32 ? 4 : 2;
+    const size_t qk = (size_t)c->n_k_heads * c->d_k, vz = (size_t)c->n_v_heads * c->d_v, g = c->n_v_heads;
+    const size_t widths[6] = {qk, qk, vz, g, g, vz};
+    for (int i = 0; i < 6; ++i) L.row_in[i] = widths[i] * ab;
+    L.row_out = vz * ob;
+    const size_t rows = (size_t)L.plan.seg_len;
+    size_t off = 0;
+    for (int i = 0; i < 6; ++i) {
+        L.in_off[i] = off;
+        off = align_up(off + rows * L.row_in[i], 256);
+    }
+    L.out_off = off;
+    off = align_up(off + rows * L.row_out, 256);
+    L.slot_bytes = off;
+    L.pre_off = 0;
+    const size_t pre = workspace_layout(c, L.plan.seg_len, n_seqs).total;
+    L.cu_off = align_up(pre, 256);
+    L.seg_cu_off[0] = align_up(L.cu_off + ((size_t)n_seqs + 1) * 4, 256);
+    L.seg_cu_off[1] = align_up(L.seg_cu_off[0] + ((size_t)n_seqs + 1) * 4, 256);
+    L.slot_off[0] = align_up(L.seg_cu_off[1] + ((size_t)n_seqs + 1) * 4, 256);
+    L.slot_off[1] = L.slot_off[0] + L.slot_bytes;
+    L.total = L.slot_off[1] + L.slot_bytes;
+    return L;
+}
+
 // Opt in to > 48 KiB of dynamic shared memory, once per device and kernel.
 template <typename K>
 cudaError_t ensure_smem(K kernel, int variant, size_t bytes) {
@@ -164,17 +219,18 @@ bool z_rows_map(CUtensorMap* m, const void* base, bool bf16, int width, int dv, 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// A non-blocking stream per device for work that may overlap the caller's
-// stream (joined back to it by events).
-cudaStream_t side_stream() {
-    static cudaStream_t streams[64];
+// Non-blocking streams per device for work that may overlap the caller's stream
+// (forked from and joined back to it by events): 0 = the context-parallel
+// transition scan, 1 = host-to-device copies, 2 = device-to-host copies.
+cudaStream_t side_stream(int which = 0) {
+    static cudaStream_t streams[64][3];
     static std::mutex mu;
     int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (which < 0 || which > 2 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     std::lock_guard<std::mutex> lock(mu);
-    if (!streams[dev] && cudaStreamCreateWithFlags(&streams[dev], cudaStreamNonBlocking) != cudaSuccess)
-        streams[dev] = nullptr;
-    return streams[dev];
+    if (!streams[dev][which] && cudaStreamCreateWithFlags(&streams[dev][which], cudaStreamNonBlocking) != cudaSuccess)
+        streams[dev][which] = nullptr;
+    return streams[dev][which];
 }
 
 // Streaming multiprocessors of the current device (cached per device).
@@ -737,7 +793,7 @@ gdn_status gdn_cp_local(const gdn_config* cfg, const gdn_weights* w, const void*
     // The two scans read the same records and are independent, one CTA per head
     // each: the transition's runs on a side stream, forked from and joined back
     // to the caller's stream by events.
-    cudaStream_t side = side_stream();
+    cudaStream_t side = side_stream(0);
     if (!side) return GDN_ERR_CUDA;
     cudaEvent_t fork = nullptr, join = nullptr;
     if (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
@@ -793,6 +849,127 @@ gdn_status gdn_cp_finish(const gdn_config* cfg, const gdn_weights* w, const void
     else if (obf) e = launch_norm<float, __nv_bfloat16>(cfg, w, z, cu, 1, T_seg, out, workspace, st);
     else e = launch_norm<float, float>(cfg, w, z, cu, 1, T_seg, out, workspace, st);
     return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// Prefill from host buffers (see host_layout)
+// ---------------------------------------------------------------------------
+namespace {
+// cu of one segment: sequences s_a .. s_a + n_s - 1 clipped to tokens [t0, t1)
+__global__ void segment_seqlens_kernel(const int32_t* cu, int32_t s_a, int32_t n_s, int32_t t0, int32_t t1,
+                                       int32_t* out) {
+    for (int j = threadIdx.x; j <= n_s; j += blockDim.x) {
+        const int32_t x = cu[s_a + j];
+        out[j] = (x < t0 ? t0 : x > t1 ? t1 : x) - t0;
+    }
+}
+}  // namespace
+
+size_t gdn_prefill_host_workspace_size(const gdn_config* cfg, int64_t T_total, int32_t n_seqs) {
+    if (check_config(cfg) != GDN_OK || T_total < 0 || n_seqs < 0) return 0;
+    return host_layout(cfg, T_total, n_seqs).total;
+}
+
+gdn_status gdn_prefill_host(const gdn_config* cfg, const gdn_weights* w, const void* q, const void* k,
+                            const void* v, const void* a, const void* b, const void* z, void* conv_state,
+                            void* rec_state, const int32_t* cu_seqlens, int32_t n_seqs, int64_t T_total,
+                            void* out, void* workspace, size_t workspace_bytes, void* stream) {
+    gdn_status s = check_config(cfg);
+    if (s != GDN_OK) return s;
+    if ((s = check_weights(w)) != GDN_OK) return s;
+    if (n_seqs < 0 || T_total < 0) return GDN_ERR_INVALID_ARG;
+    if (T_total == 0 || n_seqs == 0) return GDN_OK;
+    if (!q || !k || !v || !a || !b || !z || !conv_state || !rec_state || !cu_seqlens || !out || !workspace)
+        return GDN_ERR_INVALID_ARG;
+    if (!aligned(rec_state, 16) || !aligned(workspace, 256)) return GDN_ERR_INVALID_ARG;
+    if (T_total > 0x7fffffffLL - 64) return GDN_ERR_UNSUPPORTED;
+    // the sequence offsets are on the host: check them here
+    if (cu_seqlens[0] != 0 || cu_seqlens[n_seqs] != T_total) return GDN_ERR_INVALID_ARG;
+    for (int32_t i = 0; i < n_seqs; ++i)
+        if (cu_seqlens[i + 1] < cu_seqlens[i]) return GDN_ERR_INVALID_ARG;
+    const HostLayout L = host_layout(cfg, T_total, n_seqs);
+    if (workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaStream_t sin = side_stream(1), sout = side_stream(2);
+    if (!sin || !sout) return GDN_ERR_CUDA;
+    uint8_t* wsb = static_cast<uint8_t*>(workspace);
+    const void* hin[6] = {q, k, v, a, b, z};
+    const size_t state_bytes = (size_t)cfg->n_v_heads * cfg->d_v * cfg->d_k * (cfg->state_dtype == GDN_BF16 ? 2 : 4);
+    const size_t conv_bytes = (size_t)(2 * cfg->n_k_heads * cfg->d_k + cfg->n_v_heads * cfg->d_v) *
+                              (cfg->conv_kernel - 1) * (cfg->act_dtype == GDN_F32 ? 4 : 2);
+    const int n_seg = L.plan.n_seg;
+    std::vector<cudaEvent_t> ev;      // fork, then per segment: in_ready, computed, out_done
+    auto make = [&]() -> cudaEvent_t {
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+        ev.push_back(e);
+        return e;
+    };
+    gdn_status rc = GDN_OK;
+    auto cu_err = [&](cudaError_t e) {
+        if (e != cudaSuccess && rc == GDN_OK) rc = GDN_ERR_CUDA;
+        return e == cudaSuccess;
+    };
+    cudaEvent_t fork = make();
+    std::vector<cudaEvent_t> in_ready(n_seg), computed(n_seg), out_done(n_seg);
+    for (int i = 0; i < n_seg; ++i) {
+        in_ready[i] = make();
+        computed[i] = make();
+        out_done[i] = make();
+    }
+    bool ok = fork != nullptr;
+    for (int i = 0; ok && i < n_seg; ++i) ok = in_ready[i] && computed[i] && out_done[i];
+    if (!ok) rc = GDN_ERR_CUDA;
+    int32_t* cu_dev = reinterpret_cast<int32_t*>(wsb + L.cu_off);
+    if (rc == GDN_OK)
+        ok = cu_err(cudaMemcpyAsync(cu_dev, cu_seqlens, ((size_t)n_seqs + 1) * 4, cudaMemcpyHostToDevice, st)) &&
+             cu_err(cudaEventRecord(fork, st)) && cu_err(cudaStreamWaitEvent(sin, fork, 0)) &&
+             cu_err(cudaStreamWaitEvent(sout, fork, 0));
+    int32_t s_a = 0;
+    for (int i = 0; rc == GDN_OK && i < n_seg; ++i) {
+        const int slot = i & 1;
+        const int64_t t0 = (int64_t)i * L.plan.seg_len;
+        const int64_t t1 = std::min<int64_t>(T_total, t0 + L.plan.seg_len);
+        // sequences overlapping [t0, t1): from the one holding token t0 to the one holding t1 - 1
+        while (s_a + 1 < n_seqs && cu_seqlens[s_a + 1] <= t0) ++s_a;
+        int32_t s_b = s_a;
+        while (s_b + 1 < n_seqs && cu_seqlens[s_b + 1] < t1) ++s_b;
+        const int32_t n_s = s_b - s_a + 1;
+        uint8_t* slot_p = wsb + L.slot_off[slot];
+        // inputs in, once the segment two back has read this slot
+        if (i >= 2 && !cu_err(cudaStreamWaitEvent(sin, computed[i - 2], 0))) break;
+        for (int j = 0; j < 6; ++j)
+            if (!cu_err(cudaMemcpyAsync(slot_p + L.in_off[j], static_cast<const uint8_t*>(hin[j]) + t0 * L.row_in[j],
+                                        (size_t)(t1 - t0) * L.row_in[j], cudaMemcpyHostToDevice, sin)))
+                break;
+        if (rc != GDN_OK || !cu_err(cudaEventRecord(in_ready[i], sin))) break;
+        // the segment, once its inputs are in and the segment two back has sent its output out
+        if (!cu_err(cudaStreamWaitEvent(st, in_ready[i], 0))) break;
+        if (i >= 2 && !cu_err(cudaStreamWaitEvent(st, out_done[i - 2], 0))) break;
+        int32_t* seg_cu = reinterpret_cast<int32_t*>(wsb + L.seg_cu_off[slot]);
+        segment_seqlens_kernel<<<1, 256, 0, st>>>(cu_dev, s_a, n_s, (int32_t)t0, (int32_t)t1, seg_cu);
+        if (!cu_err(cudaGetLastError())) break;
+        const gdn_status g = gdn_prefill(
+            cfg, w, slot_p + L.in_off[0], slot_p + L.in_off[1], slot_p + L.in_off[2], slot_p + L.in_off[3],
+            slot_p + L.in_off[4], slot_p + L.in_off[5], static_cast<uint8_t*>(conv_state) + (size_t)s_a * conv_bytes,
+            static_cast<uint8_t*>(rec_state) + (size_t)s_a * state_bytes, seg_cu, n_s, t1 - t0, slot_p + L.out_off,
+            wsb + L.pre_off, L.cu_off - L.pre_off, st);
+        if (g != GDN_OK) {
+            rc = g;
+            break;
+        }
+        if (!cu_err(cudaEventRecord(computed[i], st))) break;
+        // the output out
+        if (!cu_err(cudaStreamWaitEvent(sout, computed[i], 0))) break;
+        if (!cu_err(cudaMemcpyAsync(static_cast<uint8_t*>(out) + t0 * L.row_out, slot_p + L.out_off,
+                                    (size_t)(t1 - t0) * L.row_out, cudaMemcpyDeviceToHost, sout)))
+            break;
+        if (!cu_err(cudaEventRecord(out_done[i], sout))) break;
+    }
+    // join: the caller's stream waits for the last output copy (the copy streams are in order)
+    if (rc == GDN_OK) cu_err(cudaStreamWaitEvent(st, out_done[n_seg - 1], 0));
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
+    return rc;
 }
 
 gdn_status gdn_check_device_error(void* stream) {

@@ -54,7 +54,8 @@ class _CWeights(ctypes.Structure):
 _lib = None
 EXPORTS = ("gdn_config_default", "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode",
            "gdn_decode_multi", "gdn_linear", "gdn_in_proj", "gdn_out_proj", "gdn_cp_workspace_size",
-           "gdn_cp_local", "gdn_cp_finish", "gdn_check_device_error", "gdn_status_string")
+           "gdn_cp_local", "gdn_cp_finish", "gdn_prefill_host_workspace_size", "gdn_prefill_host",
+           "gdn_check_device_error", "gdn_status_string")
 DECODE_MULTI_MAX_TOKENS = 16   # GDN_DECODE_MULTI_MAX_TOKENS
 LINEAR_MAX_SEGMENTS = 8        # GDN_LINEAR_MAX_SEGMENTS
 
@@ -90,6 +91,10 @@ def lib() -> ctypes.CDLL:
         L.gdn_cp_local.restype = ctypes.c_int
         L.gdn_cp_finish.argtypes = [vp, vp, vp, vp, i32, i32, vp, i64, vp, vp, vp, sz, vp]
         L.gdn_cp_finish.restype = ctypes.c_int
+        L.gdn_prefill_host_workspace_size.argtypes = [vp, i64, i32]
+        L.gdn_prefill_host_workspace_size.restype = sz
+        L.gdn_prefill_host.argtypes = [vp, vp] + [vp] * 8 + [vp, i32, i64, vp, vp, sz, vp]
+        L.gdn_prefill_host.restype = ctypes.c_int
         L.gdn_check_device_error.argtypes = [vp]
         L.gdn_check_device_error.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
@@ -365,13 +370,39 @@ def check_device_error(stream=None) -> None:
         raise GdnError(s, "device")
 
 
-def prefill_host(cfg: Config, w: dict, host: dict, conv_state, rec_state, stream=None):
-    """End-to-end prefill from host buffers: copies the step's inputs (pinned host
-    tensors q, k, v, a, b, z, cu_seqlens) to the device, runs the layer, and copies
-    ``out`` back into host['out'] (pinned).  States stay resident on the device."""
+def prefill_host_workspace_size(cfg: Config, T_total: int, n_seqs: int) -> int:
+    c = cfg.c()
+    return int(lib().gdn_prefill_host_workspace_size(ctypes.byref(c), T_total, n_seqs))
+
+
+def prefill_host(cfg: Config, w: dict, host: dict, conv_state, rec_state, workspace=None, stream=None):
+    """End-to-end prefill from host buffers through gdn_prefill_host: ``host`` holds CPU
+    tensors q, k, v, a, b, z (act dtype), cu_seqlens (int32) and out (out dtype), page-
+    locked for the copies to overlap the work.  The states stay on the device.  Returns
+    host['out'], complete once the stream is synchronised."""
     dev = rec_state.device
-    d = {n: host[n].to(dev, non_blocking=True) for n in ("q", "k", "v", "a", "b", "z", "cu_seqlens")}
-    out = prefill(cfg, w, d["q"], d["k"], d["v"], d["a"], d["b"], d["z"], conv_state, rec_state,
-                  d["cu_seqlens"], stream=stream)
-    host["out"].copy_(out, non_blocking=True)
+    q = host["q"]
+    T = q.shape[0]
+    cu = host["cu_seqlens"]
+    N = cu.shape[0] - 1
+    for n in ("q", "k", "v", "a", "b", "z", "cu_seqlens", "out"):
+        t = host[n]
+        if t.device.type != "cpu" or not t.is_contiguous():
+            raise ValueError("host[%r] must be a contiguous CPU tensor" % n)
+    for n in ("q", "k", "v", "a", "b", "z"):
+        if host[n].dtype != cfg.act_dtype:
+            raise TypeError("host[%r]: dtype %s, expected %s" % (n, host[n].dtype, cfg.act_dtype))
+    if cu.dtype != torch.int32 or host["out"].dtype != cfg.out_dtype:
+        raise TypeError("cu_seqlens must be int32 and out of the out dtype")
+    _check(conv_state, "conv_state", cfg.act_dtype, dev)
+    _check(rec_state, "rec_state", cfg.state_dtype, dev)
+    if workspace is None:
+        workspace = torch.empty(prefill_host_workspace_size(cfg, T, N), dtype=torch.uint8, device=dev)
+    c, cw = cfg.c(), _weights(w, dev)
+    s = lib().gdn_prefill_host(ctypes.byref(c), ctypes.byref(cw), _ptr(q), _ptr(host["k"]), _ptr(host["v"]),
+                               _ptr(host["a"]), _ptr(host["b"]), _ptr(host["z"]), _ptr(conv_state),
+                               _ptr(rec_state), _ptr(cu), N, T, _ptr(host["out"]), _ptr(workspace),
+                               workspace.numel(), _stream(stream))
+    if s != 0:
+        raise GdnError(s, "gdn_prefill_host")
     return host["out"]

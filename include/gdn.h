@@ -250,6 +250,31 @@ gdn_status gdn_cp_finish(const gdn_config* cfg, const gdn_weights* w, const void
                          const void* state_in, int64_t T_seg, void* out, void* state_out,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/*
+ * gdn_prefill from HOST buffers, end to end: the inputs come from the host, the
+ * result goes back to the host, and the transfers overlap the work.  The tokens
+ * are cut into at most 8 segments (multiples of 64 rows, at least 512); segment
+ * i runs on `stream` while segment i+1's inputs are copied in and segment i-1's
+ * output is copied out on two internal copy streams (one cudaMemcpyAsync per
+ * tensor and segment).  Sequences that cross a cut continue from the states the
+ * previous segment left, so the result is gdn_prefill's (up to where the chunk
+ * boundaries fall).
+ *   q, k, v, a, b, z, out: HOST pointers, same layouts as gdn_prefill (page-locked
+ *     memory lets the copies overlap; pageable memory is correct but serialises)
+ *   cu_seqlens: HOST [n_seqs+1], 0 = cu[0] <= ... <= cu[n_seqs] = T_total (checked)
+ *   conv_state, rec_state, workspace: DEVICE, as for gdn_prefill; workspace of
+ *     gdn_prefill_host_workspace_size bytes, 256-byte aligned
+ * When the call returns, the work is queued on `stream`; synchronising `stream`
+ * waits for the last output copy too.
+ */
+size_t gdn_prefill_host_workspace_size(const gdn_config* cfg, int64_t T_total, int32_t n_seqs);
+gdn_status gdn_prefill_host(const gdn_config* cfg, const gdn_weights* w,
+                            const void* q, const void* k, const void* v,
+                            const void* a, const void* b, const void* z,
+                            void* conv_state, void* rec_state, const int32_t* cu_seqlens,
+                            int32_t n_seqs, int64_t T_total, void* out,
+                            void* workspace, size_t workspace_bytes, void* stream);
+
 /* Capacity, in bytes, of the fixed scratch array used by gdn_prefill_noalloc. */
 #define GDN_NOALLOC_SCRATCH_BYTES ((size_t)64 << 20)
 

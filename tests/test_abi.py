@@ -157,6 +157,25 @@ def test_cp_argument_errors(lib):
     assert fin(2, 1, ws=1024) == WORKSPACE
 
 
+def test_prefill_host_argument_errors(lib):
+    """gdn_prefill_host reads cu_seqlens on the host: bad offsets are refused before any launch."""
+    P = ctypes.c_void_p
+    cw = gdn._CWeights(0x2000, 0x3000, 0x4000, 0x5000)
+    c = gdn.Config().c()
+    size = lib.gdn_prefill_host_workspace_size(ctypes.byref(c), 4096, 2)
+    assert size > gdn.workspace_size(gdn.Config(), 512, 2)
+
+    def call(cu, T, ws=1 << 40):
+        arr = (ctypes.c_int32 * len(cu))(*cu)
+        return lib.gdn_prefill_host(ctypes.byref(c), ctypes.byref(cw), *[P(0x1000)] * 6, P(0x6000), P(0x7000),
+                                    arr, len(cu) - 1, T, P(0x8000), P(0x100000), ws, None)
+    assert call([1, 10, 20], 20) == INVALID          # does not start at 0
+    assert call([0, 12, 10], 10) == INVALID          # decreasing
+    assert call([0, 10, 20], 21) == INVALID          # does not end at T
+    assert call([0, 10, 20], 20, ws=4096) == WORKSPACE
+    assert call([0], 0) == OK                        # nothing to do
+
+
 def test_status_strings(lib):
     for s in range(6):
         assert gdn.status_string(s)
