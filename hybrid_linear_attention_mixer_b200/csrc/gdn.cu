@@ -221,12 +221,13 @@ bool z_rows_map(CUtensorMap* m, const void* base, bool bf16, int width, int dv, 
 
 // Non-blocking streams per device for work that may overlap the caller's stream
 // (forked from and joined back to it by events): 0 = the context-parallel
-// transition scan, 1 = host-to-device copies, 2 = device-to-host copies.
+// transition scan, 1 = host-to-device copies, 2 = device-to-host copies,
+// 3 = the prefill's small side kernels (chunk offsets, conv-state update).
 cudaStream_t side_stream(int which = 0) {
-    static cudaStream_t streams[64][3];
+    static cudaStream_t streams[64][4];
     static std::mutex mu;
     int dev = 0;
-    if (which < 0 || which > 2 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (which < 0 || which > 3 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
     std::lock_guard<std::mutex> lock(mu);
     if (!streams[dev][which] && cudaStreamCreateWithFlags(&streams[dev][which], cudaStreamNonBlocking) != cudaSuccess)
         streams[dev][which] = nullptr;
@@ -400,10 +401,16 @@ gdn_status run_linear(const void* x, const void* w, int64_t M, int32_t N, int32_
 //   stage B: the chunk scan from rec_state (in/out), then the gated norm into out
 // Set-up first: nothing is launched unless the tensor maps encode and the
 // kernels' shared-memory opt-ins succeed.
+// Stage A keeps its two small kernels off the critical path: the chunk offsets
+// (which need only cu) run on a side stream beside the conv, and the conv-state
+// update (which must follow the conv's reads of the old state) beside the intra
+// kernel.  *join receives an event recorded after the side work; the caller's
+// stream waits on it before the call ends, and the caller destroys it.
 template <typename TA>
 cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void* q, const void* k, const void* v,
                            const void* a, const void* b, void* conv_state, const int32_t* cu, int n_seqs,
-                           int64_t T, void* ws, cudaStream_t st) {
+                           int64_t T, void* ws, cudaStream_t st, cudaEvent_t* join) {
+    *join = nullptr;
     const Layout L = workspace_layout(c, T, n_seqs);
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     ConvArgs ca;
@@ -445,6 +452,25 @@ cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void
         e = ensure_smem(k_conv, 12 + (c->d_k == 32 ? 0 : c->d_k == 64 ? 1 : 2), gdn::ctile::SMEM_BYTES);
         if (e != cudaSuccess) return e;
     }
+    cudaStream_t aux = side_stream(3);
+    if (!aux) return cudaErrorNotReady;
+    cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};   // start, offsets done, conv done, join
+    for (cudaEvent_t& x : ev)
+        if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming)) != cudaSuccess) {
+            for (cudaEvent_t y : ev)
+                if (y) cudaEventDestroy(y);
+            return e;
+        }
+    auto done = [&](cudaError_t r) {
+        for (int i = 0; i < 3; ++i) cudaEventDestroy(ev[i]);
+        if (r == cudaSuccess) *join = ev[3];
+        else cudaEventDestroy(ev[3]);
+        return r;
+    };
+    if ((e = cudaEventRecord(ev[0], st)) != cudaSuccess || (e = cudaStreamWaitEvent(aux, ev[0], 0)) != cudaSuccess)
+        return done(e);
+    gdn::intra::chunk_offsets_kernel<<<1, 1024, 0, aux>>>(cu, n_seqs, chunk_off);
+    if ((e = cudaEventRecord(ev[1], aux)) != cudaSuccess) return done(e);
     if (tiled) {
         const int n_slices = Ctot / gdn::ctile::CH;
         const int64_t n_tiles = (T + gdn::ctile::TOK - 1) / gdn::ctile::TOK;
@@ -455,8 +481,11 @@ cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void
     } else {
         gdn::conv_silu_norm_kernel<TA><<<dim3((unsigned)tblocks, cblocks), gdn::kConvThreads, 0, st>>>(ca);
     }
-    gdn::conv_state_update_kernel<TA><<<dim3(n_seqs, (Ctot + 255) / 256), 256, 0, st>>>(ca, conv_state);
-    gdn::intra::chunk_offsets_kernel<<<1, 1024, 0, st>>>(cu, n_seqs, chunk_off);
+    if ((e = cudaEventRecord(ev[2], st)) != cudaSuccess || (e = cudaStreamWaitEvent(aux, ev[2], 0)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(st, ev[1], 0)) != cudaSuccess)
+        return done(e);
+    gdn::conv_state_update_kernel<TA><<<dim3(n_seqs, (Ctot + 255) / 256), 256, 0, aux>>>(ca, conv_state);
+    if ((e = cudaEventRecord(ev[3], aux)) != cudaSuccess) return done(e);
 
     gdn::intra::Args ia;
     ia.a = a; ia.b = b;
@@ -465,7 +494,15 @@ cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void
     ia.Hk = Hk; ia.Hv = Hv;
     ia.rec = recs;
     k_intra<<<(unsigned)(max_chunks * Hv), gdn::intra::NT, gdn::intra::SMEM_BYTES, st>>>(tm_q, tm_k, ia);
-    return cudaGetLastError();
+    return done(cudaGetLastError());
+}
+
+// The caller's stream waits for stage A's side work, and the event is released.
+cudaError_t join_side(cudaEvent_t join, cudaStream_t st, cudaError_t prior) {
+    if (!join) return prior;
+    const cudaError_t e = cudaStreamWaitEvent(st, join, 0);
+    cudaEventDestroy(join);
+    return prior != cudaSuccess ? prior : e;
 }
 
 // The chunk scan over the records of stage A, reading V through `v_src` (the
@@ -524,11 +561,11 @@ cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void
                            void* rec_state, const int32_t* cu, int n_seqs, int64_t T, void* out,
                            void* ws, cudaStream_t st) {
     const Layout L = workspace_layout(c, T, n_seqs);
-    cudaError_t e = launch_stage_a<TA>(c, w, q, k, v, a, b, conv_state, cu, n_seqs, T, ws, st);
-    if (e != cudaSuccess) return e;
-    e = launch_scan<TO>(c, static_cast<uint8_t*>(ws) + L.v_off, T, rec_state, cu, n_seqs, T, ws, st);
-    if (e != cudaSuccess) return e;
-    return launch_norm<TA, TO>(c, w, z, cu, n_seqs, T, out, ws, st);
+    cudaEvent_t join = nullptr;
+    cudaError_t e = launch_stage_a<TA>(c, w, q, k, v, a, b, conv_state, cu, n_seqs, T, ws, st, &join);
+    if (e == cudaSuccess) e = launch_scan<TO>(c, static_cast<uint8_t*>(ws) + L.v_off, T, rec_state, cu, n_seqs, T, ws, st);
+    if (e == cudaSuccess) e = launch_norm<TA, TO>(c, w, z, cu, n_seqs, T, out, ws, st);
+    return join_side(join, st, e);
 }
 
 template <typename TA, typename TO, typename TS, int DK>
@@ -781,9 +818,12 @@ gdn_status gdn_cp_local(const gdn_config* cfg, const gdn_weights* w, const void*
     float* S_loc = P + (size_t)Hv * d * d;
     const bool abf = cfg->act_dtype == GDN_BF16, obf = cfg->out_dtype == GDN_BF16;
     gdn::cp::segment_cu_kernel<<<1, 32, 0, st>>>(cu, (int32_t)T_seg);
-    cudaError_t e = abf ? launch_stage_a<__nv_bfloat16>(cfg, w, q, k, v, a, b, conv_state, cu, 1, T_seg, workspace, st)
-                        : launch_stage_a<float>(cfg, w, q, k, v, a, b, conv_state, cu, 1, T_seg, workspace, st);
-    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    cudaEvent_t side_join = nullptr;
+    cudaError_t e = abf ? launch_stage_a<__nv_bfloat16>(cfg, w, q, k, v, a, b, conv_state, cu, 1, T_seg, workspace, st,
+                                                        &side_join)
+                        : launch_stage_a<float>(cfg, w, q, k, v, a, b, conv_state, cu, 1, T_seg, workspace, st,
+                                                &side_join);
+    if ((e = join_side(side_join, st, e)) != cudaSuccess) return GDN_ERR_CUDA;
     // starting states: S_loc from zero, P from I; V = 0 for P: a zero block of 64
     // rows whose map reads zeros past it
     if ((e = cudaMemsetAsync(S_loc, 0, (size_t)Hv * d * d * sizeof(float), st)) != cudaSuccess) return GDN_ERR_CUDA;
