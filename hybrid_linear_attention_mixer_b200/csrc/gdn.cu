@@ -234,6 +234,35 @@ cudaStream_t side_stream(int which = 0) {
     return streams[dev][which];
 }
 
+// Events for the forks and joins above, kept per host thread, device and use and
+// reused from call to call: a stream wait refers to the record enqueued before
+// it, so recording an event again in a later call leaves earlier waits intact,
+// and no two threads share an event.
+enum EventUse { kEvStageA = 0, kEvCp = 1, kEvHost = 2, kEvUses = 3 };
+
+struct EventPool {
+    std::vector<cudaEvent_t> ev[64][kEvUses];
+    ~EventPool() {
+        for (auto& per_dev : ev)
+            for (auto& v : per_dev)
+                for (cudaEvent_t e : v) cudaEventDestroy(e);
+    }
+};
+
+// n events of the given use for this thread on the current device, or nullptr.
+cudaEvent_t* thread_events(EventUse use, size_t n) {
+    thread_local EventPool pool;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    std::vector<cudaEvent_t>& v = pool.ev[dev][use];
+    while (v.size() < n) {
+        cudaEvent_t e = nullptr;
+        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+        v.push_back(e);
+    }
+    return v.data();
+}
+
 // Streaming multiprocessors of the current device (cached per device).
 int sm_count() {
     static int count[64];
@@ -453,18 +482,10 @@ cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void
         if (e != cudaSuccess) return e;
     }
     cudaStream_t aux = side_stream(3);
-    if (!aux) return cudaErrorNotReady;
-    cudaEvent_t ev[4] = {nullptr, nullptr, nullptr, nullptr};   // start, offsets done, conv done, join
-    for (cudaEvent_t& x : ev)
-        if ((e = cudaEventCreateWithFlags(&x, cudaEventDisableTiming)) != cudaSuccess) {
-            for (cudaEvent_t y : ev)
-                if (y) cudaEventDestroy(y);
-            return e;
-        }
+    cudaEvent_t* ev = thread_events(kEvStageA, 4);   // start, offsets done, conv done, join
+    if (!aux || !ev) return cudaErrorNotReady;
     auto done = [&](cudaError_t r) {
-        for (int i = 0; i < 3; ++i) cudaEventDestroy(ev[i]);
         if (r == cudaSuccess) *join = ev[3];
-        else cudaEventDestroy(ev[3]);
         return r;
     };
     if ((e = cudaEventRecord(ev[0], st)) != cudaSuccess || (e = cudaStreamWaitEvent(aux, ev[0], 0)) != cudaSuccess)
@@ -497,11 +518,10 @@ cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void
     return done(cudaGetLastError());
 }
 
-// The caller's stream waits for stage A's side work, and the event is released.
+// The caller's stream waits for stage A's side work.
 cudaError_t join_side(cudaEvent_t join, cudaStream_t st, cudaError_t prior) {
     if (!join) return prior;
     const cudaError_t e = cudaStreamWaitEvent(st, join, 0);
-    cudaEventDestroy(join);
     return prior != cudaSuccess ? prior : e;
 }
 
@@ -834,13 +854,9 @@ gdn_status gdn_cp_local(const gdn_config* cfg, const gdn_weights* w, const void*
     // each: the transition's runs on a side stream, forked from and joined back
     // to the caller's stream by events.
     cudaStream_t side = side_stream(0);
-    if (!side) return GDN_ERR_CUDA;
-    cudaEvent_t fork = nullptr, join = nullptr;
-    if (cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess ||
-        cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
-        if (fork) cudaEventDestroy(fork);
-        return GDN_ERR_CUDA;
-    }
+    cudaEvent_t* fj = thread_events(kEvCp, 2);
+    if (!side || !fj) return GDN_ERR_CUDA;
+    cudaEvent_t fork = fj[0], join = fj[1];
     cudaError_t e2 = cudaEventRecord(fork, st);
     if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(side, fork, 0);
     if (e2 == cudaSuccess)
@@ -853,8 +869,6 @@ gdn_status gdn_cp_local(const gdn_config* cfg, const gdn_weights* w, const void*
     e = obf ? launch_scan<__nv_bfloat16>(cfg, vh, T_seg, S_loc, cu, 1, T_seg, workspace, st)
             : launch_scan<float>(cfg, vh, T_seg, S_loc, cu, 1, T_seg, workspace, st);
     if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, join, 0);
-    cudaEventDestroy(fork);
-    cudaEventDestroy(join);
     return e == cudaSuccess && e2 == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
 }
 
@@ -938,33 +952,23 @@ gdn_status gdn_prefill_host(const gdn_config* cfg, const gdn_weights* w, const v
     const size_t conv_bytes = (size_t)(2 * cfg->n_k_heads * cfg->d_k + cfg->n_v_heads * cfg->d_v) *
                               (cfg->conv_kernel - 1) * (cfg->act_dtype == GDN_F32 ? 4 : 2);
     const int n_seg = L.plan.n_seg;
-    std::vector<cudaEvent_t> ev;      // fork, then per segment: in_ready, computed, out_done
-    auto make = [&]() -> cudaEvent_t {
-        cudaEvent_t e = nullptr;
-        if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return nullptr;
-        ev.push_back(e);
-        return e;
-    };
+    // fork, then per segment: in_ready, computed, out_done
+    cudaEvent_t* ev = thread_events(kEvHost, 1 + 3 * (size_t)n_seg);
+    if (!ev) return GDN_ERR_CUDA;
     gdn_status rc = GDN_OK;
     auto cu_err = [&](cudaError_t e) {
         if (e != cudaSuccess && rc == GDN_OK) rc = GDN_ERR_CUDA;
         return e == cudaSuccess;
     };
-    cudaEvent_t fork = make();
-    std::vector<cudaEvent_t> in_ready(n_seg), computed(n_seg), out_done(n_seg);
-    for (int i = 0; i < n_seg; ++i) {
-        in_ready[i] = make();
-        computed[i] = make();
-        out_done[i] = make();
-    }
-    bool ok = fork != nullptr;
-    for (int i = 0; ok && i < n_seg; ++i) ok = in_ready[i] && computed[i] && out_done[i];
-    if (!ok) rc = GDN_ERR_CUDA;
+    cudaEvent_t fork = ev[0];
+    cudaEvent_t* in_ready = ev + 1;
+    cudaEvent_t* computed = ev + 1 + n_seg;
+    cudaEvent_t* out_done = ev + 1 + 2 * n_seg;
     int32_t* cu_dev = reinterpret_cast<int32_t*>(wsb + L.cu_off);
-    if (rc == GDN_OK)
-        ok = cu_err(cudaMemcpyAsync(cu_dev, cu_seqlens, ((size_t)n_seqs + 1) * 4, cudaMemcpyHostToDevice, st)) &&
-             cu_err(cudaEventRecord(fork, st)) && cu_err(cudaStreamWaitEvent(sin, fork, 0)) &&
-             cu_err(cudaStreamWaitEvent(sout, fork, 0));
+    // (cu_err records the first failure in rc, which ends the loop below)
+    (void)(cu_err(cudaMemcpyAsync(cu_dev, cu_seqlens, ((size_t)n_seqs + 1) * 4, cudaMemcpyHostToDevice, st)) &&
+           cu_err(cudaEventRecord(fork, st)) && cu_err(cudaStreamWaitEvent(sin, fork, 0)) &&
+           cu_err(cudaStreamWaitEvent(sout, fork, 0)));
     int32_t s_a = 0;
     for (int i = 0; rc == GDN_OK && i < n_seg; ++i) {
         const int slot = i & 1;
@@ -1008,7 +1012,6 @@ gdn_status gdn_prefill_host(const gdn_config* cfg, const gdn_weights* w, const v
     }
     // join: the caller's stream waits for the last output copy (the copy streams are in order)
     if (rc == GDN_OK) cu_err(cudaStreamWaitEvent(st, out_done[n_seg - 1], 0));
-    for (cudaEvent_t e : ev) cudaEventDestroy(e);
     return rc;
 }
 
