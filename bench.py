@@ -39,6 +39,10 @@ C_CONV = 2 * H_K * D + H_V * D
 # Algorithmic work:
 #   prefill dense FLOPs per token: H_k * 4*C*d + H_v * (6*C*d + 6*d^2), C = 64
 PREFILL_FLOP_PER_TOKEN = H_K * 4 * 64 * D + H_V * (6 * 64 * D + 6 * D * D)
+#   prefill bytes per call: q, k, v, z, a, b in and out, bf16, per token; the fp32 state read and
+#   written once (at 168 FLOP/byte the call sits below the bf16 ridge: it is bound by these bytes)
+PREFILL_BYTES_PER_TOKEN = (2 * H_K * D + 2 * H_V * D + 2 * H_V) * 2 + H_V * D * 2
+PREFILL_STATE_BYTES = 2 * H_V * D * D * 4
 #   decode bytes per step: fp32 state read + write, conv state read + write,
 #   q/k/v/a/b/z in, out, parameters
 DECODE_BYTES_PER_STEP = (2 * DECODE_N * H_V * D * D * 4 + 2 * DECODE_N * C_CONV * 3 * 2
@@ -422,6 +426,7 @@ def main():
         dec_launch_s = dec_ms / 1e3 / (K * args.decode_steps)
         dec_gbs = DECODE_BYTES_PER_STEP / dec_launch_s / 1e9
         pre_tflops = PREFILL_FLOP_PER_TOKEN * PREFILL_T / (pre_ms / 1e3 / K) / 1e12
+        pre_gbs = (PREFILL_BYTES_PER_TOKEN * PREFILL_T + PREFILL_STATE_BYTES) / (pre_ms / 1e3 / K) / 1e9
         traffic = DECODE_TRAFFIC if DECODE_SRC_SHA == src_sha("decode.cuh") else None
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -463,9 +468,12 @@ def main():
             "roofline": {"kernel": "gdn_decode_kernel", "bound": "hbm", "achieved": dec_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / pk["hbm_gbs"],
                          "traffic": traffic, "peak_source": src},
-            "prefill_roofline": {"kernels": "whole prefill call (conv, conv state, chunk offsets, intra, scan, norm)", "bound": "tensor",
-                                 "achieved": pre_tflops, "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
-                                 "frac": pre_tflops / pk["bf16_tflops"], "peak_source": src},
+            "prefill_roofline": {"kernels": "whole prefill call (conv, conv state, chunk offsets, intra, scan, norm)",
+                                 "bound": "hbm", "achieved": pre_gbs, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                                 "frac": pre_gbs / pk["hbm_gbs"],
+                                 "bytes_per_call": PREFILL_BYTES_PER_TOKEN * PREFILL_T + PREFILL_STATE_BYTES,
+                                 "tensor_achieved_tflops": pre_tflops, "tensor_peak_tflops": pk["bf16_tflops"],
+                                 "tensor_frac": pre_tflops / pk["bf16_tflops"], "peak_source": src},
             "clocks": clocks.summary(),
             "e2e": {"value": PREFILL_T * world * K / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
