@@ -3,6 +3,7 @@
     python -m hybrid_linear_attention_mixer_b200.run_case --case prefill_4k --iters 2
     python -m hybrid_linear_attention_mixer_b200.run_case --case decode_256 --batch 64 --iters 3
     python -m hybrid_linear_attention_mixer_b200.run_case --proj --tokens 4096 --iters 1
+    python -m hybrid_linear_attention_mixer_b200.run_case --case decode_256 --batch 64 --multi 4 --state bf16
 
 A small, fixed-size target for profilers such as ncu: it builds the seeded
 inputs of the named workload, runs the layer `iters` times on cuda:0 and checks
@@ -31,6 +32,9 @@ def main():
     ap.add_argument("--iters", type=int, default=2)
     ap.add_argument("--tokens", type=int, default=None, help="shrink a prefill workload to T tokens")
     ap.add_argument("--batch", type=int, default=None, help="decode batch (sequences)")
+    ap.add_argument("--multi", type=int, default=0,
+                    help="decode: this many consecutive tokens per sequence in one gdn_decode_multi call")
+    ap.add_argument("--state", default="fp32", choices=("fp32", "bf16"), help="recurrent state storage")
     ap.add_argument("--proj", action="store_true",
                     help="run the input and output projections (hidden 2560) at --tokens instead")
     args = ap.parse_args()
@@ -48,19 +52,24 @@ def main():
         print("ok proj T=%d" % T)
         return
     if args.case == "decode_256":
-        c = inputs.make_case(args.case, n_seqs=args.batch, T=1)
+        c = inputs.make_case(args.case, n_seqs=args.batch, T=max(1, args.multi))
     else:
         c = inputs.make_case(args.case, T=args.tokens)
     act = torch.bfloat16 if c.bf16 else torch.float32
     cfg = gdn.Config(c.n_k_heads, c.n_v_heads, c.d_k, c.d_v, c.conv_kernel, 64, c.l2_eps, c.norm_eps,
-                     act, act)
+                     act, act, torch.bfloat16 if args.state == "bf16" else torch.float32)
     w = {n: torch.from_numpy(np.ascontiguousarray(c.weights[n])).to(dev)
          for n in ("conv_w", "A_log", "dt_bias", "norm_w")}
     d = {n: _act(c.acts[n], dev) for n in "qkvabz"}
     cs = _act(c.conv_state, dev)
-    rs = torch.from_numpy(c.rec_state).to(dev)
+    rs = torch.from_numpy(c.rec_state).to(dev).to(cfg.state_dtype)
+    if args.case == "decode_256" and args.multi > 0:
+        m = {n: _act(np.stack([st[n] for st in c.steps], axis=1).reshape(c.n_seqs * args.multi, -1), dev)
+             for n in "qkvabz"}
     for _ in range(args.iters):
-        if args.case == "decode_256":
+        if args.case == "decode_256" and args.multi > 0:
+            gdn.decode_multi(cfg, w, m["q"], m["k"], m["v"], m["a"], m["b"], m["z"], cs, rs, args.multi)
+        elif args.case == "decode_256":
             gdn.decode(cfg, w, d["q"], d["k"], d["v"], d["a"], d["b"], d["z"], cs, rs)
         else:
             cu = torch.from_numpy(c.cu_seqlens).to(dev)
