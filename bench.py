@@ -36,7 +36,7 @@ PREFILL_T = 4096
 DECODE_N = 256
 H_K, H_V, D = 16, 48, 128
 C_CONV = 2 * H_K * D + H_V * D
-# Algorithmic work:
+# Algorithmic work per unit:
 #   prefill dense FLOPs per token: H_k * 4*C*d + H_v * (6*C*d + 6*d^2), C = 64
 PREFILL_FLOP_PER_TOKEN = H_K * 4 * 64 * D + H_V * (6 * 64 * D + 6 * D * D)
 #   prefill bytes per call: q, k, v, z, a, b in and out, bf16, per token; the fp32 state read and
