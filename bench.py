@@ -398,6 +398,34 @@ def main():
     cp_s = timed(cp_step)
     gdn.check_device_error(stream)
 
+    # ---- packed variable-length (8 sequences) and long-context (1 x 262,144) prefills ----
+    # (one rank's replica each; timed at N = 1 only, where they add about a minute of set-up)
+    def prefill_block(name, seed):
+        c = inputs.make_case(name, seed=seed)
+        cfg_c = gdn.Config()
+        wc = {n: torch.from_numpy(c.weights[n]).to(dev) for n in ("conv_w", "A_log", "dt_bias", "norm_w")}
+        dc_ = {n: act(c.acts[n]).to(dev) for n in "qkvabz"}
+        del c.acts
+        N, T = c.n_seqs, c.T
+        cu = torch.from_numpy(c.cu_seqlens).to(dev)
+        cs = act(c.conv_state).to(dev)
+        rs = torch.zeros((N, H_V, D, D), dtype=torch.float32, device=dev)
+        out = torch.empty((T, H_V * D), dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(gdn.workspace_size(cfg_c, T, N), dtype=torch.uint8, device=dev)
+        sec = timed(lambda: gdn.prefill(cfg_c, wc, dc_["q"], dc_["k"], dc_["v"], dc_["a"], dc_["b"], dc_["z"], cs,
+                                        rs, cu, out=out, workspace=ws, stream=stream))
+        gdn.check_device_error(stream)
+        nbytes = PREFILL_BYTES_PER_TOKEN * T + N * PREFILL_STATE_BYTES
+        del dc_, out, ws
+        torch.cuda.empty_cache()
+        return {"workload": name, "tokens": T, "seqs": N, "seq_lens": np.diff(c.cu_seqlens).tolist(),
+                "us_per_call": sec * 1e6, "value": T / sec, "unit": "tokens/s", "bytes_per_call": nbytes,
+                "achieved_gbs": nbytes / sec / 1e9, "roofline_us": nbytes / (peaks()[0]["hbm_gbs"] * 1e3)}
+
+    long_blocks = None
+    if world == 1:
+        long_blocks = {"varlen_8": prefill_block("varlen_8", 2), "prefill_256k": prefill_block("prefill_256k", 4)}
+
     # ---- end to end through the public API with host buffers ----
     h_ws = torch.empty(gdn.prefill_host_workspace_size(cfg, PREFILL_T, 1), dtype=torch.uint8, device=dev)
     e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
@@ -465,6 +493,10 @@ def main():
                 "note": "one rank: phase 1 and phase 2 on one segment, no exchange"
                         if world == 1 else "NCCL all-gathers inside the timed call"},
             "prefill_ms": pre_ms / K,
+            "prefill_varlen_8": None if long_blocks is None else dict(
+                long_blocks["varlen_8"], frac=long_blocks["varlen_8"]["achieved_gbs"] / pk["hbm_gbs"]),
+            "prefill_256k": None if long_blocks is None else dict(
+                long_blocks["prefill_256k"], frac=long_blocks["prefill_256k"]["achieved_gbs"] / pk["hbm_gbs"]),
             "roofline": {"kernel": "gdn_decode_kernel", "bound": "hbm", "achieved": dec_gbs,
                          "peak": pk["hbm_gbs"], "unit": "GB/s", "frac": dec_gbs / pk["hbm_gbs"],
                          "traffic": traffic, "peak_source": src},

@@ -31,7 +31,21 @@ struct ConvArgs {
     __half* qh;              // [T][Cq]
     __half* kh;              // [T][Cq]
     __half* vh;              // [T][Cv]
+    int32_t* flags;          // per-call check word: bit 0 (malformed cu_seqlens) is read here,
+                             // bit 1 is set here when an output overflows fp16
 };
+
+// fp16 keeps values below 65520 in magnitude; larger ones round to infinity.
+constexpr float kHalfOverflow = 65520.f;
+
+// The range check's outcome: v outputs are checked by magnitude (vmax), q and k
+// rows by their squared norm, which must stay finite for the L2 norm.
+__device__ __forceinline__ void report_range(const ConvArgs& p, float vmax, bool qk_bad) {
+    if (!(vmax < kHalfOverflow) || qk_bad) {
+        atomicOr(p.flags, 2);
+        record_error(kErrRange);
+    }
+}
 
 constexpr int kConvThreads = 128;   // 8 channels per thread
 constexpr int kConvRun = 32;        // tokens per thread (one run per CTA)
@@ -76,6 +90,7 @@ template <> struct Raw8<float> {
 
 template <typename TA>
 __global__ void __launch_bounds__(kConvThreads, 4) conv_silu_norm_kernel(ConvArgs p) {
+    if (*p.flags) return;   // cu_seqlens failed its check: sequence starts are not to be trusted
     const int Cq = p.Hk * p.dk, Cv = p.Hv * p.dv, Ctot = 2 * Cq + Cv;
     const int c = (blockIdx.y * kConvThreads + threadIdx.x) * 8;   // first of 8 channels
     const int64_t t_begin = (int64_t)blockIdx.x * kConvRun;
@@ -142,6 +157,8 @@ __global__ void __launch_bounds__(kConvThreads, 4) conv_silu_norm_kernel(ConvArg
     }
 
     const int group = p.dk >> 3;                    // threads per key head (4, 8 or 16)
+    float vmax = 0.f;
+    bool qk_bad = false;
 #pragma unroll
     for (int it = 0; it < kConvRun; it++) {
         if (it >= n_run) break;
@@ -170,9 +187,13 @@ __global__ void __launch_bounds__(kConvThreads, 4) conv_silu_norm_kernel(ConvArg
         // sum of squares over the key head's `group` threads (aligned lane groups)
         for (int off = 1; off < group; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
         if (is_qk) {
+            qk_bad |= !(ss <= 3.4e38f);
             const float r = rsqrtf(ss + p.l2_eps);
 #pragma unroll
             for (int i = 0; i < 8; i++) y[i] *= r;
+        } else {
+#pragma unroll
+            for (int i = 0; i < 8; i++) vmax = fmaxf(vmax, fabsf(y[i]));
         }
         if (active) {
             uint4 o;
@@ -183,6 +204,7 @@ __global__ void __launch_bounds__(kConvThreads, 4) conv_silu_norm_kernel(ConvArg
             __stcs(reinterpret_cast<uint4*>(dst + t * ld), o);
         }
     }
+    if (active) report_range(p, vmax, qk_bad);
 }
 
 // Tiled form of the same pass for bf16 activations whose q, k and v widths are
@@ -209,7 +231,8 @@ constexpr uint32_t SMEM_BYTES = OFF_START + 2 * TOK * 8 + 128;
 template <int GROUP, bool PATCH>
 __device__ __forceinline__ void rows(const uint8_t* tb, const float (&w)[8][4], uint32_t near, int n_here,
                                      int64_t t0, const int* sq, const long long* sst, const __nv_bfloat16* cst,
-                                     int64_t seq_stride, __half* out, int64_t ld, bool is_qk, float l2_eps) {
+                                     int64_t seq_stride, __half* out, int64_t ld, bool is_qk, float l2_eps,
+                                     float& vmax, bool& qk_bad) {
     auto row = [&](int r, float (&f)[8]) {
         const uint4 u = *reinterpret_cast<const uint4*>(tb + r * 128);
         const uint32_t v[4] = {u.x, u.y, u.z, u.w};
@@ -259,9 +282,13 @@ __device__ __forceinline__ void rows(const uint8_t* tb, const float (&w)[8][4], 
 #pragma unroll
         for (int off = 1; off < GROUP; off <<= 1) ss += __shfl_xor_sync(0xffffffffu, ss, off);
         if (is_qk) {
+            qk_bad |= !(ss <= 3.4e38f);
             const float r = rsqrtf(ss + l2_eps);
 #pragma unroll
             for (int e = 0; e < 8; e++) y[e] *= r;
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; e++) vmax = fmaxf(vmax, fabsf(y[e]));
         }
         uint4 o;
         o.x = pack_half2(y[0], y[1]);
@@ -300,7 +327,7 @@ conv_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     __half* dst0 = tensor == 0 ? p.qh : tensor == 1 ? p.kh : p.vh;
     const int64_t n_tiles = (p.T + TOK - 1) / TOK;
     const int count = part < n_tiles ? (int)((n_tiles - part + parts - 1) / parts) : 0;
-    if (count == 0) return;
+    if (count == 0 || *p.flags) return;   // (flags: cu_seqlens failed its check)
 
     const int tid = threadIdx.x, lane = tid & 31;
     const int tg = tid >> 6, cg = tid & 63;
@@ -346,6 +373,8 @@ conv_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     }
     __syncthreads();
 
+    float vmax = 0.f;
+    bool qk_bad = false;
     for (int jj = 0; jj < count; jj++) {
         if (!mbar_wait_bounded(bar0 + 8 * (jj % BUFS), (jj / BUFS) & 1)) atomicOr((unsigned*)s_abort, 1u);
         __syncthreads();   // every thread is done with tile jj - 1 (buffer, sequence table)
@@ -366,11 +395,12 @@ conv_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         const __nv_bfloat16* cst = static_cast<const __nv_bfloat16*>(p.conv_state) + (int64_t)c * 3;
         if (near)
             ctile::rows<GROUP, true>(tb + tg * 8 * 128, w, near, n_here, t0, sq, sst, cst, (int64_t)Ctot * 3, out, ld,
-                                     is_qk, p.l2_eps);
+                                     is_qk, p.l2_eps, vmax, qk_bad);
         else
             ctile::rows<GROUP, false>(tb + tg * 8 * 128, w, 0u, n_here, t0, sq, sst, cst, (int64_t)Ctot * 3, out, ld,
-                                      is_qk, p.l2_eps);
+                                      is_qk, p.l2_eps, vmax, qk_bad);
     }
+    report_range(p, vmax, qk_bad);
     if (*s_abort && tid == 0) {
         // a tile never arrived: report it and give the copies still in flight one more bounded wait
         record_error(kErrCopyTimeout);
@@ -381,20 +411,23 @@ conv_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
 
 // conv_state <- the last 3 raw inputs of each sequence (oldest first), keeping
 // old entries when the sequence is shorter than 3.  Runs after the conv kernel,
-// which still reads the old state.
+// which still reads the old state, and after the call's checks (*flags): a call
+// whose checks failed leaves conv_state as it was.  A sequence with cu[s+1] <
+// cu[s] (which the checks reject) would read no row outside [cu[s], cu[s+1]).
 template <typename TA>
 __global__ void __launch_bounds__(256) conv_state_update_kernel(ConvArgs p, void* conv_state) {
     const int Cq = p.Hk * p.dk, Cv = p.Hv * p.dv, Ctot = 2 * Cq + Cv;
     const int c = blockIdx.y * 256 + threadIdx.x;
     const int s = blockIdx.x;
-    if (c >= Ctot) return;
+    if (c >= Ctot || *p.flags) return;
     const int64_t t0 = p.cu[s], t1 = p.cu[s + 1];
+    if (t1 <= t0) return;
     TA* st = static_cast<TA*>(conv_state) + ((int64_t)s * Ctot + c) * 3;
     TA old[3] = {st[0], st[1], st[2]};
     TA nw[3];
 #pragma unroll
     for (int q = 0; q < 3; q++) {
-        const int64_t t = t1 - 3 + q;
+        const int64_t t = t1 - 3 + q;   // t >= t0 - 3 since t1 > t0
         nw[q] = (t >= t0) ? *conv_channel_ptr<TA>(p, t, c, Cq, Cv) : old[3 - (int)(t0 - t)];
     }
 #pragma unroll

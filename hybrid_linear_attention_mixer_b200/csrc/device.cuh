@@ -9,6 +9,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "gdn.h"
+
 namespace gdn {
 
 // ---------------------------------------------------------------------------
@@ -17,7 +19,10 @@ namespace gdn {
 // ---------------------------------------------------------------------------
 __device__ unsigned int g_device_error;
 
-enum : unsigned int { kErrMmaTimeout = 1u, kErrCopyTimeout = 2u };
+// Bits of the error word: a tensor-core commit or a copy that never arrived, a
+// malformed cu_seqlens found by the prefill's chunk-table kernel, and a conv
+// output outside the fp16 range of the prefill workspace.
+enum : unsigned int { kErrMmaTimeout = 1u, kErrCopyTimeout = 2u, kErrSeqlens = 4u, kErrRange = 8u };
 
 // A wait that has not completed after this long is treated as lost.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;   // 2 s
@@ -135,13 +140,14 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
         : "memory");
     return ok != 0;
 }
-// Waits for the phase with the given parity to complete, for at most
-// kWaitLimitNs.  Returns false if it gave up.
-__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity) {
+// Waits for the phase with the given parity to complete, for at most limit_ns
+// (kWaitLimitNs unless a caller asks for less).  Returns false if it gave up.
+__device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t parity,
+                                                  unsigned long long limit_ns = kWaitLimitNs) {
     if (mbar_try_wait(bar, parity)) return true;
     const unsigned long long t0 = global_ns();
     while (!mbar_try_wait(bar, parity)) {
-        if (global_ns() - t0 > kWaitLimitNs) return false;
+        if (global_ns() - t0 > limit_ns) return false;
     }
     return true;
 }
@@ -386,6 +392,33 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
         "tcgen05.wait::st.sync.aligned;" ::"r"(taddr),
         "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
         : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// Host side of the error word (of the module that includes this header).
+// ---------------------------------------------------------------------------
+// The status an error word stands for, most serious first: a wait that ran
+// out, then a malformed cu_seqlens, then a conv output beyond fp16.
+inline gdn_status status_of_error_word(unsigned int w) {
+    if (w & (kErrMmaTimeout | kErrCopyTimeout)) return GDN_ERR_DEVICE_TIMEOUT;
+    if (w & kErrSeqlens) return GDN_ERR_SEQLENS;
+    if (w & kErrRange) return GDN_ERR_RANGE;
+    return GDN_OK;
+}
+
+// Waits for `stream`, then reads and clears the error word: the status it
+// stands for, or GDN_ERR_CUDA if a CUDA call failed (that call's error in
+// *cuda_err when given).
+inline gdn_status take_device_error(cudaStream_t stream, cudaError_t* cuda_err = nullptr) {
+    cudaError_t e = cudaStreamSynchronize(stream);
+    unsigned int v = 0;
+    if (e == cudaSuccess) e = cudaMemcpyFromSymbol(&v, g_device_error, sizeof v);
+    if (e == cudaSuccess && v) {
+        const unsigned int zero = 0;
+        e = cudaMemcpyToSymbol(g_device_error, &zero, sizeof zero);
+    }
+    if (cuda_err) *cuda_err = e;
+    return e != cudaSuccess ? GDN_ERR_CUDA : status_of_error_word(v);
 }
 
 }  // namespace gdn

@@ -6,6 +6,7 @@
 
 #include <algorithm>
 #include <cmath>
+#include <cstdio>
 #include <cstring>
 #include <mutex>
 #include <vector>
@@ -27,6 +28,16 @@ bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) %
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 bool dim_ok(int d) { return d == 32 || d == 64 || d == 128; }
+
+// The CUDA error behind this thread's most recent GDN_ERR_CUDA (gdn_last_cuda_error).
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+// GDN_OK for cudaSuccess; otherwise remembers e for this thread and returns GDN_ERR_CUDA.
+gdn_status cuda_status(cudaError_t e) {
+    if (e == cudaSuccess) return GDN_OK;
+    t_last_cuda_error = e;
+    return GDN_ERR_CUDA;
+}
 
 gdn_status check_config(const gdn_config* c) {
     if (!c) return GDN_ERR_INVALID_ARG;
@@ -50,23 +61,25 @@ gdn_status check_weights(const gdn_weights* w) {
 }
 
 // Prefill workspace: fp16 q^, k^, v^ (conv output), the first chunk of each
-// sequence, one intra-chunk record per (chunk, value head), and the o tile
-// ([64][128], out dtype) of each (chunk, value head) before the gated norm.
+// sequence followed by the call's check word (flags), one intra-chunk record
+// per (chunk, value head), and the o tile ([64][128], out dtype) of each
+// (chunk, value head) before the gated norm.
 struct Layout {
-    size_t q_off, k_off, v_off, coff_off, rec_off, o_off, total;
+    size_t q_off, k_off, v_off, coff_off, flags_off, rec_off, o_off, total;
 };
 
 Layout workspace_layout(const gdn_config* c, int64_t T, int64_t n_seqs) {
     Layout L;
     const size_t qb = align_up((size_t)T * c->n_k_heads * c->d_k * sizeof(__half), 256);
     const size_t vb = align_up((size_t)T * c->n_v_heads * c->d_v * sizeof(__half), 256);
-    const size_t cb = align_up((size_t)(n_seqs + 1) * sizeof(int32_t), 256);
+    const size_t cb = align_up((size_t)(n_seqs + 2) * sizeof(int32_t), 256);
     const size_t max_chunks = (size_t)((T + gdn::intra::C - 1) / gdn::intra::C) + (size_t)n_seqs;
     const size_t o_tile = (size_t)gdn::intra::C * 128 * (c->out_dtype == GDN_F32 ? 4 : 2);
     L.q_off = 0;
     L.k_off = qb;
     L.v_off = 2 * qb;
     L.coff_off = 2 * qb + vb;
+    L.flags_off = L.coff_off + (size_t)(n_seqs + 1) * sizeof(int32_t);
     L.rec_off = L.coff_off + cb;
     L.o_off = L.rec_off + max_chunks * c->n_v_heads * gdn::intra::REC_BYTES;
     L.total = L.o_off + max_chunks * c->n_v_heads * o_tile;
@@ -160,7 +173,24 @@ cudaError_t ensure_smem(K kernel, int variant, size_t bytes) {
     return e;
 }
 
-// cuTensorMapEncodeTiled, fetched once from the driver through the runtime.
+// cuCtxGetCurrent, fetched once from the driver through the runtime.
+PFN_cuCtxGetCurrent_v4000 ctx_getter() {
+    static PFN_cuCtxGetCurrent_v4000 fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(f);
+    });
+    return fn;
+}
+
+// cuTensorMapEncodeTiled, fetched once from the driver through the runtime.  It
+// is a driver call and needs a current context, which a host thread that has
+// made no runtime call yet does not have: the current device's primary context
+// is made current first in that case.
 PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
     static std::once_flag once;
@@ -171,6 +201,13 @@ PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
             q == cudaDriverEntryPointSuccess)
             fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
     });
+    CUcontext ctx = nullptr;
+    auto get_ctx = ctx_getter();
+    if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS) return nullptr;
+    if (!ctx) {
+        int dev = 0;
+        if (cudaGetDevice(&dev) != cudaSuccess || cudaSetDevice(dev) != cudaSuccess) return nullptr;
+    }
     return fn;
 }
 
@@ -219,19 +256,28 @@ bool z_rows_map(CUtensorMap* m, const void* base, bool bf16, int width, int dv, 
                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Non-blocking streams per device for work that may overlap the caller's stream
-// (forked from and joined back to it by events): 0 = the context-parallel
-// transition scan, 1 = host-to-device copies, 2 = device-to-host copies,
-// 3 = the prefill's small side kernels (chunk offsets, conv-state update).
+// Non-blocking streams for work that may overlap the caller's stream (forked
+// from and joined back to it by events): 0 = the context-parallel transition
+// scan, 1 = host-to-device copies, 2 = device-to-host copies, 3 = the prefill's
+// conv-state update.  They are kept per host thread and device, like the events
+// below: a call in one thread never waits on another thread's side work, and a
+// thread that captures a CUDA graph records only its own side work.
+struct StreamPool {
+    cudaStream_t s[64][4] = {};
+    ~StreamPool() {
+        for (auto& per_dev : s)
+            for (cudaStream_t x : per_dev)
+                if (x) cudaStreamDestroy(x);
+    }
+};
+
 cudaStream_t side_stream(int which = 0) {
-    static cudaStream_t streams[64][4];
-    static std::mutex mu;
+    thread_local StreamPool pool;
     int dev = 0;
     if (which < 0 || which > 3 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-    std::lock_guard<std::mutex> lock(mu);
-    if (!streams[dev][which] && cudaStreamCreateWithFlags(&streams[dev][which], cudaStreamNonBlocking) != cudaSuccess)
-        streams[dev][which] = nullptr;
-    return streams[dev][which];
+    cudaStream_t& st = pool.s[dev][which];
+    if (!st && cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) st = nullptr;
+    return st;
 }
 
 // Events for the forks and joins above, kept per host thread, device and use and
@@ -415,26 +461,27 @@ gdn_status run_linear(const void* x, const void* w, int64_t M, int32_t N, int32_
             case 144: e = launch_linear_pair<144>(x, w, a, 30, st); break;
             default: e = launch_linear_pair<128>(x, w, a, 31, st); break;
         }
-        return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+        return cuda_status(e);
     }
     // one CTA per 128-row tile for short inputs (decode-sized batches)
     if (pick_bn(M, N, sm_count()) == 256) e = launch_linear<256>(x, w, a, 20, st);
     else e = launch_linear<128>(x, w, a, 24, st);
-    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    return cuda_status(e);
 }
 
 // Prefill, split in its two stages so that context-parallel prefill can run the
 // chunk scan more than once over one set of intra-chunk records.
-//   stage A: conv + SiLU + L2 norm into the workspace, conv-state update, chunk
-//            offsets, intra-chunk records
+//   stage A: chunk offsets and the check of cu_seqlens, conv + SiLU + L2 norm
+//            into the workspace, conv-state update, intra-chunk records
 //   stage B: the chunk scan from rec_state (in/out), then the gated norm into out
 // Set-up first: nothing is launched unless the tensor maps encode and the
 // kernels' shared-memory opt-ins succeed.
-// Stage A keeps its two small kernels off the critical path: the chunk offsets
-// (which need only cu) run on a side stream beside the conv, and the conv-state
-// update (which must follow the conv's reads of the old state) beside the intra
-// kernel.  *join receives an event recorded after the side work; the caller's
-// stream waits on it before the call ends, and the caller destroys it.
+// The chunk-offset kernel runs first: it checks cu_seqlens and writes the
+// call's check word, which every later kernel reads.  The conv-state update
+// (which must follow the conv's reads of the old state) runs on a side stream
+// beside the intra kernel.  Once the side stream has been forked, *join
+// receives an event recorded after its work, on every path, error paths
+// included; the caller's stream waits on it before the call ends.
 template <typename TA>
 cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void* q, const void* k, const void* v,
                            const void* a, const void* b, void* conv_state, const int32_t* cu, int n_seqs,
@@ -442,6 +489,7 @@ cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void
     *join = nullptr;
     const Layout L = workspace_layout(c, T, n_seqs);
     uint8_t* wsb = static_cast<uint8_t*>(ws);
+    int32_t* flags = reinterpret_cast<int32_t*>(wsb + L.flags_off);
     ConvArgs ca;
     ca.q = q; ca.k = k; ca.v = v;
     ca.conv_w = w->conv_weight;
@@ -454,6 +502,7 @@ cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void
     ca.qh = reinterpret_cast<__half*>(wsb + L.q_off);
     ca.kh = reinterpret_cast<__half*>(wsb + L.k_off);
     ca.vh = reinterpret_cast<__half*>(wsb + L.v_off);
+    ca.flags = flags;
     auto k_intra = gdn::intra::gdn_intra_kernel<TA>;
     cudaError_t e = ensure_smem(k_intra, 4 + (sizeof(TA) == 2 ? 0 : 1), gdn::intra::SMEM_BYTES);
     if (e != cudaSuccess) return e;
@@ -482,16 +531,10 @@ cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void
         if (e != cudaSuccess) return e;
     }
     cudaStream_t aux = side_stream(3);
-    cudaEvent_t* ev = thread_events(kEvStageA, 4);   // start, offsets done, conv done, join
+    cudaEvent_t* ev = thread_events(kEvStageA, 2);   // conv done (fork), side work done (join)
     if (!aux || !ev) return cudaErrorNotReady;
-    auto done = [&](cudaError_t r) {
-        if (r == cudaSuccess) *join = ev[3];
-        return r;
-    };
-    if ((e = cudaEventRecord(ev[0], st)) != cudaSuccess || (e = cudaStreamWaitEvent(aux, ev[0], 0)) != cudaSuccess)
-        return done(e);
-    gdn::intra::chunk_offsets_kernel<<<1, 1024, 0, aux>>>(cu, n_seqs, chunk_off);
-    if ((e = cudaEventRecord(ev[1], aux)) != cudaSuccess) return done(e);
+
+    gdn::intra::chunk_offsets_kernel<<<1, 1024, 0, st>>>(cu, n_seqs, T, max_chunks, chunk_off, flags);
     if (tiled) {
         const int n_slices = Ctot / gdn::ctile::CH;
         const int64_t n_tiles = (T + gdn::ctile::TOK - 1) / gdn::ctile::TOK;
@@ -502,20 +545,24 @@ cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void
     } else {
         gdn::conv_silu_norm_kernel<TA><<<dim3((unsigned)tblocks, cblocks), gdn::kConvThreads, 0, st>>>(ca);
     }
-    if ((e = cudaEventRecord(ev[2], st)) != cudaSuccess || (e = cudaStreamWaitEvent(aux, ev[2], 0)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(st, ev[1], 0)) != cudaSuccess)
-        return done(e);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(ev[0], st)) != cudaSuccess || (e = cudaStreamWaitEvent(aux, ev[0], 0)) != cudaSuccess)
+        return e;
+    // aux is forked: from here on it is joined back whatever happens
     gdn::conv_state_update_kernel<TA><<<dim3(n_seqs, (Ctot + 255) / 256), 256, 0, aux>>>(ca, conv_state);
-    if ((e = cudaEventRecord(ev[3], aux)) != cudaSuccess) return done(e);
+    const cudaError_t e_side = cudaGetLastError();
+    if ((e = cudaEventRecord(ev[1], aux)) != cudaSuccess) return e;
+    *join = ev[1];
+    if (e_side != cudaSuccess) return e_side;
 
     gdn::intra::Args ia;
     ia.a = a; ia.b = b;
     ia.A_log = w->A_log; ia.dt_bias = w->dt_bias;
-    ia.cu = cu; ia.chunk_off = chunk_off; ia.n_seqs = n_seqs;
+    ia.cu = cu; ia.chunk_off = chunk_off; ia.flags = flags; ia.n_seqs = n_seqs;
     ia.Hk = Hk; ia.Hv = Hv;
     ia.rec = recs;
     k_intra<<<(unsigned)(max_chunks * Hv), gdn::intra::NT, gdn::intra::SMEM_BYTES, st>>>(tm_q, tm_k, ia);
-    return done(cudaGetLastError());
+    return cudaGetLastError();
 }
 
 // The caller's stream waits for stage A's side work.
@@ -544,6 +591,7 @@ cudaError_t launch_scan(const gdn_config* c, const void* v_src, int64_t v_rows, 
     sa.rec_state = rec_state;
     sa.cu = cu;
     sa.chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off);
+    sa.flags = reinterpret_cast<int32_t*>(wsb + L.flags_off);
     sa.rec = wsb + L.rec_off;
     sa.o = o_dst ? o_dst : wsb + L.o_off;
     sa.Hk = c->n_k_heads; sa.Hv = c->n_v_heads; sa.dk = c->d_k; sa.dv = c->d_v;
@@ -567,6 +615,7 @@ cudaError_t launch_norm(const gdn_config* c, const gdn_weights* w, const void* z
     gdn::norm::Args na;
     na.o = wsb + L.o_off; na.norm_w = w->norm_weight;
     na.cu = cu; na.chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off); na.out = out;
+    na.flags = reinterpret_cast<int32_t*>(wsb + L.flags_off);
     na.n_seqs = n_seqs; na.Hv = Hv; na.dv = c->d_v; na.eps = c->norm_eps;
     int64_t norm_ctas = (int64_t)sm_count() * (232448 / (int64_t)gdn::norm::smem_bytes<TA, TO>());
     norm_ctas = norm_ctas < max_chunks * Hv ? norm_ctas : max_chunks * Hv;
@@ -699,7 +748,7 @@ gdn_status gdn_prefill(const gdn_config* cfg, const gdn_weights* w, const void* 
     else
         e = launch_prefill<float, float>(cfg, w, q, k, v, a, b, z, conv_state, rec_state, cu_seqlens, n_seqs,
                                          T_total, out, workspace, st);
-    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    return cuda_status(e);
 }
 
 gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w, const void* q, const void* k,
@@ -731,7 +780,7 @@ gdn_status gdn_decode(const gdn_config* cfg, const gdn_weights* w, const void* q
     else if (abf) e = launch_decode<__nv_bfloat16, float>(da, n_seqs, sbf, st);
     else if (obf) e = launch_decode<float, __nv_bfloat16>(da, n_seqs, sbf, st);
     else e = launch_decode<float, float>(da, n_seqs, sbf, st);
-    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    return cuda_status(e);
 }
 
 static_assert(gdn::dec::kMaxTok == GDN_DECODE_MULTI_MAX_TOKENS, "multi-token limit");
@@ -772,7 +821,7 @@ gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_weights* w, const v
     else if (abf) e = launch_decode_multi<__nv_bfloat16, float>(m, sbf, st);
     else if (obf) e = launch_decode_multi<float, __nv_bfloat16>(m, sbf, st);
     else e = launch_decode_multi<float, float>(m, sbf, st);
-    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    return cuda_status(e);
 }
 
 gdn_status gdn_linear(const void* x, const void* w, int64_t M, int32_t N, int32_t K, const gdn_out_segment* segs,
@@ -843,11 +892,11 @@ gdn_status gdn_cp_local(const gdn_config* cfg, const gdn_weights* w, const void*
                                                         &side_join)
                         : launch_stage_a<float>(cfg, w, q, k, v, a, b, conv_state, cu, 1, T_seg, workspace, st,
                                                 &side_join);
-    if ((e = join_side(side_join, st, e)) != cudaSuccess) return GDN_ERR_CUDA;
+    if ((e = join_side(side_join, st, e)) != cudaSuccess) return cuda_status(e);
     // starting states: S_loc from zero, P from I; V = 0 for P: a zero block of 64
     // rows whose map reads zeros past it
-    if ((e = cudaMemsetAsync(S_loc, 0, (size_t)Hv * d * d * sizeof(float), st)) != cudaSuccess) return GDN_ERR_CUDA;
-    if ((e = cudaMemsetAsync(wsb + L.zv_off, 0, L.total - L.zv_off, st)) != cudaSuccess) return GDN_ERR_CUDA;
+    if ((e = cudaMemsetAsync(S_loc, 0, (size_t)Hv * d * d * sizeof(float), st)) != cudaSuccess) return cuda_status(e);
+    if ((e = cudaMemsetAsync(wsb + L.zv_off, 0, L.total - L.zv_off, st)) != cudaSuccess) return cuda_status(e);
     gdn::cp::identity_kernel<<<(unsigned)std::max<int64_t>(1, std::min<int64_t>((int64_t)Hv * d * d / 256, 1024)), 256, 0,
                                st>>>(P, Hv, d);
     // The two scans read the same records and are independent, one CTA per head
@@ -855,7 +904,7 @@ gdn_status gdn_cp_local(const gdn_config* cfg, const gdn_weights* w, const void*
     // to the caller's stream by events.
     cudaStream_t side = side_stream(0);
     cudaEvent_t* fj = thread_events(kEvCp, 2);
-    if (!side || !fj) return GDN_ERR_CUDA;
+    if (!side || !fj) return cuda_status(cudaErrorNotReady);
     cudaEvent_t fork = fj[0], join = fj[1];
     cudaError_t e2 = cudaEventRecord(fork, st);
     if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(side, fork, 0);
@@ -869,7 +918,7 @@ gdn_status gdn_cp_local(const gdn_config* cfg, const gdn_weights* w, const void*
     e = obf ? launch_scan<__nv_bfloat16>(cfg, vh, T_seg, S_loc, cu, 1, T_seg, workspace, st)
             : launch_scan<float>(cfg, vh, T_seg, S_loc, cu, 1, T_seg, workspace, st);
     if (e2 == cudaSuccess) e2 = cudaStreamWaitEvent(st, join, 0);
-    return e == cudaSuccess && e2 == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    return cuda_status(e != cudaSuccess ? e : e2);
 }
 
 gdn_status gdn_cp_finish(const gdn_config* cfg, const gdn_weights* w, const void* z, const void* summaries,
@@ -897,12 +946,12 @@ gdn_status gdn_cp_finish(const gdn_config* cfg, const gdn_weights* w, const void
     const void* vh = wsb + L.pre.v_off;
     cudaError_t e = obf ? launch_scan<__nv_bfloat16>(cfg, vh, T_seg, state_out, cu, 1, T_seg, workspace, st)
                         : launch_scan<float>(cfg, vh, T_seg, state_out, cu, 1, T_seg, workspace, st);
-    if (e != cudaSuccess) return GDN_ERR_CUDA;
+    if (e != cudaSuccess) return cuda_status(e);
     if (abf && obf) e = launch_norm<__nv_bfloat16, __nv_bfloat16>(cfg, w, z, cu, 1, T_seg, out, workspace, st);
     else if (abf) e = launch_norm<__nv_bfloat16, float>(cfg, w, z, cu, 1, T_seg, out, workspace, st);
     else if (obf) e = launch_norm<float, __nv_bfloat16>(cfg, w, z, cu, 1, T_seg, out, workspace, st);
     else e = launch_norm<float, float>(cfg, w, z, cu, 1, T_seg, out, workspace, st);
-    return e == cudaSuccess ? GDN_OK : GDN_ERR_CUDA;
+    return cuda_status(e);
 }
 
 // ---------------------------------------------------------------------------
@@ -945,7 +994,7 @@ gdn_status gdn_prefill_host(const gdn_config* cfg, const gdn_weights* w, const v
     if (workspace_bytes < L.total) return GDN_ERR_WORKSPACE;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     cudaStream_t sin = side_stream(1), sout = side_stream(2);
-    if (!sin || !sout) return GDN_ERR_CUDA;
+    if (!sin || !sout) return cuda_status(cudaErrorNotReady);
     uint8_t* wsb = static_cast<uint8_t*>(workspace);
     const void* hin[6] = {q, k, v, a, b, z};
     const size_t state_bytes = (size_t)cfg->n_v_heads * cfg->d_v * cfg->d_k * (cfg->state_dtype == GDN_BF16 ? 2 : 4);
@@ -954,10 +1003,10 @@ gdn_status gdn_prefill_host(const gdn_config* cfg, const gdn_weights* w, const v
     const int n_seg = L.plan.n_seg;
     // fork, then per segment: in_ready, computed, out_done
     cudaEvent_t* ev = thread_events(kEvHost, 1 + 3 * (size_t)n_seg);
-    if (!ev) return GDN_ERR_CUDA;
+    if (!ev) return cuda_status(cudaErrorNotReady);
     gdn_status rc = GDN_OK;
     auto cu_err = [&](cudaError_t e) {
-        if (e != cudaSuccess && rc == GDN_OK) rc = GDN_ERR_CUDA;
+        if (e != cudaSuccess && rc == GDN_OK) rc = cuda_status(e);
         return e == cudaSuccess;
     };
     cudaEvent_t fork = ev[0];
@@ -1016,15 +1065,18 @@ gdn_status gdn_prefill_host(const gdn_config* cfg, const gdn_weights* w, const v
 }
 
 gdn_status gdn_check_device_error(void* stream) {
-    if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return GDN_ERR_CUDA;
-    unsigned int v = 0;
-    if (cudaMemcpyFromSymbol(&v, gdn::g_device_error, sizeof v) != cudaSuccess) return GDN_ERR_CUDA;
-    if (v) {
-        const unsigned int zero = 0;
-        if (cudaMemcpyToSymbol(gdn::g_device_error, &zero, sizeof zero) != cudaSuccess) return GDN_ERR_CUDA;
-        return GDN_ERR_DEVICE_TIMEOUT;
-    }
-    return GDN_OK;
+    cudaError_t e = cudaSuccess;
+    const gdn_status s = gdn::take_device_error(static_cast<cudaStream_t>(stream), &e);
+    if (e != cudaSuccess) cuda_status(e);
+    return s;
+}
+
+const char* gdn_last_cuda_error(void) {
+    thread_local char buf[256];
+    const cudaError_t e = t_last_cuda_error;
+    if (e == cudaSuccess) return "no CUDA error";
+    snprintf(buf, sizeof buf, "%s: %s", cudaGetErrorName(e), cudaGetErrorString(e));
+    return buf;
 }
 
 const char* gdn_status_string(gdn_status s) {
@@ -1035,6 +1087,8 @@ const char* gdn_status_string(gdn_status s) {
         case GDN_ERR_CUDA: return "CUDA error";
         case GDN_ERR_DEVICE_TIMEOUT: return "device wait timed out";
         case GDN_ERR_WORKSPACE: return "workspace too small";
+        case GDN_ERR_SEQLENS: return "cu_seqlens malformed (device check)";
+        case GDN_ERR_RANGE: return "conv output beyond the fp16 range of the workspace (device check)";
     }
     return "unknown status";
 }
@@ -1051,7 +1105,15 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[GDN_NOALLOC_SCRATCH_B
 
 namespace {
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[64];   // device address of g_noalloc_scratch, per device
+// Device address of g_noalloc_scratch per device, with the context it was
+// looked up in: a reset device gets a new context, and the address is looked
+// up again there.
+struct NoallocSlot {
+    CUcontext ctx;
+    void* addr;
+};
+NoallocSlot g_noalloc_slot[64];
+
 }  // namespace
 
 extern "C" gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const gdn_weights* w, const void* q,
@@ -1066,16 +1128,25 @@ extern "C" gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const gdn_weigh
     void* scratch = nullptr;
     if (T_total > 0 && n_seqs > 0) {
         int dev = 0;
-        if (cudaGetDevice(&dev) != cudaSuccess) return GDN_ERR_CUDA;
+        const cudaError_t ed = cudaGetDevice(&dev);
+        if (ed != cudaSuccess) return cuda_status(ed);
         if (dev < 0 || dev >= 64) return GDN_ERR_UNSUPPORTED;
+        auto get_ctx = ctx_getter();
+        CUcontext ctx = nullptr;   // null while this thread has no current context yet
+        if (!get_ctx || get_ctx(&ctx) != CUDA_SUCCESS) return cuda_status(cudaErrorInitializationError);
         std::lock_guard<std::mutex> lock(g_noalloc_mu);
-        if (!g_noalloc_addr[dev]) {
+        NoallocSlot& slot = g_noalloc_slot[dev];
+        if (!slot.addr || !ctx || slot.ctx != ctx) {
             // The array's name is a host-side stand-in; the kernels need its device address.
+            // The lookup also makes the device's context current, so it is read again after.
             void* p = nullptr;
-            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return GDN_ERR_CUDA;
-            g_noalloc_addr[dev] = p;
+            const cudaError_t es = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+            if (es != cudaSuccess || !p) return cuda_status(es != cudaSuccess ? es : cudaErrorInvalidSymbol);
+            if (get_ctx(&ctx) != CUDA_SUCCESS || !ctx) return cuda_status(cudaErrorInitializationError);
+            slot.ctx = ctx;
+            slot.addr = p;
         }
-        scratch = g_noalloc_addr[dev];
+        scratch = slot.addr;
     }
     return gdn_prefill(cfg, w, q, k, v, a, b, z, conv_state, rec_state, cu_seqlens, n_seqs, T_total, out,
                        scratch, GDN_NOALLOC_SCRATCH_BYTES, stream);

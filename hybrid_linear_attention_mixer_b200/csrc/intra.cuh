@@ -71,6 +71,7 @@ struct Args {
     const float* dt_bias;     // [Hv]
     const int32_t* cu;        // [N+1]
     const int32_t* chunk_off; // [N+1] first chunk of each sequence; chunk_off[N] = total
+    const int32_t* flags;     // nonzero: a device check failed, write nothing
     int n_seqs;
     int Hk, Hv;
     uint8_t* rec;             // [total chunks][Hv][REC_BYTES]
@@ -80,16 +81,28 @@ __device__ __forceinline__ void stg128(void* p, uint32_t x, uint32_t y, uint32_t
     *reinterpret_cast<uint4*>(p) = make_uint4(x, y, z, w);
 }
 
-// chunk_off[s] = sum_{i<s} ceil(len_i / C) (one CTA, any number of sequences)
-__global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int32_t* cu, int n_seqs, int32_t* chunk_off) {
+// chunk_off[s] = sum_{i<s} ceil(len_i / C) (one CTA, any number of sequences),
+// and the check of cu_seqlens that the host cannot make (it is device memory):
+// cu[0] = 0, non-decreasing, cu[N] = T_total, at most max_chunks chunks.  A
+// malformed cu sets bit 0 of *flags (every later kernel of the call then writes
+// nothing), zeroes the chunk table and records kErrSeqlens.  *flags is written
+// here on every call; the conv kernel may OR bit 1 into it afterwards.
+__global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int32_t* cu, int n_seqs, int64_t T_total,
+                                                             int64_t max_chunks, int32_t* chunk_off,
+                                                             int32_t* flags) {
     __shared__ int32_t s_sum[32];
-    __shared__ int32_t s_carry;
+    __shared__ long long s_carry;
     if (threadIdx.x == 0) s_carry = 0;
+    int bad = threadIdx.x == 0 && (cu[0] != 0 || (int64_t)cu[n_seqs] != T_total);
     __syncthreads();
     for (int base = 0; base < n_seqs; base += 1024) {
         const int s = base + threadIdx.x;
         int32_t v = 0;
-        if (s < n_seqs) v = (cu[s + 1] - cu[s] + C - 1) / C;
+        if (s < n_seqs) {
+            const int64_t len = (int64_t)cu[s + 1] - cu[s];   // 64-bit: any int32 pair subtracts safely
+            bad |= len < 0;
+            v = len > 0 ? (int32_t)((len + C - 1) / C) : 0;
+        }
         int32_t x = v;   // inclusive scan within the warp
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
@@ -109,12 +122,22 @@ __global__ void __launch_bounds__(1024) chunk_offsets_kernel(const int32_t* cu, 
         }
         __syncthreads();
         const int32_t warp_base = (threadIdx.x >> 5) ? s_sum[(threadIdx.x >> 5) - 1] : 0;
-        if (s < n_seqs) chunk_off[s] = s_carry + warp_base + x - v;
+        if (s < n_seqs) chunk_off[s] = (int32_t)(s_carry + warp_base + x - v);
         __syncthreads();
         if (threadIdx.x == 1023) s_carry += warp_base + x;
         __syncthreads();
     }
-    if (threadIdx.x == 0) chunk_off[n_seqs] = s_carry;
+    bad |= s_carry > max_chunks;
+    if (__syncthreads_or(bad)) {
+        for (int s = threadIdx.x; s <= n_seqs; s += 1024) chunk_off[s] = 0;
+        if (threadIdx.x == 0) {
+            *flags = 1;
+            record_error(kErrSeqlens);
+        }
+    } else if (threadIdx.x == 0) {
+        chunk_off[n_seqs] = (int32_t)s_carry;
+        *flags = 0;
+    }
 }
 
 // C = sgn * L R for n x n blocks (n = 16 or 32; rows 16-byte aligned), 1 x 4
@@ -171,7 +194,7 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int Hv = p.Hv;
     const int h = blockIdx.x % Hv;
     const int gc = blockIdx.x / Hv;
-    if (gc >= p.chunk_off[p.n_seqs]) return;
+    if (gc >= p.chunk_off[p.n_seqs] || *p.flags) return;
     int lo = 0, hi = p.n_seqs - 1;   // sequence of this chunk: last s with chunk_off[s] <= gc
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;

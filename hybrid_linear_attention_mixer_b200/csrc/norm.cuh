@@ -21,6 +21,7 @@ struct Args {
     const float* norm_w;        // [dv]
     const int32_t* cu;          // [N+1]
     const int32_t* chunk_off;   // [N+1]
+    const int32_t* flags;       // nonzero: a device check of the call failed, write nothing
     void* out;                  // [T][Hv][dv] out dtype
     int n_seqs, Hv, dv;
     float eps;
@@ -98,7 +99,7 @@ __global__ void __launch_bounds__(NT) gdn_gated_norm_kernel(const __grid_constan
         tma_load_2d(dst + O_BYTES, &tm_z, h * dv, (int)t0, bar);
     };
     const int count = (int)((n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
-    if (count <= 0) return;
+    if (count <= 0 || *p.flags) return;
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; i++) mbar_init(bar0 + 8 * i, 1);
         fence_mbar_init();

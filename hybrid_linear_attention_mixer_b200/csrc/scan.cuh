@@ -77,6 +77,7 @@ struct Args {
     void* rec_state;            // [N][Hv][dv][dk] state dtype (fp32 or bf16), in/out
     const int32_t* cu;          // [N+1]
     const int32_t* chunk_off;   // [N+1]
+    const int32_t* flags;       // nonzero: a device check of the call failed, write nothing
     const uint8_t* rec;         // intra-chunk records
     void* o;                    // [chunks][Hv][64][128] out dtype: o before the gated norm
     int Hk, Hv, dk, dv;
@@ -138,7 +139,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
     const int seq = blockIdx.x / Hv, h = blockIdx.x % Hv;
     const int64_t s0 = p.cu[seq], s1 = p.cu[seq + 1];
     const int nchunks = (int)((s1 - s0 + C - 1) / C);
-    if (nchunks <= 0) return;
+    if (nchunks <= 0 || *p.flags) return;
     const int64_t first = (int64_t)p.chunk_off[seq] * Hv + h;   // (chunk, head) index of chunk 0
     const uint8_t* rec0 = p.rec + first * intra::REC_BYTES;
     const int64_t rec_stride = (int64_t)Hv * intra::REC_BYTES;

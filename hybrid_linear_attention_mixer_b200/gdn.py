@@ -27,9 +27,15 @@ LIB_PATH = os.path.join(_HERE, "libgdn_b200.so")
 _DT = {torch.bfloat16: 0, torch.float32: 1}
 
 
+CUDA_ERROR = 3   # GDN_ERR_CUDA
+
+
 class GdnError(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__("%s: %s (status %d)" % (what, status_string(status), status))
+        msg = "%s: %s (status %d)" % (what, status_string(status), status)
+        if status == CUDA_ERROR:
+            msg += " [%s]" % lib().gdn_last_cuda_error().decode()
+        super().__init__(msg)
         self.status = status
 
 
@@ -55,7 +61,7 @@ _lib = None
 EXPORTS = ("gdn_config_default", "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode",
            "gdn_decode_multi", "gdn_linear", "gdn_in_proj", "gdn_out_proj", "gdn_cp_workspace_size",
            "gdn_cp_local", "gdn_cp_finish", "gdn_prefill_host_workspace_size", "gdn_prefill_host",
-           "gdn_check_device_error", "gdn_status_string")
+           "gdn_check_device_error", "gdn_status_string", "gdn_last_cuda_error")
 DECODE_MULTI_MAX_TOKENS = 16   # GDN_DECODE_MULTI_MAX_TOKENS
 LINEAR_MAX_SEGMENTS = 8        # GDN_LINEAR_MAX_SEGMENTS
 
@@ -99,6 +105,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_check_device_error.restype = ctypes.c_int
         L.gdn_status_string.argtypes = [ctypes.c_int]
         L.gdn_status_string.restype = ctypes.c_char_p
+        L.gdn_last_cuda_error.argtypes = []
+        L.gdn_last_cuda_error.restype = ctypes.c_char_p
         _lib = L
     return _lib
 
@@ -364,7 +372,9 @@ def cp_finish(cfg: Config, w: dict, z, summaries, rank: int, state_in, workspace
 
 
 def check_device_error(stream=None) -> None:
-    """Synchronise the stream and raise if a kernel's bounded wait ran out."""
+    """Synchronise the stream and raise GdnError if the device error word holds an
+    error: a bounded wait that ran out, or a failed device check of a prefill's
+    inputs (malformed cu_seqlens, conv output beyond fp16)."""
     s = lib().gdn_check_device_error(_stream(stream))
     if s != 0:
         raise GdnError(s, "device")

@@ -37,7 +37,10 @@
  *   - Argument errors are returned synchronously and launch nothing.  Launch
  *     failures return GDN_ERR_CUDA.  Kernels never trap: a bounded wait that
  *     runs out records a device error word and the kernel returns;
- *     gdn_check_device_error reports it as GDN_ERR_DEVICE_TIMEOUT.
+ *     gdn_check_device_error reports it as GDN_ERR_DEVICE_TIMEOUT.  Checks of
+ *     device-resident inputs (prefill's cu_seqlens, and the fp16 range of the
+ *     conv outputs it keeps in its workspace) report through the same word
+ *     (GDN_ERR_SEQLENS, GDN_ERR_RANGE).
  *   - No C++ exception crosses this interface.
  *
  * Supported shapes: d_k, d_v in {32, 64, 128}; n_v_heads a multiple of
@@ -60,7 +63,10 @@ typedef enum {
     GDN_ERR_UNSUPPORTED = 2,     /* shape or dtype outside the supported set     */
     GDN_ERR_CUDA = 3,            /* a CUDA launch or runtime call failed          */
     GDN_ERR_DEVICE_TIMEOUT = 4,  /* a kernel's bounded wait ran out               */
-    GDN_ERR_WORKSPACE = 5        /* workspace smaller than gdn_prefill_workspace_size */
+    GDN_ERR_WORKSPACE = 5,       /* workspace smaller than gdn_prefill_workspace_size */
+    GDN_ERR_SEQLENS = 6,         /* (device check) cu_seqlens malformed           */
+    GDN_ERR_RANGE = 7            /* (device check) a conv output beyond the fp16 range
+                                    of the prefill workspace                        */
 } gdn_status;
 
 typedef enum { GDN_BF16 = 0, GDN_F32 = 1 } gdn_dtype;
@@ -106,12 +112,20 @@ size_t gdn_prefill_workspace_size(const gdn_config* cfg, int64_t T_total, int32_
  *   conv_state  [n_seqs][2*H_k*d_k + H_v*d_v][K-1]  act_dtype, in/out, oldest first
  *   rec_state   [n_seqs][H_v][d_v][d_k] state_dtype (float32 by default), in/out
  *   cu_seqlens  [n_seqs + 1] int32 device, cu_seqlens[0] = 0, non-decreasing,
- *               cu_seqlens[n_seqs] = T_total (not checked on the host: it is
- *               device memory and reading it would synchronise)
+ *               cu_seqlens[n_seqs] = T_total.  It is device memory, so the host
+ *               cannot read it without synchronising: the first kernel checks it.
+ *               A malformed cu_seqlens records GDN_ERR_SEQLENS in the device
+ *               error word, and the call then writes neither out nor either
+ *               state (the workspace is scratch).
  *   out         [T_total][H_v][d_v]    out_dtype
  *   workspace   >= gdn_prefill_workspace_size(cfg, T_total, n_seqs) bytes,
  *               256-byte aligned; contents need not be initialised
  * Sequences of length 0 leave their states unchanged.  T_total == 0 is a no-op.
+ * Range: the conv outputs q^, k^, v^ are kept in fp16 in the workspace.  If a
+ * conv output lies beyond the fp16 range (|v^| > 65504, or a q or k row whose
+ * squared norm overflows fp32), the call records GDN_ERR_RANGE and likewise
+ * writes neither out nor either state.
+ * Both device checks are read by gdn_check_device_error.
  */
 gdn_status gdn_prefill(const gdn_config* cfg, const gdn_weights* w,
                        const void* q, const void* k, const void* v,
@@ -310,6 +324,10 @@ gdn_status gdn_prefill_host(const gdn_config* cfg, const gdn_weights* w,
  *   - Races: calls whose work overlaps on the GPU (different streams, no
  *     ordering between them) race on the array.  Order them on one stream, or
  *     with events.
+ *   - Device reset: the looked-up address belongs to the device's current
+ *     context.  The call remembers that context and looks the address up
+ *     again when a later call finds a different one (after cudaDeviceReset,
+ *     for instance).
  */
 gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const gdn_weights* w,
                                const void* q, const void* k, const void* v,
@@ -319,11 +337,18 @@ gdn_status gdn_prefill_noalloc(const gdn_config* cfg, const gdn_weights* w,
                                void* out, void* stream);
 
 /* Synchronises `stream`, then reads and clears the device error word that
- * bounded waits write.  GDN_OK, GDN_ERR_DEVICE_TIMEOUT or GDN_ERR_CUDA. */
+ * bounded waits and the prefill's device checks write.  GDN_OK, or the most
+ * serious error recorded since the last call: GDN_ERR_DEVICE_TIMEOUT, then
+ * GDN_ERR_SEQLENS, then GDN_ERR_RANGE; GDN_ERR_CUDA if a CUDA call failed. */
 gdn_status gdn_check_device_error(void* stream);
 
 /* Static string for a status code. */
 const char* gdn_status_string(gdn_status s);
+
+/* The CUDA error behind the calling thread's most recent GDN_ERR_CUDA, as
+ * "name: description" ("no CUDA error" if there was none).  The string belongs
+ * to the calling thread and stays valid until its next call of this function. */
+const char* gdn_last_cuda_error(void);
 
 #ifdef __cplusplus
 }

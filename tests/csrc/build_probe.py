@@ -5,7 +5,9 @@ import subprocess
 HERE = os.path.dirname(os.path.abspath(__file__))
 SRC = os.path.join(HERE, "umma_probe.cu")
 LIB = os.path.join(HERE, "libumma_probe.so")
-DEPS = [SRC, os.path.join(HERE, "..", "..", "hybrid_linear_attention_mixer_b200", "csrc", "device.cuh")]
+ROOT = os.path.join(HERE, "..", "..")
+DEPS = [SRC, os.path.join(ROOT, "hybrid_linear_attention_mixer_b200", "csrc", "device.cuh"),
+        os.path.join(ROOT, "include", "gdn.h")]
 
 
 def build(force=False):
@@ -14,7 +16,7 @@ def build(force=False):
         tmp = LIB + ".tmp%d" % os.getpid()
         subprocess.check_call([nvcc if os.path.exists(nvcc) else "nvcc", "-O2", "-std=c++17",
                                "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
-                               "-Xcompiler", "-fPIC", "-shared", "-o", tmp, SRC])
+                               "-Xcompiler", "-fPIC", "-shared", "-I" + os.path.join(ROOT, "include"), "-o", tmp, SRC])
         os.replace(tmp, LIB)
     return LIB
 

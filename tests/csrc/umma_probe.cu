@@ -9,6 +9,10 @@
 //   variant 4: A in TMEM  (M=128, K=128), B K-major  (N=64,  K=128)
 //   variant 5: A in TMEM  (M=128, K=64),  B MN-major (N=128, K=64)
 //   variant 6: A in TMEM  (M=128, K=128), B MN-major (N=64,  K=128)
+// It also holds a test of the bounded wait: an mbarrier wait that nothing
+// completes gives up after its limit, records its code in the error word, and
+// the kernel returns; the host side maps the word to a status (the same
+// device.cuh code as the library's kernels and gdn_check_device_error).
 #include "../../hybrid_linear_attention_mixer_b200/csrc/device.cuh"
 
 using namespace gdn;
@@ -102,7 +106,45 @@ __global__ void __launch_bounds__(128, 1) umma_probe_kernel(int variant, const f
         tmem_dealloc(tmem, 256);
     }
 }
+// One mbarrier that nothing ever arrives on, waited on for at most limit_ns.
+__global__ void __launch_bounds__(32, 1) wait_timeout_kernel(unsigned long long limit_ns, int* gave_up) {
+    __shared__ __align__(8) uint64_t bar_mem;
+    const uint32_t bar = smem_u32(&bar_mem);
+    if (threadIdx.x == 0) {
+        mbar_init(bar, 1);
+        fence_mbar_init();
+    }
+    __syncwarp();
+    if (threadIdx.x == 0) {
+        const bool done = mbar_wait_bounded(bar, 0, limit_ns);
+        if (!done) record_error(kErrCopyTimeout);
+        *gave_up = done ? 0 : 1;
+    }
+}
 }  // namespace
+
+// Runs the wait above on `stream` and returns the status the error word maps to
+// (read and cleared), with the kernel's duration in *ms and its outcome in
+// *gave_up_dev (device int: 1 if the wait gave up).
+extern "C" int probe_wait_timeout(unsigned long long limit_ns, int* gave_up_dev, float* ms, void* stream) {
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    cudaEvent_t e0, e1;
+    if (cudaEventCreate(&e0) != cudaSuccess || cudaEventCreate(&e1) != cudaSuccess) return -1;
+    cudaEventRecord(e0, st);
+    wait_timeout_kernel<<<1, 32, 0, st>>>(limit_ns, gave_up_dev);
+    const bool launched = cudaGetLastError() == cudaSuccess;
+    cudaEventRecord(e1, st);
+    const gdn_status s = take_device_error(st);
+    cudaEventElapsedTime(ms, e0, e1);
+    cudaEventDestroy(e0);
+    cudaEventDestroy(e1);
+    return launched ? (int)s : -2;
+}
+
+// The error word of this module, read and cleared (the library's check, in this module).
+extern "C" int probe_check_device_error(void* stream) {
+    return (int)take_device_error(static_cast<cudaStream_t>(stream));
+}
 
 extern "C" int umma_probe(int variant, const float* A, const float* B, float* D) {
     if (variant < 0 || variant > 6) return 1;
