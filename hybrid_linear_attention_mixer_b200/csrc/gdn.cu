@@ -515,7 +515,7 @@ cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void
     const int cblocks = (Ctot / 8 + gdn::kConvThreads - 1) / gdn::kConvThreads;
     const int64_t tblocks = (T + gdn::kConvRun - 1) / gdn::kConvRun;
     const int64_t max_chunks = (T + gdn::intra::C - 1) / gdn::intra::C + n_seqs;
-    if (tblocks > 0x7fffffff || max_chunks * Hv > 0x7fffffff) return cudaErrorInvalidValue;
+    if (tblocks > 0x7fffffff || max_chunks * Hk > 0x7fffffff) return cudaErrorInvalidValue;
     int32_t* chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off);
     uint8_t* recs = wsb + L.rec_off;
 
@@ -561,7 +561,7 @@ cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void
     ia.cu = cu; ia.chunk_off = chunk_off; ia.flags = flags; ia.n_seqs = n_seqs;
     ia.Hk = Hk; ia.Hv = Hv;
     ia.rec = recs;
-    k_intra<<<(unsigned)(max_chunks * Hv), gdn::intra::NT, gdn::intra::SMEM_BYTES, st>>>(tm_q, tm_k, ia);
+    k_intra<<<(unsigned)(max_chunks * Hk), gdn::intra::NT, gdn::intra::SMEM_BYTES, st>>>(tm_q, tm_k, ia);
     return cudaGetLastError();
 }
 
@@ -584,8 +584,9 @@ cudaError_t launch_scan(const gdn_config* c, const void* v_src, int64_t v_rows, 
     cudaError_t e = ensure_smem(k_scan, 16 + (sizeof(TO) == 2 ? 0 : 1) + (c->state_dtype == GDN_BF16 ? 2 : 0),
                                 gdn::scan::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    CUtensorMap tm_v;
-    if (!head_tile_map(&tm_v, v_src, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_v, c->n_v_heads, v_rows))
+    CUtensorMap tm_v, tm_k;
+    if (!head_tile_map(&tm_v, v_src, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_v, c->n_v_heads, v_rows) ||
+        !head_tile_map(&tm_k, wsb + L.k_off, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, c->n_k_heads, T))
         return cudaErrorInvalidValue;
     gdn::scan::Args sa;
     sa.rec_state = rec_state;
@@ -595,7 +596,7 @@ cudaError_t launch_scan(const gdn_config* c, const void* v_src, int64_t v_rows, 
     sa.rec = wsb + L.rec_off;
     sa.o = o_dst ? o_dst : wsb + L.o_off;
     sa.Hk = c->n_k_heads; sa.Hv = c->n_v_heads; sa.dk = c->d_k; sa.dv = c->d_v;
-    k_scan<<<(unsigned)n_seqs * c->n_v_heads, gdn::scan::NT, gdn::scan::SMEM_BYTES, st>>>(tm_v, sa);
+    k_scan<<<(unsigned)n_seqs * c->n_v_heads, gdn::scan::NT, gdn::scan::SMEM_BYTES, st>>>(tm_v, tm_k, sa);
     return cudaGetLastError();
 }
 

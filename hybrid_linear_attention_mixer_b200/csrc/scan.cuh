@@ -2,40 +2,43 @@
 //
 // One CTA (18 warps) walks one (sequence, value head) chain chunk by chunk
 // (C = 64 tokens).  The state-independent factors of every chunk come from the
-// intra-chunk kernel's records (intra.cuh: -W, Q~, T, g, P, K~), whose tiles are
-// already the shared-memory images the tensor cores read.  With S0 the state
-// at the chunk start:
+// intra-chunk kernel's records (intra.cuh: -W, Q~, T, the decay factors, P^T),
+// whose tiles are already the shared-memory images the tensor cores read; v^
+// and k^ come from the conv outputs by TMA.  With S0 the state at the chunk
+// start, D = diag(e^{g_C - g}) and Q~ = diag(e^g) Q:
 //     U   = T V - W S0^T                                    (exact per-token updates)
-//     O   = (diag(e^g) Q S0^T + P U) / sqrt(d_k)
-//     S_C = e^{g_C} S0 + U^T diag(e^{g_C - g}) K
+//     O   = (Q~ S0^T + P U) / sqrt(d_k)
+//     S_C = e^{g_C} S0 + (D U)^T K
 // o goes out as [chunk][head][64][128] tiles; the gated RMSNorm that follows
 // runs in norm.cuh, in parallel over all tiles.
 //
 // A tcgen05.mma costs about the same whatever its N up to 128, so products that
 // share an A operand are fused into one wide-N MMA, and A operands live in TMEM:
-//   (c)   V^T T^T,             N = 64  -> U2^T           [A: V, shared memory]
-//   MMA1  (d,e) S [-W ; Q~]^T, N = 128 -> [U2^T | O^T] += [A: S, TMEM]
-//   MMA2  (f,g) U^T [P ; K~^T]^T, N=192 -> [O^T | S]  += [A: U^T, TMEM; B MN-major]
-// with Q~ = diag(e^g) Q and K~ = diag(e^{g_C - g}) K.  (c) does not depend on the
-// state: the loading warp issues it once MMA2 of the previous chunk has completed,
-// so it runs while that chunk's new state is converted.  The fp32 state S lives in TMEM as an
-// accumulator: before MMA2 it holds e^{g_C} S0, so MMA2 leaves S_C.  The operand
-// tiles and the U, O accumulators alternate with chunk parity so that O is
-// double-buffered while both fused MMAs keep contiguous outputs:
-//   parity 0: B1 = [-W ; Q~], B2 = [P^T | K~], TMEM [U2 | O0 | S]
-//   parity 1: B1 = [Q~ ; -W], B2 = [K~ | P^T], TMEM [S | O1 | U2']
-// Per chunk, the critical chain is MMA1 -> U^T to fp16 -> MMA2 -> the fp16 copy
-// of the new state.  While MMA1 runs, the 16 worker warps write the decayed state
-// accumulator; while MMA2
-// runs, they write the previous chunk's o tile (and zero its accumulator for the
-// chunk after next).  A 17th warp issues the chain's MMAs, so that its waits on
-// the tensor pipe delay no other work, and an 18th issues every copy and (c): a bulk copy
-// holds its issuing thread for about as long as the copy engine takes to walk
-// its bytes, so copies stay off the MMA chain.  The loader meets the others
-// only through mbarriers (buffer released, o tile staged, staging buffer free),
-// never at a CTA barrier.  Loads are double-buffered two chunks ahead: v (TMA),
-// the record's B1 image with T and g (one bulk copy) and its B2 image (one
-// bulk copy).
+//   (c)   V^T T^T,              N = 64  -> U2^T          [A: V, shared memory]
+//   MMA1  S [-W ; Q~]^T,        N = 128 -> [U2^T | O^T] += [A: S, TMEM]
+//   MMA2a (D U)^T K,            N = 128 -> S  +=          [A: (D U)^T, TMEM; B: k^, MN-major]
+//   MMA2b U^T P^T,              N = 64  -> O^T +=         [A: U^T, TMEM; B: P^T, MN-major]
+// The fp32 state S lives in TMEM as an accumulator: before MMA2a the workers
+// store e^{g_C} S0 into it, so MMA2a leaves S_C.  The decay D rides on the fp16
+// copy of U that the workers make anyway (a second, scaled copy), so the raw k^
+// tile is MMA2a's operand as it arrives.  U and O accumulators alternate with
+// chunk parity, O double-buffered.
+//
+// Per chunk, the critical chain is MMA1 -> U^T to fp16 -> MMA2a -> the fp16 copy
+// of the new state.  A dedicated warp issues every MMA: right after MMA1 it
+// queues (c) of the next chunk, which runs while U is converted, and right after
+// MMA2a it queues MMA2b, which runs while the state is converted; it waits for
+// the next MMA's operands while the workers convert, so each conversion is
+// followed by an immediate issue.  While MMA1 runs, the 16 worker warps write the
+// decayed state accumulator and the previous chunk's o tile (once its MMA2b has
+// completed), and zero that O accumulator for the chunk after next; MMA2a, the
+// shortest product, is left to run alone.  An 18th warp issues
+// every copy: a bulk copy holds its issuing thread for about as long as the copy
+// engine takes to walk its bytes, so copies stay off the MMA chain.  It meets
+// the others only through mbarriers (buffer released, o tile staged, staging
+// buffer free), never at a CTA barrier.  Loads run two chunks ahead: v (TMA) and
+// the record's B1 image, T and decay factors (one bulk copy) on one barrier; k^
+// (TMA) and P^T (one bulk copy) on another.
 #pragma once
 #include "device.cuh"
 #include "intra.cuh"
@@ -51,27 +54,26 @@ constexpr int NMAIN = NW + 32;        // workers + issuer: they meet at named ba
 constexpr int NT = NMAIN + 32;
 
 // Shared memory (bytes from a 1024-aligned base); pairs are indexed by chunk parity.
-constexpr uint32_t OFF_R = 0;           // x2: the record's B1 image (32 KiB), T (8 KiB), g (256 B)
+constexpr uint32_t OFF_R = 0;           // x2: the record's B1 image (32 KiB), T (8 KiB), decay factors
 constexpr uint32_t R_STRIDE = 41984;
 constexpr uint32_t R_T = intra::REC_T - intra::REC_B1, R_G = intra::REC_G - intra::REC_B1;
 constexpr uint32_t OFF_V = OFF_R + 2 * R_STRIDE;     // V x2: 64 token rows x d_v, halves of 8192
-constexpr uint32_t OFF_B2 = OFF_V + 2 * 16384;       // x2: the record's B2 image, [P^T | K~] or [K~ | P^T]
+constexpr uint32_t OFF_B2 = OFF_V + 2 * 16384;       // x2: [K half 0 | K half 1 | P^T], MN-major atoms
 constexpr uint32_t B2_STRIDE = 24576;
 constexpr uint32_t OFF_OST = OFF_B2 + 2 * B2_STRIDE; // o tile staging: 2 x 16 KiB (or 1 x 32 KiB)
 constexpr uint32_t OFF_BAR = OFF_OST + 32768;        // mbarriers, TMEM address, abort flag, counters
 constexpr uint32_t SMEM_USED = OFF_BAR + 192;
 constexpr uint32_t SMEM_BYTES = SMEM_USED + 1024;
 static_assert(SMEM_BYTES <= 232448, "shared memory budget");
-static_assert(R_STRIDE % 1024 == 0 && R_STRIDE >= intra::REC_B1_BYTES, "record slot");
-static_assert(B2_STRIDE == intra::REC_B2_BYTES, "B2 image");
+static_assert(R_STRIDE % 1024 == 0 && R_STRIDE >= intra::REC_LD_BYTES, "record slot");
 
-// Tensor memory: U2 | O0 | S (128) | O1 | U2' | S fp16 A (64) | U^T fp16 A (32)
-constexpr uint32_t ACC_U0 = 0, ACC_O0 = 64, ACC_S = 128, ACC_O1 = 256, ACC_U1 = 320;
-constexpr uint32_t TA_S = 384, TA_U = 448, TMEM_COLS = 512;
-__host__ __device__ constexpr uint32_t acc_u(int b) { return b ? ACC_U1 : ACC_U0; }
-__host__ __device__ constexpr uint32_t acc_o(int b) { return b ? ACC_O1 : ACC_O0; }
+// Tensor memory: [U2 | O] for parity 0 and 1, S (128), S fp16 A (64), U^T fp16 A (32), (D U)^T fp16 A (32)
+constexpr uint32_t ACC_S = 256, TA_S = 384, TA_U = 448, TA_UD = 480, TMEM_COLS = 512;
+__host__ __device__ constexpr uint32_t acc_u(int b) { return b ? 128u : 0u; }
+__host__ __device__ constexpr uint32_t acc_o(int b) { return acc_u(b) + 64u; }
 
-constexpr uint32_t LD_BYTES = 2 * 8192 + intra::REC_B1_BYTES;   // v halves + B1, T, g
+constexpr uint32_t LD_BYTES = 2 * 8192 + intra::REC_LD_BYTES;   // v halves + B1, T, decay factors
+constexpr uint32_t B2_BYTES = 2 * 8192 + 8192;                  // k^ halves + P^T
 
 struct Args {
     void* rec_state;            // [N][Hv][dv][dk] state dtype (fp32 or bf16), in/out
@@ -104,32 +106,30 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 
 template <typename TO, typename TS>
 __global__ void __launch_bounds__(NT, 1)
-gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
+gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_k, Args p) {
     constexpr uint32_t O_BYTES = C * 128 * sizeof(TO);
     constexpr int kOBufs = O_BYTES <= 16384 ? 2 : 1;   // staging buffers for the o tiles
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
     const uint32_t sb = (raw + 1023u) & ~1023u;
     uint8_t* smem = smem_raw + (sb - raw);
-    const uint32_t bar = sb + OFF_BAR;                    // tensor-core commits (issuer)
-    const uint32_t bar_ld0 = sb + OFF_BAR + 8;            // [2] v, B1, T, g arrived
-    const uint32_t bar_b20 = sb + OFF_BAR + 24;           // [2] B2 arrived
+    const uint32_t bar = sb + OFF_BAR;                    // tensor-core commits of MMA1 and MMA2a (issuer)
+    const uint32_t bar_ld0 = sb + OFF_BAR + 8;            // [2] v, B1, T, decay factors arrived
+    const uint32_t bar_b20 = sb + OFF_BAR + 24;           // [2] k^, P^T arrived
     const uint32_t bar_fin = sb + OFF_BAR + 40;           // abort path: every MMA issued so far
     const uint32_t ev10 = sb + OFF_BAR + 48;              // [2] MMA1 of a chunk done: its v/record buffer is free
-    const uint32_t ev20 = sb + OFF_BAR + 64;              // [2] MMA2 done, previous o tile staged
+    const uint32_t ev20 = sb + OFF_BAR + 64;              // [2] MMA2b of a chunk done (tensor-core arrive): B2 free
     const uint32_t evo = sb + OFF_BAR + 80;               // a staging buffer is free again
     const uint32_t ev_end = sb + OFF_BAR + 88;            // the last o tile is staged
-    const uint32_t evc0 = sb + OFF_BAR + 96;              // [2] (c) of a chunk is in its U accumulator
-    const uint32_t bar_lfin = sb + OFF_BAR + 112;         // the loading warp's own MMAs (drain)
+    const uint32_t ev_st = sb + OFF_BAR + 96;             // [2] o tile of a chunk staged
     const uint32_t ev_ldone = sb + OFF_BAR + 120;         // the loading warp has drained everything
     volatile uint32_t* s_tmem = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 128);
     volatile uint32_t* s_abort = reinterpret_cast<volatile uint32_t*>(smem + OFF_BAR + 132);
     // loads issued per barrier (ld x2, B2 x2): the loader's drain waits for the last phase of each
     volatile int* s_issued = reinterpret_cast<volatile int*>(smem + OFF_BAR + 136);
-    // the issuer has issued MMA1 (phase parity 0) or MMA2 (parity 1) of the current chunk: the
+    // the issuer has issued MMA1 (phase parity 0) or MMA2a (parity 1) of the current chunk: the
     // workers' TMEM traffic waits for it so that it does not slow the issue down
     const uint32_t ev_iss = sb + OFF_BAR + 152;
-    const uint32_t ev_m20 = sb + OFF_BAR + 160;           // [2] MMA2 of a chunk issued: (c) may queue behind it
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const bool worker = tid < NW;
@@ -137,6 +137,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
     const int cs = warp >> 2;     // column slice 0..3 (worker warps)
     const int Hv = p.Hv, dk = p.dk, dv = p.dv;
     const int seq = blockIdx.x / Hv, h = blockIdx.x % Hv;
+    const int kh = h / (Hv / p.Hk);
     const int64_t s0 = p.cu[seq], s1 = p.cu[seq + 1];
     const int nchunks = (int)((s1 - s0 + C - 1) / C);
     if (nchunks <= 0 || *p.flags) return;
@@ -147,7 +148,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
     const int64_t o_stride = (int64_t)Hv * O_BYTES;
 
     // ---- the loading warp's copies ----
-    auto issue_chunk = [&](int ci) {   // v tile and the record's B1 image, T and g of chunk ci
+    auto issue_chunk = [&](int ci) {   // v tile and the record's B1 image, T and decay factors of chunk ci
         const int bb = ci & 1;
         if (lane == 0) s_issued[bb]++;
         mbar_arrive_expect_tx_w(bar_ld0 + 8 * bb, LD_BYTES);
@@ -155,14 +156,18 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         for (int hf = 0; hf < 2; hf++)
             tma_load_3d_w(sb + OFF_V + bb * 16384 + hf * 8192, &tm_v, 64 * hf, h, (int)(s0 + (int64_t)ci * C),
                           bar_ld0 + 8 * bb);
-        bulk_g2s_w(sb + OFF_R + bb * R_STRIDE, rec0 + ci * rec_stride + intra::REC_B1, intra::REC_B1_BYTES,
+        bulk_g2s_w(sb + OFF_R + bb * R_STRIDE, rec0 + ci * rec_stride + intra::REC_B1, intra::REC_LD_BYTES,
                    bar_ld0 + 8 * bb);
     };
-    auto issue_b2 = [&](int ci) {   // the record's B2 image of chunk ci
+    auto issue_b2 = [&](int ci) {   // k^ tile and the record's P^T of chunk ci
         const int bb = ci & 1;
         if (lane == 0) s_issued[2 + bb]++;
-        mbar_arrive_expect_tx_w(bar_b20 + 8 * bb, intra::REC_B2_BYTES);
-        bulk_g2s_w(sb + OFF_B2 + bb * B2_STRIDE, rec0 + ci * rec_stride + intra::REC_B2, intra::REC_B2_BYTES,
+        mbar_arrive_expect_tx_w(bar_b20 + 8 * bb, B2_BYTES);
+#pragma unroll
+        for (int hf = 0; hf < 2; hf++)
+            tma_load_3d_w(sb + OFF_B2 + bb * B2_STRIDE + hf * 8192, &tm_k, 64 * hf, kh, (int)(s0 + (int64_t)ci * C),
+                          bar_b20 + 8 * bb);
+        bulk_g2s_w(sb + OFF_B2 + bb * B2_STRIDE + 16384, rec0 + ci * rec_stride + intra::REC_P, 8192,
                    bar_b20 + 8 * bb);
     };
     auto issue_o = [&](int ce) {
@@ -176,10 +181,8 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         if (lane == 0) {
             mbar_init(bar, 1);
 #pragma unroll
-            for (int i = 0; i < 15; i++) mbar_init(bar_ld0 + 8 * i, 1);   // ld, B2, fin, ev1, ev2, evo, end, evc, lfin, ldone
+            for (int i = 0; i < 15; i++) mbar_init(bar_ld0 + 8 * i, 1);   // ld, B2, fin, ev1, ev2, evo, end, st, -, ldone
             mbar_init(ev_iss, 1);
-            mbar_init(ev_m20, 1);
-            mbar_init(ev_m20 + 8, 1);
             fence_mbar_init();
             *s_abort = 0;
             for (int i = 0; i < 4; i++) s_issued[i] = 0;
@@ -210,23 +213,6 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
     const uint32_t tmem = *s_tmem;
 
     if (warp == LW) {
-        // (c) of chunk ce: U2^T = V^T T^T into its U accumulator, committed to evc[ce & 1].  It
-        // is issued once MMA2 of the chunk before has completed, so it runs while that chunk's
-        // new state is converted, and MMA1 of chunk ce accumulates onto it.
-        const uint64_t dV0 = sdesc(sb + OFF_V, 8192, 1024);
-        const uint64_t dT0 = sdesc(sb + OFF_R + R_T, 16, 1024);
-        constexpr uint32_t ID_C = idesc_f16(128, 64, 1, 0);
-        int c_issued = 0;
-        auto issue_c = [&](int ce) {
-            const int bb = ce & 1;
-            tc_fence_after();
-#pragma unroll
-            for (int ks = 0; ks < 4; ks++)
-                mma_f16_w(tmem + acc_u(bb), dV0 + bb * 1024 + ks * 128, dT0 + bb * (R_STRIDE >> 4) + ks * 2, ID_C,
-                          ks > 0);
-            mma_commit_w(evc0 + 8 * bb);
-            c_issued++;
-        };
         // Waits for an event of the other warps; gives up on their abort or after the time limit.
         auto lwait = [&](uint32_t b, uint32_t parity) -> bool {
             if (mbar_try_wait(b, parity)) return true;
@@ -240,31 +226,28 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
             }
             return true;
         };
-        bool ok = lwait(bar_ld0, 0);
-        if (ok) issue_c(0);
-        if (ok && nchunks > 1) {
+        if (nchunks > 1) {
             issue_chunk(1);
             issue_b2(1);
         }
+        bool ok = true;
         for (int ci = 0; ci < nchunks && ok; ci++) {
-            ok = lwait(ev10 + 8 * (ci & 1), (ci >> 1) & 1);         // MMA1 of chunk ci is done with buffer ci & 1
-            if (!ok) break;
-            if (ci + 2 < nchunks) {
-                fence_async_smem();
-                issue_chunk(ci + 2);
-            }
-            if (ci + 1 < nchunks) {   // U accumulator (ci + 1) & 1 was read by the U conversion of chunk ci - 1
-                ok = lwait(ev_m20 + 8 * (ci & 1), (ci >> 1) & 1);   // queued behind MMA2 of chunk ci
-                if (ok) ok = lwait(bar_ld0 + 8 * ((ci + 1) & 1), ((ci + 1) >> 1) & 1);
+            if (ci > 0) {   // o of chunk ci - 1 was staged while MMA1 of chunk ci ran
+                ok = lwait(ev_st + 8 * ((ci - 1) & 1), ((ci - 1) >> 1) & 1);
                 if (!ok) break;
-                issue_c(ci + 1);      // the next MMA1 waits for it
+                issue_o(ci - 1);
             }
-            ok = lwait(ev20 + 8 * (ci & 1), (ci >> 1) & 1);         // MMA2 of chunk ci done; o of chunk ci - 1 staged
-            if (!ok) break;
-            if (ci + 2 < nchunks) issue_b2(ci + 2);
-            if (ci > 0) issue_o(ci - 1);
             if (kOBufs == 2) bulk_wait_read<1>(); else bulk_wait_read<0>();   // the staging buffer of o(ci) is free
             if (lane == 0) mbar_arrive(evo);
+            if (ci + 2 < nchunks) {
+                ok = lwait(ev10 + 8 * (ci & 1), (ci >> 1) & 1);     // MMA1 of chunk ci is done with buffer ci & 1
+                if (!ok) break;
+                fence_async_smem();
+                issue_chunk(ci + 2);
+                ok = lwait(ev20 + 8 * (ci & 1), (ci >> 1) & 1);     // MMA2b of chunk ci is done with B2 buffer ci & 1
+                if (!ok) break;
+                issue_b2(ci + 2);
+            }
         }
         if (ok && lwait(ev_end, 0)) issue_o(nchunks - 1);
         // drain: every copy this warp issued completes before the CTA may exit
@@ -272,10 +255,6 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         if (lane == 0)
             for (int i = 0; i < 4; i++)   // the last phase issued on each load barrier (returns at once if complete)
                 if (s_issued[i] > 0) mbar_wait_bounded(bar_ld0 + 8 * i, (uint32_t)(s_issued[i] - 1) & 1u);
-        if (c_issued > 0) {   // every MMA of this warp has completed
-            mma_commit_w(bar_lfin);
-            mbar_wait_bounded(bar_lfin, 0);
-        }
         __syncwarp();
         if (lane == 0) mbar_arrive(ev_ldone);
         return;
@@ -285,10 +264,23 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
     const uint32_t tl = tmem + ((uint32_t)(32 * qd) << 16);
     const float inv_sqrt_dk = rsqrtf((float)dk);
     uint32_t mphase = 0;
-    const uint64_t dB10 = sdesc(sb + OFF_R, 16, 1024);
-    const uint64_t dB20 = sdesc(sb + OFF_B2, 8192, 1024);
-    constexpr uint32_t ID_DE = idesc_f16(128, 128, 0, 0);    // (d,e)
-    constexpr uint32_t ID_FG = idesc_f16(128, 192, 0, 1);    // (f,g)
+    const uint64_t dB1 = sdesc(sb + OFF_R, 16, 1024);
+    const uint64_t dK = sdesc(sb + OFF_B2, 8192, 1024);
+    const uint64_t dP = sdesc(sb + OFF_B2 + 16384, 8192, 1024);
+    const uint64_t dV0 = sdesc(sb + OFF_V, 8192, 1024);
+    const uint64_t dT0 = sdesc(sb + OFF_R + R_T, 16, 1024);
+    constexpr uint32_t ID_1 = idesc_f16(128, 128, 0, 0);    // MMA1
+    constexpr uint32_t ID_2A = idesc_f16(128, 128, 0, 1);   // MMA2a
+    constexpr uint32_t ID_2B = idesc_f16(128, 64, 0, 1);    // MMA2b
+    constexpr uint32_t ID_C = idesc_f16(128, 64, 1, 0);     // (c)
+    // (c) of chunk ce: U2^T = V^T T^T into its U accumulator (MMA1 of chunk ce accumulates onto it;
+    // the tensor pipe runs one thread's MMAs in order)
+    auto issue_c = [&](int ce) {
+        const int bb = ce & 1;
+#pragma unroll
+        for (int ks = 0; ks < 4; ks++)
+            mma_f16_w(tmem + acc_u(bb), dV0 + bb * 1024 + ks * 128, dT0 + bb * (R_STRIDE >> 4) + ks * 2, ID_C, ks > 0);
+    };
     // fp16 copy of the state: the A operand of MMA1
     auto put_state_a = [&]() {
         uint32_t h16[16];
@@ -296,7 +288,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         for (int i = 0; i < 16; i++) h16[i] = pack_half2(Sv[2 * i], Sv[2 * i + 1]);
         tmem_st16(tl + TA_S + 16 * cs, h16);
     };
-    // decayed state e^{g_C} S: the accumulator that MMA2 completes
+    // decayed state e^{g_C} S: the accumulator that MMA2a completes
     auto put_state_acc = [&](float decay) {
         uint32_t d[32];
 #pragma unroll
@@ -316,14 +308,19 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         tmem_st16(tl + acc_o(ce & 1) + 16 * cs, o);
     };
 
-    // ---- prologue: zero O accumulators, fp16 S0 ----
+    // ---- prologue: zero O accumulators, fp16 S0; (c) of chunk 0 ----
     if (worker) {
         uint32_t z[16];
 #pragma unroll
         for (int i = 0; i < 16; i++) z[i] = 0u;
-        tmem_st16(tl + ACC_O0 + 16 * cs, z);
-        tmem_st16(tl + ACC_O1 + 16 * cs, z);
+        tmem_st16(tl + acc_o(0) + 16 * cs, z);
+        tmem_st16(tl + acc_o(1) + 16 * cs, z);
         put_state_a();
+    }
+    if (warp == IW) {
+        wait_par(bar_ld0, 0);
+        tc_fence_after();
+        issue_c(0);
     }
     tc_fence_before();
     main_sync();
@@ -341,66 +338,81 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
 
     for (int ci = 0; ci < nchunks; ci++) {
         const int b = ci & 1;
+        float dU[16];   // e^{g_C - g_c} for this worker's 16 chunk positions c = 16 cs + i
 
-        // ---- MMA1: (d,e) [U2^T | O^T] += S [-W ; Q~]^T ((c) and zeroed O are already there) ----
+        // ---- MMA1: [U2^T | O^T] += S [-W ; Q~]^T ((c) and the zeroed O are already there) ----
         if (warp == IW) {
-            wait_par(bar_ld0, ci);
-            wait_par(evc0, ci);   // (c) of chunk ci
             tc_fence_after();
-            const uint32_t d1 = tmem + (b ? ACC_O1 : ACC_U0);
 #pragma unroll
             for (int ks = 0; ks < 8; ks++)
-                mma_f16_ta_w(d1, tmem + TA_S + ks * 8, dB10 + b * (R_STRIDE >> 4) + (ks >> 2) * 1024 + (ks & 3) * 2,
-                             ID_DE, 1);
+                mma_f16_ta_w(tmem + acc_u(b), tmem + TA_S + ks * 8,
+                             dB1 + b * (R_STRIDE >> 4) + (ks >> 2) * 1024 + (ks & 3) * 2, ID_1, 1);
             mma_commit_w(bar);
             if (lane == 0) mbar_arrive(ev_iss);
+            if (ci + 1 < nchunks) {   // (c) of the next chunk runs while U is converted
+                wait_par(bar_ld0, ci + 1);
+                tc_fence_after();
+                issue_c(ci + 1);
+            }
         }
-        // ---- workers, while MMA1 runs: the decayed state accumulator ----
+        // ---- workers, while MMA1 runs: the decayed state accumulator and the U^T decay factors ----
         if (worker) {
-            wait_par(bar_ld0, ci);   // g
-            const float decay = __expf(reinterpret_cast<const float*>(smem + OFF_R + b * R_STRIDE + R_G)[C - 1]);
+            wait_par(bar_ld0, ci);
+            const float* gf = reinterpret_cast<const float*>(smem + OFF_R + b * R_STRIDE + R_G);
+            const float decay = gf[C];
+#pragma unroll
+            for (int i4 = 0; i4 < 4; i4++) {
+                const float4 f = *reinterpret_cast<const float4*>(gf + 16 * cs + 4 * i4);
+                dU[4 * i4] = f.x; dU[4 * i4 + 1] = f.y; dU[4 * i4 + 2] = f.z; dU[4 * i4 + 3] = f.w;
+            }
             if (!mbar_wait_bounded(ev_iss, 0)) atomicOr((unsigned*)s_abort, 1u);
             put_state_acc(decay);
+            if (ci > 0) {   // O of the previous chunk is final once its MMA2b has completed
+                wait_par(ev20, ci - 1);
+                stage_o(ci - 1);
+            }
         }
         GDN_MMA_WAIT();
 
-        // ---- U^T -> fp16 A operand ----
-        if (warp == IW && ci > 0 && !mbar_wait_bounded(evo, (ci - 1) & 1))   // staging buffer for o(ci - 1)
-            atomicOr((unsigned*)s_abort, 2u);
+        // ---- U^T and (D U)^T -> fp16 A operands; the issuer meanwhile waits for MMA2's operands ----
+        if (warp == IW) wait_par(bar_b20, ci);
         if (worker) {
-            uint32_t r16[16], u[8];
+            uint32_t r16[16], u[8], ud[8];
             tmem_ld16(tl + acc_u(b) + 16 * cs, r16);
 #pragma unroll
-            for (int i = 0; i < 8; i++) u[i] = pack_half2(__uint_as_float(r16[2 * i]), __uint_as_float(r16[2 * i + 1]));
-            tmem_st8(tl + TA_U + 8 * cs, u);
+            for (int i = 0; i < 8; i++) {
+                const float u0 = __uint_as_float(r16[2 * i]), u1 = __uint_as_float(r16[2 * i + 1]);
+                u[i] = pack_half2(u0, u1);
+                ud[i] = pack_half2(u0 * dU[2 * i], u1 * dU[2 * i + 1]);
+            }
+            tmem_st8x2(tl + TA_U + 8 * cs, u, tl + TA_UD + 8 * cs, ud);
         }
         tc_fence_before();
         main_sync();
         if (*s_abort) goto abort_;
-        if (warp == IW && lane == 0) mbar_arrive(ev10 + 8 * b);   // MMA1, (c) and the decay are done with buffer b
 
-        // ---- MMA2: [O^T | S] (parity 0) or [S | O^T] (parity 1) += U^T [P ; K~^T]^T ----
+        // ---- MMA2a: S += (D U)^T K; then MMA2b: O^T += U^T P^T, which runs while S is converted ----
         if (warp == IW) {
-            wait_par(bar_b20, ci);
+            if (lane == 0) {
+                mbar_arrive(ev10 + 8 * b);                                // MMA1 and (c) are done with buffer b
+                if (ci > 0) mbar_arrive(ev_st + 8 * ((ci - 1) & 1));      // o(ci - 1) is staged
+            }
             tc_fence_after();
-            const uint32_t d2 = tmem + (b ? ACC_S : ACC_O0);
 #pragma unroll
             for (int ks = 0; ks < 4; ks++)
-                mma_f16_ta_w(d2, tmem + TA_U + ks * 8, dB20 + b * (B2_STRIDE >> 4) + ks * 128, ID_FG, 1);
+                mma_f16_ta_w(tmem + ACC_S, tmem + TA_UD + ks * 8, dK + b * (B2_STRIDE >> 4) + ks * 128, ID_2A, 1);
             mma_commit_w(bar);
-            if (lane == 0) {
-                mbar_arrive(ev_iss);
-                mbar_arrive(ev_m20 + 8 * b);
-            }
-        }
-        // ---- workers, while MMA2 runs: the previous chunk's o tile ----
-        if (worker && ci > 0) {
-            if (!mbar_wait_bounded(ev_iss, 1)) atomicOr((unsigned*)s_abort, 1u);
-            stage_o(ci - 1);
+            if (lane == 0) mbar_arrive(ev_iss);
+#pragma unroll
+            for (int ks = 0; ks < 4; ks++)
+                mma_f16_ta_w(tmem + acc_o(b), tmem + TA_U + ks * 8, dP + b * (B2_STRIDE >> 4) + ks * 128, ID_2B, 1);
+            mma_commit_w(ev20 + 8 * b);   // B2 buffer b is free once MMA2b has read P^T
         }
         GDN_MMA_WAIT();
 
-        // ---- new state: its fp16 copy for the next MMA1, or the final state ----
+        // ---- new state: its fp16 copy for the next MMA1, or the final state; the issuer
+        // meanwhile makes sure the staging buffer for o(ci) is free ----
+        if (warp == IW && !mbar_wait_bounded(evo, ci & 1)) atomicOr((unsigned*)s_abort, 2u);
         if (worker) {
             uint32_t r32[32];
             tmem_ld32(tl + ACC_S + 32 * cs, r32);
@@ -421,17 +433,17 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, Args p) {
         tc_fence_before();
         main_sync();
         if (*s_abort) goto abort_;
-        if (warp == IW && lane == 0) mbar_arrive(ev20 + 8 * b);   // B2 buffer b free; o(ci - 1) staged
     }
-    if (warp == IW && !mbar_wait_bounded(evo, (nchunks - 1) & 1)) atomicOr((unsigned*)s_abort, 2u);
-    main_sync();
-    if (*s_abort) goto abort_;
-    if (worker) stage_o(nchunks - 1);
+    // the last o tile (its staging buffer was checked in the last chunk's state window)
+    if (worker) {
+        wait_par(ev20, nchunks - 1);
+        stage_o(nchunks - 1);
+    }
     tc_fence_before();
     main_sync();
     if (warp == IW && lane == 0) mbar_arrive(ev_end);   // the loader stores the last tile
     if (warp == 0) {
-        mbar_wait_bounded(ev_ldone, 0);   // the loading warp's MMAs and copies are done
+        mbar_wait_bounded(ev_ldone, 0);   // the loading warp's copies are done
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }
@@ -450,7 +462,7 @@ abort_:
     tc_fence_before();
     main_sync();
     if (warp == 0) {
-        mbar_wait_bounded(ev_ldone, 0);   // the loading warp sees the flag and drains its MMAs and copies
+        mbar_wait_bounded(ev_ldone, 0);   // the loading warp sees the flag and drains its copies
         tc_fence_after();
         tmem_dealloc(tmem, TMEM_COLS);
     }

@@ -311,8 +311,8 @@ gdn_status gdn_prefill_host(const gdn_config* cfg, const gdn_weights* w,
  *   - Size limit: a request needing more than GDN_NOALLOC_SCRATCH_BYTES of
  *     workspace is rejected with GDN_ERR_WORKSPACE, before any launch.  The
  *     needed size is gdn_prefill_workspace_size(cfg, T_total, n_seqs).  At the
- *     published shape that is 82,688 bytes per token plus about 4.0 MB per
- *     sequence, so up to 749 tokens in one sequence.  Longer prompts can be
+ *     published shape that is 70,400 bytes per token plus about 3.2 MB per
+ *     sequence, so up to 896 tokens in one sequence.  Longer prompts can be
  *     split into consecutive calls, since the states carry from one call to
  *     the next.
  *   - First call on a device: it looks up the array's device address with

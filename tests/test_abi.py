@@ -48,15 +48,16 @@ def test_default_config_is_the_published_shape(lib):
 def test_workspace_size(lib):
     cfg = gdn.Config()
     T = 4096
-    # fp16 q^, k^ [T, 16*128] and v^ [T, 48*128]; chunk offsets [N+1] int32 (256-byte
-    # rounded); per (chunk, value head) a 65 KiB intra-chunk record and a [64][128]
-    # o tile of the output dtype, with at most ceil(T / 64) + N chunks
+    # fp16 q^, k^ [T, 16*128] and v^ [T, 48*128]; chunk offsets [N+1] and the check word,
+    # int32 (256-byte rounded); per (chunk, value head) a 49 KiB intra-chunk record and a
+    # [64][128] o tile of the output dtype, with at most ceil(T / 64) + N chunks
     conv = 2 * T * 2048 * 2 + T * 6144 * 2
-    per_chunk = 48 * (66560 + 64 * 128 * 2)
+    per_chunk = 48 * (50176 + 64 * 128 * 2)
     assert gdn.workspace_size(cfg, T, 1) == conv + 256 + (T // 64 + 1) * per_chunk
     assert gdn.workspace_size(cfg, T, 3) == conv + 256 + (T // 64 + 3) * per_chunk
     f32 = gdn.Config(out_dtype=__import__("torch").float32)
-    assert gdn.workspace_size(f32, T, 1) == conv + 256 + (T // 64 + 1) * 48 * (66560 + 64 * 128 * 4)
+    assert gdn.workspace_size(f32, T, 1) == conv + 256 + (T // 64 + 1) * 48 * (50176 + 64 * 128 * 4)
+    assert gdn.workspace_size(cfg, T, 63) == conv + 512 + (T // 64 + 63) * per_chunk
     assert gdn.workspace_size(cfg, 0, 0) == 256
     assert gdn.workspace_size(gdn.Config(d_k=48), T, 1) == 0
 
