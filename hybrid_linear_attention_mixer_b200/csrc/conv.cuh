@@ -33,7 +33,21 @@ struct ConvArgs {
     __half* vh;              // [T][Cv]
     int32_t* flags;          // per-call check word: bit 0 (malformed cu_seqlens) is read here,
                              // bit 1 is set here when an output overflows fp16
+    const int32_t* chunk_off;  // [N+1] first global chunk of each sequence (chunk_offsets_kernel)
+    int64_t g_lo, g_hi;      // this launch convolves the tokens of global chunks [g_lo, g_hi)
 };
+
+// The 32-token tiles (or runs) a launch over global chunks [g_lo, g_hi) owns:
+// those that start in its token range.  A tile that starts before the range
+// and reaches into it belongs to the launch before, so the launches over
+// consecutive chunk ranges write disjoint tiles, and the tokens of chunks
+// [g_lo, g_hi) are all written once this launch and the ones before it are done.
+__device__ __forceinline__ void conv_tile_range(const ConvArgs& p, int64_t& first, int64_t& count) {
+    const int64_t t_lo = chunk_first_token(p.cu, p.chunk_off, p.n_seqs, p.T, p.g_lo);
+    const int64_t t_hi = chunk_first_token(p.cu, p.chunk_off, p.n_seqs, p.T, p.g_hi);
+    first = (t_lo + 31) / 32;
+    count = (t_hi + 31) / 32 - first;
+}
 
 // fp16 keeps values below 65520 in magnitude; larger ones round to infinity.
 constexpr float kHalfOverflow = 65520.f;
@@ -49,6 +63,7 @@ __device__ __forceinline__ void report_range(const ConvArgs& p, float vmax, bool
 
 constexpr int kConvThreads = 128;   // 8 channels per thread
 constexpr int kConvRun = 32;        // tokens per thread (one run per CTA)
+static_assert(kConvRun == 32, "conv_tile_range counts 32-token runs");
 // input rows in flight per thread
 template <typename TA> __host__ __device__ constexpr int conv_depth() { return sizeof(TA) == 2 ? 8 : 4; }
 
@@ -93,7 +108,10 @@ __global__ void __launch_bounds__(kConvThreads, 4) conv_silu_norm_kernel(ConvArg
     if (*p.flags) return;   // cu_seqlens failed its check: sequence starts are not to be trusted
     const int Cq = p.Hk * p.dk, Cv = p.Hv * p.dv, Ctot = 2 * Cq + Cv;
     const int c = (blockIdx.y * kConvThreads + threadIdx.x) * 8;   // first of 8 channels
-    const int64_t t_begin = (int64_t)blockIdx.x * kConvRun;
+    int64_t run0, n_runs;
+    conv_tile_range(p, run0, n_runs);
+    if (blockIdx.x >= n_runs) return;
+    const int64_t t_begin = (run0 + blockIdx.x) * kConvRun;
     // sequence of each token of the run and its first token
     __shared__ int s_seq[kConvRun];
     __shared__ long long s_start[kConvRun];
@@ -216,6 +234,7 @@ __global__ void __launch_bounds__(kConvThreads, 4) conv_silu_norm_kernel(ConvArg
 namespace ctile {
 constexpr int NT = 256;
 constexpr int CH = 512, TOK = 32, ROWS = TOK + 3, BOXW = 64, BOXES = CH / BOXW;
+static_assert(TOK == 32, "conv_tile_range counts 32-token tiles");
 constexpr uint32_t BOX_BYTES = ROWS * BOXW * 2;          // 4480
 constexpr uint32_t TILE_BYTES = BOXES * BOX_BYTES;        // 35840
 constexpr int BUFS = 3;
@@ -325,7 +344,8 @@ conv_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const CUtensorMap* tm = tensor == 0 ? &tm_q : tensor == 1 ? &tm_k : &tm_v;
     const int64_t ld = tensor == 2 ? Cv : Cq;
     __half* dst0 = tensor == 0 ? p.qh : tensor == 1 ? p.kh : p.vh;
-    const int64_t n_tiles = (p.T + TOK - 1) / TOK;
+    int64_t tile0, n_tiles;
+    conv_tile_range(p, tile0, n_tiles);
     const int count = part < n_tiles ? (int)((n_tiles - part + parts - 1) / parts) : 0;
     if (count == 0 || *p.flags) return;   // (flags: cu_seqlens failed its check)
 
@@ -333,7 +353,7 @@ conv_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int tg = tid >> 6, cg = tid & 63;
     const int c = c0 + cg * 8, cl = cl0 + cg * 8;
     const bool is_qk = tensor < 2;
-    auto tile_t0 = [&](int jj) { return (int64_t)(part + (int64_t)jj * parts) * TOK; };
+    auto tile_t0 = [&](int jj) { return (tile0 + part + (int64_t)jj * parts) * TOK; };
     auto issue = [&](int jj) {
         const uint32_t buf = sb + (jj % BUFS) * TILE_BYTES, bar = bar0 + 8 * (jj % BUFS);
         mbar_arrive_expect_tx(bar, TILE_BYTES);

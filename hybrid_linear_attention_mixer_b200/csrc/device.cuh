@@ -37,6 +37,26 @@ __device__ __forceinline__ void record_error(unsigned int code) {
     atomicOr(&g_device_error, code);
 }
 
+// Prefill chunk length (tokens): every sequence of a packed batch is cut into
+// chunks of this many tokens, the last one possibly shorter.
+constexpr int kChunk = 64;
+
+// First token of global chunk gc of a packed batch, whose sequence s starts at
+// cu[s] and owns global chunks [chunk_off[s], chunk_off[s+1]); T_total for gc
+// at or past the batch's last chunk.  Launches that cover a range of chunks
+// turn it into a token range with this.
+__device__ __forceinline__ int64_t chunk_first_token(const int32_t* cu, const int32_t* chunk_off, int n_seqs,
+                                                     int64_t T_total, int64_t gc) {
+    if (gc <= 0) return 0;
+    if (gc >= chunk_off[n_seqs]) return T_total;
+    int lo = 0, hi = n_seqs - 1;   // last s with chunk_off[s] <= gc
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (chunk_off[mid] <= gc) lo = mid; else hi = mid - 1;
+    }
+    return (int64_t)cu[lo] + (gc - chunk_off[lo]) * kChunk;
+}
+
 // ---------------------------------------------------------------------------
 // Activation loads / stores
 // ---------------------------------------------------------------------------
@@ -105,6 +125,18 @@ __device__ __forceinline__ void sts128(uint32_t addr, uint32_t x, uint32_t y, ui
     asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(x), "r"(y), "r"(z), "r"(w)
                  : "memory");
 }
+// Zeroes rows [r0, 64) of the 64-row x 128-byte tiles at tile + i * 8192, i < n_tiles
+// (TMA tiles with the 128-byte swizzle keep each row in its own 128 bytes), with
+// nt threads, t = 0 .. nt-1.  For the rows a tile load read past a sequence's end.
+__device__ __forceinline__ void zero_tile_rows(uint32_t tile, int n_tiles, int r0, int t, int nt) {
+    const int per_tile = (64 - r0) * 8;   // 16-byte pieces
+    for (int i = t; i < n_tiles * per_tile; i += nt) {
+        const int ti = i / per_tile, j = i % per_tile;
+        asm volatile("st.shared.v4.u32 [%0], {%1, %1, %1, %1};" ::"r"(tile + ti * 8192 + (r0 + j / 8) * 128 + (j % 8) * 16),
+                     "r"(0u) : "memory");
+    }
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr) {
     uint4 v;
     asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];"

@@ -51,6 +51,7 @@ gdn_status check_config(const gdn_config* c) {
     if (c->n_v_heads % c->n_k_heads != 0) return GDN_ERR_UNSUPPORTED;
     if (!dim_ok(c->d_k) || !dim_ok(c->d_v)) return GDN_ERR_UNSUPPORTED;
     if (c->conv_kernel != 4 || c->chunk != gdn::intra::C) return GDN_ERR_UNSUPPORTED;
+    if (c->prefill_segments < 0 || c->prefill_segments > GDN_PREFILL_MAX_SEGMENTS) return GDN_ERR_INVALID_ARG;
     return GDN_OK;
 }
 
@@ -60,12 +61,34 @@ gdn_status check_weights(const gdn_weights* w) {
     return GDN_OK;
 }
 
+// Chunk ranges a prefill is pipelined over (gdn_config.prefill_segments): range
+// s is global chunks [s len, (s+1) len), the last one running to the end.
+struct SegPlan {
+    int n;
+    int32_t len;
+};
+
+SegPlan seg_plan(const gdn_config* c, int64_t T, int64_t n_seqs) {
+    const int64_t chunks = (T + gdn::kChunk - 1) / gdn::kChunk;   // of one sequence of T tokens
+    int64_t want = c->prefill_segments;
+    if (want == 0)   // automatic: chains too few to fill the GPU, in at most 8 ranges of at least 32 chunks
+        want = n_seqs * c->n_v_heads <= 96 ? (chunks / 32 < 8 ? chunks / 32 : 8) : 1;
+    if (want > GDN_PREFILL_MAX_SEGMENTS) want = GDN_PREFILL_MAX_SEGMENTS;
+    if (want > chunks) want = chunks;
+    if (want <= 1) return SegPlan{1, 0x7fffffff};
+    SegPlan p;
+    p.len = (int32_t)((chunks + want - 1) / want);
+    p.n = (int)((chunks + p.len - 1) / p.len);
+    return p;
+}
+
 // Prefill workspace: fp16 q^, k^, v^ (conv output), the first chunk of each
 // sequence followed by the call's check word (flags), one intra-chunk record
-// per (chunk, value head), and the o tile ([64][128], out dtype) of each
-// (chunk, value head) before the gated norm.
+// per (chunk, value head), the o tile ([64][128], out dtype) of each (chunk,
+// value head) before the gated norm, and, for a pipelined call, the fp32 state
+// of every chain between the launches over consecutive chunk ranges.
 struct Layout {
-    size_t q_off, k_off, v_off, coff_off, flags_off, rec_off, o_off, total;
+    size_t q_off, k_off, v_off, coff_off, flags_off, rec_off, o_off, carry_off, total;
 };
 
 Layout workspace_layout(const gdn_config* c, int64_t T, int64_t n_seqs) {
@@ -82,7 +105,9 @@ Layout workspace_layout(const gdn_config* c, int64_t T, int64_t n_seqs) {
     L.flags_off = L.coff_off + (size_t)(n_seqs + 1) * sizeof(int32_t);
     L.rec_off = L.coff_off + cb;
     L.o_off = L.rec_off + max_chunks * c->n_v_heads * gdn::intra::REC_BYTES;
-    L.total = L.o_off + max_chunks * c->n_v_heads * o_tile;
+    L.carry_off = align_up(L.o_off + max_chunks * c->n_v_heads * o_tile, 256);
+    L.total = L.carry_off;
+    if (seg_plan(c, T, n_seqs).n > 1) L.total += (size_t)n_seqs * c->n_v_heads * c->d_v * c->d_k * sizeof(float);
     return L;
 }
 
@@ -259,11 +284,15 @@ bool z_rows_map(CUtensorMap* m, const void* base, bool bf16, int width, int dv, 
 // Non-blocking streams for work that may overlap the caller's stream (forked
 // from and joined back to it by events): 0 = the context-parallel transition
 // scan, 1 = host-to-device copies, 2 = device-to-host copies, 3 = the prefill's
-// conv-state update.  They are kept per host thread and device, like the events
-// below: a call in one thread never waits on another thread's side work, and a
-// thread that captures a CUDA graph records only its own side work.
+// conv-state update, 4 = a pipelined prefill's state chain (the device's
+// greatest priority: when the kernel before it completes, its CTAs take the
+// freed SMs ahead of the caller's next producer kernel), 5 = a pipelined
+// prefill's gated norm.  They are kept per host thread and device, like the
+// events below: a call in one thread never waits on another thread's side work,
+// and a thread that captures a CUDA graph records only its own side work.
+constexpr int kSideStreams = 6;
 struct StreamPool {
-    cudaStream_t s[64][4] = {};
+    cudaStream_t s[64][kSideStreams] = {};
     ~StreamPool() {
         for (auto& per_dev : s)
             for (cudaStream_t x : per_dev)
@@ -274,9 +303,14 @@ struct StreamPool {
 cudaStream_t side_stream(int which = 0) {
     thread_local StreamPool pool;
     int dev = 0;
-    if (which < 0 || which > 3 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+    if (which < 0 || which >= kSideStreams || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64)
+        return nullptr;
     cudaStream_t& st = pool.s[dev][which];
-    if (!st && cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) st = nullptr;
+    if (!st) {
+        int least = 0, greatest = 0;
+        if (which != 4 || cudaDeviceGetStreamPriorityRange(&least, &greatest) != cudaSuccess) greatest = 0;
+        if (cudaStreamCreateWithPriority(&st, cudaStreamNonBlocking, greatest) != cudaSuccess) st = nullptr;
+    }
     return st;
 }
 
@@ -284,7 +318,7 @@ cudaStream_t side_stream(int which = 0) {
 // reused from call to call: a stream wait refers to the record enqueued before
 // it, so recording an event again in a later call leaves earlier waits intact,
 // and no two threads share an event.
-enum EventUse { kEvStageA = 0, kEvCp = 1, kEvHost = 2, kEvUses = 3 };
+enum EventUse { kEvStageA = 0, kEvCp = 1, kEvHost = 2, kEvPipe = 3, kEvUses = 4 };
 
 struct EventPool {
     std::vector<cudaEvent_t> ev[64][kEvUses];
@@ -475,22 +509,29 @@ gdn_status run_linear(const void* x, const void* w, int64_t M, int32_t N, int32_
 //            into the workspace, conv-state update, intra-chunk records
 //   stage B: the chunk scan from rec_state (in/out), then the gated norm into out
 // Set-up first: nothing is launched unless the tensor maps encode and the
-// kernels' shared-memory opt-ins succeed.
-// The chunk-offset kernel runs first: it checks cu_seqlens and writes the
-// call's check word, which every later kernel reads.  The conv-state update
-// (which must follow the conv's reads of the old state) runs on a side stream
-// beside the intra kernel.  Once the side stream has been forked, *join
-// receives an event recorded after its work, on every path, error paths
-// included; the caller's stream waits on it before the call ends.
+// kernels' shared-memory opt-ins succeed.  The conv, intra-chunk, scan and norm
+// launches each take a range of global chunks, so that a pipelined call
+// (launch_prefill) can run them range by range on three streams.
 template <typename TA>
-cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void* q, const void* k, const void* v,
-                           const void* a, const void* b, void* conv_state, const int32_t* cu, int n_seqs,
-                           int64_t T, void* ws, cudaStream_t st, cudaEvent_t* join) {
-    *join = nullptr;
+struct StageA {
+    ConvArgs ca;
+    gdn::intra::Args ia;
+    CUtensorMap tm_q, tm_k, tm_cq, tm_ck, tm_cv;
+    bool tiled;
+    int n_slices, cblocks;
+    int64_t max_chunks;
+    decltype(&gdn::conv_tile_kernel<16>) k_conv;
+};
+
+template <typename TA>
+cudaError_t prepare_stage_a(const gdn_config* c, const gdn_weights* w, const void* q, const void* k, const void* v,
+                            const void* a, const void* b, void* conv_state, const int32_t* cu, int n_seqs,
+                            int64_t T, void* ws, StageA<TA>* S) {
     const Layout L = workspace_layout(c, T, n_seqs);
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     int32_t* flags = reinterpret_cast<int32_t*>(wsb + L.flags_off);
-    ConvArgs ca;
+    int32_t* chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off);
+    ConvArgs& ca = S->ca;
     ca.q = q; ca.k = k; ca.v = v;
     ca.conv_w = w->conv_weight;
     ca.conv_state = conv_state;
@@ -503,66 +544,122 @@ cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void
     ca.kh = reinterpret_cast<__half*>(wsb + L.k_off);
     ca.vh = reinterpret_cast<__half*>(wsb + L.v_off);
     ca.flags = flags;
+    ca.chunk_off = chunk_off;
+    ca.g_lo = 0;
+    ca.g_hi = 0x7fffffff;
     auto k_intra = gdn::intra::gdn_intra_kernel<TA>;
     cudaError_t e = ensure_smem(k_intra, 4 + (sizeof(TA) == 2 ? 0 : 1), gdn::intra::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    CUtensorMap tm_q, tm_k;
     const int Hk = c->n_k_heads, Hv = c->n_v_heads;
-    if (!head_tile_map(&tm_q, ca.qh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, Hk, T) ||
-        !head_tile_map(&tm_k, ca.kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, Hk, T))
+    if (!head_tile_map(&S->tm_q, ca.qh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, Hk, T) ||
+        !head_tile_map(&S->tm_k, ca.kh, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, Hk, T))
         return cudaErrorInvalidValue;
     const int Ctot = 2 * c->n_k_heads * c->d_k + c->n_v_heads * c->d_v;
-    const int cblocks = (Ctot / 8 + gdn::kConvThreads - 1) / gdn::kConvThreads;
-    const int64_t tblocks = (T + gdn::kConvRun - 1) / gdn::kConvRun;
-    const int64_t max_chunks = (T + gdn::intra::C - 1) / gdn::intra::C + n_seqs;
-    if (tblocks > 0x7fffffff || max_chunks * Hk > 0x7fffffff) return cudaErrorInvalidValue;
-    int32_t* chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off);
-    uint8_t* recs = wsb + L.rec_off;
+    S->cblocks = (Ctot / 8 + gdn::kConvThreads - 1) / gdn::kConvThreads;
+    S->max_chunks = (T + gdn::intra::C - 1) / gdn::intra::C + n_seqs;
+    if ((T + gdn::kConvRun - 1) / gdn::kConvRun > 0x7fffffff || S->max_chunks * Hk > 0x7fffffff)
+        return cudaErrorInvalidValue;
 
     // the tiled conv for bf16 activations whose q, k and v widths are multiples of its slice
     const int Cq = c->n_k_heads * c->d_k, Cv = c->n_v_heads * c->d_v;
-    bool tiled = sizeof(TA) == 2 && Cq % gdn::ctile::CH == 0 && Cv % gdn::ctile::CH == 0;
-    CUtensorMap tm_cq, tm_ck, tm_cv;
-    auto k_conv = c->d_k == 32 ? gdn::conv_tile_kernel<4> : c->d_k == 64 ? gdn::conv_tile_kernel<8>
-                                                                           : gdn::conv_tile_kernel<16>;
-    if (tiled) {
-        tiled = conv_tile_map(&tm_cq, q, Cq, T) && conv_tile_map(&tm_ck, k, Cq, T) && conv_tile_map(&tm_cv, v, Cv, T);
-        e = ensure_smem(k_conv, 12 + (c->d_k == 32 ? 0 : c->d_k == 64 ? 1 : 2), gdn::ctile::SMEM_BYTES);
+    S->tiled = sizeof(TA) == 2 && Cq % gdn::ctile::CH == 0 && Cv % gdn::ctile::CH == 0;
+    S->n_slices = Ctot / gdn::ctile::CH;
+    S->k_conv = c->d_k == 32 ? gdn::conv_tile_kernel<4> : c->d_k == 64 ? gdn::conv_tile_kernel<8>
+                                                                        : gdn::conv_tile_kernel<16>;
+    if (S->tiled) {
+        S->tiled = conv_tile_map(&S->tm_cq, q, Cq, T) && conv_tile_map(&S->tm_ck, k, Cq, T) &&
+                   conv_tile_map(&S->tm_cv, v, Cv, T);
+        e = ensure_smem(S->k_conv, 12 + (c->d_k == 32 ? 0 : c->d_k == 64 ? 1 : 2), gdn::ctile::SMEM_BYTES);
         if (e != cudaSuccess) return e;
     }
-    cudaStream_t aux = side_stream(3);
-    cudaEvent_t* ev = thread_events(kEvStageA, 2);   // conv done (fork), side work done (join)
-    if (!aux || !ev) return cudaErrorNotReady;
 
-    gdn::intra::chunk_offsets_kernel<<<1, 1024, 0, st>>>(cu, n_seqs, T, max_chunks, chunk_off, flags);
-    if (tiled) {
-        const int n_slices = Ctot / gdn::ctile::CH;
-        const int64_t n_tiles = (T + gdn::ctile::TOK - 1) / gdn::ctile::TOK;
-        int64_t parts = (int64_t)2 * sm_count() / n_slices;
-        parts = parts < 1 ? 1 : parts > n_tiles ? n_tiles : parts;
-        k_conv<<<(unsigned)(n_slices * parts), gdn::ctile::NT, gdn::ctile::SMEM_BYTES, st>>>(
-            tm_cq, tm_ck, tm_cv, ca, (int)parts);
-    } else {
-        gdn::conv_silu_norm_kernel<TA><<<dim3((unsigned)tblocks, cblocks), gdn::kConvThreads, 0, st>>>(ca);
-    }
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    if ((e = cudaEventRecord(ev[0], st)) != cudaSuccess || (e = cudaStreamWaitEvent(aux, ev[0], 0)) != cudaSuccess)
-        return e;
-    // aux is forked: from here on it is joined back whatever happens
-    gdn::conv_state_update_kernel<TA><<<dim3(n_seqs, (Ctot + 255) / 256), 256, 0, aux>>>(ca, conv_state);
-    const cudaError_t e_side = cudaGetLastError();
-    if ((e = cudaEventRecord(ev[1], aux)) != cudaSuccess) return e;
-    *join = ev[1];
-    if (e_side != cudaSuccess) return e_side;
-
-    gdn::intra::Args ia;
+    gdn::intra::Args& ia = S->ia;
     ia.a = a; ia.b = b;
     ia.A_log = w->A_log; ia.dt_bias = w->dt_bias;
     ia.cu = cu; ia.chunk_off = chunk_off; ia.flags = flags; ia.n_seqs = n_seqs;
     ia.Hk = Hk; ia.Hv = Hv;
-    ia.rec = recs;
-    k_intra<<<(unsigned)(max_chunks * Hk), gdn::intra::NT, gdn::intra::SMEM_BYTES, st>>>(tm_q, tm_k, ia);
+    ia.rec = wsb + L.rec_off;
+    ia.g_lo = 0;
+    return cudaSuccess;
+}
+
+// The chunk table and the check of cu_seqlens: the first kernel of every prefill.
+template <typename TA>
+cudaError_t launch_chunk_offsets(const StageA<TA>& S, cudaStream_t st) {
+    gdn::intra::chunk_offsets_kernel<<<1, 1024, 0, st>>>(S.ca.cu, S.ca.n_seqs, S.ca.T, S.max_chunks,
+                                                         const_cast<int32_t*>(S.ia.chunk_off), S.ca.flags);
     return cudaGetLastError();
+}
+
+// Conv + SiLU + L2 norm of the tokens of global chunks [g_lo, g_hi) (see conv_tile_range).
+template <typename TA>
+cudaError_t launch_conv(const StageA<TA>& S, int64_t g_lo, int64_t g_hi, cudaStream_t st) {
+    ConvArgs ca = S.ca;
+    ca.g_lo = g_lo;
+    ca.g_hi = g_hi;
+    const int64_t chunks = (g_hi < S.max_chunks ? g_hi : S.max_chunks) - g_lo;
+    const int64_t all_tiles = (S.ca.T + 31) / 32;
+    int64_t tiles = 2 * chunks + 1;   // 32-token tiles that start in the range's tokens (<= 64 per chunk)
+    tiles = tiles < all_tiles ? tiles : all_tiles;
+    if (tiles <= 0) return cudaSuccess;
+    if (S.tiled) {
+        int64_t parts = (int64_t)2 * sm_count() / S.n_slices;
+        parts = parts < 1 ? 1 : parts > tiles ? tiles : parts;
+        S.k_conv<<<(unsigned)(S.n_slices * parts), gdn::ctile::NT, gdn::ctile::SMEM_BYTES, st>>>(
+            S.tm_cq, S.tm_ck, S.tm_cv, ca, (int)parts);
+    } else {
+        gdn::conv_silu_norm_kernel<TA><<<dim3((unsigned)tiles, S.cblocks), gdn::kConvThreads, 0, st>>>(ca);
+    }
+    return cudaGetLastError();
+}
+
+// conv_state <- the last 3 inputs of each sequence: after every conv launch of the call.
+template <typename TA>
+cudaError_t launch_conv_state(const StageA<TA>& S, cudaStream_t st) {
+    const int Ctot = 2 * S.ca.Hk * S.ca.dk + S.ca.Hv * S.ca.dv;
+    gdn::conv_state_update_kernel<TA><<<dim3(S.ca.n_seqs, (Ctot + 255) / 256), 256, 0, st>>>(
+        S.ca, const_cast<void*>(S.ca.conv_state));
+    return cudaGetLastError();
+}
+
+// Intra-chunk records of global chunks [g_lo, g_hi).
+template <typename TA>
+cudaError_t launch_intra(const StageA<TA>& S, int64_t g_lo, int64_t g_hi, cudaStream_t st) {
+    gdn::intra::Args ia = S.ia;
+    ia.g_lo = (int32_t)g_lo;
+    const int64_t n = (g_hi < S.max_chunks ? g_hi : S.max_chunks) - g_lo;
+    if (n <= 0) return cudaSuccess;
+    gdn::intra::gdn_intra_kernel<TA><<<(unsigned)(n * S.ia.Hk), gdn::intra::NT, gdn::intra::SMEM_BYTES, st>>>(
+        S.tm_q, S.tm_k, ia);
+    return cudaGetLastError();
+}
+
+// Stage A over every chunk on `st`.  The conv-state update (which must follow the
+// conv's reads of the old state) runs on a side stream beside the intra kernel.
+// Once the side stream has been forked, *join receives an event recorded after
+// its work, on every path, error paths included; the caller's stream waits on
+// it before the call ends.
+template <typename TA>
+cudaError_t launch_stage_a(const gdn_config* c, const gdn_weights* w, const void* q, const void* k, const void* v,
+                           const void* a, const void* b, void* conv_state, const int32_t* cu, int n_seqs,
+                           int64_t T, void* ws, cudaStream_t st, cudaEvent_t* join) {
+    *join = nullptr;
+    StageA<TA> S;
+    cudaError_t e = prepare_stage_a<TA>(c, w, q, k, v, a, b, conv_state, cu, n_seqs, T, ws, &S);
+    if (e != cudaSuccess) return e;
+    cudaStream_t aux = side_stream(3);
+    cudaEvent_t* ev = thread_events(kEvStageA, 2);   // conv done (fork), side work done (join)
+    if (!aux || !ev) return cudaErrorNotReady;
+    if ((e = launch_chunk_offsets(S, st)) != cudaSuccess) return e;
+    if ((e = launch_conv(S, 0, S.max_chunks, st)) != cudaSuccess) return e;
+    if ((e = cudaEventRecord(ev[0], st)) != cudaSuccess || (e = cudaStreamWaitEvent(aux, ev[0], 0)) != cudaSuccess)
+        return e;
+    // aux is forked: from here on it is joined back whatever happens
+    const cudaError_t e_side = launch_conv_state(S, aux);
+    if ((e = cudaEventRecord(ev[1], aux)) != cudaSuccess) return e;
+    *join = ev[1];
+    if (e_side != cudaSuccess) return e_side;
+    return launch_intra(S, 0, S.max_chunks, st);
 }
 
 // The caller's stream waits for stage A's side work.
@@ -574,9 +671,16 @@ cudaError_t join_side(cudaEvent_t join, cudaStream_t st, cudaError_t prior) {
 
 // The chunk scan over the records of stage A, reading V through `v_src` (the
 // workspace's v^, or a zero block whose map reads zeros past its 64 rows).
+struct ScanSetup {
+    CUtensorMap tm_v, tm_k;
+    gdn::scan::Args sa;
+    unsigned grid;
+    decltype(&gdn::scan::gdn_scan_kernel<float, float>) kernel;   // (every instance has this signature)
+};
+
 template <typename TO>
-cudaError_t launch_scan(const gdn_config* c, const void* v_src, int64_t v_rows, void* rec_state, const int32_t* cu,
-                        int n_seqs, int64_t T, void* ws, cudaStream_t st, void* o_dst = nullptr) {
+cudaError_t prepare_scan(const gdn_config* c, const void* v_src, int64_t v_rows, void* rec_state, const int32_t* cu,
+                         int n_seqs, int64_t T, void* ws, void* o_dst, ScanSetup* S) {
     const Layout L = workspace_layout(c, T, n_seqs);
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     auto k_scan = c->state_dtype == GDN_BF16 ? gdn::scan::gdn_scan_kernel<TO, __nv_bfloat16>
@@ -584,58 +688,172 @@ cudaError_t launch_scan(const gdn_config* c, const void* v_src, int64_t v_rows, 
     cudaError_t e = ensure_smem(k_scan, 16 + (sizeof(TO) == 2 ? 0 : 1) + (c->state_dtype == GDN_BF16 ? 2 : 0),
                                 gdn::scan::SMEM_BYTES);
     if (e != cudaSuccess) return e;
-    CUtensorMap tm_v, tm_k;
-    if (!head_tile_map(&tm_v, v_src, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_v, c->n_v_heads, v_rows) ||
-        !head_tile_map(&tm_k, wsb + L.k_off, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, c->n_k_heads, T))
+    S->kernel = k_scan;
+    if (!head_tile_map(&S->tm_v, v_src, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_v, c->n_v_heads, v_rows) ||
+        !head_tile_map(&S->tm_k, wsb + L.k_off, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, c->d_k, c->n_k_heads, T))
         return cudaErrorInvalidValue;
-    gdn::scan::Args sa;
+    gdn::scan::Args& sa = S->sa;
     sa.rec_state = rec_state;
+    sa.carry = L.total > L.carry_off ? reinterpret_cast<float*>(wsb + L.carry_off) : nullptr;
+    sa.g_lo = 0;
+    sa.g_hi = 0x7fffffff;
+    sa.final_launch = 1;
     sa.cu = cu;
     sa.chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off);
     sa.flags = reinterpret_cast<int32_t*>(wsb + L.flags_off);
     sa.rec = wsb + L.rec_off;
     sa.o = o_dst ? o_dst : wsb + L.o_off;
     sa.Hk = c->n_k_heads; sa.Hv = c->n_v_heads; sa.dk = c->d_k; sa.dv = c->d_v;
-    k_scan<<<(unsigned)n_seqs * c->n_v_heads, gdn::scan::NT, gdn::scan::SMEM_BYTES, st>>>(tm_v, tm_k, sa);
+    S->grid = (unsigned)n_seqs * c->n_v_heads;
+    return cudaSuccess;
+}
+
+// The scan over global chunks [g_lo, g_hi) of every chain; `final` for the call's
+// last scan launch, which leaves the final states in rec_state.
+cudaError_t launch_scan_range(const ScanSetup& S, int64_t g_lo, int64_t g_hi, bool final, cudaStream_t st) {
+    gdn::scan::Args sa = S.sa;
+    sa.g_lo = (int32_t)g_lo;
+    sa.g_hi = (int32_t)(g_hi < 0x7fffffff ? g_hi : 0x7fffffff);
+    sa.final_launch = final ? 1 : 0;
+    S.kernel<<<S.grid, gdn::scan::NT, gdn::scan::SMEM_BYTES, st>>>(S.tm_v, S.tm_k, sa);
     return cudaGetLastError();
 }
 
+template <typename TO>
+cudaError_t launch_scan(const gdn_config* c, const void* v_src, int64_t v_rows, void* rec_state, const int32_t* cu,
+                        int n_seqs, int64_t T, void* ws, cudaStream_t st, void* o_dst = nullptr) {
+    ScanSetup S;
+    const cudaError_t e = prepare_scan<TO>(c, v_src, v_rows, rec_state, cu, n_seqs, T, ws, o_dst, &S);
+    return e != cudaSuccess ? e : launch_scan_range(S, 0, 0x7fffffff, true, st);
+}
+
+struct NormSetup {
+    CUtensorMap tm_z;
+    gdn::norm::Args na;
+    int64_t ctas, max_chunks;
+};
+
 template <typename TA, typename TO>
-cudaError_t launch_norm(const gdn_config* c, const gdn_weights* w, const void* z, const int32_t* cu, int n_seqs,
-                        int64_t T, void* out, void* ws, cudaStream_t st) {
+cudaError_t prepare_norm(const gdn_config* c, const gdn_weights* w, const void* z, const int32_t* cu, int n_seqs,
+                         int64_t T, void* out, void* ws, NormSetup* S) {
     const Layout L = workspace_layout(c, T, n_seqs);
     uint8_t* wsb = static_cast<uint8_t*>(ws);
     cudaError_t e = ensure_smem(gdn::norm::gdn_gated_norm_kernel<TA, TO>,
                                 8 + (sizeof(TA) == 4 ? 2 : 0) + (sizeof(TO) == 4 ? 1 : 0),
                                 gdn::norm::smem_bytes<TA, TO>());
     if (e != cudaSuccess) return e;
-    CUtensorMap tm_z;
     const int Hv = c->n_v_heads;
-    if (!z_rows_map(&tm_z, z, sizeof(TA) == 2, Hv * c->d_v, c->d_v, T)) return cudaErrorInvalidValue;
-    const int64_t max_chunks = (T + gdn::intra::C - 1) / gdn::intra::C + n_seqs;
-    gdn::norm::Args na;
+    if (!z_rows_map(&S->tm_z, z, sizeof(TA) == 2, Hv * c->d_v, c->d_v, T)) return cudaErrorInvalidValue;
+    S->max_chunks = (T + gdn::intra::C - 1) / gdn::intra::C + n_seqs;
+    gdn::norm::Args& na = S->na;
     na.o = wsb + L.o_off; na.norm_w = w->norm_weight;
     na.cu = cu; na.chunk_off = reinterpret_cast<int32_t*>(wsb + L.coff_off); na.out = out;
     na.flags = reinterpret_cast<int32_t*>(wsb + L.flags_off);
     na.n_seqs = n_seqs; na.Hv = Hv; na.dv = c->d_v; na.eps = c->norm_eps;
-    int64_t norm_ctas = (int64_t)sm_count() * (232448 / (int64_t)gdn::norm::smem_bytes<TA, TO>());
-    norm_ctas = norm_ctas < max_chunks * Hv ? norm_ctas : max_chunks * Hv;
+    na.g_lo = 0;
+    na.g_hi = 0x7fffffff;
+    S->ctas = (int64_t)sm_count() * (232448 / (int64_t)gdn::norm::smem_bytes<TA, TO>());
+    return cudaSuccess;
+}
+
+// The gated norm of the tiles of global chunks [g_lo, g_hi).
+template <typename TA, typename TO>
+cudaError_t launch_norm_range(const NormSetup& S, int64_t g_lo, int64_t g_hi, cudaStream_t st) {
+    gdn::norm::Args na = S.na;
+    na.g_lo = (int32_t)g_lo;
+    na.g_hi = (int32_t)(g_hi < 0x7fffffff ? g_hi : 0x7fffffff);
+    const int64_t tiles = ((g_hi < S.max_chunks ? g_hi : S.max_chunks) - g_lo) * na.Hv;
+    if (tiles <= 0) return cudaSuccess;
+    const int64_t ctas = S.ctas < tiles ? S.ctas : tiles;
     gdn::norm::gdn_gated_norm_kernel<TA, TO>
-        <<<(unsigned)norm_ctas, gdn::norm::NT, gdn::norm::smem_bytes<TA, TO>(), st>>>(tm_z, na);
+        <<<(unsigned)ctas, gdn::norm::NT, gdn::norm::smem_bytes<TA, TO>(), st>>>(S.tm_z, na);
     return cudaGetLastError();
 }
 
+template <typename TA, typename TO>
+cudaError_t launch_norm(const gdn_config* c, const gdn_weights* w, const void* z, const int32_t* cu, int n_seqs,
+                        int64_t T, void* out, void* ws, cudaStream_t st) {
+    NormSetup S;
+    const cudaError_t e = prepare_norm<TA, TO>(c, w, z, cu, n_seqs, T, out, ws, &S);
+    return e != cudaSuccess ? e : launch_norm_range<TA, TO>(S, 0, S.max_chunks, st);
+}
+
+// A whole prefill.  One range: stage A then stage B on `st`.  Several ranges
+// (seg_plan): a pipeline over three streams, ordered by events only.
+//   st (the caller's):   chunk offsets; for each range s: conv(s), intra(s)
+//   side 4 (priority):   scan(s) after intra(s) and scan(s-1)
+//   side 5:              norm(s) after scan(s) and after the last conv
+//   side 3:              the conv-state update after the last conv
+// Intra(s) needs the conv output of range s and of the tile that range s-1 ends
+// with, both before it on `st`; scan(s) carries each chain's fp32 state to
+// scan(s+1) through the workspace.  Nothing the caller sees is written before
+// the last conv has checked its range: out is written by the norms, which wait
+// for it; conv_state by the update, which waits for it; rec_state by the last
+// scan, which follows the last intra on `st` (the carry holds the states of the
+// chains that end earlier until then).  A call whose checks fail therefore
+// leaves out and the states as they were.  Every side stream that has been
+// forked is joined back to `st` on every path.
 template <typename TA, typename TO>
 cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void* q, const void* k,
                            const void* v, const void* a, const void* b, const void* z, void* conv_state,
                            void* rec_state, const int32_t* cu, int n_seqs, int64_t T, void* out,
                            void* ws, cudaStream_t st) {
     const Layout L = workspace_layout(c, T, n_seqs);
-    cudaEvent_t join = nullptr;
-    cudaError_t e = launch_stage_a<TA>(c, w, q, k, v, a, b, conv_state, cu, n_seqs, T, ws, st, &join);
-    if (e == cudaSuccess) e = launch_scan<TO>(c, static_cast<uint8_t*>(ws) + L.v_off, T, rec_state, cu, n_seqs, T, ws, st);
-    if (e == cudaSuccess) e = launch_norm<TA, TO>(c, w, z, cu, n_seqs, T, out, ws, st);
-    return join_side(join, st, e);
+    const SegPlan P = seg_plan(c, T, n_seqs);
+    if (P.n == 1) {
+        cudaEvent_t join = nullptr;
+        cudaError_t e = launch_stage_a<TA>(c, w, q, k, v, a, b, conv_state, cu, n_seqs, T, ws, st, &join);
+        if (e == cudaSuccess)
+            e = launch_scan<TO>(c, static_cast<uint8_t*>(ws) + L.v_off, T, rec_state, cu, n_seqs, T, ws, st);
+        if (e == cudaSuccess) e = launch_norm<TA, TO>(c, w, z, cu, n_seqs, T, out, ws, st);
+        return join_side(join, st, e);
+    }
+    StageA<TA> A;
+    ScanSetup B;
+    NormSetup N;
+    cudaError_t e = prepare_stage_a<TA>(c, w, q, k, v, a, b, conv_state, cu, n_seqs, T, ws, &A);
+    if (e == cudaSuccess)
+        e = prepare_scan<TO>(c, static_cast<uint8_t*>(ws) + L.v_off, T, rec_state, cu, n_seqs, T, ws, nullptr, &B);
+    if (e == cudaSuccess) e = prepare_norm<TA, TO>(c, w, z, cu, n_seqs, T, out, ws, &N);
+    if (e != cudaSuccess) return e;
+    if (!B.sa.carry) return cudaErrorInvalidValue;
+    cudaStream_t side[3] = {side_stream(4), side_stream(5), side_stream(3)};   // scan, norm, conv state
+    // events: [0, n) intra(s) done; [n, 2n) scan(s) done; 2n: last conv done; 2n+1 .. 2n+3: joins
+    const int n = P.n;
+    cudaEvent_t* ev = thread_events(kEvPipe, 2 * (size_t)n + 4);
+    if (!side[0] || !side[1] || !side[2] || !ev) return cudaErrorNotReady;
+    bool forked[3] = {false, false, false};
+    auto fork = [&](int i, cudaEvent_t after) -> cudaError_t {
+        const cudaError_t r = cudaStreamWaitEvent(side[i], after, 0);
+        if (r == cudaSuccess) forked[i] = true;
+        return r;
+    };
+    auto range_lo = [&](int s) -> int64_t { return (int64_t)s * P.len; };
+    auto range_hi = [&](int s) -> int64_t { return s == n - 1 ? A.max_chunks : (int64_t)(s + 1) * P.len; };
+
+    e = launch_chunk_offsets(A, st);
+    for (int s = 0; s < n && e == cudaSuccess; s++) {
+        if ((e = launch_conv(A, range_lo(s), range_hi(s), st)) != cudaSuccess) break;
+        if (s == n - 1 && (e = cudaEventRecord(ev[2 * n], st)) != cudaSuccess) break;
+        if ((e = launch_intra(A, range_lo(s), range_hi(s), st)) != cudaSuccess) break;
+        if ((e = cudaEventRecord(ev[s], st)) != cudaSuccess) break;
+        if ((e = fork(0, ev[s])) != cudaSuccess) break;
+        if ((e = launch_scan_range(B, range_lo(s), range_hi(s), s == n - 1, side[0])) != cudaSuccess) break;
+        if ((e = cudaEventRecord(ev[n + s], side[0])) != cudaSuccess) break;
+    }
+    if (e == cudaSuccess && (e = fork(2, ev[2 * n])) == cudaSuccess) e = launch_conv_state(A, side[2]);
+    if (e == cudaSuccess) e = fork(1, ev[2 * n]);
+    for (int s = 0; s < n && e == cudaSuccess; s++) {
+        if ((e = cudaStreamWaitEvent(side[1], ev[n + s], 0)) != cudaSuccess) break;
+        e = launch_norm_range<TA, TO>(N, range_lo(s), range_hi(s), side[1]);
+    }
+    for (int i = 0; i < 3; i++) {   // join every forked stream, whatever happened above
+        if (!forked[i]) continue;
+        cudaError_t r = cudaEventRecord(ev[2 * n + 1 + i], side[i]);
+        if (r == cudaSuccess) r = cudaStreamWaitEvent(st, ev[2 * n + 1 + i], 0);
+        if (e == cudaSuccess) e = r;
+    }
+    return e;
 }
 
 template <typename TA, typename TO, typename TS, int DK>
@@ -709,11 +927,17 @@ void gdn_config_default(gdn_config* cfg) {
     cfg->act_dtype = GDN_BF16;
     cfg->out_dtype = GDN_BF16;
     cfg->state_dtype = GDN_F32;
+    cfg->prefill_segments = 0;
 }
 
 size_t gdn_prefill_workspace_size(const gdn_config* cfg, int64_t T_total, int32_t n_seqs) {
     if (check_config(cfg) != GDN_OK || T_total < 0 || n_seqs < 0) return 0;
     return workspace_layout(cfg, T_total, n_seqs).total;
+}
+
+int32_t gdn_prefill_segments(const gdn_config* cfg, int64_t T_total, int32_t n_seqs) {
+    if (check_config(cfg) != GDN_OK || T_total < 0 || n_seqs < 0) return 0;
+    return seg_plan(cfg, T_total, n_seqs).n;
 }
 
 gdn_status gdn_prefill(const gdn_config* cfg, const gdn_weights* w, const void* q, const void* k,

@@ -27,9 +27,10 @@
 // written straight from registers:
 //     +0      B1   per 64-wide d_k half (16384 B): [-W rows | Q~ rows], K-major,
 //                  64 + 64 rows c; Q~ = diag(e^g) Q                      fp16  32768 B
-//     +32768  T    K-major [64 rows c][64 columns j]                    fp16  8192 B
-//     +40960  decay factors: e^{g_C - g_c} for c < 64, then e^{g_C}     fp32  (65 used of 1024 B)
-//     +41984  P^T  MN-major atom: row j holds P[0..63][j]               fp16  8192 B
+//     +32768  T    K-major [64 rows c][64 columns j], as fp16(T), then  fp16  2 x 8192 B
+//                  fp16(T - fp16(T)): the pair carries T to about 22 bits
+//     +49152  decay factors: e^{g_C - g_c} for c < 64, then e^{g_C}     fp32  (65 used of 1024 B)
+//     +50176  P^T  MN-major atom: row j holds P[0..63][j]               fp16  8192 B
 // (g rows past the sequence end repeat the last g, so their factors are 1.)
 // The scan applies e^{g_C - g} to U rather than to K, so K needs no copy here.
 #pragma once
@@ -38,11 +39,11 @@
 namespace gdn {
 namespace intra {
 
-constexpr int C = 64;
+constexpr int C = kChunk;
 constexpr int GH = 3;                      // value heads per round: one 4-warp group each
 constexpr int NT = 128 * GH;
-constexpr uint32_t REC_B1 = 0, REC_T = 32768, REC_G = 40960, REC_P = 41984;
-constexpr uint32_t REC_BYTES = 50176;      // 49 x 1024: every tile of a record stays 1024-aligned
+constexpr uint32_t REC_B1 = 0, REC_T = 32768, REC_G = 49152, REC_P = 50176;
+constexpr uint32_t REC_BYTES = 58368;      // 57 x 1024: every tile of a record stays 1024-aligned
 constexpr uint32_t REC_LD_BYTES = REC_G + 512 - REC_B1;   // B1, T and the decay factors: one copy
 
 constexpr uint32_t OFF_QK = 0;             // [K;Q]: 128 token rows x d_k, halves of 16384 (k rows first)
@@ -73,6 +74,7 @@ struct Args {
     int n_seqs;
     int Hk, Hv;
     uint8_t* rec;             // [total chunks][Hv][REC_BYTES]
+    int32_t g_lo;             // CTA x takes global chunk g_lo + x / Hk
 };
 
 __device__ __forceinline__ void stg128(void* p, uint32_t x, uint32_t y, uint32_t z, uint32_t w) {
@@ -185,7 +187,7 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
     const int grp = warp >> 2, qd = warp & 3, tg = tid & 127;   // value-head slot, TMEM lane quadrant
     const int Hk = p.Hk, Hv = p.Hv, G = Hv / Hk;
     const int kh = blockIdx.x % Hk;
-    const int gc = blockIdx.x / Hk;
+    const int gc = p.g_lo + (int)(blockIdx.x / Hk);
     if (gc >= p.chunk_off[p.n_seqs] || *p.flags) return;
     int lo = 0, hi = p.n_seqs - 1;   // sequence of this chunk: last s with chunk_off[s] <= gc
     while (lo < hi) {
@@ -257,9 +259,18 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
             s_b[tg] = bt;
         }
         // ---- [K;Q] [K;Q]^T: lane j holds row j of [K K^T | K Q^T] (lanes 0..63) ----
-        if (tid == 0) {
-            if (h0 == 0 && !mbar_wait_bounded(bar_ld, 0)) atomicOr((unsigned*)s_abort, 2u);
-            if (*s_abort == 0) {
+        if (warp == 0) {
+            if (h0 == 0) {
+                if (!mbar_wait_bounded(bar_ld, 0)) atomicOr((unsigned*)s_abort, 2u);
+                // rows past the sequence's end hold another sequence's tokens, or rows a later
+                // launch has yet to write: zeros, so that only finite values meet the zero gates
+                if (n < C) {
+                    zero_tile_rows(sb + OFF_QK, 4, n, lane, 32);
+                    fence_async_smem();
+                }
+                __syncwarp();
+            }
+            if (lane == 0 && *s_abort == 0) {
                 tc_fence_after();
                 constexpr uint32_t ID = idesc_f16(128, 128, 0, 0);
 #pragma unroll
@@ -367,18 +378,23 @@ gdn_intra_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         uint32_t tq[16];
         const int c = tg >> 1, jq = (tg & 1) * 32;   // row c, columns jq .. jq + 31
         if (act) {
-            uint32_t tp[16];
+            uint32_t tp[16], tl[16];
 #pragma unroll
             for (int i = 0; i < 16; i++) {
                 const int jj = jq + 2 * i;
                 const float x0 = jj <= c ? AX[c * LDA + jj] * s_b[jj] : 0.f;
                 const float x1 = jj + 1 <= c ? AX[c * LDA + jj + 1] * s_b[jj + 1] : 0.f;
                 tp[i] = pack_half2(x0, x1);
+                const float2 hi = unpack_half2(tp[i]);
+                tl[i] = pack_half2(x0 - hi.x, x1 - hi.y);   // (exact differences)
                 tq[i] = pack_half2(x0 * s_eg[jj], x1 * s_eg[jj + 1]);
             }
 #pragma unroll
-            for (int q4 = 0; q4 < 4; q4++)
-                stg128(rec + REC_T + swz128(c, jq / 8 + q4), tp[4 * q4], tp[4 * q4 + 1], tp[4 * q4 + 2], tp[4 * q4 + 3]);
+            for (int q4 = 0; q4 < 4; q4++) {
+                const uint32_t o = swz128(c, jq / 8 + q4);
+                stg128(rec + REC_T + o, tp[4 * q4], tp[4 * q4 + 1], tp[4 * q4 + 2], tp[4 * q4 + 3]);
+                stg128(rec + REC_T + 8192 + o, tl[4 * q4], tl[4 * q4 + 1], tl[4 * q4 + 2], tl[4 * q4 + 3]);
+            }
         }
         __syncthreads();   // every group is done with its X: the T' tiles overwrite the work matrices
         if (act) {

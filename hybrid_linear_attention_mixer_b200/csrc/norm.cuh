@@ -13,7 +13,7 @@
 namespace gdn {
 namespace norm {
 
-constexpr int C = 64;
+constexpr int C = kChunk;
 constexpr int NT = 256;             // 4 threads per row, d_v / 4 channels each
 
 struct Args {
@@ -25,6 +25,7 @@ struct Args {
     void* out;                  // [T][Hv][dv] out dtype
     int n_seqs, Hv, dv;
     float eps;
+    int32_t g_lo, g_hi;         // the tiles of global chunks [g_lo, g_hi)
 };
 
 template <typename TA, typename TO> __host__ __device__ constexpr uint32_t stage_bytes() {
@@ -77,11 +78,13 @@ __global__ void __launch_bounds__(NT) gdn_gated_norm_kernel(const __grid_constan
     int* s_n = reinterpret_cast<int*>(smem + STAGES * STAGE + 24);               // [STAGES] rows of the tile
     long long* s_t0 = reinterpret_cast<long long*>(smem + STAGES * STAGE + 40);  // [STAGES] first token
     const int Hv = p.Hv, dv = p.dv;
-    const int64_t n_tiles = (int64_t)p.chunk_off[p.n_seqs] * Hv;
+    const int64_t g_end = p.chunk_off[p.n_seqs] < p.g_hi ? p.chunk_off[p.n_seqs] : p.g_hi;
+    const int64_t tile0 = (int64_t)p.g_lo * Hv;
+    const int64_t n_tiles = g_end > p.g_lo ? (g_end - p.g_lo) * Hv : 0;
     const uint32_t z_bytes = (uint32_t)(C * dv * sizeof(TA));
-    // this CTA's tile i is (chunk, head) index blockIdx.x + i * gridDim.x; thread 0 issues its loads
+    // this CTA's tile i is (chunk, head) index tile0 + blockIdx.x + i * gridDim.x; thread 0 issues its loads
     auto issue = [&](int i) {
-        const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
+        const int64_t tile = tile0 + blockIdx.x + (int64_t)i * gridDim.x;
         const int st = i % STAGES;
         const int h = (int)(tile % Hv), gc = (int)(tile / Hv);
         int lo = 0, hi = p.n_seqs - 1;   // sequence of this chunk: last s with chunk_off[s] <= gc
@@ -98,7 +101,7 @@ __global__ void __launch_bounds__(NT) gdn_gated_norm_kernel(const __grid_constan
         bulk_g2s(dst, static_cast<const uint8_t*>(p.o) + tile * O_BYTES, O_BYTES, bar);
         tma_load_2d(dst + O_BYTES, &tm_z, h * dv, (int)t0, bar);
     };
-    const int count = (int)((n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x);
+    const int count = n_tiles > blockIdx.x ? (int)((n_tiles - blockIdx.x + gridDim.x - 1) / gridDim.x) : 0;
     if (count <= 0 || *p.flags) return;
     if (threadIdx.x == 0) {
         for (int i = 0; i < STAGES; i++) mbar_init(bar0 + 8 * i, 1);
@@ -124,7 +127,7 @@ __global__ void __launch_bounds__(NT) gdn_gated_norm_kernel(const __grid_constan
             fence_async_smem();
             issue(i + STAGES - 1);
         }
-        const int64_t tile = blockIdx.x + (int64_t)i * gridDim.x;
+        const int64_t tile = tile0 + blockIdx.x + (int64_t)i * gridDim.x;
         const int h = (int)(tile % Hv);
         const int64_t t0 = s_t0[st];
         const int n = s_n[st];

@@ -10,11 +10,14 @@
 //     O   = (Q~ S0^T + P U) / sqrt(d_k)
 //     S_C = e^{g_C} S0 + (D U)^T K
 // o goes out as [chunk][head][64][128] tiles; the gated RMSNorm that follows
-// runs in norm.cuh, in parallel over all tiles.
+// runs in norm.cuh, in parallel over all tiles.  A launch may walk only a range
+// of global chunks (a pipelined prefill): the state then passes to the next
+// launch in fp32 through a carry buffer, so the arithmetic is the same as in
+// one launch, bit for bit.
 //
 // A tcgen05.mma costs about the same whatever its N up to 128, so products that
 // share an A operand are fused into one wide-N MMA, and A operands live in TMEM:
-//   (c)   V^T T^T,              N = 64  -> U2^T          [A: V, shared memory]
+//   (c)   V^T T^T,              N = 64  -> U2^T          [A: V, shared memory; T as fp16 hi + lo]
 //   MMA1  S [-W ; Q~]^T,        N = 128 -> [U2^T | O^T] += [A: S, TMEM]
 //   MMA2a (D U)^T K,            N = 128 -> S  +=          [A: (D U)^T, TMEM; B: k^, MN-major]
 //   MMA2b U^T P^T,              N = 64  -> O^T +=         [A: U^T, TMEM; B: P^T, MN-major]
@@ -46,7 +49,7 @@
 namespace gdn {
 namespace scan {
 
-constexpr int C = 64;
+constexpr int C = kChunk;
 constexpr int NW = 512;               // 16 worker warps: 4 per TMEM lane quadrant
 constexpr int IW = NW / 32;           // the issuing warp: every MMA
 constexpr int LW = IW + 1;            // the loading warp: every copy
@@ -54,8 +57,8 @@ constexpr int NMAIN = NW + 32;        // workers + issuer: they meet at named ba
 constexpr int NT = NMAIN + 32;
 
 // Shared memory (bytes from a 1024-aligned base); pairs are indexed by chunk parity.
-constexpr uint32_t OFF_R = 0;           // x2: the record's B1 image (32 KiB), T (8 KiB), decay factors
-constexpr uint32_t R_STRIDE = 41984;
+constexpr uint32_t OFF_R = 0;           // x2: the record's B1 image (32 KiB), T hi and lo (16 KiB), decay factors
+constexpr uint32_t R_STRIDE = 50176;
 constexpr uint32_t R_T = intra::REC_T - intra::REC_B1, R_G = intra::REC_G - intra::REC_B1;
 constexpr uint32_t OFF_V = OFF_R + 2 * R_STRIDE;     // V x2: 64 token rows x d_v, halves of 8192
 constexpr uint32_t OFF_B2 = OFF_V + 2 * 16384;       // x2: [K half 0 | K half 1 | P^T], MN-major atoms
@@ -77,6 +80,9 @@ constexpr uint32_t B2_BYTES = 2 * 8192 + 8192;                  // k^ halves + P
 
 struct Args {
     void* rec_state;            // [N][Hv][dv][dk] state dtype (fp32 or bf16), in/out
+    float* carry;               // [N][Hv][dv][dk] fp32: the state from one launch over a chunk range to the next
+    int32_t g_lo, g_hi;         // this launch walks global chunks [g_lo, g_hi) of every chain
+    int32_t final_launch;       // nonzero: the call's last launch, which writes the final states
     const int32_t* cu;          // [N+1]
     const int32_t* chunk_off;   // [N+1]
     const int32_t* flags;       // nonzero: a device check of the call failed, write nothing
@@ -138,10 +144,32 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant_
     const int Hv = p.Hv, dk = p.dk, dv = p.dv;
     const int seq = blockIdx.x / Hv, h = blockIdx.x % Hv;
     const int kh = h / (Hv / p.Hk);
-    const int64_t s0 = p.cu[seq], s1 = p.cu[seq + 1];
-    const int nchunks = (int)((s1 - s0 + C - 1) / C);
-    if (nchunks <= 0 || *p.flags) return;
-    const int64_t first = (int64_t)p.chunk_off[seq] * Hv + h;   // (chunk, head) index of chunk 0
+    const int n_all = (int)((p.cu[seq + 1] - (int64_t)p.cu[seq] + C - 1) / C);   // chunks of the sequence
+    if (n_all <= 0 || *p.flags) return;
+    // This launch walks chunks [c0, c1) of the sequence.  Its start state is rec_state at the
+    // sequence's first chunk, else the carry a launch before left; its end state goes to
+    // rec_state after the sequence's last chunk in the call's last launch, else to the carry.
+    const int cfirst = p.chunk_off[seq];
+    const int c0 = p.g_lo > cfirst ? p.g_lo - cfirst : 0;
+    const int c1 = p.g_hi - cfirst < n_all ? p.g_hi - cfirst : n_all;
+    TS* gstate = static_cast<TS*>(p.rec_state) + ((int64_t)seq * Hv + h) * dv * dk;
+    float* cstate = p.carry ? p.carry + ((int64_t)seq * Hv + h) * dv * dk : nullptr;
+    if (c0 >= c1) {
+        // a sequence that ended before this range: the last launch moves its end state from the carry
+        if (p.final_launch && c0 >= n_all && p.g_lo > cfirst && cstate) {
+            for (int i = 4 * threadIdx.x; i < dv * dk; i += 4 * NT)
+                st_state4(gstate + i, ld_state4(cstate + i));
+        }
+        return;
+    }
+    const bool from_rec = c0 == 0, to_rec = c1 == n_all && p.final_launch;
+    if ((!from_rec || !to_rec) && !cstate) return;   // (the host always passes a carry when it splits a chain)
+    const int nchunks = c1 - c0;
+    // tokens in this launch's last chunk: the rows after them are zeroed before the tensor cores
+    // read them (they hold another sequence's tokens, or rows a later launch has yet to write)
+    const int n_tail = c1 == n_all ? (int)(p.cu[seq + 1] - p.cu[seq] - (int64_t)(n_all - 1) * C) : C;
+    const int64_t s0 = p.cu[seq] + (int64_t)c0 * C;
+    const int64_t first = ((int64_t)cfirst + c0) * Hv + h;   // (chunk, head) index of chunk c0
     const uint8_t* rec0 = p.rec + first * intra::REC_BYTES;
     const int64_t rec_stride = (int64_t)Hv * intra::REC_BYTES;
     uint8_t* otile0 = static_cast<uint8_t*>(p.o) + first * O_BYTES;
@@ -196,14 +224,14 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant_
         tmem_relinquish();
     }
     const int dv_r = 32 * qd + lane;   // this worker's state row; columns [32 cs, 32 cs + 32)
-    TS* gstate = static_cast<TS*>(p.rec_state) + ((int64_t)seq * Hv + h) * dv * dk;
     float Sv[32];   // this worker's slice of the state at the start of the current chunk
     if (worker) {
 #pragma unroll
         for (int i4 = 0; i4 < 8; i4++) {   // 16-byte loads (d_k and the slice start are multiples of 4)
             const int col = 32 * cs + 4 * i4;
             float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
-            if (dv_r < dv && col < dk) v = ld_state4(gstate + (int64_t)dv_r * dk + col);
+            if (dv_r < dv && col < dk)
+                v = from_rec ? ld_state4(gstate + (int64_t)dv_r * dk + col) : ld_state4(cstate + (int64_t)dv_r * dk + col);
             Sv[4 * i4] = v.x; Sv[4 * i4 + 1] = v.y; Sv[4 * i4 + 2] = v.z; Sv[4 * i4 + 3] = v.w;
         }
     }
@@ -277,9 +305,15 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant_
     // the tensor pipe runs one thread's MMAs in order)
     auto issue_c = [&](int ce) {
         const int bb = ce & 1;
+        if (ce == nchunks - 1 && n_tail < C) {
+            zero_tile_rows(sb + OFF_V + bb * 16384, 2, n_tail, lane, 32);
+            fence_async_smem();
+            __syncwarp();
+        }
 #pragma unroll
-        for (int ks = 0; ks < 4; ks++)
-            mma_f16_w(tmem + acc_u(bb), dV0 + bb * 1024 + ks * 128, dT0 + bb * (R_STRIDE >> 4) + ks * 2, ID_C, ks > 0);
+        for (int ks = 0; ks < 8; ks++)   // T = fp16(T) + its fp16 remainder: two passes over K
+            mma_f16_w(tmem + acc_u(bb), dV0 + bb * 1024 + (ks & 3) * 128,
+                      dT0 + bb * (R_STRIDE >> 4) + (ks >> 2) * (8192 >> 4) + (ks & 3) * 2, ID_C, ks > 0);
     };
     // fp16 copy of the state: the A operand of MMA1
     auto put_state_a = [&]() {
@@ -375,7 +409,14 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant_
         GDN_MMA_WAIT();
 
         // ---- U^T and (D U)^T -> fp16 A operands; the issuer meanwhile waits for MMA2's operands ----
-        if (warp == IW) wait_par(bar_b20, ci);
+        if (warp == IW) {
+            wait_par(bar_b20, ci);
+            if (ci == nchunks - 1 && n_tail < C) {
+                zero_tile_rows(sb + OFF_B2 + b * B2_STRIDE, 2, n_tail, lane, 32);
+                fence_async_smem();
+                __syncwarp();
+            }
+        }
         if (worker) {
             uint32_t r16[16], u[8], ud[8];
             tmem_ld16(tl + acc_u(b) + 16 * cs, r16);
@@ -424,9 +465,11 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant_
 #pragma unroll
                 for (int i4 = 0; i4 < 8; i4++) {
                     const int col = 32 * cs + 4 * i4;
-                    if (dv_r < dv && col < dk)
-                        st_state4(gstate + (int64_t)dv_r * dk + col,
-                                  make_float4(Sv[4 * i4], Sv[4 * i4 + 1], Sv[4 * i4 + 2], Sv[4 * i4 + 3]));
+                    const float4 x = make_float4(Sv[4 * i4], Sv[4 * i4 + 1], Sv[4 * i4 + 2], Sv[4 * i4 + 3]);
+                    if (dv_r < dv && col < dk) {
+                        if (to_rec) st_state4(gstate + (int64_t)dv_r * dk + col, x);
+                        else st_state4(cstate + (int64_t)dv_r * dk + col, x);
+                    }
                 }
             }
         }

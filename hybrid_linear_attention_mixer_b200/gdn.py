@@ -45,7 +45,7 @@ class _CConfig(ctypes.Structure):
                 ("conv_kernel", ctypes.c_int32), ("chunk", ctypes.c_int32),
                 ("l2_eps", ctypes.c_float), ("norm_eps", ctypes.c_float),
                 ("act_dtype", ctypes.c_int32), ("out_dtype", ctypes.c_int32),
-                ("state_dtype", ctypes.c_int32)]
+                ("state_dtype", ctypes.c_int32), ("prefill_segments", ctypes.c_int32)]
 
 
 class _CSegment(ctypes.Structure):
@@ -58,7 +58,7 @@ class _CWeights(ctypes.Structure):
 
 
 _lib = None
-EXPORTS = ("gdn_config_default", "gdn_prefill_workspace_size", "gdn_prefill", "gdn_decode",
+EXPORTS = ("gdn_config_default", "gdn_prefill_workspace_size", "gdn_prefill_segments", "gdn_prefill", "gdn_decode",
            "gdn_decode_multi", "gdn_linear", "gdn_in_proj", "gdn_out_proj", "gdn_cp_workspace_size",
            "gdn_cp_local", "gdn_cp_finish", "gdn_prefill_host_workspace_size", "gdn_prefill_host",
            "gdn_check_device_error", "gdn_status_string", "gdn_last_cuda_error")
@@ -79,6 +79,8 @@ def lib() -> ctypes.CDLL:
         L.gdn_config_default.restype = None
         L.gdn_prefill_workspace_size.argtypes = [vp, i64, i32]
         L.gdn_prefill_workspace_size.restype = sz
+        L.gdn_prefill_segments.argtypes = [vp, i64, i32]
+        L.gdn_prefill_segments.restype = i32
         L.gdn_prefill.argtypes = [vp, vp] + [vp] * 8 + [vp, i32, i64, vp, vp, sz, vp]
         L.gdn_prefill.restype = ctypes.c_int
         L.gdn_decode.argtypes = [vp, vp] + [vp] * 8 + [i32, vp, vp]
@@ -129,6 +131,7 @@ class Config:
     act_dtype: torch.dtype = torch.bfloat16
     out_dtype: torch.dtype = torch.bfloat16
     state_dtype: torch.dtype = torch.float32   # bf16: the recurrent state stored in bf16
+    prefill_segments: int = 0                  # chunk ranges a prefill is pipelined over; 0: automatic
 
     @property
     def channels(self) -> int:
@@ -137,7 +140,7 @@ class Config:
     def c(self) -> _CConfig:
         return _CConfig(self.n_k_heads, self.n_v_heads, self.d_k, self.d_v, self.conv_kernel,
                         self.chunk, self.l2_eps, self.norm_eps, _DT[self.act_dtype],
-                        _DT[self.out_dtype], _DT[self.state_dtype])
+                        _DT[self.out_dtype], _DT[self.state_dtype], self.prefill_segments)
 
 
 def _ptr(t):
@@ -169,6 +172,13 @@ def _weights(w: dict, device) -> _CWeights:
 def workspace_size(cfg: Config, T_total: int, n_seqs: int) -> int:
     c = cfg.c()
     return int(lib().gdn_prefill_workspace_size(ctypes.byref(c), int(T_total), int(n_seqs)))
+
+
+def prefill_segments(cfg: Config, T_total: int, n_seqs: int) -> int:
+    """Chunk ranges a prefill of this size is pipelined over (1: one piece); a call
+    launches 2 + 4 n kernels (6 for n = 1)."""
+    c = cfg.c()
+    return int(lib().gdn_prefill_segments(ctypes.byref(c), int(T_total), int(n_seqs)))
 
 
 def prefill(cfg: Config, w: dict, q, k, v, a, b, z, conv_state, rec_state, cu_seqlens,

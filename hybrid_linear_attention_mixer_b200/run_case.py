@@ -1,6 +1,7 @@
 """Run one synthetic workload through the public API (no timing, no oracle).
 
     python -m hybrid_linear_attention_mixer_b200.run_case --case prefill_4k --iters 2
+    python -m hybrid_linear_attention_mixer_b200.run_case --case prefill_256k --tokens 16384 --segments 1
     python -m hybrid_linear_attention_mixer_b200.run_case --case decode_256 --batch 64 --iters 3
     python -m hybrid_linear_attention_mixer_b200.run_case --proj --tokens 4096 --iters 1
     python -m hybrid_linear_attention_mixer_b200.run_case --case decode_256 --batch 64 --multi 4 --state bf16
@@ -35,6 +36,8 @@ def main():
     ap.add_argument("--multi", type=int, default=0,
                     help="decode: this many consecutive tokens per sequence in one gdn_decode_multi call")
     ap.add_argument("--state", default="fp32", choices=("fp32", "bf16"), help="recurrent state storage")
+    ap.add_argument("--segments", type=int, default=0,
+                    help="prefill: chunk ranges the call is pipelined over (0: automatic, 1: one piece)")
     ap.add_argument("--proj", action="store_true",
                     help="run the input and output projections (hidden 2560) at --tokens instead")
     args = ap.parse_args()
@@ -57,7 +60,7 @@ def main():
         c = inputs.make_case(args.case, T=args.tokens)
     act = torch.bfloat16 if c.bf16 else torch.float32
     cfg = gdn.Config(c.n_k_heads, c.n_v_heads, c.d_k, c.d_v, c.conv_kernel, 64, c.l2_eps, c.norm_eps,
-                     act, act, torch.bfloat16 if args.state == "bf16" else torch.float32)
+                     act, act, torch.bfloat16 if args.state == "bf16" else torch.float32, args.segments)
     w = {n: torch.from_numpy(np.ascontiguousarray(c.weights[n])).to(dev)
          for n in ("conv_w", "A_log", "dt_bias", "norm_w")}
     d = {n: _act(c.acts[n], dev) for n in "qkvabz"}

@@ -86,7 +86,16 @@ typedef struct {
                              (the layer's fp32 state).  GDN_BF16 stores the state in bf16
                              (half the bytes a decode step moves); every step still
                              computes in fp32 and rounds the stored state to nearest even */
+    int32_t prefill_segments; /* chunk ranges a prefill is pipelined over (0 = automatic,
+                             the default; 1 = none; at most GDN_PREFILL_MAX_SEGMENTS).  The
+                             ranges' conv and intra-chunk kernels run on the caller's stream
+                             while the state chain walks the ranges before them on a
+                             high-priority stream of the library's own, so chains too few to
+                             fill the GPU overlap the work that feeds them.  The results do
+                             not depend on it, bit for bit */
 } gdn_config;
+
+#define GDN_PREFILL_MAX_SEGMENTS 32
 
 typedef struct {
     const float* conv_weight;  /* [2*H_k*d_k + H_v*d_v][K], channel order q | k | v;
@@ -103,6 +112,13 @@ void gdn_config_default(gdn_config* cfg);
 /* Bytes of device workspace gdn_prefill needs for T_total packed tokens.
  * Returns 0 for an invalid or unsupported config. */
 size_t gdn_prefill_workspace_size(const gdn_config* cfg, int64_t T_total, int32_t n_seqs);
+
+/* Chunk ranges gdn_prefill pipelines a call of this size over (see
+ * gdn_config.prefill_segments): 1 when it runs in one piece; with n > 1 ranges a
+ * call launches 2 + 4 n kernels (else 6).  Automatic (prefill_segments 0): at
+ * most 8 ranges of at least 32 chunks when the call has at most 96 chains
+ * (n_seqs x H_v); else 1.  Returns 0 for an invalid config. */
+int32_t gdn_prefill_segments(const gdn_config* cfg, int64_t T_total, int32_t n_seqs);
 
 /*
  * Packed variable-length prefill.
@@ -311,8 +327,8 @@ gdn_status gdn_prefill_host(const gdn_config* cfg, const gdn_weights* w,
  *   - Size limit: a request needing more than GDN_NOALLOC_SCRATCH_BYTES of
  *     workspace is rejected with GDN_ERR_WORKSPACE, before any launch.  The
  *     needed size is gdn_prefill_workspace_size(cfg, T_total, n_seqs).  At the
- *     published shape that is 70,400 bytes per token plus about 3.2 MB per
- *     sequence, so up to 896 tokens in one sequence.  Longer prompts can be
+ *     published shape that is 76,544 bytes per token plus about 3.6 MB per
+ *     sequence, so up to 823 tokens in one sequence.  Longer prompts can be
  *     split into consecutive calls, since the states carry from one call to
  *     the next.
  *   - First call on a device: it looks up the array's device address with

@@ -49,17 +49,46 @@ def test_workspace_size(lib):
     cfg = gdn.Config()
     T = 4096
     # fp16 q^, k^ [T, 16*128] and v^ [T, 48*128]; chunk offsets [N+1] and the check word,
-    # int32 (256-byte rounded); per (chunk, value head) a 49 KiB intra-chunk record and a
+    # int32 (256-byte rounded); per (chunk, value head) a 57 KiB intra-chunk record and a
     # [64][128] o tile of the output dtype, with at most ceil(T / 64) + N chunks
+    # A call pipelined over chunk ranges (automatic for up to 2 sequences and T_total of 64
+    # chunks or more; prefill_segments > 1 asks for it) adds each chain's fp32 state,
+    # [N][48][128][128].
     conv = 2 * T * 2048 * 2 + T * 6144 * 2
-    per_chunk = 48 * (50176 + 64 * 128 * 2)
-    assert gdn.workspace_size(cfg, T, 1) == conv + 256 + (T // 64 + 1) * per_chunk
+    per_chunk = 48 * (58368 + 64 * 128 * 2)
+    carry = 48 * 128 * 128 * 4
+    assert gdn.workspace_size(cfg, T, 1) == conv + 256 + (T // 64 + 1) * per_chunk + carry
+    assert gdn.workspace_size(gdn.Config(prefill_segments=1), T, 1) == conv + 256 + (T // 64 + 1) * per_chunk
+    assert gdn.workspace_size(cfg, T, 2) == conv + 256 + (T // 64 + 2) * per_chunk + 2 * carry
     assert gdn.workspace_size(cfg, T, 3) == conv + 256 + (T // 64 + 3) * per_chunk
+    assert gdn.workspace_size(gdn.Config(prefill_segments=4), T, 3) == conv + 256 + (T // 64 + 3) * per_chunk + 3 * carry
+    assert gdn.workspace_size(cfg, 4032, 1) == 2 * 4032 * 2048 * 2 + 4032 * 6144 * 2 + 256 + 64 * per_chunk
+    assert gdn.workspace_size(cfg, 4033, 1) == 2 * 4033 * 2048 * 2 + 4033 * 6144 * 2 + 256 + 65 * per_chunk + carry
     f32 = gdn.Config(out_dtype=__import__("torch").float32)
-    assert gdn.workspace_size(f32, T, 1) == conv + 256 + (T // 64 + 1) * 48 * (50176 + 64 * 128 * 4)
+    assert gdn.workspace_size(f32, T, 1) == conv + 256 + (T // 64 + 1) * 48 * (58368 + 64 * 128 * 4) + carry
     assert gdn.workspace_size(cfg, T, 63) == conv + 512 + (T // 64 + 63) * per_chunk
     assert gdn.workspace_size(cfg, 0, 0) == 256
     assert gdn.workspace_size(gdn.Config(d_k=48), T, 1) == 0
+    assert gdn.workspace_size(gdn.Config(prefill_segments=-1), T, 1) == 0
+    assert gdn.workspace_size(gdn.Config(prefill_segments=33), T, 1) == 0
+
+
+def test_prefill_segments_plan(lib):
+    cfg = gdn.Config()
+    # automatic: at most 8 ranges of at least 32 chunks for at most 96 chains (2 sequences of 48 heads)
+    assert gdn.prefill_segments(cfg, 4096, 1) == 2
+    assert gdn.prefill_segments(cfg, 4096, 2) == 2
+    assert gdn.prefill_segments(cfg, 4096, 3) == 1
+    assert gdn.prefill_segments(cfg, 4032, 1) == 1 and gdn.prefill_segments(cfg, 4033, 1) == 2
+    assert gdn.prefill_segments(cfg, 16384, 1) == 8
+    assert gdn.prefill_segments(cfg, 262144, 1) == 8
+    assert gdn.prefill_segments(cfg, 0, 0) == 1
+    # asked for: ranges of ceil(chunks / n) chunks, never more ranges than chunks
+    assert gdn.prefill_segments(gdn.Config(prefill_segments=7), 4096, 1) == 7
+    assert gdn.prefill_segments(gdn.Config(prefill_segments=32), 4096, 5) == 32
+    assert gdn.prefill_segments(gdn.Config(prefill_segments=3), 100, 1) == 2
+    assert gdn.prefill_segments(gdn.Config(prefill_segments=1), 262144, 1) == 1
+    assert gdn.prefill_segments(gdn.Config(prefill_segments=33), 4096, 1) == 0
 
 
 def _call_prefill(lib, cfg, w=True, ptr=0x1000, T=16, n=1, ws_bytes=1 << 30, ws=0x100000):

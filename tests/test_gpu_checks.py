@@ -62,11 +62,14 @@ def test_bounded_wait_runs_out_reports_timeout_and_the_gpu_stays_usable():
     gdn.check_device_error()
 
 
-def _prefill_raw(c, cu, acts=None):
+def _prefill_raw(c, cu, acts=None, segments=0):
     """gdn_prefill with cu_seqlens given as is; returns the device tensors and the
-    status gdn_check_device_error reports."""
+    status gdn_check_device_error reports.  segments > 1 pipelines the call over
+    that many chunk ranges, whose scans run before the last range's conv checks
+    its outputs."""
     acts = c.acts if acts is None else acts
     cfg = L.config_of(c)
+    cfg.prefill_segments = segments
     w = L.weights_on(c, DEV)
     d = {n: L.t_act(acts[n], DEV) for n in "qkvabz"}
     cs = L.t_act(c.conv_state, DEV)
@@ -89,12 +92,13 @@ def _case(T, seed):
     return c
 
 
+@pytest.mark.parametrize("segments", [1, 3])
 @pytest.mark.parametrize("cu", [[0, 200, 100, 300],     # decreasing
                                 [0, 100, 160, 250],     # does not end at T_total
                                 [0, 100, 160, 290]])
-def test_malformed_cu_seqlens_is_reported_and_nothing_is_written(cu):
+def test_malformed_cu_seqlens_is_reported_and_nothing_is_written(cu, segments):
     c = _case(300, 61)
-    s, after, before = _prefill_raw(c, cu)
+    s, after, before = _prefill_raw(c, cu, segments=segments)
     assert s == SEQLENS, gdn.status_string(s)
     for x, y in zip(after, before):
         assert torch.equal(x, y)
@@ -105,19 +109,24 @@ def test_malformed_cu_seqlens_is_reported_and_nothing_is_written(cu):
     L.assert_parity(g, r)
 
 
-def test_conv_output_beyond_fp16_is_reported_and_nothing_is_written():
+# 200 tokens in 4 ranges of one chunk: [0, 1), [1, 2), [2, 3) and [3, end) of the global
+# chunks of cu_seqlens [0, 70, 120, 200] (two, one and two chunks).  Rows 50..59 fall in
+# the first range's conv; rows 185..194 (the second sequence's second chunk) in the last
+# one's, which runs after the other ranges' scans.
+@pytest.mark.parametrize("segments,rows", [(1, (50, 60)), (4, (50, 60)), (4, (185, 195))])
+def test_conv_output_beyond_fp16_is_reported_and_nothing_is_written(segments, rows):
     c = _case(200, 62)
     acts = dict(c.acts)
     v = inputs.bf16_bits_to_f32(acts["v"]).copy()
-    v[50:60] = 3.0e6          # the conv of these rows reaches millions on half the channels
+    v[rows[0]:rows[1]] = 3.0e6   # the conv of these rows reaches millions on half the channels
     acts["v"] = inputs.f32_to_bf16_bits(v)
     cu = np.array([0, 70, 120, 200], np.int32)
-    s, after, before = _prefill_raw(c, cu, acts=acts)
+    s, after, before = _prefill_raw(c, cu, acts=acts, segments=segments)
     assert s == RANGE, gdn.status_string(s)
     for x, y in zip(after, before):
         assert torch.equal(x, y)
     # large q and k are normalised, so they are in range
     acts = dict(c.acts)
     acts["q"] = inputs.f32_to_bf16_bits(inputs.bf16_bits_to_f32(c.acts["q"]) * 1.0e4)
-    s, _, _ = _prefill_raw(c, cu, acts=acts)
+    s, _, _ = _prefill_raw(c, cu, acts=acts, segments=segments)
     assert s == 0, gdn.status_string(s)

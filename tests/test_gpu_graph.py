@@ -1,7 +1,8 @@
 """The library's calls inside a CUDA graph.
 
-gdn_prefill forks two small kernels onto an internal side stream and joins them
-back with events, and gdn_cp_local runs its second scan on another; under stream
+gdn_prefill forks work onto internal side streams and joins it back with events
+(the conv-state update; when pipelined over chunk ranges, the scans and the
+norms too), and gdn_cp_local runs its second scan on another; under stream
 capture those forks become graph branches.  A captured prefill + decode step,
 replayed, must give exactly what the same calls give when run directly from the
 same starting states.
@@ -18,11 +19,13 @@ pytestmark = pytest.mark.gpu
 DEV = "cuda:0"
 
 
-def test_prefill_and_decode_replay_from_a_graph():
+@pytest.mark.parametrize("segments", [1, 3])   # 3: the prefill pipelined over three streams
+def test_prefill_and_decode_replay_from_a_graph(segments):
     lens = [300, 0, 129]
     c = inputs.make_case("prefill_4k", T=sum(lens), seed=17)
     c.cu_seqlens = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
     cfg, w = L.config_of(c), L.weights_on(c, DEV)
+    cfg.prefill_segments = segments
     N = len(lens)
     rng = np.random.default_rng(17)
     cs0 = L.t_act(inputs.f32_to_bf16_bits(rng.normal(size=(N, c.channels, 3)).astype(np.float32)), DEV)

@@ -97,7 +97,7 @@ def test_noalloc_rejects_requests_beyond_its_scratch():
     c = _case([8], 43)
     cfg = gdn.Config()
     fits = _largest_single_sequence()
-    assert fits == 896   # the limit include/gdn.h states for one sequence
+    assert fits == 823   # the limit include/gdn.h states for one sequence
     cc, cw = cfg.c(), gdn._weights(L.weights_on(c, DEV), torch.device(DEV))
     dummy = torch.zeros(16, device=DEV)
     P = ctypes.c_void_p(dummy.data_ptr())
