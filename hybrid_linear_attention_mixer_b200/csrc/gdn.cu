@@ -882,12 +882,38 @@ cudaError_t launch_decode_multi_dk(const gdn::dec::MultiArgs& m, cudaStream_t st
     return cudaGetLastError();
 }
 
+// The decode with the state streamed through shared memory (one or several tokens).
+// Persistent: as many CTAs as fit at once (at most one per unit); shapes whose
+// buffers do not fit in shared memory take the multi-token kernel instead.
+template <typename TA, typename TO, typename TS, int DK>
+cudaError_t launch_decode_stream_dk(const gdn::dec::MultiArgs& m_in, cudaStream_t st) {
+    const int G = m_in.a.Hv / m_in.a.Hk;
+    gdn::dec::MultiArgs m = m_in;
+    // the deepest ring that lets two CTAs share an SM (228 KiB, 1 KiB reserved per CTA), else one
+    auto smem_of = [&](int ns) { return gdn::dec::stream_smem_bytes<TA, TS, DK>(G, m.a.dv, m.n_tok, ns); };
+    m.stages = gdn::dec::stream_stages<TS>();
+    while (m.stages > 2 && 2 * (smem_of(m.stages) + 1024) > 233472) m.stages--;
+    const size_t smem = smem_of(m.stages);
+    if (smem > 232448) return launch_decode_multi_dk<TA, TO, TS, DK>(m, st);
+    auto kern = gdn::dec::gdn_decode_stream_kernel<TA, TO, TS, DK>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    int per_sm = 0;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, gdn::dec::SNT, smem);
+    if (e != cudaSuccess) return e;
+    const int64_t units = (int64_t)m.n_seqs * m.a.Hk;
+    int64_t grid = (int64_t)(per_sm > 0 ? per_sm : 1) * sm_count();
+    grid = grid < units ? grid : units;
+    kern<<<(unsigned)grid, gdn::dec::SNT, smem, st>>>(m);
+    return cudaGetLastError();
+}
+
 template <typename TA, typename TO, typename TS>
 cudaError_t launch_decode_multi_ts(const gdn::dec::MultiArgs& m, cudaStream_t st) {
     switch (m.a.dk) {
-        case 32: return launch_decode_multi_dk<TA, TO, TS, 32>(m, st);
-        case 64: return launch_decode_multi_dk<TA, TO, TS, 64>(m, st);
-        default: return launch_decode_multi_dk<TA, TO, TS, 128>(m, st);
+        case 32: return launch_decode_stream_dk<TA, TO, TS, 32>(m, st);
+        case 64: return launch_decode_stream_dk<TA, TO, TS, 64>(m, st);
+        default: return launch_decode_stream_dk<TA, TO, TS, 128>(m, st);
     }
 }
 template <typename TA, typename TO>
@@ -896,13 +922,27 @@ cudaError_t launch_decode_multi(const gdn::dec::MultiArgs& m, bool bf16_state, c
                       : launch_decode_multi_ts<TA, TO, float>(m, st);
 }
 
+// One token: the fp32 state streams best through registers (gdn_decode_kernel,
+// measured about 0.9 of the HBM copy rate at batch 256); the bf16 state, whose
+// rows cost as many instructions for half the bytes, through the warp-specialised
+// streamed kernel.
 template <typename TA, typename TO, typename TS>
 cudaError_t launch_decode_ts(const gdn::dec::Args& a, int n_seqs, cudaStream_t st) {
-    switch (a.dk) {
-        case 32: return launch_decode_dk<TA, TO, TS, 32>(a, n_seqs, st);
-        case 64: return launch_decode_dk<TA, TO, TS, 64>(a, n_seqs, st);
-        default: return launch_decode_dk<TA, TO, TS, 128>(a, n_seqs, st);
+    if (sizeof(TS) == 4) {
+        switch (a.dk) {
+            case 32: return launch_decode_dk<TA, TO, TS, 32>(a, n_seqs, st);
+            case 64: return launch_decode_dk<TA, TO, TS, 64>(a, n_seqs, st);
+            default: return launch_decode_dk<TA, TO, TS, 128>(a, n_seqs, st);
+        }
     }
+    gdn::dec::MultiArgs m;
+    m.a = a;
+    m.n_tok = 1;
+    m.state_snap = nullptr;
+    m.conv_snap = nullptr;
+    m.n_seqs = n_seqs;
+    m.stages = 0;   // (chosen at launch)
+    return launch_decode_multi_ts<TA, TO, TS>(m, st);
 }
 template <typename TA, typename TO>
 cudaError_t launch_decode(const gdn::dec::Args& a, int n_seqs, bool bf16_state, cudaStream_t st) {
@@ -1034,6 +1074,7 @@ gdn_status gdn_decode_multi(const gdn_config* cfg, const gdn_weights* w, const v
     da.out = out;
     da.Hk = cfg->n_k_heads; da.Hv = cfg->n_v_heads; da.dk = cfg->d_k; da.dv = cfg->d_v;
     da.l2_eps = cfg->l2_eps; da.norm_eps = cfg->norm_eps;
+    m.stages = 0;   // (chosen at launch)
     m.n_tok = n_tok;
     m.state_snap = state_snapshots;
     m.conv_snap = conv_snapshots;
