@@ -63,9 +63,12 @@ PROJ_IN_FLOP = 2 * PREFILL_T * D_MODEL * PROJ_IN_N
 PROJ_OUT_FLOP = 2 * PREFILL_T * H_V * D * D_MODEL
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 # ncu DRAM bytes (read + write) per decode launch at batch 256, taken on the
-# decode kernel whose source hashes to DECODE_SRC_SHA; null once it changes.
+# fp32-state decode kernel (gdn_decode_kernel) whose source text hashes to
+# DECODE_SRC_SHA; null once that kernel's text changes.
 DECODE_TRAFFIC = 1593363968          # mean of 3 launches at batch 256
-DECODE_SRC_SHA = "1ad3fb952dfab07f"
+DECODE_SRC_SHA = "4315b287d18a287c"
+DECODE_KERNEL_TEXT = ("template <typename TA, typename TO, typename TS, int DK>\n"
+                      "__global__ void __launch_bounds__(NT) gdn_decode_kernel", "// Multi-token rows")
 
 
 def peaks():
@@ -77,9 +80,17 @@ def peaks():
     return dict(FALLBACK_PEAKS), "fallback"
 
 
-def src_sha(name):
-    with open(os.path.join(ROOT, "hybrid_linear_attention_mixer_b200", "csrc", name), "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+def src_sha(name, section=None):
+    """sha256 (16 hex digits) of a source file, or of the text from section[0] up to section[1]."""
+    with open(os.path.join(ROOT, "hybrid_linear_attention_mixer_b200", "csrc", name)) as f:
+        text = f.read()
+    if section is not None:
+        a = text.find(section[0])
+        b = text.find(section[1], a) if a >= 0 else -1
+        if b < 0:
+            return None
+        text = text[a:b]
+    return hashlib.sha256(text.encode()).hexdigest()[:16]
 
 
 class ClockSampler:
@@ -456,7 +467,7 @@ def main():
         dec_gbs = DECODE_BYTES_PER_STEP / dec_launch_s / 1e9
         pre_tflops = PREFILL_FLOP_PER_TOKEN * PREFILL_T / (pre_ms / 1e3 / K) / 1e12
         pre_gbs = (PREFILL_BYTES_PER_TOKEN * PREFILL_T + PREFILL_STATE_BYTES) / (pre_ms / 1e3 / K) / 1e9
-        traffic = DECODE_TRAFFIC if DECODE_SRC_SHA == src_sha("decode.cuh") else None
+        traffic = DECODE_TRAFFIC if DECODE_SRC_SHA == src_sha("decode.cuh", DECODE_KERNEL_TEXT) else None
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": (pre_ms + dec_ms) / K, "higher_is_better": True,
