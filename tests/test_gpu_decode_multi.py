@@ -6,7 +6,9 @@ state (checking tokens that a multi-token-prediction head drafted).
   to the order of fp32 additions inside a state row's dot products.
 * It matches the fp64 oracle run over the same tokens as one prefill per sequence,
   and every state snapshot matches the oracle run over that prefix of the tokens.
-* The largest n_tok at the small head shape with fp32 activations.
+* The largest n_tok at the small head shape with fp32 activations, and at the
+  published shape, whose 16-token buffers exceed the streamed kernel's shared
+  memory (the call takes the register-streaming multi-token kernel instead).
 """
 import numpy as np
 import pytest
@@ -54,7 +56,7 @@ def _decode_steps_f32(c, steps):
     return outs, cs, rs, snaps, csnaps
 
 
-@pytest.mark.parametrize("n_tok", [1, 4, 7])
+@pytest.mark.parametrize("n_tok", [1, 4, 7, 16])
 def test_decode_multi_equals_decode_steps(n_tok):
     c = inputs.make_case("decode_256", T=n_tok, n_seqs=64)
     outs, cs1, rs1, snaps, csnaps = _decode_steps_f32(c, c.steps)
