@@ -29,8 +29,9 @@
 //
 // Per chunk, the critical chain is MMA1 -> U^T to fp16 -> MMA2a -> the fp16 copy
 // of the new state.  A dedicated warp issues every MMA: right after MMA1 it
-// queues (c) of the next chunk, which runs while U is converted, and right after
-// MMA2a it queues MMA2b, which runs while the state is converted; it waits for
+// queues the first half of (c) of the next chunk, which runs while U is
+// converted, and right after MMA2a it queues MMA2b and then the second half of
+// (c), which run while the state is converted; it waits for
 // the next MMA's operands while the workers convert, so each conversion is
 // followed by an immediate issue.  While MMA1 runs, the 16 worker warps write the
 // decayed state accumulator and the previous chunk's o tile (once its MMA2b has
@@ -303,17 +304,21 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant_
     constexpr uint32_t ID_C = idesc_f16(128, 64, 1, 0);     // (c)
     // (c) of chunk ce: U2^T = V^T T^T into its U accumulator (MMA1 of chunk ce accumulates onto it;
     // the tensor pipe runs one thread's MMAs in order)
-    auto issue_c = [&](int ce) {
+    // T = fp16(T) + its fp16 remainder: pass 0 over fp16(T) (which starts the accumulator), pass 1
+    // over the remainder.  They are queued where the tensor pipe would otherwise idle: pass 0 of
+    // the next chunk right after MMA1 (it runs while U is converted), pass 1 right after MMA2b
+    // (while the state is converted); MMA1 of that chunk follows both in the pipe.
+    auto issue_c = [&](int ce, int pass) {
         const int bb = ce & 1;
-        if (ce == nchunks - 1 && n_tail < C) {
+        if (pass == 0 && ce == nchunks - 1 && n_tail < C) {
             zero_tile_rows(sb + OFF_V + bb * 16384, 2, n_tail, lane, 32);
             fence_async_smem();
             __syncwarp();
         }
 #pragma unroll
-        for (int ks = 0; ks < 8; ks++)   // T = fp16(T) + its fp16 remainder: two passes over K
-            mma_f16_w(tmem + acc_u(bb), dV0 + bb * 1024 + (ks & 3) * 128,
-                      dT0 + bb * (R_STRIDE >> 4) + (ks >> 2) * (8192 >> 4) + (ks & 3) * 2, ID_C, ks > 0);
+        for (int ks = 0; ks < 4; ks++)
+            mma_f16_w(tmem + acc_u(bb), dV0 + bb * 1024 + ks * 128,
+                      dT0 + bb * (R_STRIDE >> 4) + pass * (8192 >> 4) + ks * 2, ID_C, pass > 0 || ks > 0);
     };
     // fp16 copy of the state: the A operand of MMA1
     auto put_state_a = [&]() {
@@ -354,7 +359,8 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant_
     if (warp == IW) {
         wait_par(bar_ld0, 0);
         tc_fence_after();
-        issue_c(0);
+        issue_c(0, 0);
+        issue_c(0, 1);
     }
     tc_fence_before();
     main_sync();
@@ -383,10 +389,10 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant_
                              dB1 + b * (R_STRIDE >> 4) + (ks >> 2) * 1024 + (ks & 3) * 2, ID_1, 1);
             mma_commit_w(bar);
             if (lane == 0) mbar_arrive(ev_iss);
-            if (ci + 1 < nchunks) {   // (c) of the next chunk runs while U is converted
+            if (ci + 1 < nchunks) {   // (c) of the next chunk, pass 0, runs while U is converted
                 wait_par(bar_ld0, ci + 1);
                 tc_fence_after();
-                issue_c(ci + 1);
+                issue_c(ci + 1, 0);
             }
         }
         // ---- workers, while MMA1 runs: the decayed state accumulator and the U^T decay factors ----
@@ -448,6 +454,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant_
             for (int ks = 0; ks < 4; ks++)
                 mma_f16_ta_w(tmem + acc_o(b), tmem + TA_U + ks * 8, dP + b * (B2_STRIDE >> 4) + ks * 128, ID_2B, 1);
             mma_commit_w(ev20 + 8 * b);   // B2 buffer b is free once MMA2b has read P^T
+            if (ci + 1 < nchunks) issue_c(ci + 1, 1);   // (c) of the next chunk, pass 1, while S is converted
         }
         GDN_MMA_WAIT();
 
