@@ -380,9 +380,7 @@ conv_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         for (int i = 0; i < BUFS; i++) mbar_init(bar0 + 8 * i, 1);
         fence_mbar_init();
         *s_abort = 0;
-        issue(0);
-        issued = 1;
-        if (count > 1) issue(1), issued = 2;
+        for (; issued < BUFS - 1 && issued < count; issued++) issue(issued);
     }
     if (tid < 32) search(0);
     float w[8][4];
@@ -399,10 +397,10 @@ conv_tile_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant
         if (!mbar_wait_bounded(bar0 + 8 * (jj % BUFS), (jj / BUFS) & 1)) atomicOr((unsigned*)s_abort, 1u);
         __syncthreads();   // every thread is done with tile jj - 1 (buffer, sequence table)
         if (*s_abort) break;
-        if (tid == 0 && jj + 2 < count) {            // into the buffer of tile jj - 1
+        if (tid == 0 && jj + BUFS - 1 < count) {     // into the buffer of tile jj - 1
             fence_async_smem();
-            issue(jj + 2);
-            issued = jj + 3;
+            issue(jj + BUFS - 1);
+            issued = jj + BUFS;
         }
         if (tid < 32 && jj + 1 < count) search(jj + 1);
         const uint8_t* tb = smem + (jj % BUFS) * TILE_BYTES + (cg >> 3) * BOX_BYTES + (cg & 7) * 16;
