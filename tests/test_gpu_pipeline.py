@@ -69,8 +69,10 @@ def test_range_counts_give_the_same_bits_as_one_piece(state_dtype):
 # The first sequence ends 10 tokens into its 16th chunk, right where the 2-range
 # plan of 2,048 tokens in 2 ranges (32 chunks, ranges of 16) cuts: that chunk's tile loads
 # reach rows 992..1023, which only the second range's conv writes.
+# The last case packs 20 one-chunk sequences of 40 tokens before a long one, so that every
+# range boundary among the first 20 chunks falls right after a partial chunk.
 @pytest.mark.parametrize("lens,segments", [([970, 1078], 2), ([100, 1, 1500, 63, 384], 5),
-                                           ([0, 2048, 0], 3)])
+                                           ([0, 2048, 0], 3), ([40] * 20 + [1000], 7)])
 def test_partial_chunks_at_range_boundaries(lens, segments):
     c, d, cs0, rs0, cu = _problem(lens, 83 + len(lens))
     ref = _run(c, d, cs0, rs0, cu, 1)
