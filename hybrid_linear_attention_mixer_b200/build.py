@@ -9,7 +9,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "libgdn_b200.so")
 SOURCES = [os.path.join(HERE, "csrc", f) for f in
-           ("gdn.cu", "device.cuh", "conv.cuh", "intra.cuh", "scan.cuh", "norm.cuh", "decode.cuh", "gemm.cuh", "cp.cuh")]
+           ("gdn.cu", "device.cuh", "conv.cuh", "intra.cuh", "scan.cuh", "norm.cuh", "decode.cuh", "gemm.cuh", "cp.cuh",
+            "fixup.cuh")]
 HEADERS = [os.path.join(ROOT, "include", "gdn.h")]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo",
               "-Xcompiler", "-fPIC", "-shared"]

@@ -44,7 +44,8 @@ constexpr int CT = 128;   // threads: one per column (d <= 128)
 // Rows are independent, so one CTA takes CR rows of one head through every
 // step; thread k holds column k.  state_out may alias state_in.
 __global__ void __launch_bounds__(CT) fold_kernel(const float* state_in, const float* summaries, int rank, int Hv,
-                                                  int d, float* state_out) {
+                                                  int d, float* state_out, const int32_t* flags = nullptr) {
+    if (flags && *flags) return;   // (a prefill whose device checks failed writes nothing)
     __shared__ float s[CR][CT];
     const int blocks_per_head = d / CR;
     const int h = blockIdx.x / blocks_per_head, r0 = (blockIdx.x % blocks_per_head) * CR;
@@ -60,6 +61,7 @@ __global__ void __launch_bounds__(CT) fold_kernel(const float* state_in, const f
         float acc[CR];
 #pragma unroll
         for (int i = 0; i < CR; ++i) acc[i] = on ? B[(size_t)(r0 + i) * d + k] : 0.f;
+#pragma unroll 8   // eight P rows' loads in flight (d is a multiple of 32)
         for (int m = 0; m < d; ++m) {
             const float pm = on ? P[(size_t)m * d + k] : 0.f;
 #pragma unroll

@@ -15,6 +15,7 @@
 #include "cp.cuh"
 #include "decode.cuh"
 #include "device.cuh"
+#include "fixup.cuh"
 #include "gemm.cuh"
 #include "intra.cuh"
 #include "norm.cuh"
@@ -51,7 +52,8 @@ gdn_status check_config(const gdn_config* c) {
     if (c->n_v_heads % c->n_k_heads != 0) return GDN_ERR_UNSUPPORTED;
     if (!dim_ok(c->d_k) || !dim_ok(c->d_v)) return GDN_ERR_UNSUPPORTED;
     if (c->conv_kernel != 4 || c->chunk != gdn::intra::C) return GDN_ERR_UNSUPPORTED;
-    if (c->prefill_segments < 0 || c->prefill_segments > GDN_PREFILL_MAX_SEGMENTS) return GDN_ERR_INVALID_ARG;
+    if (c->prefill_segments < GDN_PREFILL_SPLIT || c->prefill_segments > GDN_PREFILL_MAX_SEGMENTS)
+        return GDN_ERR_INVALID_ARG;
     return GDN_OK;
 }
 
@@ -59,6 +61,21 @@ gdn_status check_weights(const gdn_weights* w) {
     if (!w || !w->conv_weight || !w->A_log || !w->dt_bias || !w->norm_weight) return GDN_ERR_INVALID_ARG;
     if (!aligned(w->conv_weight, 16)) return GDN_ERR_INVALID_ARG;
     return GDN_OK;
+}
+
+// Split-chain prefill (fixup.cuh): one sequence's chain cut in two at its middle
+// chunk, the second half scanned from zero and, at the same time, as the
+// transition map from the identity; its outputs and end state are then
+// corrected with the first half's end state.  Taken when asked for
+// (GDN_PREFILL_SPLIT), for one sequence at the published head size with bf16
+// activations and output and an fp32 state.  Not chosen automatically: at 4096
+// tokens it measured 363 us against 333 us for two pipelined chunk ranges (the
+// three concurrent scans read records, v and k at a rate that HBM does not
+// sustain, so each runs well below half the chain's time).
+bool split_mode(const gdn_config* c, int64_t T, int64_t n_seqs) {
+    const int64_t chunks = (T + gdn::kChunk - 1) / gdn::kChunk;
+    return c->prefill_segments == GDN_PREFILL_SPLIT && n_seqs == 1 && chunks >= 2 && c->d_k == 128 &&
+           c->d_v == 128 && c->state_dtype == GDN_F32 && c->act_dtype == GDN_BF16 && c->out_dtype == GDN_BF16;
 }
 
 // Chunk ranges a prefill is pipelined over (gdn_config.prefill_segments): range
@@ -77,6 +94,7 @@ struct SegPlan {
 SegPlan seg_plan(const gdn_config* c, int64_t T, int64_t n_seqs) {
     const int64_t chunks = (T + gdn::kChunk - 1) / gdn::kChunk;   // of one sequence of T tokens
     int64_t want = c->prefill_segments;
+    if (want < 0 || split_mode(c, T, n_seqs)) want = 1;   // (the split chain is not range-pipelined)
     if (want == 0)   // automatic: chains too few to fill the GPU, in at most 8 ranges, 32 chunks a range on average
         want = n_seqs * c->n_v_heads <= 96 ? (chunks / 32 < 8 ? chunks / 32 : 8) : 1;
     if (want > GDN_PREFILL_MAX_SEGMENTS) want = GDN_PREFILL_MAX_SEGMENTS;
@@ -111,6 +129,8 @@ SegPlan seg_plan(const gdn_config* c, int64_t T, int64_t n_seqs) {
 // of every chain between the launches over consecutive chunk ranges.
 struct Layout {
     size_t q_off, k_off, v_off, coff_off, flags_off, rec_off, o_off, carry_off, total;
+    // split chain: [P | S_loc] fp32, S0 as bf16, the o^P tiles, a zeroed 64-row v block
+    size_t summ_off = 0, s0b_off = 0, op_off = 0, zv_off = 0;
 };
 
 Layout workspace_layout(const gdn_config* c, int64_t T, int64_t n_seqs) {
@@ -129,7 +149,16 @@ Layout workspace_layout(const gdn_config* c, int64_t T, int64_t n_seqs) {
     L.o_off = L.rec_off + max_chunks * c->n_v_heads * gdn::intra::REC_BYTES;
     L.carry_off = align_up(L.o_off + max_chunks * c->n_v_heads * o_tile, 256);
     L.total = L.carry_off;
-    if (seg_plan(c, T, n_seqs).n > 1) L.total += (size_t)n_seqs * c->n_v_heads * c->d_v * c->d_k * sizeof(float);
+    const size_t st_f32 = (size_t)c->n_v_heads * c->d_v * c->d_k * sizeof(float);
+    if (split_mode(c, T, n_seqs)) {   // carry: the first half's end state
+        L.summ_off = L.carry_off + st_f32;
+        L.s0b_off = L.summ_off + 2 * st_f32;
+        L.op_off = align_up(L.s0b_off + st_f32 / 2, 256);
+        L.zv_off = L.op_off + max_chunks * c->n_v_heads * o_tile;
+        L.total = align_up(L.zv_off + (size_t)gdn::intra::C * c->n_v_heads * c->d_v * sizeof(__half), 256);
+    } else if (seg_plan(c, T, n_seqs).n > 1) {
+        L.total += (size_t)n_seqs * st_f32;
+    }
     return L;
 }
 
@@ -210,7 +239,8 @@ HostLayout host_layout(const gdn_config* c, int64_t T, int32_t n_seqs) {
 // Opt in to > 48 KiB of dynamic shared memory, once per device and kernel.
 template <typename K>
 cudaError_t ensure_smem(K kernel, int variant, size_t bytes) {
-    static bool done[64][32];
+    static bool done[64][32];   // variants in use: 4-6, 8-20, 24-31
+    if (variant < 0 || variant >= 32) return cudaErrorInvalidValue;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
@@ -340,7 +370,7 @@ cudaStream_t side_stream(int which = 0) {
 // reused from call to call: a stream wait refers to the record enqueued before
 // it, so recording an event again in a later call leaves earlier waits intact,
 // and no two threads share an event.
-enum EventUse { kEvStageA = 0, kEvCp = 1, kEvHost = 2, kEvPipe = 3, kEvUses = 4 };
+enum EventUse { kEvStageA = 0, kEvCp = 1, kEvHost = 2, kEvPipe = 3, kEvSplit = 4, kEvUses = 5 };
 
 struct EventPool {
     std::vector<cudaEvent_t> ev[64][kEvUses];
@@ -815,11 +845,154 @@ cudaError_t launch_norm(const gdn_config* c, const gdn_weights* w, const void* z
 // chains that end earlier until then).  A call whose checks fail therefore
 // leaves out and the states as they were.  Every side stream that has been
 // forked is joined back to `st` on every path.
+// 2-D tensor map over row-major [rows][128] bf16 with boxes of 64 columns x box_rows,
+// 128-byte swizzle (the split chain's o^P tiles and bf16 start state).
+bool rows128_map(CUtensorMap* m, const void* base, int64_t rows, int box_rows) {
+    auto enc = tensor_map_encoder();
+    if (!enc) return false;
+    cuuint64_t dims[2] = {128, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {128 * 2};
+    cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+    cuuint32_t estr[2] = {1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// The split chain (split_mode; one sequence, bf16 activations and output, fp32 state):
+//   st:      stage A (conv-state update on its side stream), the start states of the
+//            second half (zero and identity) and the zero v block, the first half's scan
+//            (its end state into the carry), its end state to bf16, then (after the two
+//            side scans) the second half's correction and gated norm (fixup.cuh), and the
+//            fold of the end state into rec_state;
+//   side 5:  the first half's gated norm, after its scan;
+//   side 4:  the second half scanned from zero (S_loc; o^loc tiles);
+//   side 0:  the second half scanned from the identity with V = 0 (the transition P;
+//            o^P tiles).
+// The three scans take 48 SMs each at the same time.  Nothing the caller sees is
+// written before every device check has passed (every kernel reads the check word).
+template <typename TA, typename TO>
+cudaError_t launch_prefill_split(const gdn_config* c, const gdn_weights* w, const void* q, const void* k,
+                                 const void* v, const void* a, const void* b, const void* z, void* conv_state,
+                                 void* rec_state, const int32_t* cu, int64_t T, void* out, void* ws, cudaStream_t st) {
+    const Layout L = workspace_layout(c, T, 1);
+    uint8_t* wsb = static_cast<uint8_t*>(ws);
+    const int Hv = c->n_v_heads, d = c->d_k;
+    const int64_t chunks = (T + gdn::kChunk - 1) / gdn::kChunk, mid = chunks / 2;
+    const int64_t per = (int64_t)Hv * d * d;
+    float* C0 = reinterpret_cast<float*>(wsb + L.carry_off);
+    float* summ = reinterpret_cast<float*>(wsb + L.summ_off);   // [P | S_loc]
+    __nv_bfloat16* s0b = reinterpret_cast<__nv_bfloat16*>(wsb + L.s0b_off);
+    const int32_t* flags = reinterpret_cast<const int32_t*>(wsb + L.flags_off);
+
+    StageA<TA> A;
+    ScanSetup B0, B1, B2;
+    NormSetup N;
+    CUtensorMap tm_p, tm_s;
+    cudaError_t e = prepare_stage_a<TA>(c, w, q, k, v, a, b, conv_state, cu, 1, T, ws, &A);
+    if (e == cudaSuccess)
+        e = prepare_scan<TO>(c, wsb + L.v_off, T, rec_state, cu, 1, T, ws, nullptr, &B0);
+    if (e == cudaSuccess) e = prepare_scan<TO>(c, wsb + L.v_off, T, summ + per, cu, 1, T, ws, nullptr, &B1);
+    if (e == cudaSuccess) e = prepare_scan<TO>(c, wsb + L.zv_off, gdn::intra::C, summ, cu, 1, T, ws, wsb + L.op_off, &B2);
+    if (e == cudaSuccess) e = prepare_norm<TA, TO>(c, w, z, cu, 1, T, out, ws, &N);
+    if (e == cudaSuccess)
+        e = ensure_smem(gdn::fix::gdn_fixup_norm_kernel, 6, gdn::fix::SMEM_BYTES);
+    if (e != cudaSuccess) return e;
+    if (!rows128_map(&tm_p, wsb + L.op_off, (int64_t)A.max_chunks * Hv * 64, 64) ||
+        !rows128_map(&tm_s, s0b, (int64_t)Hv * 128, 128))
+        return cudaErrorInvalidValue;
+    B0.sa.carry = C0;                        // the first half's end state
+    B1.sa.carry = summ + per;                // S_loc: starts at zero, ends there
+    B2.sa.carry = summ;                      // P: starts at the identity, ends there
+    cudaStream_t side[3] = {side_stream(4), side_stream(0), side_stream(5)};
+    // start states ready; the two side scans done; the first half's scan done; its norm done
+    cudaEvent_t* ev = thread_events(kEvSplit, 5);
+    if (!side[0] || !side[1] || !side[2] || !ev) return cudaErrorNotReady;
+
+    cudaEvent_t join = nullptr;   // the conv-state update's side stream
+    cudaStream_t aux = side_stream(3);
+    cudaEvent_t* evA = thread_events(kEvStageA, 2);
+    if (!aux || !evA) return cudaErrorNotReady;
+    e = launch_chunk_offsets(A, st);
+    if (e == cudaSuccess) e = launch_conv(A, 0, A.max_chunks, st);
+    if (e == cudaSuccess && (e = cudaEventRecord(evA[0], st)) == cudaSuccess &&
+        (e = cudaStreamWaitEvent(aux, evA[0], 0)) == cudaSuccess) {
+        const cudaError_t e_side = launch_conv_state(A, aux);
+        if ((e = cudaEventRecord(evA[1], aux)) == cudaSuccess) join = evA[1];
+        if (e == cudaSuccess) e = e_side;
+    }
+    if (e == cudaSuccess) e = launch_intra(A, 0, A.max_chunks, st);
+    if (e == cudaSuccess) {
+        gdn::fix::split_init_kernel<<<(unsigned)std::min<int64_t>((2 * per + 255) / 256, 1024), 256, 0, st>>>(
+            summ, Hv, d, flags);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess)
+        e = cudaMemsetAsync(wsb + L.zv_off, 0, (size_t)gdn::intra::C * Hv * c->d_v * sizeof(__half), st);
+    bool forked[3] = {false, false, false};
+    if (e == cudaSuccess) e = cudaEventRecord(ev[0], st);
+    for (int i = 0; i < 2 && e == cudaSuccess; i++) {
+        if ((e = cudaStreamWaitEvent(side[i], ev[0], 0)) != cudaSuccess) break;
+        forked[i] = true;
+        e = launch_scan_range(i == 0 ? B1 : B2, mid, 0x7fffffff, false, side[i]);
+        const cudaError_t r = cudaEventRecord(ev[1 + i], side[i]);
+        if (e == cudaSuccess) e = r;
+    }
+    if (e == cudaSuccess) e = launch_scan_range(B0, 0, mid, false, st);
+    // the first half's norm beside the second half's scans
+    if (e == cudaSuccess && (e = cudaEventRecord(ev[3], st)) == cudaSuccess &&
+        (e = cudaStreamWaitEvent(side[2], ev[3], 0)) == cudaSuccess) {
+        forked[2] = true;
+        e = launch_norm_range<TA, TO>(N, 0, mid, side[2]);
+        const cudaError_t r = cudaEventRecord(ev[4], side[2]);
+        if (e == cudaSuccess) e = r;
+    }
+    if (e == cudaSuccess) {
+        gdn::fix::state_to_bf16_kernel<<<(unsigned)std::min<int64_t>((per / 4 + 255) / 256, 1024), 256, 0, st>>>(
+            C0, s0b, per, flags);
+        e = cudaGetLastError();
+    }
+    for (int i = 0; i < 2; i++) {   // join the side scans, whatever happened above
+        if (!forked[i]) continue;
+        const cudaError_t r = cudaStreamWaitEvent(st, ev[1 + i], 0);
+        if (e == cudaSuccess) e = r;
+    }
+    if (e == cudaSuccess) {
+        gdn::fix::Args fa;
+        fa.o_loc = reinterpret_cast<const __nv_bfloat16*>(wsb + L.o_off);
+        fa.z = static_cast<const __nv_bfloat16*>(z);
+        fa.norm_w = w->norm_weight;
+        fa.out = static_cast<__nv_bfloat16*>(out);
+        fa.flags = flags;
+        fa.T = T;
+        fa.Hv = Hv;
+        fa.c_lo = (int)mid;
+        fa.c_hi = (int)chunks;
+        fa.eps = c->norm_eps;
+        const int64_t pairs = (chunks - mid + 1) / 2;
+        gdn::fix::gdn_fixup_norm_kernel<<<(unsigned)(pairs * Hv), gdn::fix::NT, gdn::fix::SMEM_BYTES, st>>>(tm_p, tm_s,
+                                                                                                         fa);
+        e = cudaGetLastError();
+    }
+    if (e == cudaSuccess) {
+        gdn::cp::fold_kernel<<<(unsigned)(Hv * (d / gdn::cp::CR)), gdn::cp::CT, 0, st>>>(
+            C0, summ, 1, Hv, d, static_cast<float*>(rec_state), flags);
+        e = cudaGetLastError();
+    }
+    if (forked[2]) {   // the first half's norm
+        const cudaError_t r = cudaStreamWaitEvent(st, ev[4], 0);
+        if (e == cudaSuccess) e = r;
+    }
+    return join_side(join, st, e);
+}
+
 template <typename TA, typename TO>
 cudaError_t launch_prefill(const gdn_config* c, const gdn_weights* w, const void* q, const void* k,
                            const void* v, const void* a, const void* b, const void* z, void* conv_state,
                            void* rec_state, const int32_t* cu, int n_seqs, int64_t T, void* out,
                            void* ws, cudaStream_t st) {
+    if (sizeof(TA) == 2 && sizeof(TO) == 2 && split_mode(c, T, n_seqs))
+        return launch_prefill_split<TA, TO>(c, w, q, k, v, a, b, z, conv_state, rec_state, cu, T, out, ws, st);
     const Layout L = workspace_layout(c, T, n_seqs);
     const SegPlan P = seg_plan(c, T, n_seqs);
     if (P.n == 1) {
@@ -999,6 +1172,7 @@ size_t gdn_prefill_workspace_size(const gdn_config* cfg, int64_t T_total, int32_
 
 int32_t gdn_prefill_segments(const gdn_config* cfg, int64_t T_total, int32_t n_seqs) {
     if (check_config(cfg) != GDN_OK || T_total < 0 || n_seqs < 0) return 0;
+    if (split_mode(cfg, T_total, n_seqs)) return GDN_PREFILL_SPLIT;
     return seg_plan(cfg, T_total, n_seqs).n;
 }
 

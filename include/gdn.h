@@ -86,16 +86,28 @@ typedef struct {
                              (the layer's fp32 state).  GDN_BF16 stores the state in bf16
                              (half the bytes a decode step moves); every step still
                              computes in fp32 and rounds the stored state to nearest even */
-    int32_t prefill_segments; /* chunk ranges a prefill is pipelined over (0 = automatic,
-                             the default; 1 = none; at most GDN_PREFILL_MAX_SEGMENTS).  The
-                             ranges' conv and intra-chunk kernels run on the caller's stream
-                             while the state chain walks the ranges before them on a
-                             high-priority stream of the library's own, so chains too few to
-                             fill the GPU overlap the work that feeds them.  The results do
-                             not depend on it, bit for bit */
+    int32_t prefill_segments; /* how a prefill overlaps its state chain with other work.
+                             n >= 2: pipelined over n chunk ranges (at most
+                             GDN_PREFILL_MAX_SEGMENTS): the ranges' conv and intra-chunk
+                             kernels run on the caller's stream while the state chain walks
+                             the ranges before them on a high-priority stream of the
+                             library's own; the results are those of one range, bit for bit.
+                             1: one range.  GDN_PREFILL_SPLIT (-1): for one sequence at
+                             d_k = d_v = 128 with bf16 activations and output and an fp32
+                             state, the chain is cut in two at its middle chunk and the
+                             halves run at the same time (the second from a zero state and as
+                             its transition map), then the second half's outputs and end state
+                             are corrected with the first half's end state; other calls take
+                             one range.  The results then differ from one range's within the
+                             rounding of the bf16 correction (well inside the layer's
+                             tolerances).  0 (the default): automatic, at most 8 ranges of at
+                             least 32 chunks when the call has at most 96 chains
+                             (n_seqs x H_v), else one range */
 } gdn_config;
 
 #define GDN_PREFILL_MAX_SEGMENTS 32
+/* gdn_config.prefill_segments: split one sequence's state chain in two (see gdn_prefill) */
+#define GDN_PREFILL_SPLIT (-1)
 
 typedef struct {
     const float* conv_weight;  /* [2*H_k*d_k + H_v*d_v][K], channel order q | k | v;
@@ -113,11 +125,10 @@ void gdn_config_default(gdn_config* cfg);
  * Returns 0 for an invalid or unsupported config. */
 size_t gdn_prefill_workspace_size(const gdn_config* cfg, int64_t T_total, int32_t n_seqs);
 
-/* Chunk ranges gdn_prefill pipelines a call of this size over (see
- * gdn_config.prefill_segments): 1 when it runs in one piece; with n > 1 ranges a
- * call launches 2 + 4 n kernels (else 6).  Automatic (prefill_segments 0): at
- * most 8 ranges of at least 32 chunks when the call has at most 96 chains
- * (n_seqs x H_v); else 1.  Returns 0 for an invalid config. */
+/* How gdn_prefill runs a call of this size (see gdn_config.prefill_segments): the
+ * number of chunk ranges it is pipelined over (1 when it runs in one piece; with
+ * n > 1 ranges a call launches 2 + 4 n kernels, else 6), or GDN_PREFILL_SPLIT when
+ * it splits the chain (13 kernels).  Returns 0 for an invalid config. */
 int32_t gdn_prefill_segments(const gdn_config* cfg, int64_t T_total, int32_t n_seqs);
 
 /*

@@ -58,31 +58,46 @@ def test_workspace_size(lib):
     per_chunk = 48 * (58368 + 64 * 128 * 2)
     carry = 48 * 128 * 128 * 4
     assert gdn.workspace_size(cfg, T, 1) == conv + 256 + (T // 64 + 1) * per_chunk + carry
+    # the split chain (asked for): the first half's end state, [P | S_loc], S0 in bf16, a second
+    # set of o tiles and a zeroed 64-row v block
+    split = 3 * carry + carry // 2 + (T // 64 + 1) * 48 * 64 * 128 * 2 + 64 * 48 * 128 * 2
+    assert gdn.workspace_size(gdn.Config(prefill_segments=-1), T, 1) == conv + 256 + (T // 64 + 1) * per_chunk + split
     assert gdn.workspace_size(gdn.Config(prefill_segments=1), T, 1) == conv + 256 + (T // 64 + 1) * per_chunk
     assert gdn.workspace_size(cfg, T, 2) == conv + 256 + (T // 64 + 2) * per_chunk + 2 * carry
     assert gdn.workspace_size(cfg, T, 3) == conv + 256 + (T // 64 + 3) * per_chunk
     assert gdn.workspace_size(gdn.Config(prefill_segments=4), T, 3) == conv + 256 + (T // 64 + 3) * per_chunk + 3 * carry
-    assert gdn.workspace_size(cfg, 4032, 1) == 2 * 4032 * 2048 * 2 + 4032 * 6144 * 2 + 256 + 64 * per_chunk
-    assert gdn.workspace_size(cfg, 4033, 1) == 2 * 4033 * 2048 * 2 + 4033 * 6144 * 2 + 256 + 65 * per_chunk + carry
-    f32 = gdn.Config(out_dtype=__import__("torch").float32)
+    w = lambda T_, n: 2 * T_ * 2048 * 2 + T_ * 6144 * 2 + 256 + (-(-T_ // 64) + n) * per_chunk
+    assert gdn.workspace_size(cfg, 4032, 2) == w(4032, 2)
+    assert gdn.workspace_size(cfg, 4033, 2) == w(4033, 2) + 2 * carry
+    f32 = gdn.Config(out_dtype=__import__("torch").float32)   # (no split chain with an fp32 output)
     assert gdn.workspace_size(f32, T, 1) == conv + 256 + (T // 64 + 1) * 48 * (58368 + 64 * 128 * 4) + carry
     assert gdn.workspace_size(cfg, T, 63) == conv + 512 + (T // 64 + 63) * per_chunk
     assert gdn.workspace_size(cfg, 0, 0) == 256
     assert gdn.workspace_size(gdn.Config(d_k=48), T, 1) == 0
-    assert gdn.workspace_size(gdn.Config(prefill_segments=-1), T, 1) == 0
+    assert gdn.workspace_size(gdn.Config(prefill_segments=-2), T, 1) == 0
     assert gdn.workspace_size(gdn.Config(prefill_segments=33), T, 1) == 0
 
 
 def test_prefill_segments_plan(lib):
     cfg = gdn.Config()
+    SPLIT = -1
     # automatic: at most 8 ranges of at least 32 chunks for at most 96 chains (2 sequences of 48 heads)
     assert gdn.prefill_segments(cfg, 4096, 1) == 2
+    assert gdn.prefill_segments(cfg, 4032, 1) == 1 and gdn.prefill_segments(cfg, 4033, 1) == 2
     assert gdn.prefill_segments(cfg, 4096, 2) == 2
     assert gdn.prefill_segments(cfg, 4096, 3) == 1
-    assert gdn.prefill_segments(cfg, 4032, 1) == 1 and gdn.prefill_segments(cfg, 4033, 1) == 2
+    assert gdn.prefill_segments(cfg, 4032, 2) == 1 and gdn.prefill_segments(cfg, 4033, 2) == 2
     assert gdn.prefill_segments(cfg, 16384, 1) == 8
     assert gdn.prefill_segments(cfg, 262144, 1) == 8
     assert gdn.prefill_segments(cfg, 0, 0) == 1
+    # asked for: the split chain where it applies (one sequence, published head size, bf16 in and
+    # out, fp32 state), else one range
+    assert gdn.prefill_segments(gdn.Config(prefill_segments=SPLIT), 200, 1) == SPLIT
+    assert gdn.prefill_segments(gdn.Config(prefill_segments=SPLIT), 64, 1) == 1
+    assert gdn.prefill_segments(gdn.Config(prefill_segments=SPLIT), 4096, 2) == 1
+    import torch
+    assert gdn.prefill_segments(gdn.Config(prefill_segments=SPLIT, state_dtype=torch.bfloat16), 4096, 1) == 1
+    assert gdn.prefill_segments(gdn.Config(prefill_segments=SPLIT, d_k=64, d_v=64), 4096, 1) == 1
     # asked for: ranges of ceil(chunks / n) chunks, never more ranges than chunks
     assert gdn.prefill_segments(gdn.Config(prefill_segments=7), 4096, 1) == 7
     assert gdn.prefill_segments(gdn.Config(prefill_segments=32), 4096, 5) == 32
