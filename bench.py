@@ -69,6 +69,12 @@ DECODE_TRAFFIC = 1593363968          # mean of 3 launches at batch 256
 DECODE_SRC_SHA = "4315b287d18a287c"
 DECODE_KERNEL_TEXT = ("template <typename TA, typename TO, typename TS, int DK>\n"
                       "__global__ void __launch_bounds__(NT) gdn_decode_kernel", "// Multi-token rows")
+# Tensor-pipe activity of the prefill's tensor-core kernels (ncu
+# sm__pipe_tensor_cycles_active.avg.pct_of_peak_sustained_active, one --set full capture of the
+# 4K prefill in one chunk range; the scan's average is over the SMs that run it), taken on the
+# sources that hash to the given values; null once a file changes.
+TENSOR_PIPE_NCU = {"gdn_intra_kernel": ("intra.cuh", "b1f14988bf943661", 0.0411),
+                   "gdn_scan_kernel": ("scan.cuh", "4ce0eddd0125a8b0", 0.2811)}
 
 
 def peaks():
@@ -525,6 +531,9 @@ def main():
                                  "bytes_per_call": PREFILL_BYTES_PER_TOKEN * PREFILL_T + PREFILL_STATE_BYTES,
                                  "tensor_achieved_tflops": pre_tflops, "tensor_peak_tflops": pk["bf16_tflops"],
                                  "tensor_frac": pre_tflops / pk["bf16_tflops"], "peak_source": src},
+            "tensor_pipe": dict({k: (v[2] if src_sha(v[0]) == v[1] else None) for k, v in TENSOR_PIPE_NCU.items()},
+                                target=0.40, source="ncu captures in profiles/gdn_intra_kernel_prefill_4k.md and "
+                                                    "profiles/gdn_scan_kernel_prefill_4k.md"),
             "clocks": clocks.summary(),
             "e2e": {"value": PREFILL_T * world * K / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
