@@ -34,8 +34,8 @@
 // (c), which run while the state is converted; it waits for
 // the next MMA's operands while the workers convert, so each conversion is
 // followed by an immediate issue.  While MMA1 runs, the 16 worker warps write the
-// decayed state accumulator and the previous chunk's o tile (once its MMA2b has
-// completed), and zero that O accumulator for the chunk after next; MMA2a, the
+// decayed state accumulator and stage the previous chunk's o tile (once its MMA2b
+// has completed; MMA1's first K step restarts each O accumulator); MMA2a, the
 // shortest product, is left to run alone.  An 18th warp issues
 // every copy: a bulk copy holds its issuing thread for about as long as the copy
 // engine takes to walk its bytes, so copies stay off the MMA chain.  It meets
@@ -299,6 +299,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant_
     const uint64_t dV0 = sdesc(sb + OFF_V, 8192, 1024);
     const uint64_t dT0 = sdesc(sb + OFF_R + R_T, 16, 1024);
     constexpr uint32_t ID_1 = idesc_f16(128, 128, 0, 0);    // MMA1
+    constexpr uint32_t ID_1H = idesc_f16(128, 64, 0, 0);    // MMA1's first K step, one half at a time
     constexpr uint32_t ID_2A = idesc_f16(128, 128, 0, 1);   // MMA2a
     constexpr uint32_t ID_2B = idesc_f16(128, 64, 0, 1);    // MMA2b
     constexpr uint32_t ID_C = idesc_f16(128, 64, 1, 0);     // (c)
@@ -334,7 +335,7 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant_
         for (int i = 0; i < 32; i++) d[i] = __float_as_uint(decay * Sv[i]);
         tmem_st32(tl + ACC_S + 32 * cs, d);
     };
-    // o = O / sqrt(d_k) of chunk ce -> staging, and its accumulator zeroed for chunk ce + 2
+    // o = O / sqrt(d_k) of chunk ce -> staging (MMA1 of chunk ce + 2 restarts the accumulator)
     auto stage_o = [&](int ce) {
         uint32_t o[16];
         tmem_ld16(tl + acc_o(ce & 1) + 16 * cs, o);
@@ -342,20 +343,10 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant_
 #pragma unroll
         for (int i = 0; i < 16; i++) from_f32(__uint_as_float(o[i]) * inv_sqrt_dk, st + (16 * cs + i) * 128 + dv_r);
         fence_async_smem();
-#pragma unroll
-        for (int i = 0; i < 16; i++) o[i] = 0u;
-        tmem_st16(tl + acc_o(ce & 1) + 16 * cs, o);
     };
 
-    // ---- prologue: zero O accumulators, fp16 S0; (c) of chunk 0 ----
-    if (worker) {
-        uint32_t z[16];
-#pragma unroll
-        for (int i = 0; i < 16; i++) z[i] = 0u;
-        tmem_st16(tl + acc_o(0) + 16 * cs, z);
-        tmem_st16(tl + acc_o(1) + 16 * cs, z);
-        put_state_a();
-    }
+    // ---- prologue: fp16 S0; (c) of chunk 0 ----
+    if (worker) put_state_a();
     if (warp == IW) {
         wait_par(bar_ld0, 0);
         tc_fence_after();
@@ -380,11 +371,14 @@ gdn_scan_kernel(const __grid_constant__ CUtensorMap tm_v, const __grid_constant_
         const int b = ci & 1;
         float dU[16];   // e^{g_C - g_c} for this worker's 16 chunk positions c = 16 cs + i
 
-        // ---- MMA1: [U2^T | O^T] += S [-W ; Q~]^T ((c) and the zeroed O are already there) ----
+        // ---- MMA1: U2^T += S (-W)^T onto (c)'s result, O^T = S Q~^T; the first K step in halves,
+        // so that the O half starts its accumulator, the rest at N = 128 ----
         if (warp == IW) {
             tc_fence_after();
+            mma_f16_ta_w(tmem + acc_u(b), tmem + TA_S, dB1 + b * (R_STRIDE >> 4), ID_1H, 1);
+            mma_f16_ta_w(tmem + acc_o(b), tmem + TA_S, dB1 + b * (R_STRIDE >> 4) + (8192 >> 4), ID_1H, 0);
 #pragma unroll
-            for (int ks = 0; ks < 8; ks++)
+            for (int ks = 1; ks < 8; ks++)
                 mma_f16_ta_w(tmem + acc_u(b), tmem + TA_S + ks * 8,
                              dB1 + b * (R_STRIDE >> 4) + (ks >> 2) * 1024 + (ks & 3) * 2, ID_1, 1);
             mma_commit_w(bar);
