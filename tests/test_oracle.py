@@ -375,6 +375,30 @@ def test_linear_reads_bf16_exactly():
 # Segment state maps (context-parallel prefill)
 # ---------------------------------------------------------------------------
 
+def test_segment_outputs_are_affine_in_the_start_state():
+    """Over a segment the pre-norm outputs are affine in the start state too:
+    o_t = o_t^loc + S_0 o_t^P, with o^loc the outputs of the run from 0 and o^P those of
+    the v = 0 run from I (the transported queries).  This is what the split-chain prefill
+    computes for the second half of a sequence; the end state is the segment map's."""
+    rng = np.random.default_rng(37)
+    shape, w, acts, cs, rs, cu = _random_case(rng, Hk=1, G=2, d=4, T=11, n_seqs=1, state_std=0.5)
+    Hv, d = shape.n_v_heads, shape.d_k
+    loc = _run(shape, w, acts, cs, np.zeros_like(rs), cu, want_o_pre=True)["o_pre"]
+    cs0 = cs.copy()
+    cs0[:, 2 * shape.n_k_heads * d:] = 0.0   # v = 0 in the conv window too
+    acts0 = dict(acts, v=np.zeros_like(acts["v"]))
+    eye = np.broadcast_to(np.eye(d), (1, Hv, d, d)).copy()
+    oP = _run(shape, w, acts0, cs0, eye, cu, want_o_pre=True)["o_pre"]
+    for trial in range(3):
+        S0 = rng.normal(0, 0.7, (1, Hv, d, d))
+        true = _run(shape, w, acts, cs, S0, cu, want_o_pre=True)["o_pre"]
+        np.testing.assert_allclose(true, loc + np.einsum("hvk,thk->thv", S0[0], oP), rtol=0, atol=1e-12)
+    # and a wrong transport (S0^T instead of S0) does not satisfy it
+    S0 = rng.normal(0, 0.7, (1, Hv, d, d))
+    true = _run(shape, w, acts, cs, S0, cu, want_o_pre=True)["o_pre"]
+    assert np.abs(true - (loc + np.einsum("hkv,thk->thv", S0[0], oP))).max() > 1e-3
+
+
 def test_segment_map_is_the_affine_state_map():
     """For any S_0 the segment's end state is S_0 . P + S_loc, with (P, S_loc) from the
     v = 0 run from I and the run from 0; folding two segments' maps equals one run over
