@@ -63,6 +63,7 @@ EXPORTS = ("gdn_config_default", "gdn_prefill_workspace_size", "gdn_prefill_segm
            "gdn_cp_local", "gdn_cp_finish", "gdn_prefill_host_workspace_size", "gdn_prefill_host",
            "gdn_check_device_error", "gdn_status_string", "gdn_last_cuda_error")
 DECODE_MULTI_MAX_TOKENS = 16   # GDN_DECODE_MULTI_MAX_TOKENS
+PREFILL_SPLIT = -1             # GDN_PREFILL_SPLIT: Config.prefill_segments value that splits the chain
 LINEAR_MAX_SEGMENTS = 8        # GDN_LINEAR_MAX_SEGMENTS
 
 
@@ -131,7 +132,8 @@ class Config:
     act_dtype: torch.dtype = torch.bfloat16
     out_dtype: torch.dtype = torch.bfloat16
     state_dtype: torch.dtype = torch.float32   # bf16: the recurrent state stored in bf16
-    prefill_segments: int = 0                  # chunk ranges a prefill is pipelined over; 0: automatic
+    prefill_segments: int = 0                  # chunk ranges a prefill is pipelined over; 0: automatic;
+                                               # PREFILL_SPLIT: one sequence's chain split in two
 
     @property
     def channels(self) -> int:
