@@ -128,7 +128,7 @@ size_t gdn_prefill_workspace_size(const gdn_config* cfg, int64_t T_total, int32_
 /* How gdn_prefill runs a call of this size (see gdn_config.prefill_segments): the
  * number of chunk ranges it is pipelined over (1 when it runs in one piece; with
  * n > 1 ranges a call launches 2 + 4 n kernels, else 6), or GDN_PREFILL_SPLIT when
- * it splits the chain (13 kernels).  Returns 0 for an invalid config. */
+ * it splits the chain (12 kernels and one memset).  Returns 0 for an invalid config. */
 int32_t gdn_prefill_segments(const gdn_config* cfg, int64_t T_total, int32_t n_seqs);
 
 /*
